@@ -1,0 +1,290 @@
+"""Pins of the CPU oracle against things other than itself.
+
+Each test ties one oracle function to a value the pages print, a closed form, a library
+routine on a special case, or brute force, chosen so that a dropped term, a wrong sign or
+index, or a transposed operand in the oracle fails at least one of them.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+from sparse_fp32_softmax_b200 import inputs
+from sparse_fp32_softmax_b200.roofline import moe_parameter_split
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+def logits_of(probs):
+    """FP32 logits whose softmax is ``probs`` (up to FP32 rounding of the logarithm)."""
+    return np.log(np.asarray(probs, np.float64)).astype(np.float32)[None, :]
+
+
+# ------------------------------------------------------------------ router: pages' values
+
+def test_worked_example(oracle_mod):
+    g = golden("worked_example.json")
+    l = logits_of(g["probs"])
+    idx, w = oracle_mod.select(l, g["k"], norm=True)
+    assert idx[0].tolist() == g["experts"]
+    assert np.abs(w[0] - np.array(g["weights_renorm"])).max() <= 1e-6
+    idx, w = oracle_mod.select(l, g["k"], norm=False)
+    assert idx[0].tolist() == g["experts"]
+    assert np.abs(w[0] - np.array(g["weights_plain"])).max() <= 1e-6
+
+
+def test_renorm_example(oracle_mod):
+    g = golden("renorm_example.json")
+    idx, w = oracle_mod.select(logits_of(g["probs"]), g["k"], norm=True)
+    assert idx[0].tolist() == g["experts"]
+    assert np.abs(w[0] - np.array(g["weights_renorm"])).max() <= 1e-6
+    # the page's printed rounding of the same values
+    assert sorted(np.floor(w[0] * 100) / 100) == sorted(g["printed_rounded"])
+
+
+def test_worked_example_k3_index_tiebreak(oracle_mod):
+    # Same probabilities, k = 3: experts 0 and 3 tie at 0.1; the lower index wins.
+    idx, w = oracle_mod.select(logits_of([0.1, 0.5, 0.3, 0.1]), 3, norm=True)
+    assert idx[0].tolist() == [1, 2, 0]
+    assert np.abs(w[0] - np.array([5 / 9, 1 / 3, 1 / 9])).max() <= 1e-6
+    assert abs(float(w[0].sum()) - 1.0) <= 1e-6
+
+
+# ------------------------------------------------------------------ router: closed forms
+
+def test_softmax_closed_form(oracle_mod):
+    l = np.array([[0.0, math.log(2.0), math.log(3.0)]], np.float32)
+    idx, w = oracle_mod.select(l, 3, norm=False)
+    assert idx[0].tolist() == [2, 1, 0]
+    assert np.abs(w[0] - np.array([3 / 6, 2 / 6, 1 / 6])).max() <= 1e-7
+
+
+def test_softmax_matches_library_when_k_equals_E(oracle_mod):
+    from scipy.special import softmax
+    rng = np.random.default_rng(5)
+    l = rng.normal(size=(7, 13)).astype(np.float32)
+    for norm in (False, True):
+        idx, w = oracle_mod.select(l, 13, norm=norm)
+        ref = softmax(l.astype(np.float64), axis=1)
+        got = np.zeros_like(ref)
+        np.put_along_axis(got, idx.astype(np.int64), w.astype(np.float64), axis=1)
+        assert np.abs(got - ref).max() <= 1e-7          # renorm of the full set is a no-op
+        order = np.argsort(-l, axis=1, kind="stable")    # library stable sort, lower index first
+        assert (idx == order).all()
+
+
+def test_k1_renorm_is_exactly_one(oracle_mod):
+    rng = np.random.default_rng(6)
+    l = rng.normal(size=(9, 6)).astype(np.float32)
+    idx, w = oracle_mod.select(l, 1, norm=True)
+    assert (w == 1.0).all()
+    assert (idx[:, 0] == np.argmax(l, axis=1)).all()
+
+
+def test_renorm_sums_to_one(oracle_mod):
+    rng = np.random.default_rng(7)
+    l = rng.normal(size=(50, 64)).astype(np.float32)
+    _, w = oracle_mod.select(l, 8, norm=True)
+    assert np.abs(w.astype(np.float64).sum(1) - 1.0).max() <= 1e-6
+
+
+@pytest.mark.parametrize("k", [1, 2, 3])
+def test_index_tiebreak(oracle_mod, k):
+    l = np.array([[1.0, 3.0, 3.0, 0.0, 3.0]], np.float32)
+    idx, _ = oracle_mod.select(l, k, norm=True)
+    assert idx[0].tolist() == [1, 2, 4][:k]
+    z = np.zeros((1, 6), np.float32)
+    idx, w = oracle_mod.select(z, 4, norm=True)
+    assert idx[0].tolist() == [0, 1, 2, 3]
+    assert np.abs(w - 0.25).max() == 0.0
+    # -0.0 and +0.0 are the same value: the lower index ranks first
+    s = np.array([[-0.0, 0.0, -1.0]], np.float32)
+    assert oracle_mod.select(s, 1)[0][0].tolist() == [0]
+    s = np.array([[0.0, -0.0, -1.0]], np.float32)
+    assert oracle_mod.select(s, 2)[0][0].tolist() == [0, 1]
+
+
+def test_router_logits_one_hot_rows(oracle_mod):
+    rng = np.random.default_rng(8)
+    E, D = 10, 64
+    W = torch.from_numpy(rng.normal(scale=0.02, size=(E, D)).astype(np.float32)).to(torch.bfloat16)
+    x = torch.zeros(D, D, dtype=torch.bfloat16)
+    for j in range(D):
+        x[j, j] = 1.0
+    l = oracle_mod.router_logits(x, W)
+    assert np.array_equal(l, W.float().numpy().T)       # l[t=j, e] = W[e, j], exactly
+    b = rng.normal(size=E).astype(np.float32)
+    lb = oracle_mod.router_logits(x, W, b)
+    assert np.array_equal(lb, (W.float().numpy().T + b[None, :]).astype(np.float32))
+
+
+def test_router_logits_match_library_matmul(oracle_mod):
+    g = torch.Generator().manual_seed(9)
+    x = torch.randn(33, 96, generator=g).to(torch.bfloat16)
+    W = (0.02 * torch.randn(17, 96, generator=g)).to(torch.bfloat16)
+    l = oracle_mod.router_logits(x, W)
+    ref = (x.double() @ W.double().T).float().numpy()
+    # both are the exact dot product rounded once to FP32 (sums of <= 96 exact products in
+    # double are exact to far below FP32's last bit, barring a double-rounding tie)
+    ulp = np.spacing(np.abs(ref))
+    assert (np.abs(l - ref) <= ulp).all()
+
+
+def test_tiny_tie_rows(oracle_mod):
+    cfg = inputs.CONFIGS["tiny"]
+    L = inputs.make_layer(cfg)
+    logits, idx, w = oracle_mod.route(L["x"], L["W_r"], cfg.k, cfg.norm_topk_prob)
+    for row, (_, vals, expect) in inputs.TINY_TIES.items():
+        assert tuple(idx[row].tolist()) == expect, row
+    for row in (5, 42, 63):
+        assert (w[row] == 0.5).all(), row
+    y, _, _, _ = oracle_mod.forward_rows(L["x"], L["W_r"], L["W_gate_up"], L["W_down"], cfg.k, [63])
+    assert np.abs(y).max() == 0.0                       # zero token -> silu(0) * 0 = 0
+
+
+# ------------------------------------------------------------------ experts
+
+def _small_layer(T=12, D=64, E=5, I=32, seed=11):
+    g = torch.Generator().manual_seed(seed)
+    x = torch.randn(T, D, generator=g).to(torch.bfloat16)
+    W_r = (0.3 * torch.randn(E, D, generator=g)).to(torch.bfloat16)
+    W_gu = (0.1 * torch.randn(E, 2 * I, D, generator=g)).to(torch.bfloat16)
+    W_dn = (0.1 * torch.randn(E, D, I, generator=g)).to(torch.bfloat16)
+    return x, W_r, W_gu, W_dn
+
+
+def _swiglu_ffn_library(x, W_gu, W_dn):
+    """Textbook SwiGLU FFN with torch.nn.functional in float64."""
+    I = W_gu.shape[0] // 2
+    gate, up = F.linear(x.double(), W_gu.double()).split(I, dim=-1)
+    return F.linear(F.silu(gate) * up, W_dn.double())
+
+
+def test_single_expert_is_swiglu_ffn(oracle_mod):
+    x, W_r, W_gu, W_dn = _small_layer(E=1)
+    y, idx, w, _ = oracle_mod.forward_rows(x, W_r, W_gu, W_dn, 1, list(range(x.shape[0])))
+    assert (idx == 0).all() and (w == 1.0).all()
+    ref = _swiglu_ffn_library(x, W_gu[0], W_dn[0]).numpy()
+    assert np.abs(y - ref).max() <= 1e-12 * max(1.0, np.abs(ref).max())
+
+
+def test_dense_bruteforce_bmm_formulation(oracle_mod):
+    """The all-experts bmm inference path of the HF module (transposed stacked layout
+    (E, D, 2I) / (E, I, D), x repeated E times, sum over E of a [T, E] weight matrix that is
+    zero off the top-k) equals the sparse per-token oracle."""
+    x, W_r, W_gu, W_dn = _small_layer(T=16, E=6)
+    k = 2
+    T, D = x.shape
+    E, I2, _ = W_gu.shape
+    I = I2 // 2
+    y, idx, w, _ = oracle_mod.forward_rows(x, W_r, W_gu, W_dn, k, list(range(T)))
+    dense_w = torch.zeros(T, E, dtype=torch.float64).scatter_(1, torch.from_numpy(idx).long(),
+                                                              torch.from_numpy(w).double())
+    gate_up_proj = W_gu.double().transpose(1, 2)            # (E, D, 2I)
+    down_proj = W_dn.double().transpose(1, 2)               # (E, I, D)
+    hs = x.double().repeat(E, 1).view(E, T, D)
+    gu = torch.bmm(hs, gate_up_proj)
+    gate, up = gu[..., :I], gu[..., I:]
+    nxt = torch.bmm(up * F.silu(gate), down_proj)            # (E, T, D)
+    ref = (nxt * dense_w.transpose(0, 1)[..., None]).sum(0).numpy()
+    assert np.abs(y - ref).max() <= 1e-12 * max(1.0, np.abs(ref).max())
+
+
+def test_loop_dispatch_equals_per_token(oracle_mod):
+    g = golden("loop_vs_grouped.json")                      # the pages' invariant
+    assert g["checksum_loop"] == g["checksum_grouped"]
+    x, W_r, W_gu, W_dn = _small_layer(T=20, E=7)
+    _, idx, w = oracle_mod.route(x, W_r, 3)
+    y_loop = oracle_mod.loop_dispatch(x, idx, w, W_gu, W_dn)
+    y_tok = oracle_mod.combine_rows(x, idx, w, list(range(20)), W_gu, W_dn)
+    assert np.abs(y_loop - y_tok).max() <= 1e-12 * max(1.0, np.abs(y_tok).max())
+
+
+def test_zero_up_projection_gives_zero(oracle_mod):
+    x, W_r, W_gu, W_dn = _small_layer()
+    I = W_gu.shape[1] // 2
+    W0 = W_gu.clone()
+    W0[:, I:, :] = 0
+    y, _, _, _ = oracle_mod.forward_rows(x, W_r, W0, W_dn, 2, list(range(x.shape[0])))
+    assert np.abs(y).max() == 0.0
+    y, _, _, _ = oracle_mod.forward_rows(torch.zeros_like(x), W_r, W_gu, W_dn, 2, [0, 3])
+    assert np.abs(y).max() == 0.0
+
+
+def test_weighted_sum_of_selected_experts(oracle_mod):
+    """y = sum_j w_j expert_{e_j}(x), each expert from the library SwiGLU."""
+    x, W_r, W_gu, W_dn = _small_layer(T=6, E=5)
+    k = 3
+    y, idx, w, _ = oracle_mod.forward_rows(x, W_r, W_gu, W_dn, k, list(range(6)), norm=False)
+    for t in range(6):
+        ref = sum(float(w[t, j]) * _swiglu_ffn_library(x[t:t + 1], W_gu[idx[t, j]], W_dn[idx[t, j]])[0]
+                  for j in range(k)).numpy()
+        assert np.abs(y[t] - ref).max() <= 1e-12
+
+
+def test_shared_expert_gate_and_residual(oracle_mod):
+    x, W_r, W_gu, W_dn = _small_layer(T=5, E=4)
+    g = torch.Generator().manual_seed(12)
+    I_s = 16
+    sgu = (0.1 * torch.randn(2 * I_s, x.shape[1], generator=g)).to(torch.bfloat16)
+    sdn = (0.1 * torch.randn(x.shape[1], I_s, generator=g)).to(torch.bfloat16)
+    sg = (0.1 * torch.randn(x.shape[1], generator=g)).to(torch.bfloat16)
+    res = torch.randn(x.shape, generator=g).to(torch.bfloat16)
+    rows = list(range(5))
+    base, _, _, _ = oracle_mod.forward_rows(x, W_r, W_gu, W_dn, 2, rows)
+    S = _swiglu_ffn_library(x, sgu, sdn).numpy()
+    y, _, _, _ = oracle_mod.forward_rows(x, W_r, W_gu, W_dn, 2, rows, shared_gate_up=sgu, shared_down=sdn)
+    assert np.abs(y - (base + S)).max() <= 1e-12           # ungated shared expert
+    y, _, _, _ = oracle_mod.forward_rows(x, W_r, W_gu, W_dn, 2, rows, shared_gate_up=sgu,
+                                         shared_down=sdn, shared_gate=torch.zeros_like(sg))
+    assert np.abs(y - (base + 0.5 * S)).max() <= 1e-12     # sigmoid(0) = 1/2
+    y, _, _, _ = oracle_mod.forward_rows(x, W_r, W_gu, W_dn, 2, rows, shared_gate_up=sgu,
+                                         shared_down=sdn, shared_gate=sg, residual=res)
+    gate = torch.sigmoid(x.double() @ sg.double()).numpy()[:, None]
+    assert np.abs(y - (base + gate * S + res.double().numpy())).max() <= 1e-12
+
+
+# ------------------------------------------------------------------ permute
+
+@pytest.mark.parametrize("tile_m", [1, 4, 16])
+def test_permute_matches_library_stable_sort(oracle_mod, tile_m):
+    rng = np.random.default_rng(13)
+    T, k, E = 37, 3, 9
+    idx = np.stack([rng.choice(E, size=k, replace=False) for _ in range(T)]).astype(np.int32)
+    counts, offsets, row_token, slot_row = oracle_mod.permute(idx, E, tile_m)
+    flat = idx.reshape(-1)
+    assert counts.tolist() == np.bincount(flat, minlength=E).tolist()
+    assert counts.sum() == T * k
+    order = sorted(range(T * k), key=lambda a: flat[a])     # Python's sort is stable
+    assert offsets[0] == 0 and all((offsets[1:] - offsets[:-1]) % tile_m == 0)
+    assert all(offsets[e + 1] - offsets[e] == -(-counts[e] // tile_m) * tile_m for e in range(E))
+    pos = 0
+    for e in range(E):
+        seg = order[pos:pos + counts[e]]
+        pos += counts[e]
+        rows = list(range(offsets[e], offsets[e] + counts[e]))
+        assert [row_token[r] for r in rows] == [a // k for a in seg]
+        assert [slot_row[a] for a in seg] == rows
+        assert all(row_token[r] == -1 for r in range(offsets[e] + counts[e], offsets[e + 1]))
+
+
+# ------------------------------------------------------------------ byte accounting
+
+def test_parameter_split_matches_page():
+    g = golden("parameter_split.json")
+    s = g["shape"]
+    stored, active = moe_parameter_split(s["hidden"], s["layers"], s["experts"], s["top_k"],
+                                         s["intermediate"], s["shared_intermediate"])
+    p = g["printed"]
+    assert round(stored / 1e9, 1) == p["expert_params_stored_B"]
+    assert round(active / 1e9, 2) == p["expert_params_active_B"]
+    assert round(active / stored, 3) == p["active_fraction"]
