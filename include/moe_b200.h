@@ -1,0 +1,151 @@
+/*
+ * moe_b200.h -- C ABI of the B200 (sm_100a) forward pass of a Qwen-family sparse MoE FFN
+ * block: router, expert-contiguous permutation, SwiGLU experts and the weighted combine.
+ *
+ * The operation ("27. Mixture of experts", inference.shantanugoel.com):
+ *   section "The router":  logits = W_r x; softmax over all E experts in FP32; keep the k
+ *                          largest with their indices, ties broken by index; with
+ *                          norm_topk_prob, divide the kept weights by their sum;
+ *                          y = sum_{i in top-k} w_i expert_i(x).
+ *   section "Dispatch":    experts stacked as gate_up [E, 2I, D] (gate rows first) and
+ *                          down [E, D, I]; expert(x) = down(silu(gate x) * up x); grouped
+ *                          dispatch sorts the N*k assignments by expert (stable) so each
+ *                          expert's rows are contiguous.
+ *   section "The shared expert": optionally y += sigmoid(w_s . x) * shared(x).
+ *
+ * Conventions shared by every entry point:
+ *  - All tensor pointers are DEVICE pointers owned by the caller, row-major and contiguous,
+ *    16-byte aligned.  bf16 tensors are passed as their 16-bit patterns (moe_bf16).
+ *  - The library allocates no memory and never synchronises the host on these calls: all
+ *    work is enqueued on `stream` (a cudaStream_t; NULL = the legacy default stream).
+ *    Scratch comes from the caller's workspace `ws` of `ws_bytes` bytes, sized with
+ *    moe_workspace_size().  The workspace must not be used by two calls that can run at the
+ *    same time.
+ *  - Arguments are validated before anything is enqueued; an invalid call returns an error
+ *    status and enqueues nothing.  There is no CPU fallback: a call that cannot run on the
+ *    GPU fails with MOE_ERR_CUDA.
+ *  - Inputs must be finite; NaN or Inf inputs give undefined outputs (never a fault).
+ *  - Supported shapes: 1 <= E <= 512, 1 <= k <= min(E, 16), D and I (and I_s) multiples of
+ *    128, T >= 1, T * (k + 1) < 2^31.  Other shapes return MOE_ERR_UNSUPPORTED.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t moe_bf16;                /* raw bfloat16 bits */
+typedef struct CUstream_st *moe_stream_t; /* identical to cudaStream_t */
+typedef struct CUevent_st *moe_event_t;   /* identical to cudaEvent_t */
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1,    /* null / misaligned pointer, T < 1, bad struct */
+    MOE_ERR_UNSUPPORTED = 2,    /* shape outside the supported set above */
+    MOE_ERR_WORKSPACE = 3,      /* ws_bytes smaller than moe_workspace_size() */
+    MOE_ERR_CUDA = 4,           /* a CUDA call failed (no GPU, launch error, ...) */
+    MOE_ERR_DEVICE_TIMEOUT = 5  /* a kernel gave up a bounded wait (see moe_get_device_status) */
+} moe_status;
+
+/* Problem shape.  No field has a default: every one must be set.
+ *   T  tokens, D hidden size, E routed experts, k experts per token, I expert width;
+ *   norm_topk_prob  1 = renormalise the k kept weights to sum to 1, 0 = keep softmax values;
+ *   tile_m  row padding of each expert segment in moe_permute (1 = none; 1..256).  The
+ *           forward pass does not use it. */
+typedef struct {
+    int T, D, E, k, I;
+    int norm_topk_prob;
+    int tile_m;
+} moe_dims;
+
+/* Which expert path moe_forward_ex takes. */
+enum {
+    MOE_PATH_AUTO = 0,    /* streaming path for small T, grouped tensor-core path otherwise */
+    MOE_PATH_STREAM = 1,  /* stream each touched expert's weights once (decode) */
+    MOE_PATH_GROUPED = 2  /* permute + tcgen05 grouped GEMMs (prefill) */
+};
+
+/* Options of moe_forward_ex.  Zero-initialise and set what is needed. */
+typedef struct {
+    const float *router_bias;        /* [E] FP32 added to the logits before the softmax, or NULL */
+    const moe_bf16 *shared_gate_up;  /* [2*I_s, D] shared expert (gate rows first), or NULL */
+    const moe_bf16 *shared_down;     /* [D, I_s]; required with shared_gate_up */
+    const moe_bf16 *shared_gate;     /* [D] w_s: y += sigmoid(w_s . x) * shared(x); NULL = ungated */
+    int I_s;                         /* shared expert width (multiple of 128) */
+    const moe_bf16 *residual;        /* [T, D]: out = residual + block(x), or NULL */
+    float *logits_out;               /* [T, E] FP32 router logits (bias included), or NULL */
+    int32_t *topk_idx_out;           /* [T, k] selected experts, slot order, or NULL */
+    float *topk_w_out;               /* [T, k] FP32 routing weights, or NULL */
+    int path;                        /* MOE_PATH_* */
+    moe_event_t *stage_events;       /* if n_stage_events == 6: recorded on `stream` at the start,
+                                        after routing, after the permutation, after gate_up,
+                                        after down and after the combine */
+    int n_stage_events;
+} moe_opts;
+
+/* Bytes of workspace that moe_route, moe_permute and moe_forward(_ex) need for `dims`
+ * (and `opts`, which may be NULL).  Returns 0 for invalid or unsupported arguments. */
+size_t moe_workspace_size(const moe_dims *dims, const moe_opts *opts);
+
+/* Router ("27. Mixture of experts", section "The router"):
+ *   logits[t, e] = sum_d x[t, d] W_r[e, d] (FP32 accumulate) (+ bias[e]);
+ *   topk_idx[t, j] = expert of rank j by FP32 logit, equal logits -> lower index;
+ *   topk_w[t, j] = softmax(logits[t])[idx] in FP32, divided by the sum of the k kept values
+ *                  when dims->norm_topk_prob.
+ * x [T, D] bf16, W_r [E, D] bf16 (nn.Linear layout), bias [E] FP32 or NULL,
+ * logits [T, E] FP32 or NULL (then the workspace holds them), topk_idx [T, k] int32,
+ * topk_w [T, k] FP32. */
+moe_status moe_route(const moe_bf16 *x, const moe_bf16 *W_r, const float *bias,
+                     const moe_dims *dims, float *logits, int32_t *topk_idx, float *topk_w,
+                     void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Stable expert-contiguous permutation ("27. Mixture of experts", section "Dispatch",
+ * grouped dispatch; counting sort over a = t*k + j):
+ *   counts[e]  = number of assignments to expert e                       [E] int32
+ *   offsets[0] = 0, offsets[e+1] = offsets[e] + ceil(counts[e]/tile_m)*tile_m   [E+1]
+ *   rows offsets[e] .. offsets[e]+counts[e]-1 hold expert e's assignments in increasing a;
+ *   row_token[r] = token of row r, -1 on padding rows                    [cap] int32
+ *   slot_row[a]  = row of assignment a                                   [T*k] int32
+ *   row_weight[r] = topk_w of row r (0 on padding), written when both are non-NULL [cap]
+ *   x_perm[r, :] = x[row_token[r], :] (zeros on padding rows), written when x and x_perm
+ *                  are non-NULL                                          [cap, D] bf16
+ * cap must be >= T*k + E*(tile_m - 1).  topk_idx values outside [0, E) set
+ * MOE_ERR_DEVICE_TIMEOUT's sibling bit in the device status (reported by
+ * moe_get_device_status as MOE_ERR_INVALID_ARG). */
+moe_status moe_permute(const int32_t *topk_idx, const float *topk_w, const moe_bf16 *x,
+                       const moe_dims *dims, int32_t *counts, int32_t *offsets,
+                       int32_t *row_token, int32_t *slot_row, float *row_weight,
+                       moe_bf16 *x_perm, int cap, void *ws, size_t ws_bytes,
+                       moe_stream_t stream);
+
+/* The whole block: out[t] = sum_j w[t,j] * expert_{idx[t,j]}(x[t]).
+ * x [T, D] bf16, W_r [E, D] bf16, W_gate_up [E, 2I, D] bf16 (gate rows 0..I-1, up rows
+ * I..2I-1), W_down [E, D, I] bf16, out [T, D] bf16 (fully overwritten; must not alias x).
+ * The k weighted outputs are summed in slot order in FP32 and rounded once to bf16. */
+moe_status moe_forward(const moe_bf16 *x, const moe_bf16 *W_r, const moe_bf16 *W_gate_up,
+                       const moe_bf16 *W_down, const moe_dims *dims, moe_bf16 *out, void *ws,
+                       size_t ws_bytes, moe_stream_t stream);
+
+/* moe_forward with options (router bias, gated shared expert, residual, routing outputs,
+ * path choice, stage events).  out may alias opts->residual but not x. */
+moe_status moe_forward_ex(const moe_bf16 *x, const moe_bf16 *W_r, const moe_bf16 *W_gate_up,
+                          const moe_bf16 *W_down, const moe_dims *dims, const moe_opts *opts,
+                          moe_bf16 *out, void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Synchronises `stream` and reports the device error word that the last call using `ws`
+ * left: MOE_OK, MOE_ERR_DEVICE_TIMEOUT (a bounded wait expired), MOE_ERR_INVALID_ARG (an
+ * expert index outside [0, E) reached moe_permute) or MOE_ERR_CUDA. */
+moe_status moe_get_device_status(const void *ws, moe_stream_t stream);
+
+/* Static, human-readable name of a status. */
+const char *moe_status_string(moe_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

@@ -1,0 +1,130 @@
+// internal.h -- declarations shared by the library's translation units (not public API).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace moe {
+
+// Every bounded wait gives up after this long and reports it in the device error word.
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
+
+// Bits of the device error word (first int of the workspace).
+enum : int {
+    kErrWaitProducer = 1,   // TMA producer gave up waiting for a free stage
+    kErrWaitMma = 2,        // MMA issuer gave up waiting for data or a free accumulator
+    kErrWaitEpilogue = 4,   // epilogue gave up waiting for an accumulator
+    kErrBadIndex = 8,       // an expert index outside [0, E) reached the permute stage
+    kErrWaitTail = 16,      // producer gave up draining its last stages
+};
+
+// Tile geometry of the tcgen05 grouped GEMMs (swap-AB: weights on M, tokens on N).
+constexpr int kTcM = 128;       // weight rows per tile (MMA M)
+constexpr int kTcK = 64;        // K elements per pipeline stage (one 128-byte swizzle row)
+constexpr int kGuBN = 128;      // token columns per gate_up tile (two accumulators per tile)
+constexpr int kDnBN = 256;      // token columns per down tile
+constexpr int kRtBN = 128;      // token columns per router-logit tile
+constexpr int kStages = 4;      // shared-memory pipeline depth
+
+// Largest supported expert count (and segments: experts + one shared expert).
+constexpr int kMaxE = 512;
+constexpr int kMaxK = 16;
+constexpr int kMaxSegments = kMaxE + 1;
+
+// Permute-stage geometry.
+constexpr int kPermChunk = 4096;   // assignments per histogram / scatter block
+constexpr int kPermThreads = 1024;
+
+// Device tables written by the permute stage.  Segment s < E is routed expert s; when a
+// shared expert is present it is segment E and owns the last T rows in token order.
+struct SegTables {
+    int* seg_count;   // [nseg] rows of each segment
+    int* seg_start;   // [nseg] first permuted row of each segment
+    int* gu_items;    // [nseg + 1] prefix sums of tcgen05 gate_up work items
+    int* dn_items;    // [nseg + 1] prefix sums of tcgen05 down work items
+    int* gu_tasks;    // [nseg + 1] prefix sums of streaming gate_up warp tasks
+    int* dn_tasks;    // [nseg + 1] prefix sums of streaming down warp tasks
+};
+
+struct PermuteArgs {
+    const int32_t* topk_idx;  // [T, k]
+    const float* topk_w;      // [T, k] or null
+    int T, k, E, tile_m;
+    int has_shared;           // adds segment E = all T tokens in order
+    int slots_per_token;      // k (+1 with a shared expert): row_dest = t * S + j
+    int D, I, I_s;
+    int* chunk_counts;        // [nchunks, E] scratch
+    int nchunks;
+    int* counts;              // [E] (caller-visible), may alias tables.seg_count
+    int* offsets;             // [E + 1] (caller-visible)
+    int32_t* row_token;       // [cap]
+    float* row_weight;        // [cap] or null
+    int32_t* row_dest;        // [cap] or null
+    int32_t* slot_row;        // [T * k]
+    int cap;                  // rows available in row_* arrays
+    SegTables tables;         // may be all-null (moe_permute alone)
+    int* err;
+};
+
+struct StreamArgs {
+    const uint16_t* x;        // [T, D]
+    const uint16_t* W_gu;     // [E, 2I, D]
+    const uint16_t* W_dn;     // [E, D, I]
+    const uint16_t* S_gu;     // [2I_s, D] or null
+    const uint16_t* S_dn;     // [D, I_s] or null
+    int D, I, I_s, E, nseg;
+    SegTables tables;
+    const int32_t* row_token;
+    const float* row_weight;
+    const int32_t* row_dest;
+    uint16_t* h;              // [rows, ld_h] bf16
+    int ld_h;
+    float* slots;             // [T * S, D] FP32
+    int* err;
+};
+
+struct TcArgs {
+    int D, I, I_s, E, nseg;
+    SegTables tables;
+    // gate_up epilogue
+    uint16_t* h;              // [rows, ld_h]
+    int ld_h;
+    // down epilogue
+    const float* row_weight;
+    const int32_t* row_dest;
+    uint16_t* slots_bf16;     // [T * S, D]
+    // dense (router) epilogue
+    float* logits;            // [T, E]
+    const float* bias;        // [E] or null
+    int T;
+    int* err;
+};
+
+// Raise a kernel's dynamic shared-memory limit once per device (host-side attribute; done
+// outside stream capture by the first call on each device).
+cudaError_t ensure_smem_attr(const void* kernel, int bytes, int slot);
+
+// ---------------------------------------------------------------- launchers (return the
+// launch error, cudaSuccess when all kernels were enqueued)
+cudaError_t launch_router_small(const uint16_t* x, const uint16_t* W_r, const float* bias, int T,
+                                int D, int E, float* logits, cudaStream_t s);
+cudaError_t launch_select(const float* logits, int T, int E, int k, int norm, int32_t* idx,
+                          float* w, cudaStream_t s);
+cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t s);
+cudaError_t launch_gather_rows(const uint16_t* x, const int32_t* row_token, int rows, int D,
+                               uint16_t* x_perm, cudaStream_t s);
+cudaError_t launch_stream_gate_up(const StreamArgs& a, int max_rows, cudaStream_t s);
+cudaError_t launch_stream_down(const StreamArgs& a, int max_rows, cudaStream_t s);
+cudaError_t launch_tc_router(const CUtensorMap& mapA, const CUtensorMap& mapB, const TcArgs& a,
+                             int num_sms, cudaStream_t s);
+cudaError_t launch_tc_gate_up(const CUtensorMap& mapA, const CUtensorMap& mapA_shared,
+                              const CUtensorMap& mapB, const TcArgs& a, int num_sms,
+                              cudaStream_t s);
+cudaError_t launch_tc_down(const CUtensorMap& mapA, const CUtensorMap& mapA_shared,
+                           const CUtensorMap& mapB, const TcArgs& a, int num_sms, cudaStream_t s);
+cudaError_t launch_combine(const void* slots, int slots_bf16, int T, int D, int k, int has_shared,
+                           const uint16_t* x, const uint16_t* shared_gate,
+                           const uint16_t* residual, uint16_t* out, cudaStream_t s);
+
+}  // namespace moe

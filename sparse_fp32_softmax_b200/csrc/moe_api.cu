@@ -1,0 +1,427 @@
+// moe_api.cu -- the C ABI: argument validation, workspace layout, TMA tensor maps and the
+// launch sequence of the MoE block forward pass.  Host code only; kernels live in the other
+// translation units.  Nothing here allocates device memory or synchronises the host, except
+// moe_get_device_status, whose job is to synchronise.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "../../include/moe_b200.h"
+#include "internal.h"
+
+using namespace moe;
+
+namespace moe {
+
+cudaError_t ensure_smem_attr(const void* kernel, int bytes, int slot) {
+    static std::mutex mu;
+    static unsigned char done[64][8] = {};
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return err;
+    if (dev < 0 || dev >= 64 || slot < 0 || slot >= 8) return cudaErrorInvalidValue;
+    std::lock_guard<std::mutex> lock(mu);
+    if (done[dev][slot]) return cudaSuccess;
+    err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (err == cudaSuccess) done[dev][slot] = 1;
+    return err;
+}
+
+}  // namespace moe
+
+namespace {
+
+constexpr size_t kAlign = 256;
+constexpr int kRouterSmallMaxT = 64;     // below: CUDA-core router; above: tcgen05 router GEMM
+constexpr int kStreamMaxAssignments = 2048;  // AUTO path: streaming while T*k <= this
+
+size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Byte offsets of every workspace region.
+struct Plan {
+    int T, D, E, k, I, I_s, has_shared, S, R, ld_h, nchunks, nseg;
+    size_t err, logits, idx, w, counts, offsets, chunk, seg_count, seg_start, gu_items, dn_items,
+        gu_tasks, dn_tasks, row_token, row_weight, row_dest, slot_row, x_perm, h, slots, total;
+};
+
+Plan make_plan(const moe_dims& d, const moe_opts* o) {
+    Plan p{};
+    p.T = d.T; p.D = d.D; p.E = d.E; p.k = d.k; p.I = d.I;
+    p.has_shared = (o && o->shared_gate_up) ? 1 : 0;
+    p.I_s = p.has_shared ? o->I_s : 0;
+    p.S = p.k + p.has_shared;
+    p.R = p.T * p.k + (p.has_shared ? p.T : 0);
+    p.ld_h = p.I > p.I_s ? p.I : p.I_s;
+    p.nchunks = (int)(((long)p.T * p.k + kPermChunk - 1) / kPermChunk);
+    p.nseg = p.E + p.has_shared;
+    size_t off = 0;
+    auto take = [&](size_t bytes) { size_t at = off; off += align_up(bytes); return at; };
+    p.err = take(kAlign);
+    p.logits = take((size_t)p.T * p.E * 4);
+    p.idx = take((size_t)p.T * p.k * 4);
+    p.w = take((size_t)p.T * p.k * 4);
+    p.counts = take((size_t)(p.E + 1) * 4);
+    p.offsets = take((size_t)(p.E + 2) * 4);
+    p.chunk = take((size_t)p.nchunks * p.E * 4);
+    p.seg_count = take((size_t)(p.nseg + 1) * 4);
+    p.seg_start = take((size_t)(p.nseg + 1) * 4);
+    p.gu_items = take((size_t)(p.nseg + 2) * 4);
+    p.dn_items = take((size_t)(p.nseg + 2) * 4);
+    p.gu_tasks = take((size_t)(p.nseg + 2) * 4);
+    p.dn_tasks = take((size_t)(p.nseg + 2) * 4);
+    p.row_token = take((size_t)p.R * 4);
+    p.row_weight = take((size_t)p.R * 4);
+    p.row_dest = take((size_t)p.R * 4);
+    p.slot_row = take((size_t)p.T * p.k * 4);
+    p.x_perm = take((size_t)p.R * p.D * 2);
+    p.h = take((size_t)p.R * p.ld_h * 2);
+    p.slots = take((size_t)p.T * p.S * p.D * 4);
+    p.total = off;
+    return p;
+}
+
+moe_status check_dims(const moe_dims* d) {
+    if (!d) return MOE_ERR_INVALID_ARG;
+    if (d->T < 1 || d->D < 1 || d->E < 1 || d->k < 1 || d->I < 1) return MOE_ERR_INVALID_ARG;
+    if (d->norm_topk_prob != 0 && d->norm_topk_prob != 1) return MOE_ERR_INVALID_ARG;
+    if (d->E > kMaxE || d->k > kMaxK || d->k > d->E) return MOE_ERR_UNSUPPORTED;
+    if (d->D % 128 != 0 || d->I % 128 != 0) return MOE_ERR_UNSUPPORTED;
+    if (d->tile_m < 1 || d->tile_m > 256) return MOE_ERR_UNSUPPORTED;
+    if ((long long)d->T * (d->k + 1) >= (1ll << 31)) return MOE_ERR_UNSUPPORTED;
+    if ((long long)d->T * d->D >= (1ll << 40)) return MOE_ERR_UNSUPPORTED;
+    return MOE_OK;
+}
+
+moe_status check_opts(const moe_dims* d, const moe_opts* o) {
+    if (!o) return MOE_OK;
+    if (o->shared_gate_up) {
+        if (!o->shared_down) return MOE_ERR_INVALID_ARG;
+        if (o->I_s < 1) return MOE_ERR_INVALID_ARG;
+        if (o->I_s % 128 != 0) return MOE_ERR_UNSUPPORTED;
+        if (!aligned(o->shared_gate_up, 16) || !aligned(o->shared_down, 16)) return MOE_ERR_INVALID_ARG;
+        if (o->shared_gate && !aligned(o->shared_gate, 16)) return MOE_ERR_INVALID_ARG;
+    } else if (o->shared_down || o->shared_gate) {
+        return MOE_ERR_INVALID_ARG;
+    }
+    if (o->router_bias && !aligned(o->router_bias, 4)) return MOE_ERR_INVALID_ARG;
+    if (o->residual && !aligned(o->residual, 16)) return MOE_ERR_INVALID_ARG;
+    if (o->logits_out && !aligned(o->logits_out, 4)) return MOE_ERR_INVALID_ARG;
+    if (o->topk_idx_out && !aligned(o->topk_idx_out, 4)) return MOE_ERR_INVALID_ARG;
+    if (o->topk_w_out && !aligned(o->topk_w_out, 4)) return MOE_ERR_INVALID_ARG;
+    if (o->path < MOE_PATH_AUTO || o->path > MOE_PATH_GROUPED) return MOE_ERR_INVALID_ARG;
+    if (o->n_stage_events != 0 && o->n_stage_events != 6) return MOE_ERR_INVALID_ARG;
+    if (o->n_stage_events == 6 && !o->stage_events) return MOE_ERR_INVALID_ARG;
+    (void)d;
+    return MOE_OK;
+}
+
+// ------------------------------------------------------------------ device properties / TMA
+
+int num_sms_of_current_device() {
+    static int cache[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    if (dev < 0 || dev >= 64) return 0;
+    if (cache[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+        cache[dev] = n;
+    }
+    return cache[dev];
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// 2-D bf16 map over a row-major [rows, cols] tensor, box {64 columns, box_rows rows}, in the
+// 128-byte swizzle layout that the tcgen05 shared-memory descriptors expect.
+bool make_map(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint32_t box_rows) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * 2};
+    cuuint32_t box[2] = {(cuuint32_t)kTcK, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <typename T>
+T* at(void* ws, size_t off) {
+    return reinterpret_cast<T*>(static_cast<char*>(ws) + off);
+}
+
+#define MOE_CUDA(expr)                                       \
+    do {                                                     \
+        if ((expr) != cudaSuccess) return MOE_ERR_CUDA;      \
+    } while (0)
+
+moe_status record(const moe_opts* o, int i, cudaStream_t s) {
+    if (o && o->n_stage_events == 6)
+        MOE_CUDA(cudaEventRecord(reinterpret_cast<cudaEvent_t>(o->stage_events[i]), s));
+    return MOE_OK;
+}
+
+SegTables tables_of(const Plan& p, void* ws) {
+    SegTables t;
+    t.seg_count = at<int>(ws, p.seg_count);
+    t.seg_start = at<int>(ws, p.seg_start);
+    t.gu_items = at<int>(ws, p.gu_items);
+    t.dn_items = at<int>(ws, p.dn_items);
+    t.gu_tasks = at<int>(ws, p.gu_tasks);
+    t.dn_tasks = at<int>(ws, p.dn_tasks);
+    return t;
+}
+
+// Router: logits (CUDA-core for small T, tcgen05 GEMM otherwise), then selection.
+moe_status run_route(const moe_bf16* x, const moe_bf16* W_r, const float* bias, const Plan& p,
+                     int norm, float* logits, int32_t* idx, float* w, void* ws,
+                     cudaStream_t s) {
+    if (p.T <= kRouterSmallMaxT) {
+        MOE_CUDA(launch_router_small(x, W_r, bias, p.T, p.D, p.E, logits, s));
+    } else {
+        CUtensorMap mA, mB;
+        if (!make_map(&mA, W_r, p.D, p.E, kTcM)) return MOE_ERR_CUDA;
+        if (!make_map(&mB, x, p.D, p.T, kRtBN)) return MOE_ERR_CUDA;
+        TcArgs a{};
+        a.D = p.D; a.E = p.E; a.T = p.T; a.I = p.I; a.nseg = 1;
+        a.logits = logits;
+        a.bias = bias;
+        a.err = at<int>(ws, p.err);
+        const int sms = num_sms_of_current_device();
+        if (sms <= 0) return MOE_ERR_CUDA;
+        MOE_CUDA(launch_tc_router(mA, mB, a, sms, s));
+    }
+    MOE_CUDA(launch_select(logits, p.T, p.E, p.k, norm, idx, w, s));
+    return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t moe_workspace_size(const moe_dims* dims, const moe_opts* opts) {
+    if (check_dims(dims) != MOE_OK || check_opts(dims, opts) != MOE_OK) return 0;
+    return make_plan(*dims, opts).total;
+}
+
+const char* moe_status_string(moe_status s) {
+    switch (s) {
+        case MOE_OK: return "MOE_OK";
+        case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG";
+        case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED";
+        case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE";
+        case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+        case MOE_ERR_DEVICE_TIMEOUT: return "MOE_ERR_DEVICE_TIMEOUT";
+    }
+    return "MOE_ERR_UNKNOWN";
+}
+
+moe_status moe_route(const moe_bf16* x, const moe_bf16* W_r, const float* bias,
+                     const moe_dims* dims, float* logits, int32_t* topk_idx, float* topk_w,
+                     void* ws, size_t ws_bytes, moe_stream_t stream) {
+    moe_status st = check_dims(dims);
+    if (st != MOE_OK) return st;
+    if (!x || !W_r || !topk_idx || !topk_w || !ws) return MOE_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(W_r, 16) || !aligned(ws, kAlign)) return MOE_ERR_INVALID_ARG;
+    if ((bias && !aligned(bias, 4)) || (logits && !aligned(logits, 4)) ||
+        !aligned(topk_idx, 4) || !aligned(topk_w, 4))
+        return MOE_ERR_INVALID_ARG;
+    const Plan p = make_plan(*dims, nullptr);
+    if (ws_bytes < p.total) return MOE_ERR_WORKSPACE;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    MOE_CUDA(cudaMemsetAsync(at<int>(ws, p.err), 0, sizeof(int), s));
+    float* lg = logits ? logits : at<float>(ws, p.logits);
+    return run_route(x, W_r, bias, p, dims->norm_topk_prob, lg, topk_idx, topk_w, ws, s);
+}
+
+moe_status moe_permute(const int32_t* topk_idx, const float* topk_w, const moe_bf16* x,
+                       const moe_dims* dims, int32_t* counts, int32_t* offsets,
+                       int32_t* row_token, int32_t* slot_row, float* row_weight,
+                       moe_bf16* x_perm, int cap, void* ws, size_t ws_bytes,
+                       moe_stream_t stream) {
+    moe_status st = check_dims(dims);
+    if (st != MOE_OK) return st;
+    if (!topk_idx || !counts || !offsets || !row_token || !slot_row || !ws) return MOE_ERR_INVALID_ARG;
+    if (!aligned(topk_idx, 4) || !aligned(counts, 4) || !aligned(offsets, 4) ||
+        !aligned(row_token, 4) || !aligned(slot_row, 4) || !aligned(ws, kAlign))
+        return MOE_ERR_INVALID_ARG;
+    if ((topk_w && !aligned(topk_w, 4)) || (row_weight && !aligned(row_weight, 4)))
+        return MOE_ERR_INVALID_ARG;
+    if ((x_perm && !x) || (x && !aligned(x, 16)) || (x_perm && !aligned(x_perm, 16)))
+        return MOE_ERR_INVALID_ARG;
+    const long long need = (long long)dims->T * dims->k + (long long)dims->E * (dims->tile_m - 1);
+    if (cap < need) return MOE_ERR_INVALID_ARG;
+    const Plan p = make_plan(*dims, nullptr);
+    if (ws_bytes < p.total) return MOE_ERR_WORKSPACE;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    MOE_CUDA(cudaMemsetAsync(at<int>(ws, p.err), 0, sizeof(int), s));
+    PermuteArgs a{};
+    a.topk_idx = topk_idx;
+    a.topk_w = topk_w;
+    a.T = p.T; a.k = p.k; a.E = p.E; a.tile_m = dims->tile_m;
+    a.has_shared = 0;
+    a.slots_per_token = p.k;
+    a.D = p.D; a.I = p.I; a.I_s = 0;
+    a.chunk_counts = at<int>(ws, p.chunk);
+    a.nchunks = p.nchunks;
+    a.counts = counts;
+    a.offsets = offsets;
+    a.row_token = row_token;
+    a.row_weight = topk_w ? row_weight : nullptr;
+    a.row_dest = nullptr;
+    a.slot_row = slot_row;
+    a.cap = cap;
+    a.tables = SegTables{nullptr, nullptr, nullptr, nullptr, nullptr, nullptr};
+    a.err = at<int>(ws, p.err);
+    // padding rows are only written per expert segment; rows past offsets[E] stay as given,
+    // so mark every row as padding first
+    MOE_CUDA(cudaMemsetAsync(row_token, 0xFF, (size_t)cap * sizeof(int32_t), s));
+    MOE_CUDA(launch_permute(a, s));
+    if (x_perm) MOE_CUDA(launch_gather_rows(x, row_token, cap, p.D, x_perm, s));
+    return MOE_OK;
+}
+
+moe_status moe_forward_ex(const moe_bf16* x, const moe_bf16* W_r, const moe_bf16* W_gate_up,
+                          const moe_bf16* W_down, const moe_dims* dims, const moe_opts* opts,
+                          moe_bf16* out, void* ws, size_t ws_bytes, moe_stream_t stream) {
+    moe_status st = check_dims(dims);
+    if (st != MOE_OK) return st;
+    st = check_opts(dims, opts);
+    if (st != MOE_OK) return st;
+    if (!x || !W_r || !W_gate_up || !W_down || !out || !ws) return MOE_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(W_r, 16) || !aligned(W_gate_up, 16) || !aligned(W_down, 16) ||
+        !aligned(out, 16) || !aligned(ws, kAlign))
+        return MOE_ERR_INVALID_ARG;
+    if (out == x) return MOE_ERR_INVALID_ARG;
+    const Plan p = make_plan(*dims, opts);
+    if (ws_bytes < p.total) return MOE_ERR_WORKSPACE;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const int path_req = opts ? opts->path : MOE_PATH_AUTO;
+    const bool streaming = path_req == MOE_PATH_STREAM ||
+                           (path_req == MOE_PATH_AUTO && (long)p.T * p.k <= kStreamMaxAssignments);
+    const int sms = num_sms_of_current_device();
+    if (sms <= 0) return MOE_ERR_CUDA;
+
+    int* err = at<int>(ws, p.err);
+    float* logits = (opts && opts->logits_out) ? opts->logits_out : at<float>(ws, p.logits);
+    int32_t* idx = (opts && opts->topk_idx_out) ? opts->topk_idx_out : at<int32_t>(ws, p.idx);
+    float* w = (opts && opts->topk_w_out) ? opts->topk_w_out : at<float>(ws, p.w);
+    const float* bias = opts ? opts->router_bias : nullptr;
+    const moe_bf16* sgu = opts ? opts->shared_gate_up : nullptr;
+    const moe_bf16* sdn = opts ? opts->shared_down : nullptr;
+    const moe_bf16* sg = opts ? opts->shared_gate : nullptr;
+    const moe_bf16* residual = opts ? opts->residual : nullptr;
+
+    // tensor maps of the grouped path are encoded before anything is enqueued
+    CUtensorMap mGuA, mGuAs, mGuB, mDnA, mDnAs, mDnB;
+    if (!streaming) {
+        uint16_t* x_perm = at<uint16_t>(ws, p.x_perm);
+        uint16_t* h = at<uint16_t>(ws, p.h);
+        if (!make_map(&mGuA, W_gate_up, p.D, (uint64_t)p.E * 2 * p.I, kTcM) ||
+            !make_map(&mGuAs, sgu ? sgu : W_gate_up, p.D, sgu ? 2 * (uint64_t)p.I_s : 2 * (uint64_t)p.I, kTcM) ||
+            !make_map(&mGuB, x_perm, p.D, p.R, kGuBN) ||
+            !make_map(&mDnA, W_down, p.I, (uint64_t)p.E * p.D, kTcM) ||
+            !make_map(&mDnAs, sdn ? sdn : W_down, sdn ? p.I_s : p.I, p.D, kTcM) ||
+            !make_map(&mDnB, h, p.ld_h, p.R, kDnBN))
+            return MOE_ERR_CUDA;
+    }
+
+    MOE_CUDA(cudaMemsetAsync(err, 0, sizeof(int), s));
+    if ((st = record(opts, 0, s)) != MOE_OK) return st;
+    if ((st = run_route(x, W_r, bias, p, dims->norm_topk_prob, logits, idx, w, ws, s)) != MOE_OK)
+        return st;
+    if ((st = record(opts, 1, s)) != MOE_OK) return st;
+
+    PermuteArgs pa{};
+    pa.topk_idx = idx;
+    pa.topk_w = w;
+    pa.T = p.T; pa.k = p.k; pa.E = p.E; pa.tile_m = 1;
+    pa.has_shared = p.has_shared;
+    pa.slots_per_token = p.S;
+    pa.D = p.D; pa.I = p.I; pa.I_s = p.I_s;
+    pa.chunk_counts = at<int>(ws, p.chunk);
+    pa.nchunks = p.nchunks;
+    pa.counts = at<int>(ws, p.counts);
+    pa.offsets = at<int>(ws, p.offsets);
+    pa.row_token = at<int32_t>(ws, p.row_token);
+    pa.row_weight = at<float>(ws, p.row_weight);
+    pa.row_dest = at<int32_t>(ws, p.row_dest);
+    pa.slot_row = at<int32_t>(ws, p.slot_row);
+    pa.cap = p.R;
+    pa.tables = tables_of(p, ws);
+    pa.err = err;
+    MOE_CUDA(launch_permute(pa, s));
+    if (!streaming)
+        MOE_CUDA(launch_gather_rows(x, pa.row_token, p.R, p.D, at<uint16_t>(ws, p.x_perm), s));
+    if ((st = record(opts, 2, s)) != MOE_OK) return st;
+
+    if (streaming) {
+        StreamArgs sa{};
+        sa.x = x; sa.W_gu = W_gate_up; sa.W_dn = W_down; sa.S_gu = sgu; sa.S_dn = sdn;
+        sa.D = p.D; sa.I = p.I; sa.I_s = p.I_s; sa.E = p.E; sa.nseg = p.nseg;
+        sa.tables = pa.tables;
+        sa.row_token = pa.row_token;
+        sa.row_weight = pa.row_weight;
+        sa.row_dest = pa.row_dest;
+        sa.h = at<uint16_t>(ws, p.h);
+        sa.ld_h = p.ld_h;
+        sa.slots = at<float>(ws, p.slots);
+        sa.err = err;
+        MOE_CUDA(launch_stream_gate_up(sa, p.T, s));
+        if ((st = record(opts, 3, s)) != MOE_OK) return st;
+        MOE_CUDA(launch_stream_down(sa, p.T, s));
+        if ((st = record(opts, 4, s)) != MOE_OK) return st;
+        MOE_CUDA(launch_combine(sa.slots, 0, p.T, p.D, p.k, p.has_shared, x, sg, residual, out, s));
+    } else {
+        TcArgs ta{};
+        ta.D = p.D; ta.I = p.I; ta.I_s = p.I_s; ta.E = p.E; ta.nseg = p.nseg; ta.T = p.T;
+        ta.tables = pa.tables;
+        ta.h = at<uint16_t>(ws, p.h);
+        ta.ld_h = p.ld_h;
+        ta.row_weight = pa.row_weight;
+        ta.row_dest = pa.row_dest;
+        ta.slots_bf16 = at<uint16_t>(ws, p.slots);
+        ta.err = err;
+        MOE_CUDA(launch_tc_gate_up(mGuA, mGuAs, mGuB, ta, sms, s));
+        if ((st = record(opts, 3, s)) != MOE_OK) return st;
+        MOE_CUDA(launch_tc_down(mDnA, mDnAs, mDnB, ta, sms, s));
+        if ((st = record(opts, 4, s)) != MOE_OK) return st;
+        MOE_CUDA(launch_combine(ta.slots_bf16, 1, p.T, p.D, p.k, p.has_shared, x, sg, residual, out, s));
+    }
+    return record(opts, 5, s);
+}
+
+moe_status moe_forward(const moe_bf16* x, const moe_bf16* W_r, const moe_bf16* W_gate_up,
+                       const moe_bf16* W_down, const moe_dims* dims, moe_bf16* out, void* ws,
+                       size_t ws_bytes, moe_stream_t stream) {
+    return moe_forward_ex(x, W_r, W_gate_up, W_down, dims, nullptr, out, ws, ws_bytes, stream);
+}
+
+moe_status moe_get_device_status(const void* ws, moe_stream_t stream) {
+    if (!ws || !aligned(ws, kAlign)) return MOE_ERR_INVALID_ARG;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
+    int word = 0;
+    if (cudaMemcpy(&word, ws, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+    if (word & kErrBadIndex) return MOE_ERR_INVALID_ARG;
+    if (word) return MOE_ERR_DEVICE_TIMEOUT;
+    return MOE_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,105 @@
+"""Shared helpers of the parity tests: tolerances and the routing comparison.
+
+Tolerances (the block's correctness criteria):
+  * selected expert indices, per-expert counts and the permutation: bit-exact;
+  * routing weights: within 1e-6 absolute;
+  * block output y (bf16) against the FP64 oracle: relative L2 error <= 5e-3 and max-abs
+    error <= 2e-2 * rms(y).
+
+Routing against FP64 oracle logits.  The GPU sums bf16 x bf16 products (exact in FP32) in
+FP32 in its own order; the oracle sums them exactly and rounds once.  For logit e of token t
+the two differ by at most
+    delta[t, e] = gamma_D * sum_d |x[t, d] W_r[e, d]| + 2^-23 * |l[t, e]|,
+    gamma_D = D u / (1 - D u), u = 2^-24
+(the classic bound on recursive FP32 summation, plus one rounding of each result).  A
+token is *decisive* when, in the oracle's ranking, every adjacent gap from rank 0 down to
+rank k (the boundary between kept and dropped) exceeds the sum of the two deltas: then any
+correct FP32 evaluation must select the same experts in the same order, and the GPU must
+match exactly.  Tokens that are not decisive are counted; their GPU selection must still be
+a valid top-k of the oracle logits within those deltas.
+"""
+import numpy as np
+import torch
+
+U = 2.0 ** -24
+W_ATOL = 1e-6
+Y_REL_L2 = 5e-3
+Y_MAX_ABS_RMS = 2e-2
+
+
+def to_u16(t: torch.Tensor) -> np.ndarray:
+    return t.detach().contiguous().cpu().view(torch.int16).numpy().view(np.uint16)
+
+
+def logit_deltas(x, W_r, logits):
+    """delta[t, e] for the given rows (x: [n, D] bf16 CPU/GPU tensor)."""
+    xd = x.detach().cpu().double().numpy()
+    wd = W_r.detach().cpu().double().numpy()
+    D = xd.shape[1]
+    gamma = D * U / (1 - D * U)
+    return gamma * (np.abs(xd) @ np.abs(wd).T) + 2 * U * np.abs(np.asarray(logits, np.float64))
+
+
+def ranking(l):
+    """Experts of one token by (logit desc, index asc)."""
+    return np.lexsort((np.arange(l.shape[0]), -l.astype(np.float64)))
+
+
+def is_decisive(l, delta, k):
+    order = ranking(l)
+    last = min(k, l.shape[0] - 1)
+    for r in range(last):
+        a, b = order[r], order[r + 1]
+        if not (l[a] - l[b] > delta[a] + delta[b]):
+            return False
+    return True
+
+
+def valid_topk(l, delta, sel):
+    """Is `sel` (in slot order) a correct top-k of logits known only to within delta?"""
+    sel = list(sel)
+    E = l.shape[0]
+    if len(set(sel)) != len(sel):
+        return False
+    rest = [e for e in range(E) if e not in sel]
+    for a in sel:
+        for b in rest:
+            if l[a] < l[b] - (delta[a] + delta[b]):
+                return False
+    for a, b in zip(sel[:-1], sel[1:]):
+        if l[a] < l[b] - (delta[a] + delta[b]):
+            return False
+    return True
+
+
+def check_routing(gpu_idx, oracle_idx, oracle_logits, delta, k):
+    """Bit-exact on decisive tokens, valid elsewhere.  Returns (n_decisive, n_other)."""
+    gpu_idx = np.asarray(gpu_idx)
+    nd = no = 0
+    for t in range(gpu_idx.shape[0]):
+        if is_decisive(oracle_logits[t], delta[t], k):
+            nd += 1
+            assert gpu_idx[t].tolist() == oracle_idx[t].tolist(), (t, gpu_idx[t], oracle_idx[t])
+        else:
+            no += 1
+            assert valid_topk(oracle_logits[t], delta[t], gpu_idx[t]), (t, gpu_idx[t], oracle_idx[t])
+    return nd, no
+
+
+def y_errors(y_gpu, y_ref):
+    y_gpu = np.asarray(y_gpu, np.float64)
+    y_ref = np.asarray(y_ref, np.float64)
+    diff = y_gpu - y_ref
+    ref_norm = np.linalg.norm(y_ref)
+    rel_l2 = np.linalg.norm(diff) / ref_norm if ref_norm > 0 else np.linalg.norm(diff)
+    rms = np.sqrt(np.mean(y_ref ** 2)) if y_ref.size else 0.0
+    max_abs = np.abs(diff).max() if diff.size else 0.0
+    return rel_l2, max_abs, rms
+
+
+def assert_y_close(y_gpu, y_ref, what=""):
+    rel_l2, max_abs, rms = y_errors(y_gpu, y_ref)
+    assert rel_l2 <= Y_REL_L2, f"{what}: relative L2 error {rel_l2:.3e} > {Y_REL_L2}"
+    assert max_abs <= Y_MAX_ABS_RMS * rms + 1e-30, \
+        f"{what}: max-abs error {max_abs:.3e} > {Y_MAX_ABS_RMS} * rms {rms:.3e}"
+    return rel_l2, max_abs / rms if rms else 0.0
