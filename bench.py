@@ -175,7 +175,7 @@ def build_workload(args, device):
     if spec["layers"] > 1:
         for l in range(spec["layers"]):
             W.append(inputs.make_layer(cfg, T=Tmax, layer=l, device=device, gen_device=device, with_x=False))
-        x0 = inputs.make_layer(cfg, T=Tmax, with_x=True)["x"].to(device)
+        x0 = inputs.normal_bf16((Tmax, cfg.D), 1.0, 1000 * cfg.seed + inputs.TID_X).to(device)
     else:
         L = inputs.make_layer(cfg, T=Tmax)
         x0 = L["x"].to(device)

@@ -25,6 +25,11 @@
  *    status and enqueues nothing.  There is no CPU fallback: a call that cannot run on the
  *    GPU fails with MOE_ERR_CUDA.
  *  - Inputs must be finite; NaN or Inf inputs give undefined outputs (never a fault).
+ *  - Precision: router logits, softmax, routing weights and every accumulation are FP32;
+ *    the SwiGLU intermediate h = silu(g) * u is rounded to bf16 (the down projection's MMA
+ *    operand type); the k weighted expert outputs are summed in FP32 and the block output
+ *    is rounded once to bf16 (round to nearest even).  opts->out_f32 returns that FP32 sum
+ *    before its rounding.
  *  - Supported shapes: 1 <= E <= 512, 1 <= k <= min(E, 16), D and I (and I_s) multiples of
  *    128, T >= 1, T * (k + 1) < 2^31.  Other shapes return MOE_ERR_UNSUPPORTED.
  */
@@ -83,8 +88,11 @@ typedef struct {
     int path;                        /* MOE_PATH_* */
     moe_event_t *stage_events;       /* if n_stage_events == 6: recorded on `stream` at the start,
                                         after routing, after the permutation, after gate_up,
-                                        after down and after the combine */
+                                        after down and after the combine (as external events,
+                                        so they become graph nodes under stream capture) */
     int n_stage_events;
+    float *out_f32;                  /* [T, D] FP32 block output before its rounding to bf16
+                                        (residual and shared expert included), or NULL */
 } moe_opts;
 
 /* Bytes of workspace that moe_route, moe_permute and moe_forward(_ex) need for `dims`
@@ -113,9 +121,9 @@ moe_status moe_route(const moe_bf16 *x, const moe_bf16 *W_r, const float *bias,
  *   row_weight[r] = topk_w of row r (0 on padding), written when both are non-NULL [cap]
  *   x_perm[r, :] = x[row_token[r], :] (zeros on padding rows), written when x and x_perm
  *                  are non-NULL                                          [cap, D] bf16
- * cap must be >= T*k + E*(tile_m - 1).  topk_idx values outside [0, E) set
- * MOE_ERR_DEVICE_TIMEOUT's sibling bit in the device status (reported by
- * moe_get_device_status as MOE_ERR_INVALID_ARG). */
+ * cap must be >= T*k + E*(tile_m - 1).  topk_idx values outside [0, E) are skipped and
+ * recorded in the device error word; moe_get_device_status then returns
+ * MOE_ERR_INVALID_ARG. */
 moe_status moe_permute(const int32_t *topk_idx, const float *topk_w, const moe_bf16 *x,
                        const moe_dims *dims, int32_t *counts, int32_t *offsets,
                        int32_t *row_token, int32_t *slot_row, float *row_weight,

@@ -34,7 +34,7 @@ class moe_opts(ctypes.Structure):
     _fields_ = [("router_bias", _vp), ("shared_gate_up", _vp), ("shared_down", _vp),
                 ("shared_gate", _vp), ("I_s", _c_int), ("residual", _vp), ("logits_out", _vp),
                 ("topk_idx_out", _vp), ("topk_w_out", _vp), ("path", _c_int),
-                ("stage_events", _vp), ("n_stage_events", _c_int)]
+                ("stage_events", _vp), ("n_stage_events", _c_int), ("out_f32", _vp)]
 
 
 class MoeError(RuntimeError):
@@ -117,7 +117,7 @@ def make_dims(T, D, E, k, I, norm_topk_prob=True, tile_m=1) -> moe_dims:
 
 def make_opts(router_bias=None, shared_gate_up=None, shared_down=None, shared_gate=None,
               residual=None, logits_out=None, topk_idx_out=None, topk_w_out=None, path="auto",
-              stage_events=None):
+              stage_events=None, out_f32=None):
     o = moe_opts()
     o.router_bias = _ptr(router_bias)
     o.shared_gate_up = _ptr(shared_gate_up)
@@ -129,6 +129,7 @@ def make_opts(router_bias=None, shared_gate_up=None, shared_down=None, shared_ga
     o.topk_idx_out = _ptr(topk_idx_out)
     o.topk_w_out = _ptr(topk_w_out)
     o.path = PATHS[path] if isinstance(path, str) else int(path)
+    o.out_f32 = _ptr(out_f32)
     o._events_keepalive = None
     if stage_events is not None:
         handles = (ctypes.c_void_p * len(stage_events))(*[ev.cuda_event for ev in stage_events])
@@ -215,7 +216,7 @@ def moe_forward_ex(x, W_r, W_gate_up, W_down, k, norm_topk_prob=True, out=None, 
                    stream=None, opts: moe_opts | None = None, **opt_kwargs):
     """moe_forward with options; pass a prepared ``opts`` or the keyword arguments of
     ``make_opts`` (router_bias, shared_gate_up, shared_down, shared_gate, residual,
-    logits_out, topk_idx_out, topk_w_out, path, stage_events)."""
+    logits_out, topk_idx_out, topk_w_out, path, stage_events, out_f32)."""
     dims = _dims_of(x, W_r, W_gate_up, W_down, k, norm_topk_prob)
     if opts is None:
         opts = make_opts(**opt_kwargs)

@@ -34,7 +34,7 @@ template <typename SlotT>
 __global__ void __launch_bounds__(kCombineThreads) combine_kernel(
     const SlotT* __restrict__ slots, int T, int D, int k, int has_shared,
     const uint16_t* __restrict__ x, const uint16_t* __restrict__ shared_gate,
-    const uint16_t* __restrict__ residual, uint16_t* __restrict__ out) {
+    const uint16_t* __restrict__ residual, uint16_t* __restrict__ out, float* __restrict__ out_f32) {
     __shared__ float red[kCombineThreads / 32];
     const int S = k + has_shared;
     for (int t = blockIdx.x; t < T; t += gridDim.x) {
@@ -77,6 +77,11 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(
 #pragma unroll
                 for (int i = 0; i < 8; ++i) acc[i] += v[i];
             }
+            if (out_f32) {
+                float4* of = reinterpret_cast<float4*>(out_f32 + (size_t)t * D + d);
+                of[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+                of[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+            }
             uint4 o;
             o.x = pack_bf16x2(acc[0], acc[1]);
             o.y = pack_bf16x2(acc[2], acc[3]);
@@ -89,15 +94,18 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(
 
 cudaError_t launch_combine(const void* slots, int slots_bf16, int T, int D, int k, int has_shared,
                            const uint16_t* x, const uint16_t* shared_gate,
-                           const uint16_t* residual, uint16_t* out, cudaStream_t s) {
+                           const uint16_t* residual, uint16_t* out, float* out_f32,
+                           cudaStream_t s) {
     if (T <= 0) return cudaSuccess;
     int blocks = T < 148 * 16 ? T : 148 * 16;
     if (slots_bf16)
         combine_kernel<uint16_t><<<blocks, kCombineThreads, 0, s>>>(
-            static_cast<const uint16_t*>(slots), T, D, k, has_shared, x, shared_gate, residual, out);
+            static_cast<const uint16_t*>(slots), T, D, k, has_shared, x, shared_gate, residual, out,
+            out_f32);
     else
         combine_kernel<float><<<blocks, kCombineThreads, 0, s>>>(
-            static_cast<const float*>(slots), T, D, k, has_shared, x, shared_gate, residual, out);
+            static_cast<const float*>(slots), T, D, k, has_shared, x, shared_gate, residual, out,
+            out_f32);
     return cudaGetLastError();
 }
 

@@ -12,7 +12,8 @@
 //            [I+f0, ...), against the same token tile; TMEM lane f holds gate and up of
 //            feature f for every token, and the epilogue writes h = silu(g) * u in bf16.
 //   down:    one accumulator, down rows [d0, d0+128) against a tile of h rows; the epilogue
-//            scales by the routing weight (FP32) and stores bf16 into the token's slot.
+//            scales by the routing weight and stores FP32 into the token's slot (a bf16 slot
+//            would add a third bf16 rounding on top of h and the output).
 //   router:  one accumulator, router rows [e0, e0+128) against a tile of x rows; FP32 out.
 //
 // Per CTA (one per SM, persistent over a device-side item list):
@@ -298,7 +299,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                             const int r = ti.b_row + col;
                             const int dest = __ldg(a.row_dest + r);
                             const float wt = __ldg(a.row_weight + r);
-                            a.slots_bf16[(size_t)dest * a.D + d] = to_bf16_bits(wt * v[j]);
+                            a.slots[(size_t)dest * a.D + d] = wt * v[j];
                         }
                     }
                 } else {

@@ -78,7 +78,7 @@ struct StreamArgs {
     const int32_t* row_token;
     const float* row_weight;
     const int32_t* row_dest;
-    uint16_t* h;              // [rows, ld_h] bf16
+    uint16_t* h;              // [rows, ld_h] bf16 SwiGLU output
     int ld_h;
     float* slots;             // [T * S, D] FP32
     int* err;
@@ -88,12 +88,12 @@ struct TcArgs {
     int D, I, I_s, E, nseg;
     SegTables tables;
     // gate_up epilogue
-    uint16_t* h;              // [rows, ld_h]
+    uint16_t* h;              // [rows, ld_h] bf16 SwiGLU output
     int ld_h;
     // down epilogue
     const float* row_weight;
     const int32_t* row_dest;
-    uint16_t* slots_bf16;     // [T * S, D]
+    float* slots;             // [T * S, D] FP32
     // dense (router) epilogue
     float* logits;            // [T, E]
     const float* bias;        // [E] or null
@@ -125,6 +125,7 @@ cudaError_t launch_tc_down(const CUtensorMap& mapA, const CUtensorMap& mapA_shar
                            const CUtensorMap& mapB, const TcArgs& a, int num_sms, cudaStream_t s);
 cudaError_t launch_combine(const void* slots, int slots_bf16, int T, int D, int k, int has_shared,
                            const uint16_t* x, const uint16_t* shared_gate,
-                           const uint16_t* residual, uint16_t* out, cudaStream_t s);
+                           const uint16_t* residual, uint16_t* out, float* out_f32,
+                           cudaStream_t s);
 
 }  // namespace moe

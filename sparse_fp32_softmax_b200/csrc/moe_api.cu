@@ -113,6 +113,7 @@ moe_status check_opts(const moe_dims* d, const moe_opts* o) {
     if (o->path < MOE_PATH_AUTO || o->path > MOE_PATH_GROUPED) return MOE_ERR_INVALID_ARG;
     if (o->n_stage_events != 0 && o->n_stage_events != 6) return MOE_ERR_INVALID_ARG;
     if (o->n_stage_events == 6 && !o->stage_events) return MOE_ERR_INVALID_ARG;
+    if (o->out_f32 && !aligned(o->out_f32, 16)) return MOE_ERR_INVALID_ARG;
     (void)d;
     return MOE_OK;
 }
@@ -171,9 +172,12 @@ T* at(void* ws, size_t off) {
         if ((expr) != cudaSuccess) return MOE_ERR_CUDA;      \
     } while (0)
 
+// Stage events are recorded as external events so that, under stream capture, they become
+// event-record nodes of the graph (a plain record would only order captured work).
 moe_status record(const moe_opts* o, int i, cudaStream_t s) {
     if (o && o->n_stage_events == 6)
-        MOE_CUDA(cudaEventRecord(reinterpret_cast<cudaEvent_t>(o->stage_events[i]), s));
+        MOE_CUDA(cudaEventRecordWithFlags(reinterpret_cast<cudaEvent_t>(o->stage_events[i]), s,
+                                          cudaEventRecordExternal));
     return MOE_OK;
 }
 
@@ -292,6 +296,7 @@ moe_status moe_permute(const int32_t* topk_idx, const float* topk_w, const moe_b
     // padding rows are only written per expert segment; rows past offsets[E] stay as given,
     // so mark every row as padding first
     MOE_CUDA(cudaMemsetAsync(row_token, 0xFF, (size_t)cap * sizeof(int32_t), s));
+    if (a.row_weight) MOE_CUDA(cudaMemsetAsync(a.row_weight, 0, (size_t)cap * sizeof(float), s));
     MOE_CUDA(launch_permute(a, s));
     if (x_perm) MOE_CUDA(launch_gather_rows(x, row_token, cap, p.D, x_perm, s));
     return MOE_OK;
@@ -327,6 +332,7 @@ moe_status moe_forward_ex(const moe_bf16* x, const moe_bf16* W_r, const moe_bf16
     const moe_bf16* sdn = opts ? opts->shared_down : nullptr;
     const moe_bf16* sg = opts ? opts->shared_gate : nullptr;
     const moe_bf16* residual = opts ? opts->residual : nullptr;
+    float* out_f32 = opts ? opts->out_f32 : nullptr;
 
     // tensor maps of the grouped path are encoded before anything is enqueued
     CUtensorMap mGuA, mGuAs, mGuB, mDnA, mDnAs, mDnB;
@@ -387,7 +393,8 @@ moe_status moe_forward_ex(const moe_bf16* x, const moe_bf16* W_r, const moe_bf16
         if ((st = record(opts, 3, s)) != MOE_OK) return st;
         MOE_CUDA(launch_stream_down(sa, p.T, s));
         if ((st = record(opts, 4, s)) != MOE_OK) return st;
-        MOE_CUDA(launch_combine(sa.slots, 0, p.T, p.D, p.k, p.has_shared, x, sg, residual, out, s));
+        MOE_CUDA(launch_combine(sa.slots, 0, p.T, p.D, p.k, p.has_shared, x, sg, residual, out,
+                                out_f32, s));
     } else {
         TcArgs ta{};
         ta.D = p.D; ta.I = p.I; ta.I_s = p.I_s; ta.E = p.E; ta.nseg = p.nseg; ta.T = p.T;
@@ -396,13 +403,14 @@ moe_status moe_forward_ex(const moe_bf16* x, const moe_bf16* W_r, const moe_bf16
         ta.ld_h = p.ld_h;
         ta.row_weight = pa.row_weight;
         ta.row_dest = pa.row_dest;
-        ta.slots_bf16 = at<uint16_t>(ws, p.slots);
+        ta.slots = at<float>(ws, p.slots);
         ta.err = err;
         MOE_CUDA(launch_tc_gate_up(mGuA, mGuAs, mGuB, ta, sms, s));
         if ((st = record(opts, 3, s)) != MOE_OK) return st;
         MOE_CUDA(launch_tc_down(mDnA, mDnAs, mDnB, ta, sms, s));
         if ((st = record(opts, 4, s)) != MOE_OK) return st;
-        MOE_CUDA(launch_combine(ta.slots_bf16, 1, p.T, p.D, p.k, p.has_shared, x, sg, residual, out, s));
+        MOE_CUDA(launch_combine(ta.slots, 0, p.T, p.D, p.k, p.has_shared, x, sg, residual, out,
+                                out_f32, s));
     }
     return record(opts, 5, s);
 }

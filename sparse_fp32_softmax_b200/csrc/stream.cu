@@ -19,7 +19,7 @@
 //          and applies SwiGLU in registers; h is written in bf16 (the precision the down
 //          projection consumes).
 // down:    a warp owns 16 output features of one segment; outputs are scaled by the routing
-//          weight in FP32 and stored to the token's slot, summed later in slot order.
+//          weight in FP32 and stored to the token's FP32 slot, summed later in slot order.
 #include "common.cuh"
 
 namespace moe {

@@ -3,8 +3,15 @@
 Tolerances (the block's correctness criteria):
   * selected expert indices, per-expert counts and the permutation: bit-exact;
   * routing weights: within 1e-6 absolute;
-  * block output y (bf16) against the FP64 oracle: relative L2 error <= 5e-3 and max-abs
-    error <= 2e-2 * rms(y).
+  * block output y against the FP64 oracle: relative L2 error <= 5e-3 and max-abs error
+    <= 2e-2 * rms(y).
+Reading of the output criterion: the block computes y in FP32 and rounds it once to the
+bf16 output format.  That rounding alone moves a value by up to 2^-8 of its magnitude, so
+for outputs beyond ~5 rms (present in these workloads) it exceeds 2e-2 * rms by itself and
+no bf16-output implementation could meet a literal max-abs bound on the stored values.  The
+checks are therefore: max-abs (and relative L2) on the FP32 value before the rounding
+(returned through opts->out_f32); the bf16 output bit-exactly equal to that value rounded
+to nearest even; and relative L2 <= 5e-3 on the bf16 output itself.
 
 Routing against FP64 oracle logits.  The GPU sums bf16 x bf16 products (exact in FP32) in
 FP32 in its own order; the oracle sums them exactly and rounds once.  For logit e of token t
@@ -95,6 +102,15 @@ def y_errors(y_gpu, y_ref):
     rms = np.sqrt(np.mean(y_ref ** 2)) if y_ref.size else 0.0
     max_abs = np.abs(diff).max() if diff.size else 0.0
     return rel_l2, max_abs, rms
+
+
+def assert_block_output(y_bf16, y_f32, y_ref, what=""):
+    """The three checks of the output criterion (see the module docstring).
+    y_bf16: bf16 torch tensor [n, D]; y_f32: FP32 torch tensor [n, D]; y_ref: float64."""
+    assert torch.equal(y_f32.to(torch.bfloat16), y_bf16), f"{what}: bf16 output is not RNE of its FP32 value"
+    rel_b, _, _ = y_errors(y_bf16.double().numpy(), y_ref)
+    assert rel_b <= Y_REL_L2, f"{what}: bf16 output relative L2 error {rel_b:.3e} > {Y_REL_L2}"
+    return assert_y_close(y_f32.double().numpy(), y_ref, what)
 
 
 def assert_y_close(y_gpu, y_ref, what=""):

@@ -13,7 +13,8 @@ import torch
 from oracle import oracle as O
 from sparse_fp32_softmax_b200 import binding as B
 from sparse_fp32_softmax_b200 import inputs
-from tests.parity_util import (W_ATOL, assert_y_close, check_routing, logit_deltas)
+from tests.parity_util import (W_ATOL, assert_block_output, assert_y_close, check_routing,
+                               logit_deltas, y_errors)
 
 pytestmark = pytest.mark.gpu
 
@@ -49,12 +50,14 @@ def run_forward(cfg, G, path="auto", x=None, residual=None, k=None, norm=None):
     idx = torch.empty(T, k, dtype=torch.int32, device="cuda")
     w = torch.empty(T, k, dtype=torch.float32, device="cuda")
     logits = torch.empty(T, E, dtype=torch.float32, device="cuda")
+    y32 = torch.empty(x.shape, dtype=torch.float32, device="cuda")
     out = B.moe_forward_ex(x, G["W_r"], G["W_gate_up"], G["W_down"], k, norm,
                            router_bias=G.get("bias"), shared_gate_up=G.get("shared_gate_up"),
                            shared_down=G.get("shared_down"), shared_gate=G.get("shared_gate"),
                            residual=residual, logits_out=logits, topk_idx_out=idx, topk_w_out=w,
-                           path=path)
+                           path=path, out_f32=y32)
     torch.cuda.synchronize()
+    run_forward.last_f32 = y32.cpu()
     return out.cpu(), idx.cpu().numpy(), w.cpu().numpy(), logits.cpu().numpy()
 
 
@@ -66,6 +69,7 @@ def compare_block(cfg, L, G, rows, path="auto", x_cpu=None, residual_cpu=None, k
     x_cpu = L["x"] if x_cpu is None else x_cpu
     res_gpu = residual_cpu.cuda() if residual_cpu is not None else None
     y, idx, w, logits = run_forward(cfg, G, path, x=x_cpu.cuda(), residual=res_gpu, k=k, norm=norm)
+    y32 = run_forward.last_f32
     rows = np.asarray(sorted(set(int(r) for r in rows)), np.int32)
     # selection from the GPU's own logits is bit-exact; weights within 1e-6
     o_idx, o_w = O.select(logits, k, norm)
@@ -91,8 +95,8 @@ def compare_block(cfg, L, G, rows, path="auto", x_cpu=None, residual_cpu=None, k
                                           shared_down=L.get("shared_down"),
                                           shared_gate=L.get("shared_gate"),
                                           residual=residual_cpu, threads=THREADS)
-    yg = y[torch.from_numpy(rows).long()].double().numpy()
-    rel, mx = assert_y_close(yg, y_ref, what)
+    sel = torch.from_numpy(rows).long()
+    rel, mx = assert_block_output(y[sel], y32[sel], y_ref, what)
     return dict(rel_l2=rel, max_abs_over_rms=mx, decisive=nd, other=nother, idx=idx, y=y)
 
 
@@ -266,18 +270,26 @@ def test_forward_zero_input(path):
 
 @pytest.mark.parametrize("path", ["stream", "grouped"])
 def test_determinism_and_batch_invariance(path):
+    """Bitwise-equal reruns, and a token's output independent of the other tokens in the
+    batch for a given router kernel (T <= 64 runs the CUDA-core router, larger T the
+    tensor-core one; the two sum the logits in different FP32 orders)."""
     cfg, L, G = _small_layer(256)
     y1, *_ = run_forward(cfg, G, path)
     y2, *_ = run_forward(cfg, G, path)
     assert torch.equal(y1, y2)
+    y100, *_ = run_forward(cfg, G, path, x=G["x"][:100].contiguous())
+    assert torch.equal(y100, y1[:100])
+    y64, *_ = run_forward(cfg, G, path, x=G["x"][:64].contiguous())
     y8, *_ = run_forward(cfg, G, path, x=G["x"][:8].contiguous())
-    assert torch.equal(y8, y1[:8])
+    assert torch.equal(y8, y64[:8])
 
 
 def test_paths_agree_and_status_ok():
     cfg, L, G = layer("decode", 128)
-    ys, *_ = run_forward(cfg, G, "stream")
-    yg, *_ = run_forward(cfg, G, "grouped")
+    run_forward(cfg, G, "stream")
+    ys = run_forward.last_f32
+    run_forward(cfg, G, "grouped")
+    yg = run_forward.last_f32
     assert_y_close(ys.double().numpy(), yg.double().numpy(), "stream vs grouped")
     dims = B.make_dims(128, cfg.D, cfg.E, cfg.k, cfg.I)
     ws = B.workspace(dims)
@@ -298,23 +310,33 @@ def test_gpu_errors_before_launch():
 
 
 def test_residual_chain_short():
-    """Three residual blocks of the 48-block chain's shape: x_{l+1} = x_l + MoE_l(x_l),
-    compared row by row with the oracle's own trajectory (rows are independent)."""
+    """Three residual blocks of the 48-block chain's shape, x_{l+1} = x_l + MoE_l(x_l).
+    Each layer is checked on the oracle's own layer input (teacher forcing: the oracle's
+    bf16 trajectory is fed to the GPU, never the reverse) with the full output criterion;
+    the free-running GPU chain is compared with the oracle trajectory in relative L2 (its
+    max-abs is dominated by one-ulp bf16 flips of the residual stream, ~3% of rms at |x|>4,
+    which no bf16 chain can avoid)."""
     cfg = inputs.CONFIGS["keras"]
     T, nl = 256, 3
-    x0 = inputs.make_layer(cfg, T=T, layer=0)["x"]
-    rows = list(range(0, T, 8))
-    x_gpu = x0.cuda()
-    x_o = x0.clone()
+    x_o = inputs.make_layer(cfg, T=T, layer=0)["x"]
+    rows = list(range(T))
+    x_free = x_o.cuda()
     for l in range(nl):
         Ll = inputs.make_layer(cfg, T=T, layer=l, with_x=False)
         Gl = {k: (v.cuda() if v is not None else None) for k, v in Ll.items()}
-        out = torch.empty_like(x_gpu)
-        B.moe_forward_ex(x_gpu, Gl["W_r"], Gl["W_gate_up"], Gl["W_down"], cfg.k, True, out=out,
-                         residual=x_gpu)
-        x_gpu = out
-        y, *_ = O.forward_rows(x_o, Ll["W_r"], Ll["W_gate_up"], Ll["W_down"], cfg.k, list(range(T)),
+        x_in = x_o.cuda()
+        y32 = torch.empty(x_in.shape, dtype=torch.float32, device="cuda")
+        out = B.moe_forward_ex(x_in, Gl["W_r"], Gl["W_gate_up"], Gl["W_down"], cfg.k, True,
+                               residual=x_in, out_f32=y32)
+        free = torch.empty_like(x_free)
+        B.moe_forward_ex(x_free, Gl["W_r"], Gl["W_gate_up"], Gl["W_down"], cfg.k, True, out=free,
+                         residual=x_free)
+        x_free = free
+        y, *_ = O.forward_rows(x_o, Ll["W_r"], Ll["W_gate_up"], Ll["W_down"], cfg.k, rows,
                                residual=x_o, threads=THREADS)
+        torch.cuda.synchronize()
+        assert_block_output(out.cpu(), y32.cpu(), y, f"chain layer {l}")
         x_o = torch.from_numpy(y).to(torch.bfloat16)
-    torch.cuda.synchronize()
-    assert_y_close(x_gpu.cpu()[rows].double().numpy(), x_o[rows].double().numpy(), "chain")
+    rel, _, _ = y_errors(x_free.cpu().double().numpy(), x_o.double().numpy())
+    print(f"free-running chain vs oracle trajectory after {nl} layers: relative L2 {rel:.2e}")
+    assert rel <= 5e-2, rel     # divergence diagnostic: near-tie routing flips compound
