@@ -144,6 +144,24 @@ moe_status moe_forward_ex(const moe_bf16 *x, const moe_bf16 *W_r, const moe_bf16
                           const moe_bf16 *W_down, const moe_dims *dims, const moe_opts *opts,
                           moe_bf16 *out, void *ws, size_t ws_bytes, moe_stream_t stream);
 
+/* moe_forward for callers that cannot allocate device memory: code that enqueues work
+ * while a stream is being captured into a CUDA graph, plugin hosts that give a kernel only
+ * its input and output buffers, runtimes that forbid allocation after start-up.  The pages
+ * have no counterpart: this is a deployment variant of moe_forward, same arguments minus
+ * the workspace, same results.
+ * Scratch: a 32 MiB array in the library's own device memory (a file-scope device
+ * variable), held by every GPU that loads this part of the library until the process
+ * exits.  Calls whose moe_workspace_size(dims, NULL) exceeds 32 MiB return
+ * MOE_ERR_WORKSPACE before enqueuing anything (the decode shapes fit: D=2048, E=128, k=8,
+ * I=768 up to T=256).  Nothing is allocated or freed.
+ * The first call on a device looks up the array's device address (once per device); make
+ * that first call before any stream capture.  All calls on a device share the array and it
+ * keeps the last call's contents; each call clears what must start at zero.  Calls that can
+ * overlap on the GPU (other streams, unordered host threads) race on the array. */
+moe_status moe_forward_noalloc(const moe_bf16 *x, const moe_bf16 *W_r, const moe_bf16 *W_gate_up,
+                               const moe_bf16 *W_down, const moe_dims *dims, moe_bf16 *out,
+                               moe_stream_t stream);
+
 /* Synchronises `stream` and reports the device error word that the last call using `ws`
  * left: MOE_OK, MOE_ERR_DEVICE_TIMEOUT (a bounded wait expired), MOE_ERR_INVALID_ARG (an
  * expert index outside [0, E) reached moe_permute) or MOE_ERR_CUDA. */

@@ -62,10 +62,12 @@ def load():
         lib.moe_permute.argtypes = [_vp, _vp, _vp, dp, _vp, _vp, _vp, _vp, _vp, _vp, _c_int, _vp, _sz, _vp]
         lib.moe_forward.argtypes = [_vp, _vp, _vp, _vp, dp, _vp, _vp, _sz, _vp]
         lib.moe_forward_ex.argtypes = [_vp, _vp, _vp, _vp, dp, op, _vp, _vp, _sz, _vp]
+        lib.moe_forward_noalloc.argtypes = [_vp, _vp, _vp, _vp, dp, _vp, _vp]
         lib.moe_get_device_status.argtypes = [_vp, _vp]
         lib.moe_status_string.argtypes = [_c_int]
         lib.moe_status_string.restype = ctypes.c_char_p
-        for n in ("moe_route", "moe_permute", "moe_forward", "moe_forward_ex", "moe_get_device_status"):
+        for n in ("moe_route", "moe_permute", "moe_forward", "moe_forward_ex", "moe_forward_noalloc",
+                  "moe_get_device_status"):
             getattr(lib, n).restype = _c_int
         _lib = lib
     return _lib
@@ -227,6 +229,18 @@ def moe_forward_ex(x, W_r, W_gate_up, W_down, k, norm_topk_prob=True, out=None, 
     _check(load().moe_forward_ex(_ptr(x), _ptr(W_r), _ptr(W_gate_up), _ptr(W_down), ctypes.byref(dims),
                                  ctypes.byref(opts), _ptr(out), _ptr(ws), ws.numel(), _stream(stream)),
            "moe_forward_ex")
+    return out
+
+
+def moe_forward_noalloc(x, W_r, W_gate_up, W_down, k, norm_topk_prob=True, out=None, stream=None):
+    """moe_forward without a workspace argument: for callers that cannot allocate device
+    memory, the library uses its own fixed 32 MiB device array (see the header)."""
+    dims = _dims_of(x, W_r, W_gate_up, W_down, k, norm_topk_prob)
+    if out is None:
+        out = torch.empty_like(x)
+    _check(load().moe_forward_noalloc(_ptr(x), _ptr(W_r), _ptr(W_gate_up), _ptr(W_down),
+                                      ctypes.byref(dims), _ptr(out), _stream(stream)),
+           "moe_forward_noalloc")
     return out
 
 

@@ -26,7 +26,8 @@ def lib():
 def test_library_exports_every_declared_function(lib):
     declared = B.header_functions()
     assert set(declared) == {"moe_workspace_size", "moe_route", "moe_permute", "moe_forward",
-                             "moe_forward_ex", "moe_get_device_status", "moe_status_string"}
+                             "moe_forward_ex", "moe_forward_noalloc", "moe_get_device_status",
+                             "moe_status_string"}
     out = subprocess.run(["nm", "-D", "--defined-only", LIB], capture_output=True, text=True, check=True).stdout
     exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
     for name in declared:
