@@ -175,9 +175,14 @@ T* at(void* ws, size_t off) {
 // Stage events are recorded as external events so that, under stream capture, they become
 // event-record nodes of the graph (a plain record would only order captured work).
 moe_status record(const moe_opts* o, int i, cudaStream_t s) {
-    if (o && o->n_stage_events == 6)
+    if (o && o->n_stage_events == 6) {
+        cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+        MOE_CUDA(cudaStreamIsCapturing(s, &cs));
+        const unsigned flags =
+            cs == cudaStreamCaptureStatusActive ? cudaEventRecordExternal : cudaEventRecordDefault;
         MOE_CUDA(cudaEventRecordWithFlags(reinterpret_cast<cudaEvent_t>(o->stage_events[i]), s,
-                                          cudaEventRecordExternal));
+                                          flags));
+    }
     return MOE_OK;
 }
 
