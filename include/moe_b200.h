@@ -69,9 +69,10 @@ typedef struct {
 
 /* Which expert path moe_forward_ex takes. */
 enum {
-    MOE_PATH_AUTO = 0,    /* streaming path for small T, grouped tensor-core path otherwise */
-    MOE_PATH_STREAM = 1,  /* stream each touched expert's weights once (decode) */
-    MOE_PATH_GROUPED = 2  /* permute + tcgen05 grouped GEMMs (prefill) */
+    MOE_PATH_AUTO = 0,    /* the library's choice (currently the grouped path at every T) */
+    MOE_PATH_STREAM = 1,  /* warp-MMA kernels that stream each touched expert's weights once
+                             straight into registers (no permuted copy of x) */
+    MOE_PATH_GROUPED = 2  /* permute + tcgen05 grouped GEMMs, TMA-fed, TMEM accumulators */
 };
 
 /* Options of moe_forward_ex.  Zero-initialise and set what is needed. */

@@ -249,6 +249,37 @@ __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint3
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// Segment tables copied into shared memory at kernel start, so that decoding a work item
+// costs a few shared-memory loads instead of a chain of dependent global loads.
+struct SmemTables {
+    int prefix[kMaxSegments + 1];
+    int count[kMaxSegments];
+    int start[kMaxSegments];
+};
+
+// Cooperative copy by all threads of the block (caller synchronises afterwards).
+__device__ __forceinline__ void load_tables(SmemTables* st, const int* prefix, const int* count,
+                                            const int* start, int nseg) {
+    for (int i = threadIdx.x; i <= nseg; i += blockDim.x) st->prefix[i] = __ldg(prefix + i);
+    for (int i = threadIdx.x; i < nseg; i += blockDim.x) {
+        st->count[i] = __ldg(count + i);
+        st->start[i] = __ldg(start + i);
+    }
+}
+
+// Largest s with prefix[s] <= item, searching a shared-memory prefix array.
+__device__ __forceinline__ int find_segment_smem(const int* prefix, int nseg, int item) {
+    int lo = 0, hi = nseg - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (prefix[mid] <= item)
+            lo = mid;
+        else
+            hi = mid - 1;
+    }
+    return lo;
+}
+
 // Index of the segment s with prefix[s] <= item < prefix[s+1] (prefix non-decreasing,
 // prefix[0] = 0, item < prefix[nseg]).
 __device__ __forceinline__ int find_segment(const int* prefix, int nseg, int item) {

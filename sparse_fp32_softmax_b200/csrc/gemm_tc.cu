@@ -57,10 +57,12 @@ constexpr int tc_stage_bytes() {
 }
 template <int MODE>
 constexpr int tc_smem_bytes() {
-    return kStages * tc_stage_bytes<MODE>() + 1024 + 256;
+    return kStages * tc_stage_bytes<MODE>() + 1024 + 256 + (int)sizeof(SmemTables) +
+           (MODE == kModeDown ? 4 * 2 * 4 * kDnBN : 0);
 }
 
 struct TileInfo {
+    int bi;       // token-operand box: 16 << bi rows
     int shared;   // A comes from the shared-expert tensor map
     int a_row0;   // first A row (gate rows for gate_up)
     int a_row1;   // first up row (gate_up only)
@@ -78,8 +80,16 @@ __device__ __forceinline__ int tc_total_items(const TcArgs& a) {
     return __ldg(prefix + a.nseg);
 }
 
+// Smallest token box (16 << bi rows, bi <= log2(BN/16)) that covers n valid rows.
+template <int BN>
+__device__ __forceinline__ int box_index(int n) {
+    int bi = 0;
+    while ((16 << bi) < n && (16 << bi) < BN) ++bi;
+    return bi;
+}
+
 template <int MODE>
-__device__ __forceinline__ TileInfo tc_decode_item(const TcArgs& a, int item) {
+__device__ __forceinline__ TileInfo tc_decode_item(const TcArgs& a, const SmemTables* st, int item) {
     constexpr int BN = TcTraits<MODE>::BN;
     TileInfo ti;
     if (MODE == kModeRouter) {
@@ -92,17 +102,17 @@ __device__ __forceinline__ TileInfo tc_decode_item(const TcArgs& a, int item) {
         ti.n_valid = min(BN, a.T - tt * BN);
         ti.nk = a.D / kTcK;
         ti.m0 = mt * kTcM;
+        ti.bi = box_index<BN>(ti.n_valid);
         return ti;
     }
-    const int* prefix = (MODE == kModeGateUp) ? a.tables.gu_items : a.tables.dn_items;
-    const int s = find_segment(prefix, a.nseg, item);
-    const int local = item - __ldg(prefix + s);
+    const int s = find_segment_smem(st->prefix, a.nseg, item);
+    const int local = item - st->prefix[s];
     const int sh = (s == a.E);
     const int Iseg = sh ? a.I_s : a.I;
     const int mtc = (MODE == kModeGateUp) ? Iseg / kTcM : a.D / kTcM;
     const int tt = local / mtc, mt = local % mtc;
-    const int cnt = __ldg(a.tables.seg_count + s);
-    const int start = __ldg(a.tables.seg_start + s);
+    const int cnt = st->count[s];
+    const int start = st->start[s];
     ti.shared = sh;
     ti.b_row = start + tt * BN;
     ti.n_valid = min(BN, cnt - tt * BN);
@@ -118,6 +128,7 @@ __device__ __forceinline__ TileInfo tc_decode_item(const TcArgs& a, int item) {
         ti.a_row1 = 0;
         ti.nk = Iseg / kTcK;
     }
+    ti.bi = box_index<BN>(ti.n_valid);
     return ti;
 }
 
@@ -133,9 +144,7 @@ __device__ __forceinline__ void tma_load(void* dst, const CUtensorMap* map, uint
 
 template <int MODE>
 __global__ void __launch_bounds__(kTcThreads, 1)
-    tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA,
-                   const __grid_constant__ CUtensorMap mapA_sh,
-                   const __grid_constant__ CUtensorMap mapB, const TcArgs a) {
+    tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
     using Tr = TcTraits<MODE>;
     constexpr int BN = Tr::BN, NA = Tr::NA, ACC = Tr::ACC;
     constexpr int SB = tc_stage_bytes<MODE>();
@@ -148,6 +157,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     uint64_t* tempty = tfull + 2;       // [2]
     uint64_t* drain = tempty + 2;       // [1]
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    SmemTables* tabs = reinterpret_cast<SmemTables*>(smem + kStages * SB + 256);
+    // down: per epilogue warp, the current tile's row destinations and weights
+    int* ep_dest_all = reinterpret_cast<int*>(tabs + 1);       // [4][BN]
+    float* ep_wt_all = reinterpret_cast<float*>(ep_dest_all + 4 * BN);  // [4][BN]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int total = tc_total_items<MODE>(a);
@@ -165,12 +178,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         mbar_init(drain, 1);
         mbar_fence_init();
     }
-    if (warp == 0 && lane == 0) {
-        tma_prefetch_desc(&mapA);
-        tma_prefetch_desc(&mapA_sh);
-        tma_prefetch_desc(&mapB);
+    if (warp == 0 && lane < 2 + kNumBBoxes) {
+        const CUtensorMap* m = lane == 0 ? &maps.A : (lane == 1 ? &maps.A_shared : &maps.B[lane - 2]);
+        tma_prefetch_desc(m);
     }
     if (warp == 1) tmem_alloc(tmem_slot, Tr::TMEM);
+    if (MODE != kModeRouter) {
+        const int* prefix = (MODE == kModeGateUp) ? a.tables.gu_items : a.tables.dn_items;
+        load_tables(tabs, prefix, a.tables.seg_count, a.tables.seg_start, a.nseg);
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -185,8 +201,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
             for (int s = 0; s < kStages; ++s) last_round[s] = -1;
             for (int item = blockIdx.x; item < total && ok; item += gridDim.x) {
-                const TileInfo ti = tc_decode_item<MODE>(a, item);
-                const CUtensorMap* mA = ti.shared ? &mapA_sh : &mapA;
+                const TileInfo ti = tc_decode_item<MODE>(a, tabs, item);
+                const CUtensorMap* mA = ti.shared ? &maps.A_shared : &maps.A;
+                const CUtensorMap* mB = &maps.B[ti.bi];
+                const uint32_t bytes = NA * kATileBytes + (16u << ti.bi) * kTcK * 2;
                 for (int kb = 0; kb < ti.nk; ++kb, ++it) {
                     const int s = it % kStages;
                     const int round = it / kStages;
@@ -195,10 +213,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         break;
                     }
                     uint8_t* st = smem + s * SB;
-                    mbar_arrive_expect_tx(full + s, SB);
+                    mbar_arrive_expect_tx(full + s, bytes);
                     tma_load(st, mA, full + s, kb * kTcK, ti.a_row0);
                     if (NA == 2) tma_load(st + kATileBytes, mA, full + s, kb * kTcK, ti.a_row1);
-                    tma_load(st + NA * kATileBytes, &mapB, full + s, kb * kTcK, ti.b_row);
+                    tma_load(st + NA * kATileBytes, mB, full + s, kb * kTcK, ti.b_row);
 #pragma unroll
                     for (int q = 0; q < kStages; ++q)
                         if (q == s) last_round[q] = round;
@@ -224,7 +242,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             int it = 0, tc = 0;
             bool ok = true;
             for (int item = blockIdx.x; item < total && ok; item += gridDim.x, ++tc) {
-                const TileInfo ti = tc_decode_item<MODE>(a, item);
+                const TileInfo ti = tc_decode_item<MODE>(a, tabs, item);
                 const int b = tc & 1;
                 const int use = tc >> 1;
                 if (!mbar_wait(tempty + b, (use & 1) ^ 1, a.err, kErrWaitMma)) {
@@ -269,7 +287,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const int row = quarter * 32 + lane;  // TMEM lane = weight row within the tile
         int tc = 0;
         for (int item = blockIdx.x; item < total; item += gridDim.x, ++tc) {
-            const TileInfo ti = tc_decode_item<MODE>(a, item);
+            const TileInfo ti = tc_decode_item<MODE>(a, tabs, item);
             const int b = tc & 1;
             const int use = tc >> 1;
             const bool got = mbar_wait(tfull + b, use & 1, a.err, kErrWaitEpilogue);
@@ -277,6 +295,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             tc_fence_after();
             const uint32_t tb = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(b * ACC);
             const int nchunks = (ti.n_valid + 31) >> 5;
+            int* ep_dest = ep_dest_all + quarter * BN;
+            float* ep_wt = ep_wt_all + quarter * BN;
+            if (MODE == kModeDown) {
+                // each epilogue warp keeps its own copy: no barrier across warps
+                __syncwarp();
+                for (int c = lane; c < ti.n_valid; c += 32) {
+                    ep_dest[c] = __ldg(a.row_dest + ti.b_row + c);
+                    ep_wt[c] = __ldg(a.row_weight + ti.b_row + c);
+                }
+                __syncwarp();
+            }
             for (int c = 0; c < nchunks; ++c) {
                 float v[32];
                 tmem_ld32(tb + c * 32, v);
@@ -295,12 +324,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
                         const int col = c * 32 + j;
-                        if (col < ti.n_valid) {
-                            const int r = ti.b_row + col;
-                            const int dest = __ldg(a.row_dest + r);
-                            const float wt = __ldg(a.row_weight + r);
-                            a.slots[(size_t)dest * a.D + d] = wt * v[j];
-                        }
+                        if (col < ti.n_valid)
+                            a.slots[(size_t)ep_dest[col] * a.D + d] = ep_wt[col] * v[j];
                     }
                 } else {
                     tmem_ld_wait();
@@ -329,31 +354,26 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 }
 
 template <int MODE>
-static cudaError_t launch_tc(const CUtensorMap& mapA, const CUtensorMap& mapA_sh,
-                             const CUtensorMap& mapB, const TcArgs& a, int grid, cudaStream_t s) {
+static cudaError_t launch_tc(const TcMaps& maps, const TcArgs& a, int grid, cudaStream_t s) {
     constexpr int smem = tc_smem_bytes<MODE>();
     cudaError_t err = ensure_smem_attr((const void*)tc_gemm_kernel<MODE>, smem, 1 + MODE);
     if (err != cudaSuccess) return err;
     if (grid < 1) grid = 1;
-    tc_gemm_kernel<MODE><<<grid, kTcThreads, smem, s>>>(mapA, mapA_sh, mapB, a);
+    tc_gemm_kernel<MODE><<<grid, kTcThreads, smem, s>>>(maps, a);
     return cudaGetLastError();
 }
 
-cudaError_t launch_tc_router(const CUtensorMap& mapA, const CUtensorMap& mapB, const TcArgs& a,
-                             int num_sms, cudaStream_t s) {
+cudaError_t launch_tc_router(const TcMaps& maps, const TcArgs& a, int num_sms, cudaStream_t s) {
     const int items = ((a.T + kRtBN - 1) / kRtBN) * ((a.E + kTcM - 1) / kTcM);
-    return launch_tc<kModeRouter>(mapA, mapA, mapB, a, items < num_sms ? items : num_sms, s);
+    return launch_tc<kModeRouter>(maps, a, items < num_sms ? items : num_sms, s);
 }
 
-cudaError_t launch_tc_gate_up(const CUtensorMap& mapA, const CUtensorMap& mapA_shared,
-                              const CUtensorMap& mapB, const TcArgs& a, int num_sms,
-                              cudaStream_t s) {
-    return launch_tc<kModeGateUp>(mapA, mapA_shared, mapB, a, num_sms, s);
+cudaError_t launch_tc_gate_up(const TcMaps& maps, const TcArgs& a, int num_sms, cudaStream_t s) {
+    return launch_tc<kModeGateUp>(maps, a, num_sms, s);
 }
 
-cudaError_t launch_tc_down(const CUtensorMap& mapA, const CUtensorMap& mapA_shared,
-                           const CUtensorMap& mapB, const TcArgs& a, int num_sms, cudaStream_t s) {
-    return launch_tc<kModeDown>(mapA, mapA_shared, mapB, a, num_sms, s);
+cudaError_t launch_tc_down(const TcMaps& maps, const TcArgs& a, int num_sms, cudaStream_t s) {
+    return launch_tc<kModeDown>(maps, a, num_sms, s);
 }
 
 }  // namespace moe

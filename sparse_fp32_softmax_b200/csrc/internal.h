@@ -43,8 +43,8 @@ struct SegTables {
     int* seg_start;   // [nseg] first permuted row of each segment
     int* gu_items;    // [nseg + 1] prefix sums of tcgen05 gate_up work items
     int* dn_items;    // [nseg + 1] prefix sums of tcgen05 down work items
-    int* gu_tasks;    // [nseg + 1] prefix sums of streaming gate_up warp tasks
-    int* dn_tasks;    // [nseg + 1] prefix sums of streaming down warp tasks
+    int* gu_tasks;    // [nseg + 1] prefix sums of streaming gate_up tasks
+    int* dn_tasks;    // [nseg + 1] prefix sums of streaming down tasks
 };
 
 struct PermuteArgs {
@@ -84,6 +84,16 @@ struct StreamArgs {
     int* err;
 };
 
+// Tensor maps of one grouped GEMM: the weight operand (routed experts, shared expert) and
+// the token operand encoded at five box heights (16, 32, 64, 128, 256 rows), so that a work
+// item loads only as many token rows as it has (rounded up to the next height).
+constexpr int kNumBBoxes = 5;
+struct alignas(64) TcMaps {
+    CUtensorMap A;
+    CUtensorMap A_shared;
+    CUtensorMap B[kNumBBoxes];
+};
+
 struct TcArgs {
     int D, I, I_s, E, nseg;
     SegTables tables;
@@ -116,13 +126,9 @@ cudaError_t launch_gather_rows(const uint16_t* x, const int32_t* row_token, int 
                                uint16_t* x_perm, cudaStream_t s);
 cudaError_t launch_stream_gate_up(const StreamArgs& a, int max_rows, cudaStream_t s);
 cudaError_t launch_stream_down(const StreamArgs& a, int max_rows, cudaStream_t s);
-cudaError_t launch_tc_router(const CUtensorMap& mapA, const CUtensorMap& mapB, const TcArgs& a,
-                             int num_sms, cudaStream_t s);
-cudaError_t launch_tc_gate_up(const CUtensorMap& mapA, const CUtensorMap& mapA_shared,
-                              const CUtensorMap& mapB, const TcArgs& a, int num_sms,
-                              cudaStream_t s);
-cudaError_t launch_tc_down(const CUtensorMap& mapA, const CUtensorMap& mapA_shared,
-                           const CUtensorMap& mapB, const TcArgs& a, int num_sms, cudaStream_t s);
+cudaError_t launch_tc_router(const TcMaps& maps, const TcArgs& a, int num_sms, cudaStream_t s);
+cudaError_t launch_tc_gate_up(const TcMaps& maps, const TcArgs& a, int num_sms, cudaStream_t s);
+cudaError_t launch_tc_down(const TcMaps& maps, const TcArgs& a, int num_sms, cudaStream_t s);
 cudaError_t launch_combine(const void* slots, int slots_bf16, int T, int D, int k, int has_shared,
                            const uint16_t* x, const uint16_t* shared_gate,
                            const uint16_t* residual, uint16_t* out, float* out_f32,

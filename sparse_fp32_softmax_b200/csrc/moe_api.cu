@@ -33,7 +33,6 @@ namespace {
 
 constexpr size_t kAlign = 256;
 constexpr int kRouterSmallMaxT = 64;     // below: CUDA-core router; above: tcgen05 router GEMM
-constexpr int kStreamMaxAssignments = 2048;  // AUTO path: streaming while T*k <= this
 
 size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
@@ -162,6 +161,19 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, ui
     return r == CUDA_SUCCESS;
 }
 
+// The token-operand map at every box height up to max_rows.
+bool make_b_maps(CUtensorMap* maps, const void* base, uint64_t cols, uint64_t rows, int max_rows) {
+    for (int bi = 0; bi < kNumBBoxes; ++bi) {
+        const uint32_t box = 16u << bi;
+        if ((int)box > max_rows) {
+            maps[bi] = maps[bi - 1];
+            continue;
+        }
+        if (!make_map(&maps[bi], base, cols, rows, box)) return false;
+    }
+    return true;
+}
+
 template <typename T>
 T* at(void* ws, size_t off) {
     return reinterpret_cast<T*>(static_cast<char*>(ws) + off);
@@ -204,9 +216,10 @@ moe_status run_route(const moe_bf16* x, const moe_bf16* W_r, const float* bias, 
     if (p.T <= kRouterSmallMaxT) {
         MOE_CUDA(launch_router_small(x, W_r, bias, p.T, p.D, p.E, logits, s));
     } else {
-        CUtensorMap mA, mB;
-        if (!make_map(&mA, W_r, p.D, p.E, kTcM)) return MOE_ERR_CUDA;
-        if (!make_map(&mB, x, p.D, p.T, kRtBN)) return MOE_ERR_CUDA;
+        TcMaps maps;
+        if (!make_map(&maps.A, W_r, p.D, p.E, kTcM)) return MOE_ERR_CUDA;
+        maps.A_shared = maps.A;
+        if (!make_b_maps(maps.B, x, p.D, p.T, kRtBN)) return MOE_ERR_CUDA;
         TcArgs a{};
         a.D = p.D; a.E = p.E; a.T = p.T; a.I = p.I; a.nseg = 1;
         a.logits = logits;
@@ -214,7 +227,7 @@ moe_status run_route(const moe_bf16* x, const moe_bf16* W_r, const float* bias, 
         a.err = at<int>(ws, p.err);
         const int sms = num_sms_of_current_device();
         if (sms <= 0) return MOE_ERR_CUDA;
-        MOE_CUDA(launch_tc_router(mA, mB, a, sms, s));
+        MOE_CUDA(launch_tc_router(maps, a, sms, s));
     }
     MOE_CUDA(launch_select(logits, p.T, p.E, p.k, norm, idx, w, s));
     return MOE_OK;
@@ -323,8 +336,9 @@ moe_status moe_forward_ex(const moe_bf16* x, const moe_bf16* W_r, const moe_bf16
     if (ws_bytes < p.total) return MOE_ERR_WORKSPACE;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const int path_req = opts ? opts->path : MOE_PATH_AUTO;
-    const bool streaming = path_req == MOE_PATH_STREAM ||
-                           (path_req == MOE_PATH_AUTO && (long)p.T * p.k <= kStreamMaxAssignments);
+    // AUTO takes the tensor-core grouped path at every T: measured on B200 it beats the
+    // register-streaming path from T = 1 up (its 2-D TMA weight tiles keep HBM busier)
+    const bool streaming = path_req == MOE_PATH_STREAM;
     const int sms = num_sms_of_current_device();
     if (sms <= 0) return MOE_ERR_CUDA;
 
@@ -340,16 +354,17 @@ moe_status moe_forward_ex(const moe_bf16* x, const moe_bf16* W_r, const moe_bf16
     float* out_f32 = opts ? opts->out_f32 : nullptr;
 
     // tensor maps of the grouped path are encoded before anything is enqueued
-    CUtensorMap mGuA, mGuAs, mGuB, mDnA, mDnAs, mDnB;
+    TcMaps mGu, mDn;
     if (!streaming) {
         uint16_t* x_perm = at<uint16_t>(ws, p.x_perm);
         uint16_t* h = at<uint16_t>(ws, p.h);
-        if (!make_map(&mGuA, W_gate_up, p.D, (uint64_t)p.E * 2 * p.I, kTcM) ||
-            !make_map(&mGuAs, sgu ? sgu : W_gate_up, p.D, sgu ? 2 * (uint64_t)p.I_s : 2 * (uint64_t)p.I, kTcM) ||
-            !make_map(&mGuB, x_perm, p.D, p.R, kGuBN) ||
-            !make_map(&mDnA, W_down, p.I, (uint64_t)p.E * p.D, kTcM) ||
-            !make_map(&mDnAs, sdn ? sdn : W_down, sdn ? p.I_s : p.I, p.D, kTcM) ||
-            !make_map(&mDnB, h, p.ld_h, p.R, kDnBN))
+        if (!make_map(&mGu.A, W_gate_up, p.D, (uint64_t)p.E * 2 * p.I, kTcM) ||
+            !make_map(&mGu.A_shared, sgu ? sgu : W_gate_up, p.D,
+                      sgu ? 2 * (uint64_t)p.I_s : 2 * (uint64_t)p.I, kTcM) ||
+            !make_b_maps(mGu.B, x_perm, p.D, p.R, kGuBN) ||
+            !make_map(&mDn.A, W_down, p.I, (uint64_t)p.E * p.D, kTcM) ||
+            !make_map(&mDn.A_shared, sdn ? sdn : W_down, sdn ? p.I_s : p.I, p.D, kTcM) ||
+            !make_b_maps(mDn.B, h, p.ld_h, p.R, kDnBN))
             return MOE_ERR_CUDA;
     }
 
@@ -410,9 +425,9 @@ moe_status moe_forward_ex(const moe_bf16* x, const moe_bf16* W_r, const moe_bf16
         ta.row_dest = pa.row_dest;
         ta.slots = at<float>(ws, p.slots);
         ta.err = err;
-        MOE_CUDA(launch_tc_gate_up(mGuA, mGuAs, mGuB, ta, sms, s));
+        MOE_CUDA(launch_tc_gate_up(mGu, ta, sms, s));
         if ((st = record(opts, 3, s)) != MOE_OK) return st;
-        MOE_CUDA(launch_tc_down(mDnA, mDnAs, mDnB, ta, sms, s));
+        MOE_CUDA(launch_tc_down(mDn, ta, sms, s));
         if ((st = record(opts, 4, s)) != MOE_OK) return st;
         MOE_CUDA(launch_combine(ta.slots, 0, p.T, p.D, p.k, p.has_shared, x, sg, residual, out,
                                 out_f32, s));

@@ -124,8 +124,8 @@ __global__ void __launch_bounds__(kPermThreads) perm_scan_kernel(PermuteArgs a) 
             if (c > 0) {
                 gi = (c + kGuBN - 1) / kGuBN * (Iseg / kTcM);
                 di = (c + kDnBN - 1) / kDnBN * (a.D / kTcM);
-                gt = Iseg / 8;
-                dt = a.D / 16;
+                gt = Iseg / 8;      // streaming gate_up: one warp per 8 features
+                dt = a.D / 16;      // streaming down: one warp per 16 output rows
             }
         }
         int tot;
