@@ -325,7 +325,7 @@ def run_ours(args, rank, world, device):
             for j in range(5):
                 stage_ms[n][j] += e[j].elapsed_time(e[j + 1]) / K
     peaks = load_peaks()
-    launches_per_pass = [8 if p["streaming"] else 9 for p in passes]
+    launches_per_pass = [8 + (0 if (p["streaming"] or p["T"] <= 32) else 1) for p in passes]   # router 2, permute 3 (+ row copy), gate_up, down, combine
 
     # roofline of the dominant kernel (the gate_up expert kernel, stage 3)
     I2 = 2 * cfg.I

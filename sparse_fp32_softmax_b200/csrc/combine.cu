@@ -36,6 +36,8 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(
     const uint16_t* __restrict__ x, const uint16_t* __restrict__ shared_gate,
     const uint16_t* __restrict__ residual, uint16_t* __restrict__ out, float* __restrict__ out_f32) {
     __shared__ float red[kCombineThreads / 32];
+    pdl_wait();
+    pdl_launch_dependents();
     const int S = k + has_shared;
     for (int t = blockIdx.x; t < T; t += gridDim.x) {
         float gate = 1.0f;
@@ -94,19 +96,17 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(
 
 cudaError_t launch_combine(const void* slots, int slots_bf16, int T, int D, int k, int has_shared,
                            const uint16_t* x, const uint16_t* shared_gate,
-                           const uint16_t* residual, uint16_t* out, float* out_f32,
+                           const uint16_t* residual, uint16_t* out, float* out_f32, bool pdl,
                            cudaStream_t s) {
     if (T <= 0) return cudaSuccess;
-    int blocks = T < 148 * 16 ? T : 148 * 16;
+    const int blocks = T < 148 * 16 ? T : 148 * 16;
     if (slots_bf16)
-        combine_kernel<uint16_t><<<blocks, kCombineThreads, 0, s>>>(
-            static_cast<const uint16_t*>(slots), T, D, k, has_shared, x, shared_gate, residual, out,
-            out_f32);
-    else
-        combine_kernel<float><<<blocks, kCombineThreads, 0, s>>>(
-            static_cast<const float*>(slots), T, D, k, has_shared, x, shared_gate, residual, out,
-            out_f32);
-    return cudaGetLastError();
+        return launch_kernel(combine_kernel<uint16_t>, dim3(blocks), dim3(kCombineThreads), 0, s, pdl,
+                             static_cast<const uint16_t*>(slots), T, D, k, has_shared, x, shared_gate,
+                             residual, out, out_f32);
+    return launch_kernel(combine_kernel<float>, dim3(blocks), dim3(kCombineThreads), 0, s, pdl,
+                         static_cast<const float*>(slots), T, D, k, has_shared, x, shared_gate,
+                         residual, out, out_f32);
 }
 
 }  // namespace moe

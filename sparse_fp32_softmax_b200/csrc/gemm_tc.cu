@@ -163,9 +163,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     float* ep_wt_all = reinterpret_cast<float*>(ep_dest_all + 4 * BN);  // [4][BN]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int total = tc_total_items<MODE>(a);
-    if ((int)blockIdx.x >= total) return;  // whole CTA, before any barrier or TMEM use
 
+    // prologue: independent of earlier kernels, overlaps them under launch chaining
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(full + s, 1);
@@ -183,6 +182,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         tma_prefetch_desc(m);
     }
     if (warp == 1) tmem_alloc(tmem_slot, Tr::TMEM);
+    pdl_wait();
+    pdl_launch_dependents();
+    const int total = tc_total_items<MODE>(a);
     if (MODE != kModeRouter) {
         const int* prefix = (MODE == kModeGateUp) ? a.tables.gu_items : a.tables.dn_items;
         load_tables(tabs, prefix, a.tables.seg_count, a.tables.seg_start, a.nseg);
@@ -192,49 +194,74 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
-    if (warp == 0) {
-        // ------------------------------------------------------------ TMA producer
-        if (lane == 0) {
-            int it = 0;
-            bool ok = true;
-            int last_round[kStages];
+    if ((int)blockIdx.x >= total) {
+        // no work for this CTA: nothing was issued; fall through to the TMEM release
+    } else if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer warp
+        // Weight tiles are issued by lane 0.  Token tiles: in gather mode gate_up fetches its
+        // rows from x by row_token, lane i taking rows 4i..4i+3 of the tile (rows past the
+        // segment repeat its last row; their columns are never used); otherwise lane 0 loads
+        // a tile of the permuted rows.
+        int it = 0;
+        bool ok = true;
+        int last_round[kStages];
 #pragma unroll
-            for (int s = 0; s < kStages; ++s) last_round[s] = -1;
-            for (int item = blockIdx.x; item < total && ok; item += gridDim.x) {
-                const TileInfo ti = tc_decode_item<MODE>(a, tabs, item);
-                const CUtensorMap* mA = ti.shared ? &maps.A_shared : &maps.A;
-                const CUtensorMap* mB = &maps.B[ti.bi];
-                const uint32_t bytes = NA * kATileBytes + (16u << ti.bi) * kTcK * 2;
-                for (int kb = 0; kb < ti.nk; ++kb, ++it) {
-                    const int s = it % kStages;
-                    const int round = it / kStages;
-                    if (!mbar_wait(empty + s, (round & 1) ^ 1, a.err, kErrWaitProducer)) {
-                        ok = false;
-                        break;
-                    }
-                    uint8_t* st = smem + s * SB;
+        for (int s = 0; s < kStages; ++s) last_round[s] = -1;
+        for (int item = blockIdx.x; item < total && ok; item += gridDim.x) {
+            const TileInfo ti = tc_decode_item<MODE>(a, tabs, item);
+            const CUtensorMap* mA = ti.shared ? &maps.A_shared : &maps.A;
+            const CUtensorMap* mB = &maps.B[ti.bi];
+            const int brows = 16 << ti.bi;
+            const uint32_t bytes = NA * kATileBytes + (uint32_t)brows * kTcK * 2;
+            const bool gather = MODE == kModeGateUp && a.gather;
+            int g0 = 0, g1 = 0, g2 = 0, g3 = 0;
+            if (gather) {
+                const int base = ti.b_row + 4 * lane;
+                const int last = ti.b_row + ti.n_valid - 1;
+                g0 = __ldg(a.row_token + min(base + 0, last));
+                g1 = __ldg(a.row_token + min(base + 1, last));
+                g2 = __ldg(a.row_token + min(base + 2, last));
+                g3 = __ldg(a.row_token + min(base + 3, last));
+            }
+            for (int kb = 0; kb < ti.nk; ++kb, ++it) {
+                const int s = it % kStages;
+                const int round = it / kStages;
+                const bool got = mbar_wait(empty + s, (round & 1) ^ 1, a.err, kErrWaitProducer);
+                if (!__all_sync(0xffffffffu, got)) {
+                    ok = false;
+                    break;
+                }
+                uint8_t* st = smem + s * SB;
+                if (lane == 0) {
                     mbar_arrive_expect_tx(full + s, bytes);
                     tma_load(st, mA, full + s, kb * kTcK, ti.a_row0);
                     if (NA == 2) tma_load(st + kATileBytes, mA, full + s, kb * kTcK, ti.a_row1);
-                    tma_load(st + NA * kATileBytes, mB, full + s, kb * kTcK, ti.b_row);
-#pragma unroll
-                    for (int q = 0; q < kStages; ++q)
-                        if (q == s) last_round[q] = round;
+                    if (!gather) tma_load(st + NA * kATileBytes, mB, full + s, kb * kTcK, ti.b_row);
                 }
-            }
-            // wait until the MMA issuer has released every stage, then until every issued
-            // load has landed, so no copy is in flight when the CTA exits
-            if (ok) {
-                for (int i = 0; i < kStages; ++i, ++it) {
-                    const int s = it % kStages;
-                    const int round = it / kStages;
-                    if (!mbar_wait(empty + s, (round & 1) ^ 1, a.err, kErrWaitTail)) break;
+                if (gather) {
+                    __syncwarp();  // expect_tx is posted before any gather can complete
+                    if (4 * lane < brows)
+                        tma_gather4(st + NA * kATileBytes + lane * 4 * kTcK * 2, mB, full + s,
+                                    kb * kTcK, g0, g1, g2, g3);
                 }
-            }
 #pragma unroll
-            for (int s = 0; s < kStages; ++s)
-                if (last_round[s] >= 0) mbar_wait(full + s, last_round[s] & 1, a.err, kErrWaitTail);
+                for (int q = 0; q < kStages; ++q)
+                    if (q == s) last_round[q] = round;
+            }
         }
+        // wait until the MMA issuer has released every stage, then until every issued
+        // load has landed, so no copy is in flight when the CTA exits
+        if (ok) {
+            for (int i = 0; i < kStages; ++i, ++it) {
+                const int s = it % kStages;
+                const int round = it / kStages;
+                const bool got = mbar_wait(empty + s, (round & 1) ^ 1, a.err, kErrWaitTail);
+                if (!__all_sync(0xffffffffu, got)) break;
+            }
+        }
+#pragma unroll
+        for (int s = 0; s < kStages; ++s)
+            if (last_round[s] >= 0) mbar_wait(full + s, last_round[s] & 1, a.err, kErrWaitTail);
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
@@ -354,26 +381,28 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 }
 
 template <int MODE>
-static cudaError_t launch_tc(const TcMaps& maps, const TcArgs& a, int grid, cudaStream_t s) {
+static cudaError_t launch_tc(const TcMaps& maps, const TcArgs& a, int grid, bool pdl, cudaStream_t s) {
     constexpr int smem = tc_smem_bytes<MODE>();
     cudaError_t err = ensure_smem_attr((const void*)tc_gemm_kernel<MODE>, smem, 1 + MODE);
     if (err != cudaSuccess) return err;
     if (grid < 1) grid = 1;
-    tc_gemm_kernel<MODE><<<grid, kTcThreads, smem, s>>>(maps, a);
-    return cudaGetLastError();
+    return launch_kernel(tc_gemm_kernel<MODE>, dim3(grid), dim3(kTcThreads), smem, s, pdl, maps, a);
 }
 
-cudaError_t launch_tc_router(const TcMaps& maps, const TcArgs& a, int num_sms, cudaStream_t s) {
+cudaError_t launch_tc_router(const TcMaps& maps, const TcArgs& a, int num_sms, bool pdl,
+                             cudaStream_t s) {
     const int items = ((a.T + kRtBN - 1) / kRtBN) * ((a.E + kTcM - 1) / kTcM);
-    return launch_tc<kModeRouter>(maps, a, items < num_sms ? items : num_sms, s);
+    return launch_tc<kModeRouter>(maps, a, items < num_sms ? items : num_sms, pdl, s);
 }
 
-cudaError_t launch_tc_gate_up(const TcMaps& maps, const TcArgs& a, int num_sms, cudaStream_t s) {
-    return launch_tc<kModeGateUp>(maps, a, num_sms, s);
+cudaError_t launch_tc_gate_up(const TcMaps& maps, const TcArgs& a, int num_sms, bool pdl,
+                              cudaStream_t s) {
+    return launch_tc<kModeGateUp>(maps, a, num_sms, pdl, s);
 }
 
-cudaError_t launch_tc_down(const TcMaps& maps, const TcArgs& a, int num_sms, cudaStream_t s) {
-    return launch_tc<kModeDown>(maps, a, num_sms, s);
+cudaError_t launch_tc_down(const TcMaps& maps, const TcArgs& a, int num_sms, bool pdl,
+                           cudaStream_t s) {
+    return launch_tc<kModeDown>(maps, a, num_sms, pdl, s);
 }
 
 }  // namespace moe

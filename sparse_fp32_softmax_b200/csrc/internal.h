@@ -26,6 +26,10 @@ constexpr int kGuBN = 128;      // token columns per gate_up tile (two accumulat
 constexpr int kDnBN = 256;      // token columns per down tile
 constexpr int kRtBN = 128;      // token columns per router-logit tile
 constexpr int kStages = 4;      // shared-memory pipeline depth
+// Largest T for which gate_up gathers token rows from x instead of reading a permuted copy:
+// a tile then has at most this many rows, i.e. at most 8 four-row gathers per stage (the
+// TMA engine's cost per operation makes gathering larger tiles slower than copying).
+constexpr int kGatherMaxT = 32;
 
 // Largest supported expert count (and segments: experts + one shared expert).
 constexpr int kMaxE = 512;
@@ -67,6 +71,21 @@ struct PermuteArgs {
     int* err;
 };
 
+// Routing of T <= kFusedRouteMaxT tokens in one kernel: blocks split the experts' logits,
+// the last block to finish selects every token and performs the permutation.
+constexpr int kFusedRouteMaxT = 32;
+struct RouteArgs {
+    const uint16_t* x;        // [T, D]
+    const uint16_t* W_r;      // [E, D]
+    const float* bias;        // [E] or null
+    int T, D, E, k, norm;
+    float* logits_out;        // [T, E] (the caller's or workspace scratch)
+    int32_t* topk_idx;        // [T, k]
+    float* topk_w;            // [T, k]
+    int* ticket;              // zero before the launch
+    PermuteArgs perm;         // topk_idx / topk_w above are its inputs
+};
+
 struct StreamArgs {
     const uint16_t* x;        // [T, D]
     const uint16_t* W_gu;     // [E, 2I, D]
@@ -97,6 +116,10 @@ struct alignas(64) TcMaps {
 struct TcArgs {
     int D, I, I_s, E, nseg;
     SegTables tables;
+    // gate_up token rows: gather = 1 -> gathered from x by row_token (map B = x with a
+    // one-row box, four rows per TMA operation); gather = 0 -> tiles of the permuted copy
+    const int32_t* row_token;
+    int gather;
     // gate_up epilogue
     uint16_t* h;              // [rows, ld_h] bf16 SwiGLU output
     int ld_h;
@@ -116,22 +139,28 @@ struct TcArgs {
 cudaError_t ensure_smem_attr(const void* kernel, int bytes, int slot);
 
 // ---------------------------------------------------------------- launchers (return the
-// launch error, cudaSuccess when all kernels were enqueued)
+// launch error, cudaSuccess when all kernels were enqueued).  pdl: launch the first kernel
+// as a programmatic dependent of the previous kernel on the stream (set for every launch
+// after the first of an API call; later kernels of one launcher always chain).
 cudaError_t launch_router_small(const uint16_t* x, const uint16_t* W_r, const float* bias, int T,
-                                int D, int E, float* logits, cudaStream_t s);
+                                int D, int E, float* logits, bool pdl, cudaStream_t s);
 cudaError_t launch_select(const float* logits, int T, int E, int k, int norm, int32_t* idx,
-                          float* w, cudaStream_t s);
-cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t s);
+                          float* w, bool pdl, cudaStream_t s);
+cudaError_t launch_permute(const PermuteArgs& a, bool pdl, cudaStream_t s);
+cudaError_t launch_route_fused(const RouteArgs& a, bool pdl, cudaStream_t s);
 cudaError_t launch_gather_rows(const uint16_t* x, const int32_t* row_token, int rows, int D,
-                               uint16_t* x_perm, cudaStream_t s);
-cudaError_t launch_stream_gate_up(const StreamArgs& a, int max_rows, cudaStream_t s);
-cudaError_t launch_stream_down(const StreamArgs& a, int max_rows, cudaStream_t s);
-cudaError_t launch_tc_router(const TcMaps& maps, const TcArgs& a, int num_sms, cudaStream_t s);
-cudaError_t launch_tc_gate_up(const TcMaps& maps, const TcArgs& a, int num_sms, cudaStream_t s);
-cudaError_t launch_tc_down(const TcMaps& maps, const TcArgs& a, int num_sms, cudaStream_t s);
+                               uint16_t* x_perm, bool pdl, cudaStream_t s);
+cudaError_t launch_stream_gate_up(const StreamArgs& a, int max_rows, bool pdl, cudaStream_t s);
+cudaError_t launch_stream_down(const StreamArgs& a, int max_rows, bool pdl, cudaStream_t s);
+cudaError_t launch_tc_router(const TcMaps& maps, const TcArgs& a, int num_sms, bool pdl,
+                             cudaStream_t s);
+cudaError_t launch_tc_gate_up(const TcMaps& maps, const TcArgs& a, int num_sms, bool pdl,
+                              cudaStream_t s);
+cudaError_t launch_tc_down(const TcMaps& maps, const TcArgs& a, int num_sms, bool pdl,
+                           cudaStream_t s);
 cudaError_t launch_combine(const void* slots, int slots_bf16, int T, int D, int k, int has_shared,
                            const uint16_t* x, const uint16_t* shared_gate,
-                           const uint16_t* residual, uint16_t* out, float* out_f32,
+                           const uint16_t* residual, uint16_t* out, float* out_f32, bool pdl,
                            cudaStream_t s);
 
 }  // namespace moe

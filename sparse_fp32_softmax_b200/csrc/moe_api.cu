@@ -15,11 +15,11 @@ namespace moe {
 
 cudaError_t ensure_smem_attr(const void* kernel, int bytes, int slot) {
     static std::mutex mu;
-    static unsigned char done[64][8] = {};
+    static unsigned char done[64][16] = {};
     int dev = 0;
     cudaError_t err = cudaGetDevice(&dev);
     if (err != cudaSuccess) return err;
-    if (dev < 0 || dev >= 64 || slot < 0 || slot >= 8) return cudaErrorInvalidValue;
+    if (dev < 0 || dev >= 64 || slot < 0 || slot >= 16) return cudaErrorInvalidValue;
     std::lock_guard<std::mutex> lock(mu);
     if (done[dev][slot]) return cudaSuccess;
     err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
@@ -74,7 +74,7 @@ Plan make_plan(const moe_dims& d, const moe_opts* o) {
     p.row_weight = take((size_t)p.R * 4);
     p.row_dest = take((size_t)p.R * 4);
     p.slot_row = take((size_t)p.T * p.k * 4);
-    p.x_perm = take((size_t)p.R * p.D * 2);
+    p.x_perm = take(p.T > kGatherMaxT ? (size_t)p.R * p.D * 2 : 0);
     p.h = take((size_t)p.R * p.ld_h * 2);
     p.slots = take((size_t)p.T * p.S * p.D * 4);
     p.total = off;
@@ -210,11 +210,13 @@ SegTables tables_of(const Plan& p, void* ws) {
 }
 
 // Router: logits (CUDA-core for small T, tcgen05 GEMM otherwise), then selection.
+// The router's first kernel is launched normally (it reads the caller's x); the selection
+// chains to it.
 moe_status run_route(const moe_bf16* x, const moe_bf16* W_r, const float* bias, const Plan& p,
                      int norm, float* logits, int32_t* idx, float* w, void* ws,
                      cudaStream_t s) {
     if (p.T <= kRouterSmallMaxT) {
-        MOE_CUDA(launch_router_small(x, W_r, bias, p.T, p.D, p.E, logits, s));
+        MOE_CUDA(launch_router_small(x, W_r, bias, p.T, p.D, p.E, logits, false, s));
     } else {
         TcMaps maps;
         if (!make_map(&maps.A, W_r, p.D, p.E, kTcM)) return MOE_ERR_CUDA;
@@ -227,9 +229,9 @@ moe_status run_route(const moe_bf16* x, const moe_bf16* W_r, const float* bias, 
         a.err = at<int>(ws, p.err);
         const int sms = num_sms_of_current_device();
         if (sms <= 0) return MOE_ERR_CUDA;
-        MOE_CUDA(launch_tc_router(maps, a, sms, s));
+        MOE_CUDA(launch_tc_router(maps, a, sms, false, s));
     }
-    MOE_CUDA(launch_select(logits, p.T, p.E, p.k, norm, idx, w, s));
+    MOE_CUDA(launch_select(logits, p.T, p.E, p.k, norm, idx, w, true, s));
     return MOE_OK;
 }
 
@@ -315,8 +317,8 @@ moe_status moe_permute(const int32_t* topk_idx, const float* topk_w, const moe_b
     // so mark every row as padding first
     MOE_CUDA(cudaMemsetAsync(row_token, 0xFF, (size_t)cap * sizeof(int32_t), s));
     if (a.row_weight) MOE_CUDA(cudaMemsetAsync(a.row_weight, 0, (size_t)cap * sizeof(float), s));
-    MOE_CUDA(launch_permute(a, s));
-    if (x_perm) MOE_CUDA(launch_gather_rows(x, row_token, cap, p.D, x_perm, s));
+    MOE_CUDA(launch_permute(a, false, s));
+    if (x_perm) MOE_CUDA(launch_gather_rows(x, row_token, cap, p.D, x_perm, true, s));
     return MOE_OK;
 }
 
@@ -354,24 +356,34 @@ moe_status moe_forward_ex(const moe_bf16* x, const moe_bf16* W_r, const moe_bf16
     float* out_f32 = opts ? opts->out_f32 : nullptr;
 
     // tensor maps of the grouped path are encoded before anything is enqueued
+    // gate_up token rows: for T <= kGatherMaxT gathered straight from x (one-row box,
+    // tile::gather4: no permuted copy); above, tiles of a permuted copy.  down reads h tiles.
+    const bool gather = p.T <= kGatherMaxT;
     TcMaps mGu, mDn;
     if (!streaming) {
-        uint16_t* x_perm = at<uint16_t>(ws, p.x_perm);
         uint16_t* h = at<uint16_t>(ws, p.h);
+        const bool gu_b_ok = gather ? make_map(&mGu.B[0], x, p.D, p.T, 1)
+                                    : make_b_maps(mGu.B, at<uint16_t>(ws, p.x_perm), p.D, p.R, kGuBN);
         if (!make_map(&mGu.A, W_gate_up, p.D, (uint64_t)p.E * 2 * p.I, kTcM) ||
             !make_map(&mGu.A_shared, sgu ? sgu : W_gate_up, p.D,
                       sgu ? 2 * (uint64_t)p.I_s : 2 * (uint64_t)p.I, kTcM) ||
-            !make_b_maps(mGu.B, x_perm, p.D, p.R, kGuBN) ||
+            !gu_b_ok ||
             !make_map(&mDn.A, W_down, p.I, (uint64_t)p.E * p.D, kTcM) ||
             !make_map(&mDn.A_shared, sdn ? sdn : W_down, sdn ? p.I_s : p.I, p.D, kTcM) ||
             !make_b_maps(mDn.B, h, p.ld_h, p.R, kDnBN))
             return MOE_ERR_CUDA;
+        if (gather)
+            for (int bi = 1; bi < kNumBBoxes; ++bi) mGu.B[bi] = mGu.B[0];
     }
 
-    MOE_CUDA(cudaMemsetAsync(err, 0, sizeof(int), s));
+    // the header of the workspace: [0] device error word, [1] routing ticket
+    MOE_CUDA(cudaMemsetAsync(err, 0, 2 * sizeof(int), s));
     if ((st = record(opts, 0, s)) != MOE_OK) return st;
-    if ((st = run_route(x, W_r, bias, p, dims->norm_topk_prob, logits, idx, w, ws, s)) != MOE_OK)
-        return st;
+    const bool fused_route = p.T <= kFusedRouteMaxT;
+    if (!fused_route) {
+        if ((st = run_route(x, W_r, bias, p, dims->norm_topk_prob, logits, idx, w, ws, s)) != MOE_OK)
+            return st;
+    }
     if ((st = record(opts, 1, s)) != MOE_OK) return st;
 
     PermuteArgs pa{};
@@ -392,9 +404,24 @@ moe_status moe_forward_ex(const moe_bf16* x, const moe_bf16* W_r, const moe_bf16
     pa.cap = p.R;
     pa.tables = tables_of(p, ws);
     pa.err = err;
-    MOE_CUDA(launch_permute(pa, s));
-    if (!streaming)
-        MOE_CUDA(launch_gather_rows(x, pa.row_token, p.R, p.D, at<uint16_t>(ws, p.x_perm), s));
+    // launch chaining between the forward's kernels (not across a stage-event record)
+    const bool chain = !(opts && opts->n_stage_events == 6);
+    if (fused_route) {
+        // one kernel: logits, softmax, top-k and (in its last block) the permutation
+        RouteArgs ra{};
+        ra.x = x; ra.W_r = W_r; ra.bias = bias;
+        ra.T = p.T; ra.D = p.D; ra.E = p.E; ra.k = p.k; ra.norm = dims->norm_topk_prob;
+        ra.logits_out = logits;
+        ra.topk_idx = idx;
+        ra.topk_w = w;
+        ra.ticket = err + 1;
+        ra.perm = pa;
+        MOE_CUDA(launch_route_fused(ra, false, s));
+    } else {
+        MOE_CUDA(launch_permute(pa, chain, s));
+    }
+    if (!streaming && !gather)
+        MOE_CUDA(launch_gather_rows(x, pa.row_token, p.R, p.D, at<uint16_t>(ws, p.x_perm), true, s));
     if ((st = record(opts, 2, s)) != MOE_OK) return st;
 
     if (streaming) {
@@ -409,28 +436,30 @@ moe_status moe_forward_ex(const moe_bf16* x, const moe_bf16* W_r, const moe_bf16
         sa.ld_h = p.ld_h;
         sa.slots = at<float>(ws, p.slots);
         sa.err = err;
-        MOE_CUDA(launch_stream_gate_up(sa, p.T, s));
+        MOE_CUDA(launch_stream_gate_up(sa, p.T, chain, s));
         if ((st = record(opts, 3, s)) != MOE_OK) return st;
-        MOE_CUDA(launch_stream_down(sa, p.T, s));
+        MOE_CUDA(launch_stream_down(sa, p.T, chain, s));
         if ((st = record(opts, 4, s)) != MOE_OK) return st;
         MOE_CUDA(launch_combine(sa.slots, 0, p.T, p.D, p.k, p.has_shared, x, sg, residual, out,
-                                out_f32, s));
+                                out_f32, chain, s));
     } else {
         TcArgs ta{};
         ta.D = p.D; ta.I = p.I; ta.I_s = p.I_s; ta.E = p.E; ta.nseg = p.nseg; ta.T = p.T;
         ta.tables = pa.tables;
+        ta.row_token = pa.row_token;
+        ta.gather = gather ? 1 : 0;
         ta.h = at<uint16_t>(ws, p.h);
         ta.ld_h = p.ld_h;
         ta.row_weight = pa.row_weight;
         ta.row_dest = pa.row_dest;
         ta.slots = at<float>(ws, p.slots);
         ta.err = err;
-        MOE_CUDA(launch_tc_gate_up(mGu, ta, sms, s));
+        MOE_CUDA(launch_tc_gate_up(mGu, ta, sms, chain, s));
         if ((st = record(opts, 3, s)) != MOE_OK) return st;
-        MOE_CUDA(launch_tc_down(mDn, ta, sms, s));
+        MOE_CUDA(launch_tc_down(mDn, ta, sms, chain, s));
         if ((st = record(opts, 4, s)) != MOE_OK) return st;
         MOE_CUDA(launch_combine(ta.slots, 0, p.T, p.D, p.k, p.has_shared, x, sg, residual, out,
-                                out_f32, s));
+                                out_f32, chain, s));
     }
     return record(opts, 5, s);
 }

@@ -1,0 +1,212 @@
+// permute_block.cuh -- block-level pieces of the expert counting sort (see permute.cu):
+// block scan, offsets and work tables, stable per-warp ranking and scattering, and the
+// whole permutation by one block.  Included by the translation units that use them.
+#pragma once
+
+#include "common.cuh"
+
+namespace moe {
+
+// Block-wide exclusive scan of one int per thread (blockDim.x <= 1024, multiple of 32).
+// Returns the exclusive prefix; *total receives the sum.  Contains __syncthreads.
+static __device__ int block_exclusive_scan(int v, int* total) {
+    __shared__ int warp_sums[32];
+    __shared__ int s_total;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int nwarps = blockDim.x >> 5;
+    int inc = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += y;
+    }
+    if (lane == 31) warp_sums[warp] = inc;
+    __syncthreads();
+    if (warp == 0) {
+        int w = lane < nwarps ? warp_sums[lane] : 0;
+        int winc = w;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, winc, o);
+            if (lane >= o) winc += y;
+        }
+        if (lane < nwarps) warp_sums[lane] = winc - w;  // exclusive warp offsets
+        if (lane == 31) s_total = winc;                 // grand total
+    }
+    __syncthreads();
+    const int res = warp_sums[warp] + inc - v;
+    const int tot = s_total;
+    __syncthreads();
+    if (total) *total = tot;
+    return res;
+}
+
+// From per-expert totals s_cnt[0..E) (block-visible shared memory): write counts, the
+// tile-padded offsets (also into s_off[0..E]), the segment tables and the work-item prefix
+// sums of the expert kernels.  Whole block (1024 threads, E < 1024).
+static __device__ void finish_offsets(const PermuteArgs& a, const int* s_cnt, int* s_off) {
+    const int E = a.E;
+    const int nseg = E + (a.has_shared ? 1 : 0);
+    int total = 0;
+    const int e = threadIdx.x;
+    const int padded = (e < E) ? (s_cnt[e] + a.tile_m - 1) / a.tile_m * a.tile_m : 0;
+    const int off = block_exclusive_scan(padded, &total);
+    if (e < E) {
+        a.counts[e] = s_cnt[e];
+        a.offsets[e] = off;
+        s_off[e] = off;
+        if (a.tables.seg_count) {
+            a.tables.seg_count[e] = s_cnt[e];
+            a.tables.seg_start[e] = off;
+        }
+    }
+    if (threadIdx.x == 0) {
+        a.offsets[E] = total;
+        s_off[E] = total;
+        if (a.has_shared && a.tables.seg_count) {
+            a.tables.seg_count[E] = a.T;
+            a.tables.seg_start[E] = total;
+        }
+    }
+    if (a.tables.gu_items) {
+        const int s = threadIdx.x;
+        int gi = 0, di = 0, gt = 0, dt = 0;
+        if (s < nseg) {
+            const int c = (s == E) ? a.T : s_cnt[s];
+            const int Iseg = (s == E) ? a.I_s : a.I;
+            if (c > 0) {
+                gi = (c + kGuBN - 1) / kGuBN * (Iseg / kTcM);
+                di = (c + kDnBN - 1) / kDnBN * (a.D / kTcM);
+                gt = Iseg / 8;      // streaming gate_up: one warp per 8 features
+                dt = a.D / 16;      // streaming down: one warp per 16 output rows
+            }
+        }
+        int tot;
+        const int pgi = block_exclusive_scan(gi, &tot);
+        if (s < nseg) a.tables.gu_items[s] = pgi;
+        if (s == 0) a.tables.gu_items[nseg] = tot;
+        const int pdi = block_exclusive_scan(di, &tot);
+        if (s < nseg) a.tables.dn_items[s] = pdi;
+        if (s == 0) a.tables.dn_items[nseg] = tot;
+        const int pgt = block_exclusive_scan(gt, &tot);
+        if (s < nseg) a.tables.gu_tasks[s] = pgt;
+        if (s == 0) a.tables.gu_tasks[nseg] = tot;
+        const int pdt = block_exclusive_scan(dt, &tot);
+        if (s < nseg) a.tables.dn_tasks[s] = pdt;
+        if (s == 0) a.tables.dn_tasks[nseg] = tot;
+    }
+    __syncthreads();
+}
+
+// Warp w of a block of W warps owns assignments [a0 + w*L, a0 + w*L + L), L = 4096 / W,
+// in rounds of 32 in increasing order.  Counting pass: wb[w*E + e] += assignments of e in
+// the warp's slice.
+static __device__ void count_warp_slices(const PermuteArgs& a, long a0, int* wb) {
+    const int E = a.E;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int slice = kPermChunk / (blockDim.x >> 5);
+    const long n = (long)a.T * a.k;
+    const long w0 = a0 + (long)warp * slice;
+    const uint32_t lt_mask = (1u << lane) - 1u;
+#pragma unroll 1
+    for (int r = 0; r < slice / 32; ++r) {
+        const long as = w0 + r * 32 + lane;
+        int e = (as < n) ? __ldcg(a.topk_idx + as) : -1;
+        if (as < n && (e >= E || e < 0)) {
+            set_error(a.err, kErrBadIndex);
+            e = -1;
+        }
+        const uint32_t m = __match_any_sync(0xffffffffu, e);
+        if (e >= 0 && (m & lt_mask) == 0) wb[warp * E + e] += __popc(m);
+    }
+}
+
+// Scatter pass: wb[w*E + e] holds the first row warp w may give to expert e; each
+// assignment takes the next row of its expert (stable: lanes in order, rounds in order).
+static __device__ void scatter_warp_slices(const PermuteArgs& a, long a0, int* wb) {
+    const int E = a.E;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int slice = kPermChunk / (blockDim.x >> 5);
+    const long n = (long)a.T * a.k;
+    const long w0 = a0 + (long)warp * slice;
+    const uint32_t lt_mask = (1u << lane) - 1u;
+#pragma unroll 1
+    for (int r = 0; r < slice / 32; ++r) {
+        const long as = w0 + r * 32 + lane;
+        int e = (as < n) ? __ldcg(a.topk_idx + as) : -1;
+        if (e >= E || e < 0) e = -1;
+        const uint32_t m = __match_any_sync(0xffffffffu, e);
+        int base = 0;
+        if (e >= 0) base = wb[warp * E + e];
+        __syncwarp();
+        if (e >= 0 && (m & lt_mask) == 0) wb[warp * E + e] = base + __popc(m);
+        __syncwarp();
+        if (e >= 0) {
+            const int row = base + __popc(m & lt_mask);
+            const int t = (int)(as / a.k), j = (int)(as % a.k);
+            a.slot_row[as] = row;
+            if (row < a.cap) {
+                a.row_token[row] = t;
+                if (a.row_weight) a.row_weight[row] = a.topk_w ? __ldcg(a.topk_w + as) : 1.0f;
+                if (a.row_dest) a.row_dest[row] = t * a.slots_per_token + j;
+            }
+        }
+    }
+}
+
+// Rows of the shared expert (segment E: all tokens in order after the routed rows) and
+// padding rows of each expert segment (tile_m > 1), spread over blocks b0 of nb.
+static __device__ void write_fixed_rows(const PermuteArgs& a, int rows0, const int* offsets,
+                                 const int* counts, int b0, int nb) {
+    if (a.has_shared) {
+        for (int t = b0 * blockDim.x + threadIdx.x; t < a.T; t += nb * blockDim.x) {
+            const int row = rows0 + t;
+            if (row < a.cap) {
+                a.row_token[row] = t;
+                if (a.row_weight) a.row_weight[row] = 1.0f;
+                if (a.row_dest) a.row_dest[row] = t * a.slots_per_token + a.k;
+            }
+        }
+    }
+    if (a.tile_m > 1) {
+        for (int e = b0; e < a.E; e += nb) {
+            const int r0 = offsets[e] + counts[e], r1 = offsets[e + 1];
+            for (int row = r0 + threadIdx.x; row < r1 && row < a.cap; row += blockDim.x) {
+                a.row_token[row] = -1;
+                if (a.row_weight) a.row_weight[row] = 0.0f;
+                if (a.row_dest) a.row_dest[row] = -1;
+            }
+        }
+    }
+}
+
+// ------------------------------------------------------------------ single-block path
+
+// The whole permutation by one block of 1024 threads (T*k <= 4096).  wb: [32][E] ints of
+// shared memory.  Also called by the fused routing kernel's last block.
+static __device__ void permute_one_block(const PermuteArgs& a, int* wb) {
+    __shared__ int s_cnt[kMaxSegments];
+    __shared__ int s_off[kMaxSegments + 1];
+    const int E = a.E;
+    for (int q = threadIdx.x; q < 32 * E; q += blockDim.x) wb[q] = 0;
+    __syncthreads();
+    count_warp_slices(a, 0, wb);
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {   // per-warp exclusive prefix
+        int run = 0;
+        for (int w = 0; w < 32; ++w) {
+            const int v = wb[w * E + e];
+            wb[w * E + e] = run;
+            run += v;
+        }
+        s_cnt[e] = run;
+    }
+    __syncthreads();
+    finish_offsets(a, s_cnt, s_off);
+    for (int q = threadIdx.x; q < 32 * E; q += blockDim.x) wb[q] += s_off[q % E];
+    __syncthreads();
+    scatter_warp_slices(a, 0, wb);
+    write_fixed_rows(a, s_off[E], s_off, s_cnt, 0, 1);
+}
+
+}  // namespace moe

@@ -1,0 +1,90 @@
+// route_fused.cu -- routing of small batches (T <= 32) in a single launch.
+//
+// "27. Mixture of experts" (inference.shantanugoel.com): section "The router" (logits,
+// FP32 softmax over all experts, top-k with ties to the lower index, renormalisation) and
+// section "Dispatch" (stable grouping of the assignments by expert).  At decode sizes each
+// of these steps is a few microseconds of work, so launching them separately costs more
+// than running them; this kernel does all of them.
+#include "permute_block.cuh"
+#include "select.cuh"
+
+namespace moe {
+
+// ------------------------------------------------------------------ fused small-T routing
+//
+// Blocks split the experts: block b computes the FP32 logits of its experts for every token
+// (T <= 32), one warp per (expert, token) pair, with the same exact-product FP32
+// accumulation as the small-T router.  Logits go to global memory; each block then takes an
+// atomic ticket after a fence, and the block that draws the last ticket sees every block's
+// logits: it selects all tokens (one warp per token) and performs the whole permutation.
+// One launch replaces the router, the selection and the permutation kernels.
+template <int VPL>
+__global__ void __launch_bounds__(1024) route_fused_kernel(RouteArgs a) {
+    extern __shared__ int route_smem[];
+    int* wb = route_smem;                                               // [32][E] (last block)
+    float* lg = reinterpret_cast<float*>(route_smem + 32 * a.E);        // [T][E] (last block)
+    __shared__ int s_ticket;
+    pdl_wait();
+    pdl_launch_dependents();
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int E = a.E, D = a.D, T = a.T;
+    const int per_block = (E + gridDim.x - 1) / gridDim.x;
+    const int e0 = blockIdx.x * per_block;
+    const int e1 = min(E, e0 + per_block);
+    const int npairs = max(0, e1 - e0) * T;
+    for (int q = warp; q < npairs; q += 32) {
+        const int e = e0 + q / T, t = q % T;
+        const uint16_t* wr = a.W_r + (size_t)e * D;
+        const uint16_t* xr = a.x + (size_t)t * D;
+        float acc = 0.f;
+#pragma unroll 8
+        for (int c = lane * 8; c < D; c += 256) {
+            const uint4 wv = ld_v4(wr + c);
+            const uint4 v = ld_v4(xr + c);
+            acc = fmaf(bf16_lo(wv.x), bf16_lo(v.x), acc);
+            acc = fmaf(bf16_hi(wv.x), bf16_hi(v.x), acc);
+            acc = fmaf(bf16_lo(wv.y), bf16_lo(v.y), acc);
+            acc = fmaf(bf16_hi(wv.y), bf16_hi(v.y), acc);
+            acc = fmaf(bf16_lo(wv.z), bf16_lo(v.z), acc);
+            acc = fmaf(bf16_hi(wv.z), bf16_hi(v.z), acc);
+            acc = fmaf(bf16_lo(wv.w), bf16_lo(v.w), acc);
+            acc = fmaf(bf16_hi(wv.w), bf16_hi(v.w), acc);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        if (lane == 0) {
+            float l = acc;
+            if (a.bias) l = l + a.bias[e];
+            a.logits_out[(size_t)t * E + e] = l;
+        }
+    }
+    // publish this block's logits; the last block routes and permutes everything
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) s_ticket = atomicAdd(a.ticket, 1);
+    __syncthreads();
+    if (s_ticket != (int)gridDim.x - 1) return;
+    __threadfence();
+    for (int i = threadIdx.x; i < T * E; i += blockDim.x) lg[i] = __ldcg(a.logits_out + i);
+    __syncthreads();
+    for (int t = warp; t < T; t += 32)
+        select_token<VPL>(lg + t * E, E, a.k, a.norm, a.topk_idx + (size_t)t * a.k,
+                          a.topk_w + (size_t)t * a.k);
+    __syncthreads();
+    permute_one_block(a.perm, wb);
+}
+
+cudaError_t launch_route_fused(const RouteArgs& a, bool pdl, cudaStream_t s) {
+    if (a.T > kFusedRouteMaxT) return cudaErrorInvalidValue;
+    const int smem = (32 + a.T) * a.E * 4;
+    void (*k_)(RouteArgs) = a.E <= 32 ? route_fused_kernel<1> : a.E <= 64 ? route_fused_kernel<2>
+                          : a.E <= 128 ? route_fused_kernel<4> : a.E <= 256 ? route_fused_kernel<8>
+                          : route_fused_kernel<16>;
+    const int slot = a.E <= 32 ? 0 : a.E <= 64 ? 1 : a.E <= 128 ? 2 : a.E <= 256 ? 3 : 4;
+    cudaError_t err = ensure_smem_attr((const void*)k_, (32 + kFusedRouteMaxT) * kMaxE * 4, 8 + slot);
+    if (err != cudaSuccess) return err;
+    const int blocks = a.E < 148 ? a.E : 148;
+    return launch_kernel(k_, dim3(blocks), dim3(1024), smem, s, pdl, a);
+}
+
+}  // namespace moe

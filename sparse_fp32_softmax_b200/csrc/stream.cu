@@ -28,6 +28,8 @@ constexpr int kStreamThreads = 128;
 
 template <int NB>
 __global__ void __launch_bounds__(kStreamThreads) stream_gate_up_kernel(StreamArgs a) {
+    pdl_wait();
+    pdl_launch_dependents();
     const int lane = threadIdx.x & 31;
     const int g = lane >> 2, q = lane & 3;
     const int nseg = a.nseg;
@@ -87,6 +89,8 @@ __global__ void __launch_bounds__(kStreamThreads) stream_gate_up_kernel(StreamAr
 
 template <int NB>
 __global__ void __launch_bounds__(kStreamThreads) stream_down_kernel(StreamArgs a) {
+    pdl_wait();
+    pdl_launch_dependents();
     const int lane = threadIdx.x & 31;
     const int g = lane >> 2, q = lane & 3;
     const int nseg = a.nseg;
@@ -160,25 +164,19 @@ static int stream_blocks(int max_tasks) {
     return blocks;
 }
 
-cudaError_t launch_stream_gate_up(const StreamArgs& a, int max_rows, cudaStream_t s) {
+cudaError_t launch_stream_gate_up(const StreamArgs& a, int max_rows, bool pdl, cudaStream_t s) {
     // upper bound of warp tasks: every segment touched
     const int max_tasks = a.E * (a.I / 8) + (a.S_gu ? a.I_s / 8 : 0);
     const int blocks = stream_blocks(max_tasks);
-    if (max_rows <= 16)
-        stream_gate_up_kernel<2><<<blocks, kStreamThreads, 0, s>>>(a);
-    else
-        stream_gate_up_kernel<4><<<blocks, kStreamThreads, 0, s>>>(a);
-    return cudaGetLastError();
+    return launch_kernel(max_rows <= 16 ? stream_gate_up_kernel<2> : stream_gate_up_kernel<4>,
+                         dim3(blocks), dim3(kStreamThreads), 0, s, pdl, a);
 }
 
-cudaError_t launch_stream_down(const StreamArgs& a, int max_rows, cudaStream_t s) {
+cudaError_t launch_stream_down(const StreamArgs& a, int max_rows, bool pdl, cudaStream_t s) {
     const int max_tasks = (a.E + (a.S_dn ? 1 : 0)) * (a.D / 16);
     const int blocks = stream_blocks(max_tasks);
-    if (max_rows <= 16)
-        stream_down_kernel<2><<<blocks, kStreamThreads, 0, s>>>(a);
-    else
-        stream_down_kernel<4><<<blocks, kStreamThreads, 0, s>>>(a);
-    return cudaGetLastError();
+    return launch_kernel(max_rows <= 16 ? stream_down_kernel<2> : stream_down_kernel<4>,
+                         dim3(blocks), dim3(kStreamThreads), 0, s, pdl, a);
 }
 
 }  // namespace moe
