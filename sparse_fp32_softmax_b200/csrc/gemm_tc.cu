@@ -22,9 +22,10 @@
 //   warp 1      allocates TMEM, and one thread issues tcgen05.mma (M=128, N=tile width,
 //               K=16 x 4 per stage) with FP32 accumulation in TMEM; tcgen05.commit frees a
 //               stage when its MMAs are done and publishes an accumulator when a tile is;
-//   warps 2..5  epilogue: tcgen05.ld 32 columns at a time from the lane quarter the warp may
-//               access, apply the epilogue, store; accumulators are double-buffered so the
-//               next tile's MMAs overlap this epilogue.
+//   warps 2..9  epilogue: two warps per TMEM lane quarter (a warp may only read the quarter
+//               warp % 4), taking alternate 32-column chunks of the tile: tcgen05.ld, apply
+//               the epilogue, store; accumulators are double-buffered so the next tile's
+//               MMAs overlap this epilogue.
 // All mbarrier waits are bounded (common.cuh); on expiry the kernel records the fact in the
 // device error word and winds down without leaving TMEM allocated.
 #include "common.cuh"
@@ -49,7 +50,8 @@ struct TcTraits<kModeRouter> {
 };
 
 constexpr int kATileBytes = kTcM * kTcK * 2;  // 16 KB
-constexpr int kTcThreads = 192;
+constexpr int kEpiWarps = 8;
+constexpr int kTcThreads = (2 + kEpiWarps) * 32;
 
 template <int MODE>
 constexpr int tc_stage_bytes() {
@@ -58,7 +60,7 @@ constexpr int tc_stage_bytes() {
 template <int MODE>
 constexpr int tc_smem_bytes() {
     return kStages * tc_stage_bytes<MODE>() + 1024 + 256 + (int)sizeof(SmemTables) +
-           (MODE == kModeDown ? 4 * 2 * 4 * kDnBN : 0);
+           (MODE == kModeDown ? kEpiWarps * 2 * 4 * kDnBN : 0);
 }
 
 struct TileInfo {
@@ -159,8 +161,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
     SmemTables* tabs = reinterpret_cast<SmemTables*>(smem + kStages * SB + 256);
     // down: per epilogue warp, the current tile's row destinations and weights
-    int* ep_dest_all = reinterpret_cast<int*>(tabs + 1);       // [4][BN]
-    float* ep_wt_all = reinterpret_cast<float*>(ep_dest_all + 4 * BN);  // [4][BN]
+    int* ep_dest_all = reinterpret_cast<int*>(tabs + 1);                       // [8][BN]
+    float* ep_wt_all = reinterpret_cast<float*>(ep_dest_all + kEpiWarps * BN);  // [8][BN]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -172,7 +174,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(tfull + b, 1);
-            mbar_init(tempty + b, 128);
+            mbar_init(tempty + b, kEpiWarps * 32);
         }
         mbar_init(drain, 1);
         mbar_fence_init();
@@ -309,8 +311,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             mbar_wait(drain, 0, a.err, kErrWaitMma);
         }
     } else {
-        // ------------------------------------------------------------ epilogue warps 2..5
+        // ------------------------------------------------------------ epilogue warps 2..9
         const int quarter = warp & 3;
+        const int ew = warp - 2;               // epilogue warp 0..7
+        const int half = ew >> 2;              // which alternate chunks this warp takes
         const int row = quarter * 32 + lane;  // TMEM lane = weight row within the tile
         int tc = 0;
         for (int item = blockIdx.x; item < total; item += gridDim.x, ++tc) {
@@ -322,8 +326,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             tc_fence_after();
             const uint32_t tb = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(b * ACC);
             const int nchunks = (ti.n_valid + 31) >> 5;
-            int* ep_dest = ep_dest_all + quarter * BN;
-            float* ep_wt = ep_wt_all + quarter * BN;
+            int* ep_dest = ep_dest_all + ew * BN;
+            float* ep_wt = ep_wt_all + ew * BN;
             if (MODE == kModeDown) {
                 // each epilogue warp keeps its own copy: no barrier across warps
                 __syncwarp();
@@ -333,7 +337,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 }
                 __syncwarp();
             }
-            for (int c = 0; c < nchunks; ++c) {
+            for (int c = half; c < nchunks; c += 2) {
                 float v[32];
                 tmem_ld32(tb + c * 32, v);
                 if (MODE == kModeGateUp) {

@@ -78,9 +78,10 @@ __global__ void __launch_bounds__(kPermThreads) perm_scatter_kernel(PermuteArgs 
     pdl_launch_dependents();
     const int E = a.E;
     if (blockIdx.x < a.nchunks) {
+        const WarpSlice ws = load_warp_slice(a, (long)blockIdx.x * kPermChunk);
         for (int q = threadIdx.x; q < 32 * E; q += blockDim.x) wb[q] = 0;
         __syncthreads();
-        count_warp_slices(a, (long)blockIdx.x * kPermChunk, wb);
+        count_warp_slices(a, ws, wb);
         __syncthreads();
         for (int e = threadIdx.x; e < E; e += blockDim.x) {
             int run = a.chunk_counts[(size_t)blockIdx.x * E + e];
@@ -91,7 +92,7 @@ __global__ void __launch_bounds__(kPermThreads) perm_scatter_kernel(PermuteArgs 
             }
         }
         __syncthreads();
-        scatter_warp_slices(a, (long)blockIdx.x * kPermChunk, wb);
+        scatter_warp_slices(a, ws, wb);
     }
     write_fixed_rows(a, __ldg(a.offsets + E), a.offsets, a.counts, blockIdx.x, gridDim.x);
 }

@@ -98,24 +98,49 @@ static __device__ void finish_offsets(const PermuteArgs& a, const int* s_cnt, in
     __syncthreads();
 }
 
-// Warp w of a block of W warps owns assignments [a0 + w*L, a0 + w*L + L), L = 4096 / W,
-// in rounds of 32 in increasing order.  Counting pass: wb[w*E + e] += assignments of e in
-// the warp's slice.
-static __device__ void count_warp_slices(const PermuteArgs& a, long a0, int* wb) {
-    const int E = a.E;
+// Warp w of a block of W warps owns assignments [a0 + w*L, a0 + w*L + L), L = 4096 / W
+// (at most 256 = 8 rounds of 32), in rounds of 32 in increasing order.  A lane's experts
+// (and weights) of all rounds are loaded once, up front, so the passes below cost one memory
+// round trip instead of one per round.
+constexpr int kMaxRounds = 8;
+struct WarpSlice {
+    int e[kMaxRounds];      // expert of the lane's assignment in each round (-1: none)
+    float w[kMaxRounds];    // its routing weight
+    int rounds;
+    long w0;                // first assignment of the warp's slice
+};
+
+static __device__ __forceinline__ WarpSlice load_warp_slice(const PermuteArgs& a, long a0) {
+    WarpSlice ws;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int slice = kPermChunk / (blockDim.x >> 5);
     const long n = (long)a.T * a.k;
-    const long w0 = a0 + (long)warp * slice;
-    const uint32_t lt_mask = (1u << lane) - 1u;
-#pragma unroll 1
-    for (int r = 0; r < slice / 32; ++r) {
-        const long as = w0 + r * 32 + lane;
-        int e = (as < n) ? __ldcg(a.topk_idx + as) : -1;
-        if (as < n && (e >= E || e < 0)) {
+    ws.rounds = slice / 32;
+    ws.w0 = a0 + (long)warp * slice;
+#pragma unroll
+    for (int r = 0; r < kMaxRounds; ++r) {
+        const long as = ws.w0 + r * 32 + lane;
+        const bool in = r < ws.rounds && as < n;
+        int e = in ? __ldcg(a.topk_idx + as) : -1;
+        ws.w[r] = (in && a.topk_w) ? __ldcg(a.topk_w + as) : 1.0f;
+        if (in && (e >= a.E || e < 0)) {
             set_error(a.err, kErrBadIndex);
             e = -1;
         }
+        ws.e[r] = e;
+    }
+    return ws;
+}
+
+// Counting pass: wb[w*E + e] += assignments of e in the warp's slice.
+static __device__ void count_warp_slices(const PermuteArgs& a, const WarpSlice& ws, int* wb) {
+    const int E = a.E;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const uint32_t lt_mask = (1u << lane) - 1u;
+#pragma unroll
+    for (int r = 0; r < kMaxRounds; ++r) {
+        if (r >= ws.rounds) break;
+        const int e = ws.e[r];
         const uint32_t m = __match_any_sync(0xffffffffu, e);
         if (e >= 0 && (m & lt_mask) == 0) wb[warp * E + e] += __popc(m);
     }
@@ -123,18 +148,15 @@ static __device__ void count_warp_slices(const PermuteArgs& a, long a0, int* wb)
 
 // Scatter pass: wb[w*E + e] holds the first row warp w may give to expert e; each
 // assignment takes the next row of its expert (stable: lanes in order, rounds in order).
-static __device__ void scatter_warp_slices(const PermuteArgs& a, long a0, int* wb) {
+static __device__ void scatter_warp_slices(const PermuteArgs& a, const WarpSlice& ws, int* wb) {
     const int E = a.E;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int slice = kPermChunk / (blockDim.x >> 5);
-    const long n = (long)a.T * a.k;
-    const long w0 = a0 + (long)warp * slice;
     const uint32_t lt_mask = (1u << lane) - 1u;
-#pragma unroll 1
-    for (int r = 0; r < slice / 32; ++r) {
-        const long as = w0 + r * 32 + lane;
-        int e = (as < n) ? __ldcg(a.topk_idx + as) : -1;
-        if (e >= E || e < 0) e = -1;
+#pragma unroll
+    for (int r = 0; r < kMaxRounds; ++r) {
+        if (r >= ws.rounds) break;
+        const int e = ws.e[r];
+        const long as = ws.w0 + r * 32 + lane;
         const uint32_t m = __match_any_sync(0xffffffffu, e);
         int base = 0;
         if (e >= 0) base = wb[warp * E + e];
@@ -147,7 +169,7 @@ static __device__ void scatter_warp_slices(const PermuteArgs& a, long a0, int* w
             a.slot_row[as] = row;
             if (row < a.cap) {
                 a.row_token[row] = t;
-                if (a.row_weight) a.row_weight[row] = a.topk_w ? __ldcg(a.topk_w + as) : 1.0f;
+                if (a.row_weight) a.row_weight[row] = ws.w[r];
                 if (a.row_dest) a.row_dest[row] = t * a.slots_per_token + j;
             }
         }
@@ -188,9 +210,10 @@ static __device__ void permute_one_block(const PermuteArgs& a, int* wb) {
     __shared__ int s_cnt[kMaxSegments];
     __shared__ int s_off[kMaxSegments + 1];
     const int E = a.E;
+    const WarpSlice ws = load_warp_slice(a, 0);
     for (int q = threadIdx.x; q < 32 * E; q += blockDim.x) wb[q] = 0;
     __syncthreads();
-    count_warp_slices(a, 0, wb);
+    count_warp_slices(a, ws, wb);
     __syncthreads();
     for (int e = threadIdx.x; e < E; e += blockDim.x) {   // per-warp exclusive prefix
         int run = 0;
@@ -205,7 +228,7 @@ static __device__ void permute_one_block(const PermuteArgs& a, int* wb) {
     finish_offsets(a, s_cnt, s_off);
     for (int q = threadIdx.x; q < 32 * E; q += blockDim.x) wb[q] += s_off[q % E];
     __syncthreads();
-    scatter_warp_slices(a, 0, wb);
+    scatter_warp_slices(a, ws, wb);
     write_fixed_rows(a, s_off[E], s_off, s_cnt, 0, 1);
 }
 
