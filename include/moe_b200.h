@@ -150,9 +150,9 @@ moe_status moe_forward_ex(const moe_bf16 *x, const moe_bf16 *W_r, const moe_bf16
  * its input and output buffers, runtimes that forbid allocation after start-up.  The pages
  * have no counterpart: this is a deployment variant of moe_forward, same arguments minus
  * the workspace, same results.
- * Scratch: a 32 MiB array in the library's own device memory (a file-scope device
+ * Scratch: a 64 MiB array in the library's own device memory (a file-scope device
  * variable), held by every GPU that loads this part of the library until the process
- * exits.  Calls whose moe_workspace_size(dims, NULL) exceeds 32 MiB return
+ * exits.  Calls whose moe_workspace_size(dims, NULL) exceeds 64 MiB return
  * MOE_ERR_WORKSPACE before enqueuing anything (the decode shapes fit: D=2048, E=128, k=8,
  * I=768 up to T=256).  Nothing is allocated or freed.
  * The first call on a device looks up the array's device address (once per device); make

@@ -234,7 +234,7 @@ def moe_forward_ex(x, W_r, W_gate_up, W_down, k, norm_topk_prob=True, out=None, 
 
 def moe_forward_noalloc(x, W_r, W_gate_up, W_down, k, norm_topk_prob=True, out=None, stream=None):
     """moe_forward without a workspace argument: for callers that cannot allocate device
-    memory, the library uses its own fixed 32 MiB device array (see the header)."""
+    memory, the library uses its own fixed 64 MiB device array (see the header)."""
     dims = _dims_of(x, W_r, W_gate_up, W_down, k, norm_topk_prob)
     if out is None:
         out = torch.empty_like(x)

@@ -64,10 +64,19 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(
         for (int d = threadIdx.x * 8; d < D; d += kCombineThreads * 8) {
             float acc[8], v[8];
             load8<SlotT>(base + d, acc);
-            for (int j = 1; j < k; ++j) {
-                load8<SlotT>(base + (size_t)j * D + d, v);
+            // slots j = 1..k-1 in groups of 8: all loads of a group are in flight together,
+            // the additions still run in slot order
+            for (int j0 = 1; j0 < k; j0 += 8) {
+                float g[8][8];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) acc[i] += v[i];
+                for (int q = 0; q < 8; ++q)
+                    if (j0 + q < k) load8<SlotT>(base + (size_t)(j0 + q) * D + d, g[q]);
+#pragma unroll
+                for (int q = 0; q < 8; ++q)
+                    if (j0 + q < k) {
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) acc[i] += g[q][i];
+                    }
             }
             if (has_shared) {
                 load8<SlotT>(base + (size_t)k * D + d, v);

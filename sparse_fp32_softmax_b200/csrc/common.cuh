@@ -150,6 +150,14 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* e
 
 // ------------------------------------------------------------------ TMA
 
+// Bring one tile of a 2-D tensor map into L2 (a hint: no completion, no shared memory).
+__device__ __forceinline__ void tma_prefetch_l2(const CUtensorMap* map, int x, int y) {
+    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(x), "r"(y)
+                 : "memory");
+}
+
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -303,13 +311,15 @@ struct SmemTables {
     int start[kMaxSegments];
 };
 
-// Cooperative copy by all threads of the block (caller synchronises afterwards).
+// Cooperative copy by all threads of the block (caller synchronises afterwards).  Loads go
+// through L2 only (ld.global.cg), so the copy may also run before a kernel's dependency wait
+// on tables that an earlier kernel of the chain finished writing.
 __device__ __forceinline__ void load_tables(SmemTables* st, const int* prefix, const int* count,
                                             const int* start, int nseg) {
-    for (int i = threadIdx.x; i <= nseg; i += blockDim.x) st->prefix[i] = __ldg(prefix + i);
+    for (int i = threadIdx.x; i <= nseg; i += blockDim.x) st->prefix[i] = __ldcg(prefix + i);
     for (int i = threadIdx.x; i < nseg; i += blockDim.x) {
-        st->count[i] = __ldg(count + i);
-        st->start[i] = __ldg(start + i);
+        st->count[i] = __ldcg(count + i);
+        st->start[i] = __ldcg(start + i);
     }
 }
 

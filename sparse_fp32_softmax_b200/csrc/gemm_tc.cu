@@ -14,7 +14,9 @@
 //   down:    one accumulator, down rows [d0, d0+128) against a tile of h rows; the epilogue
 //            scales by the routing weight and stores FP32 into the token's slot (a bf16 slot
 //            would add a third bf16 rounding on top of h and the output).
-//   router:  one accumulator, router rows [e0, e0+128) against a tile of x rows; FP32 out.
+//   router:  one accumulator, router rows [e0, e0+128) against a tile of x rows over one
+//            of ksplit slices of K; FP32 partial sums out (added in slice order, with the
+//            bias, by the selection), so that a handful of token tiles still fills the SMs.
 //
 // Per CTA (one per SM, persistent over a device-side item list):
 //   warp 0      TMA producer: 4-stage ring of {A tile(s) 128x64, B tile BNx64} bf16 tiles in
@@ -34,34 +36,27 @@ namespace moe {
 
 enum { kModeGateUp = 0, kModeDown = 1, kModeRouter = 2 };
 
-template <int MODE>
-struct TcTraits;
-template <>
-struct TcTraits<kModeGateUp> {
-    static constexpr int BN = kGuBN, NA = 2, ACC = 2 * kGuBN, TMEM = 512;
-};
-template <>
-struct TcTraits<kModeDown> {
-    static constexpr int BN = kDnBN, NA = 1, ACC = kDnBN, TMEM = 512;
-};
-template <>
-struct TcTraits<kModeRouter> {
-    static constexpr int BN = kRtBN, NA = 1, ACC = kRtBN, TMEM = 256;
+// One kernel configuration: mode, token columns per tile and pipeline depth.
+template <int MODE, int BN_, int STAGES_>
+struct TcCfg {
+    static constexpr int BN = BN_, STAGES = STAGES_;
+    static constexpr int NA = MODE == kModeGateUp ? 2 : 1;   // A tiles (accumulators) per stage
+    static constexpr int ACC = NA * BN;                       // TMEM columns per accumulator set
+    // two accumulator sets, rounded up to the power-of-two allocation unit (>= 32 columns)
+    static constexpr int TMEM = 2 * ACC <= 32 ? 32 : 2 * ACC <= 64 ? 64 : 2 * ACC <= 128 ? 128
+                              : 2 * ACC <= 256 ? 256 : 512;
+    static_assert(2 * ACC <= 512, "accumulators exceed TMEM");
+    static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "token tile");
+    static constexpr int SB = NA * (kTcM * kTcK * 2) + BN * kTcK * 2;  // bytes per stage
+    static constexpr int SMEM = STAGES * SB + 1024 + 256 + (int)sizeof(SmemTables) +
+                                (MODE == kModeDown ? 8 * 2 * 4 * BN : 0);
+    static_assert(2 * STAGES + 5 <= 31, "barriers exceed their 256-byte region");
+    static_assert(SMEM <= 232448, "shared memory per block");
 };
 
 constexpr int kATileBytes = kTcM * kTcK * 2;  // 16 KB
 constexpr int kEpiWarps = 8;
 constexpr int kTcThreads = (2 + kEpiWarps) * 32;
-
-template <int MODE>
-constexpr int tc_stage_bytes() {
-    return TcTraits<MODE>::NA * kATileBytes + TcTraits<MODE>::BN * kTcK * 2;
-}
-template <int MODE>
-constexpr int tc_smem_bytes() {
-    return kStages * tc_stage_bytes<MODE>() + 1024 + 256 + (int)sizeof(SmemTables) +
-           (MODE == kModeDown ? kEpiWarps * 2 * 4 * kDnBN : 0);
-}
 
 struct TileInfo {
     int bi;       // token-operand box: 16 << bi rows
@@ -71,15 +66,51 @@ struct TileInfo {
     int b_row;    // first B (token) row
     int n_valid;  // valid token columns, 1..BN
     int nk;       // K stages
+    int k0;       // first K stage of this unit
+    int split;    // K slice index (router slices, or a split tail item's slice)
+    int nsplit;   // > 1: tail item split over K, partial sums reduced by the last slice
+    int tail;     // index of a split item among the tail items
     int m0;       // first output feature of this tile within its segment
 };
 
-template <int MODE>
-__device__ __forceinline__ int tc_total_items(const TcArgs& a) {
-    constexpr int BN = TcTraits<MODE>::BN;
-    if (MODE == kModeRouter) return ((a.T + BN - 1) / BN) * ((a.E + kTcM - 1) / kTcM);
-    const int* prefix = (MODE == kModeGateUp) ? a.tables.gu_items : a.tables.dn_items;
-    return __ldg(prefix + a.nseg);
+// Work schedule of one launch (identical in every CTA): the first `full` items -- whole
+// waves of G = gridDim.x -- run one item per unit; when the remaining tail is at most half a
+// wave, each tail item is split along K into S slices so that no CTA ends a whole item
+// after the others.  The slices come last (at most one per CTA): their reduction then reads
+// L2 while the SM's TMA engine is idle -- mid-stream, those loads would queue behind the
+// weight traffic.  A slice writes FP32 partial accumulators; the last slice of an item to
+// finish (atomic ticket) adds them in slice order and runs the epilogue, so the sums do not
+// depend on timing.
+struct Sched {
+    int n;      // items
+    int full;   // items in whole waves
+    int S;      // slices per tail item (1: no split)
+    int units;  // work units
+};
+
+template <int MODE, int BN>
+__device__ __forceinline__ int tc_total_items(const TcArgs& a, const SmemTables* st) {
+    if (MODE == kModeRouter) return ((a.T + BN - 1) / BN) * ((a.E + kTcM - 1) / kTcM) * a.ksplit;
+    return st->prefix[a.nseg];
+}
+
+template <int MODE, int BN, bool SPLIT>
+__device__ __forceinline__ Sched tc_schedule(const TcArgs& a, const SmemTables* st) {
+    Sched sc;
+    const int G = gridDim.x;
+    sc.n = tc_total_items<MODE, BN>(a, st);
+    sc.full = sc.n / G * G;
+    sc.S = 1;
+    const int tail = sc.n - sc.full;
+    if (SPLIT && tail > 0 && 2 * tail <= G) {
+        const int kmin = MODE == kModeGateUp ? a.D : (a.I_s > 0 ? min(a.I, a.I_s) : a.I);
+        int S = min(G / tail, kMaxKSplit);
+        S = min(S, kmin / kTcK);
+        S = min(S, a.partial_slots / tail);
+        if (S >= 2) sc.S = S;
+    }
+    sc.units = sc.full + tail * sc.S;
+    return sc;
 }
 
 // Smallest token box (16 << bi rows, bi <= log2(BN/16)) that covers n valid rows.
@@ -90,19 +121,27 @@ __device__ __forceinline__ int box_index(int n) {
     return bi;
 }
 
-template <int MODE>
+template <int MODE, int BN>
 __device__ __forceinline__ TileInfo tc_decode_item(const TcArgs& a, const SmemTables* st, int item) {
-    constexpr int BN = TcTraits<MODE>::BN;
     TileInfo ti;
+    ti.k0 = 0;
+    ti.split = 0;
+    ti.nsplit = 1;
+    ti.tail = 0;
     if (MODE == kModeRouter) {
+        // consecutive items are the K splits of one tile
         const int mtc = (a.E + kTcM - 1) / kTcM;
+        ti.split = item % a.ksplit;
+        item /= a.ksplit;
         const int tt = item / mtc, mt = item % mtc;
         ti.shared = 0;
         ti.a_row0 = mt * kTcM;
         ti.a_row1 = 0;
         ti.b_row = tt * BN;
         ti.n_valid = min(BN, a.T - tt * BN);
-        ti.nk = a.D / kTcK;
+        const int nkt = a.D / kTcK;
+        ti.k0 = ti.split * nkt / a.ksplit;
+        ti.nk = (ti.split + 1) * nkt / a.ksplit - ti.k0;
         ti.m0 = mt * kTcM;
         ti.bi = box_index<BN>(ti.n_valid);
         return ti;
@@ -134,6 +173,21 @@ __device__ __forceinline__ TileInfo tc_decode_item(const TcArgs& a, const SmemTa
     return ti;
 }
 
+template <int MODE, int BN>
+__device__ __forceinline__ TileInfo tc_decode_unit(const TcArgs& a, const SmemTables* st,
+                                                   const Sched& sc, int u) {
+    if (sc.S == 1 || u < sc.full) return tc_decode_item<MODE, BN>(a, st, u);
+    const int tail = (u - sc.full) / sc.S, split = (u - sc.full) % sc.S;
+    TileInfo ti = tc_decode_item<MODE, BN>(a, st, sc.full + tail);
+    const int nkt = ti.nk;
+    ti.k0 = split * nkt / sc.S;
+    ti.nk = (split + 1) * nkt / sc.S - ti.k0;
+    ti.split = split;
+    ti.nsplit = sc.S;
+    ti.tail = tail;
+    return ti;
+}
+
 // Plain 2-D TMA load without an L2 hint.
 __device__ __forceinline__ void tma_load(void* dst, const CUtensorMap* map, uint64_t* bar, int x,
                                          int y) {
@@ -144,22 +198,23 @@ __device__ __forceinline__ void tma_load(void* dst, const CUtensorMap* map, uint
         : "memory");
 }
 
-template <int MODE>
+template <int MODE, int BN, int STAGES>
 __global__ void __launch_bounds__(kTcThreads, 1)
     tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
-    using Tr = TcTraits<MODE>;
-    constexpr int BN = Tr::BN, NA = Tr::NA, ACC = Tr::ACC;
-    constexpr int SB = tc_stage_bytes<MODE>();
+    using Tr = TcCfg<MODE, BN, STAGES>;
+    constexpr int NA = Tr::NA, ACC = Tr::ACC;
+    constexpr bool SPLIT = MODE != kModeRouter && BN <= kNarrowBN;
+    constexpr int SB = Tr::SB;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * SB);
-    uint64_t* empty = full + kStages;
-    uint64_t* tfull = empty + kStages;  // [2]
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * SB);
+    uint64_t* empty = full + STAGES;
+    uint64_t* tfull = empty + STAGES;  // [2]
     uint64_t* tempty = tfull + 2;       // [2]
     uint64_t* drain = tempty + 2;       // [1]
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
-    SmemTables* tabs = reinterpret_cast<SmemTables*>(smem + kStages * SB + 256);
+    SmemTables* tabs = reinterpret_cast<SmemTables*>(smem + STAGES * SB + 256);
     // down: per epilogue warp, the current tile's row destinations and weights
     int* ep_dest_all = reinterpret_cast<int*>(tabs + 1);                       // [8][BN]
     float* ep_wt_all = reinterpret_cast<float*>(ep_dest_all + kEpiWarps * BN);  // [8][BN]
@@ -168,7 +223,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
     // prologue: independent of earlier kernels, overlaps them under launch chaining
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < STAGES; ++s) {
             mbar_init(full + s, 1);
             mbar_init(empty + s, 1);
         }
@@ -184,17 +239,30 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         tma_prefetch_desc(m);
     }
     if (warp == 1) tmem_alloc(tmem_slot, Tr::TMEM);
+    if (MODE == kModeDown) {
+        // The work tables come from the permutation, two kernels back: it completed before
+        // the gate_up kernel (this kernel's predecessor) passed its own dependency wait,
+        // which precedes the moment this kernel can start.  So they are read (through L2)
+        // before this kernel's wait, and this CTA's first tile of weights -- which does not
+        // depend on gate_up -- is requested into L2 while gate_up finishes.
+        load_tables(tabs, a.tables.dn_items, a.tables.seg_count, a.tables.seg_start, a.nseg);
+        __syncthreads();
+        if (warp == 0 && lane == 0 && (int)blockIdx.x < tabs->prefix[a.nseg]) {
+            const TileInfo t0 = tc_decode_item<MODE, BN>(a, tabs, blockIdx.x);
+            const CUtensorMap* mA = t0.shared ? &maps.A_shared : &maps.A;
+            for (int kb = 0; kb < t0.nk; ++kb) tma_prefetch_l2(mA, kb * kTcK, t0.a_row0);
+        }
+    }
     pdl_wait();
     pdl_launch_dependents();
-    const int total = tc_total_items<MODE>(a);
-    if (MODE != kModeRouter) {
-        const int* prefix = (MODE == kModeGateUp) ? a.tables.gu_items : a.tables.dn_items;
-        load_tables(tabs, prefix, a.tables.seg_count, a.tables.seg_start, a.nseg);
-    }
+    if (MODE == kModeGateUp)
+        load_tables(tabs, a.tables.gu_items, a.tables.seg_count, a.tables.seg_start, a.nseg);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    const Sched sc = tc_schedule<MODE, BN, SPLIT>(a, tabs);
+    const int total = sc.units;
 
     if ((int)blockIdx.x >= total) {
         // no work for this CTA: nothing was issued; fall through to the TMEM release
@@ -206,28 +274,37 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         // a tile of the permuted rows.
         int it = 0;
         bool ok = true;
-        int last_round[kStages];
+        int last_round[STAGES];
 #pragma unroll
-        for (int s = 0; s < kStages; ++s) last_round[s] = -1;
+        for (int s = 0; s < STAGES; ++s) last_round[s] = -1;
+        const bool gather = MODE == kModeGateUp && a.gather;
+        // the next unit's gather rows are loaded while the current unit's stages are issued
+        auto gather_rows = [&](const TileInfo& t, int (&g)[4]) {
+            const int base = t.b_row + 4 * lane;
+            const int last = t.b_row + t.n_valid - 1;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) g[q] = __ldg(a.row_token + min(base + q, last));
+        };
+        TileInfo tn{};
+        int gn[4] = {0, 0, 0, 0};
+        if ((int)blockIdx.x < total) {
+            tn = tc_decode_unit<MODE, BN>(a, tabs, sc, blockIdx.x);
+            if (gather) gather_rows(tn, gn);
+        }
         for (int item = blockIdx.x; item < total && ok; item += gridDim.x) {
-            const TileInfo ti = tc_decode_item<MODE>(a, tabs, item);
+            const TileInfo ti = tn;
+            const int g0 = gn[0], g1 = gn[1], g2 = gn[2], g3 = gn[3];
+            if (item + (int)gridDim.x < total) {
+                tn = tc_decode_unit<MODE, BN>(a, tabs, sc, item + gridDim.x);
+                if (gather) gather_rows(tn, gn);
+            }
             const CUtensorMap* mA = ti.shared ? &maps.A_shared : &maps.A;
             const CUtensorMap* mB = &maps.B[ti.bi];
             const int brows = 16 << ti.bi;
             const uint32_t bytes = NA * kATileBytes + (uint32_t)brows * kTcK * 2;
-            const bool gather = MODE == kModeGateUp && a.gather;
-            int g0 = 0, g1 = 0, g2 = 0, g3 = 0;
-            if (gather) {
-                const int base = ti.b_row + 4 * lane;
-                const int last = ti.b_row + ti.n_valid - 1;
-                g0 = __ldg(a.row_token + min(base + 0, last));
-                g1 = __ldg(a.row_token + min(base + 1, last));
-                g2 = __ldg(a.row_token + min(base + 2, last));
-                g3 = __ldg(a.row_token + min(base + 3, last));
-            }
             for (int kb = 0; kb < ti.nk; ++kb, ++it) {
-                const int s = it % kStages;
-                const int round = it / kStages;
+                const int s = it % STAGES;
+                const int round = it / STAGES;
                 const bool got = mbar_wait(empty + s, (round & 1) ^ 1, a.err, kErrWaitProducer);
                 if (!__all_sync(0xffffffffu, got)) {
                     ok = false;
@@ -236,33 +313,34 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 uint8_t* st = smem + s * SB;
                 if (lane == 0) {
                     mbar_arrive_expect_tx(full + s, bytes);
-                    tma_load(st, mA, full + s, kb * kTcK, ti.a_row0);
-                    if (NA == 2) tma_load(st + kATileBytes, mA, full + s, kb * kTcK, ti.a_row1);
-                    if (!gather) tma_load(st + NA * kATileBytes, mB, full + s, kb * kTcK, ti.b_row);
+                    const int kx = (ti.k0 + kb) * kTcK;
+                    tma_load(st, mA, full + s, kx, ti.a_row0);
+                    if (NA == 2) tma_load(st + kATileBytes, mA, full + s, kx, ti.a_row1);
+                    if (!gather) tma_load(st + NA * kATileBytes, mB, full + s, kx, ti.b_row);
                 }
                 if (gather) {
                     __syncwarp();  // expect_tx is posted before any gather can complete
                     if (4 * lane < brows)
                         tma_gather4(st + NA * kATileBytes + lane * 4 * kTcK * 2, mB, full + s,
-                                    kb * kTcK, g0, g1, g2, g3);
+                                    (ti.k0 + kb) * kTcK, g0, g1, g2, g3);
                 }
 #pragma unroll
-                for (int q = 0; q < kStages; ++q)
+                for (int q = 0; q < STAGES; ++q)
                     if (q == s) last_round[q] = round;
             }
         }
         // wait until the MMA issuer has released every stage, then until every issued
         // load has landed, so no copy is in flight when the CTA exits
         if (ok) {
-            for (int i = 0; i < kStages; ++i, ++it) {
-                const int s = it % kStages;
-                const int round = it / kStages;
+            for (int i = 0; i < STAGES; ++i, ++it) {
+                const int s = it % STAGES;
+                const int round = it / STAGES;
                 const bool got = mbar_wait(empty + s, (round & 1) ^ 1, a.err, kErrWaitTail);
                 if (!__all_sync(0xffffffffu, got)) break;
             }
         }
 #pragma unroll
-        for (int s = 0; s < kStages; ++s)
+        for (int s = 0; s < STAGES; ++s)
             if (last_round[s] >= 0) mbar_wait(full + s, last_round[s] & 1, a.err, kErrWaitTail);
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
@@ -271,7 +349,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             int it = 0, tc = 0;
             bool ok = true;
             for (int item = blockIdx.x; item < total && ok; item += gridDim.x, ++tc) {
-                const TileInfo ti = tc_decode_item<MODE>(a, tabs, item);
+                const TileInfo ti = tc_decode_unit<MODE, BN>(a, tabs, sc, item);
                 const int b = tc & 1;
                 const int use = tc >> 1;
                 if (!mbar_wait(tempty + b, (use & 1) ^ 1, a.err, kErrWaitMma)) {
@@ -284,8 +362,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 const uint32_t idesc = idesc0 | ((uint32_t)(n >> 3) << 17);
                 const uint32_t d0 = tmem_base + (uint32_t)(b * ACC);
                 for (int kb = 0; kb < ti.nk; ++kb, ++it) {
-                    const int s = it % kStages;
-                    const int round = it / kStages;
+                    const int s = it % STAGES;
+                    const int round = it / STAGES;
                     if (!mbar_wait(full + s, round & 1, a.err, kErrWaitMma)) {
                         ok = false;
                         break;
@@ -316,9 +394,56 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const int ew = warp - 2;               // epilogue warp 0..7
         const int half = ew >> 2;              // which alternate chunks this warp takes
         const int row = quarter * 32 + lane;  // TMEM lane = weight row within the tile
+        int* ep_dest = ep_dest_all + ew * BN;
+        float* ep_wt = ep_wt_all + ew * BN;
+        // The epilogue of one 32-column chunk: v (and u, the up accumulator) hold row `row`.
+        auto finish_chunk = [&](const TileInfo& ti, int c, const float* v, const float* u) {
+            if (MODE == kModeGateUp) {
+                const int f = ti.m0 + row;
+                uint16_t* hp = a.h + (size_t)(ti.b_row + c * 32) * a.ld_h + f;
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                    if (c * 32 + j < ti.n_valid) hp[(size_t)j * a.ld_h] = to_bf16_bits(silu(v[j]) * u[j]);
+            } else if (MODE == kModeDown) {
+                const int d = ti.m0 + row;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const int col = c * 32 + j;
+                    if (col < ti.n_valid) a.slots[(size_t)ep_dest[col] * a.D + d] = ep_wt[col] * v[j];
+                }
+            } else {
+                const int e = ti.m0 + row;
+                if (e < a.E) {
+                    float* part = a.logits + (size_t)ti.split * a.T * a.E;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int t = ti.b_row + c * 32 + j;
+                        if (c * 32 + j < ti.n_valid) part[(size_t)t * a.E + e] = v[j];
+                    }
+                }
+            }
+        };
+        // The same for four columns 4g..4g+3 of chunk c (the split-tail reduction).
+        auto finish_quad = [&](const TileInfo& ti, int c, int g, const float4& v4, const float4& u4) {
+            const float v[4] = {v4.x, v4.y, v4.z, v4.w};
+            const float u[4] = {u4.x, u4.y, u4.z, u4.w};
+            const int col0 = c * 32 + 4 * g;
+            if (MODE == kModeGateUp) {
+                uint16_t* hp = a.h + (size_t)(ti.b_row + col0) * a.ld_h + ti.m0 + row;
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    if (col0 + j < ti.n_valid) hp[(size_t)j * a.ld_h] = to_bf16_bits(silu(v[j]) * u[j]);
+            } else if (MODE == kModeDown) {
+                const int d = ti.m0 + row;
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    if (col0 + j < ti.n_valid)
+                        a.slots[(size_t)ep_dest[col0 + j] * a.D + d] = ep_wt[col0 + j] * v[j];
+            }
+        };
         int tc = 0;
         for (int item = blockIdx.x; item < total; item += gridDim.x, ++tc) {
-            const TileInfo ti = tc_decode_item<MODE>(a, tabs, item);
+            const TileInfo ti = tc_decode_unit<MODE, BN>(a, tabs, sc, item);
             const int b = tc & 1;
             const int use = tc >> 1;
             const bool got = mbar_wait(tfull + b, use & 1, a.err, kErrWaitEpilogue);
@@ -326,8 +451,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             tc_fence_after();
             const uint32_t tb = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(b * ACC);
             const int nchunks = (ti.n_valid + 31) >> 5;
-            int* ep_dest = ep_dest_all + ew * BN;
-            float* ep_wt = ep_wt_all + ew * BN;
             if (MODE == kModeDown) {
                 // each epilogue warp keeps its own copy: no barrier across warps
                 __syncwarp();
@@ -337,40 +460,77 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 }
                 __syncwarp();
             }
-            for (int c = half; c < nchunks; c += 2) {
-                float v[32];
-                tmem_ld32(tb + c * 32, v);
-                if (MODE == kModeGateUp) {
+            if (SPLIT && ti.nsplit > 1) {
+                // 1. this slice's partial accumulators (rows x BN per accumulator, FP32)
+                float* ps = a.partial + (size_t)(ti.tail * ti.nsplit + ti.split) * (NA * kTcM * BN);
+                for (int c = half; c < nchunks; c += 2) {
+                    float v[32];
+                    tmem_ld32(tb + c * 32, v);
                     float u[32];
-                    tmem_ld32(tb + BN + c * 32, u);
+                    if (MODE == kModeGateUp) tmem_ld32(tb + BN + c * 32, u);
                     tmem_ld_wait();
-                    const int f = ti.m0 + row;
-                    uint16_t* hp = a.h + (size_t)(ti.b_row + c * 32) * a.ld_h + f;
+                    float4* d0 = reinterpret_cast<float4*>(ps + (size_t)row * BN + c * 32);
 #pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        if (c * 32 + j < ti.n_valid) hp[(size_t)j * a.ld_h] = to_bf16_bits(silu(v[j]) * u[j]);
-                } else if (MODE == kModeDown) {
-                    tmem_ld_wait();
-                    const int d = ti.m0 + row;
+                    for (int q = 0; q < 8; ++q)
+                        d0[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+                    if (MODE == kModeGateUp) {
+                        float4* d1 = reinterpret_cast<float4*>(ps + (size_t)(kTcM + row) * BN + c * 32);
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        const int col = c * 32 + j;
-                        if (col < ti.n_valid)
-                            a.slots[(size_t)ep_dest[col] * a.D + d] = ep_wt[col] * v[j];
-                    }
-                } else {
-                    tmem_ld_wait();
-                    const int e = ti.m0 + row;
-                    if (e < a.E) {
-                        const float be = a.bias ? __ldg(a.bias + e) : 0.0f;
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) {
-                            const int t = ti.b_row + c * 32 + j;
-                            if (c * 32 + j < ti.n_valid)
-                                a.logits[(size_t)t * a.E + e] = a.bias ? v[j] + be : v[j];
-                        }
+                        for (int q = 0; q < 8; ++q)
+                            d1[q] = make_float4(u[4 * q], u[4 * q + 1], u[4 * q + 2], u[4 * q + 3]);
                     }
                 }
+                tc_fence_before();
+                mbar_arrive(tempty + b);  // the accumulator is free for the next tile
+                // 2. publish; the warp that completes this (item, warp) portion reduces it
+                __threadfence();
+                __syncwarp();
+                int old = 0;
+                int* ticket = a.tickets + ti.tail * kEpiWarps + ew;
+                if (lane == 0) old = atomicAdd(ticket, 1);
+                old = __shfl_sync(0xffffffffu, old, 0);
+                if (old != ti.nsplit - 1) continue;
+                __threadfence();
+                if (lane == 0) *ticket = 0;  // ready for the next launch
+                const float* p0 = a.partial + (size_t)(ti.tail * ti.nsplit) * (NA * kTcM * BN);
+                for (int c = half; c < nchunks; c += 2) {
+                    // valid columns only, four at a time; the loads of all slices of a group
+                    // are in flight together and are added in slice order
+                    const int ng = (min(32, ti.n_valid - c * 32) + 3) >> 2;
+#pragma unroll
+                    for (int g = 0; g < 8; ++g) {
+                        if (g >= ng) break;
+                        float4 lv[kMaxKSplit], lu[kMaxKSplit] = {};
+#pragma unroll
+                        for (int sp = 0; sp < kMaxKSplit; ++sp) {
+                            if (sp < ti.nsplit) {
+                                const float* pp = p0 + (size_t)sp * (NA * kTcM * BN) + c * 32 + 4 * g;
+                                lv[sp] = __ldcg(reinterpret_cast<const float4*>(pp + (size_t)row * BN));
+                                if (MODE == kModeGateUp)
+                                    lu[sp] = __ldcg(reinterpret_cast<const float4*>(pp + (size_t)(kTcM + row) * BN));
+                            }
+                        }
+                        float4 sv = lv[0], su = lu[0];
+#pragma unroll
+                        for (int sp = 1; sp < kMaxKSplit; ++sp) {
+                            if (sp < ti.nsplit) {
+                                sv.x += lv[sp].x; sv.y += lv[sp].y; sv.z += lv[sp].z; sv.w += lv[sp].w;
+                                if (MODE == kModeGateUp) {
+                                    su.x += lu[sp].x; su.y += lu[sp].y; su.z += lu[sp].z; su.w += lu[sp].w;
+                                }
+                            }
+                        }
+                        finish_quad(ti, c, g, sv, su);
+                    }
+                }
+                continue;
+            }
+            for (int c = half; c < nchunks; c += 2) {
+                float v[32], u[32];
+                tmem_ld32(tb + c * 32, v);
+                if (MODE == kModeGateUp) tmem_ld32(tb + BN + c * 32, u);
+                tmem_ld_wait();
+                finish_chunk(ti, c, v, u);
             }
             tc_fence_before();
             mbar_arrive(tempty + b);
@@ -384,29 +544,33 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
 }
 
-template <int MODE>
-static cudaError_t launch_tc(const TcMaps& maps, const TcArgs& a, int grid, bool pdl, cudaStream_t s) {
-    constexpr int smem = tc_smem_bytes<MODE>();
-    cudaError_t err = ensure_smem_attr((const void*)tc_gemm_kernel<MODE>, smem, 1 + MODE);
+template <int MODE, int BN, int STAGES>
+static cudaError_t launch_tc(const TcMaps& maps, const TcArgs& a, int grid, int attr_slot, bool pdl,
+                             cudaStream_t s) {
+    constexpr int smem = TcCfg<MODE, BN, STAGES>::SMEM;
+    cudaError_t err = ensure_smem_attr((const void*)tc_gemm_kernel<MODE, BN, STAGES>, smem, attr_slot);
     if (err != cudaSuccess) return err;
     if (grid < 1) grid = 1;
-    return launch_kernel(tc_gemm_kernel<MODE>, dim3(grid), dim3(kTcThreads), smem, s, pdl, maps, a);
+    return launch_kernel(tc_gemm_kernel<MODE, BN, STAGES>, dim3(grid), dim3(kTcThreads), smem, s, pdl,
+                         maps, a);
 }
 
 cudaError_t launch_tc_router(const TcMaps& maps, const TcArgs& a, int num_sms, bool pdl,
                              cudaStream_t s) {
-    const int items = ((a.T + kRtBN - 1) / kRtBN) * ((a.E + kTcM - 1) / kTcM);
-    return launch_tc<kModeRouter>(maps, a, items < num_sms ? items : num_sms, pdl, s);
+    const int items = ((a.T + kRtBN - 1) / kRtBN) * ((a.E + kTcM - 1) / kTcM) * a.ksplit;
+    return launch_tc<kModeRouter, kRtBN, kStages>(maps, a, items < num_sms ? items : num_sms, 3, pdl, s);
 }
 
-cudaError_t launch_tc_gate_up(const TcMaps& maps, const TcArgs& a, int num_sms, bool pdl,
+cudaError_t launch_tc_gate_up(const TcMaps& maps, const TcArgs& a, int num_sms, bool narrow, bool pdl,
                               cudaStream_t s) {
-    return launch_tc<kModeGateUp>(maps, a, num_sms, pdl, s);
+    if (narrow) return launch_tc<kModeGateUp, kNarrowBN, kGuNarrowStages>(maps, a, num_sms, 4, pdl, s);
+    return launch_tc<kModeGateUp, kGuBN, kStages>(maps, a, num_sms, 1, pdl, s);
 }
 
-cudaError_t launch_tc_down(const TcMaps& maps, const TcArgs& a, int num_sms, bool pdl,
+cudaError_t launch_tc_down(const TcMaps& maps, const TcArgs& a, int num_sms, bool narrow, bool pdl,
                            cudaStream_t s) {
-    return launch_tc<kModeDown>(maps, a, num_sms, pdl, s);
+    if (narrow) return launch_tc<kModeDown, kNarrowBN, kDnNarrowStages>(maps, a, num_sms, 5, pdl, s);
+    return launch_tc<kModeDown, kDnBN, kStages>(maps, a, num_sms, 2, pdl, s);
 }
 
 }  // namespace moe

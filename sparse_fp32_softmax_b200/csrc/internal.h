@@ -25,11 +25,29 @@ constexpr int kTcK = 64;        // K elements per pipeline stage (one 128-byte s
 constexpr int kGuBN = 128;      // token columns per gate_up tile (two accumulators per tile)
 constexpr int kDnBN = 256;      // token columns per down tile
 constexpr int kRtBN = 128;      // token columns per router-logit tile
-constexpr int kStages = 4;      // shared-memory pipeline depth
-// Largest T for which gate_up gathers token rows from x instead of reading a permuted copy:
-// a tile then has at most this many rows, i.e. at most 8 four-row gathers per stage (the
-// TMA engine's cost per operation makes gathering larger tiles slower than copying).
+constexpr int kStages = 4;      // shared-memory pipeline depth of the wide tiles
+// Narrow tiles for small per-expert row counts (decode): the token box is at most 64 rows,
+// so a stage is mostly weight bytes and the freed shared memory buys a deeper pipeline --
+// more weight bytes in flight per SM, which is what a weight-streaming GEMM is bound by.
+constexpr int kNarrowBN = 64;
+constexpr int kGuNarrowStages = 5;   // 5 x (2 x 16 KB + 8 KB)
+constexpr int kDnNarrowStages = 8;   // 8 x (16 KB + 8 KB)
+// The forward takes the narrow tiles when the mean rows per expert, T*k/E, is at most this.
+constexpr int kNarrowMaxMeanRows = 32;
+// Largest T for which gate_up gathers its token rows straight from x (tile::gather4, four
+// rows per TMA operation) instead of reading a permuted copy: a tile then has at most 32
+// rows, 8 gathers per stage.  Above, the TMA engine's cost per gather operation makes the
+// expert GEMM slower by more than a separate copy costs (measured on B200).
 constexpr int kGatherMaxT = 32;
+// Split tail items of the narrow-tile GEMMs: at most this many K slices per item, and
+// partial-sum slots for one wave (a tail is split only when it is at most half a wave, so
+// the tickets of at most kSplitSlots / 2 items x 8 epilogue warps are in use).
+constexpr int kMaxKSplit = 8;
+constexpr int kSplitSlots = 148;
+constexpr int kSplitTickets = 1024;
+__host__ __device__ inline bool use_narrow_tiles(long long T, int k, int E) {
+    return T * k <= (long long)kNarrowMaxMeanRows * E;
+}
 
 // Largest supported expert count (and segments: experts + one shared expert).
 constexpr int kMaxE = 512;
@@ -68,6 +86,7 @@ struct PermuteArgs {
     int32_t* slot_row;        // [T * k]
     int cap;                  // rows available in row_* arrays
     SegTables tables;         // may be all-null (moe_permute alone)
+    int gu_bn, dn_bn;         // token columns per gate_up / down tile (work-item tables)
     int* err;
 };
 
@@ -84,7 +103,25 @@ struct RouteArgs {
     float* topk_w;            // [T, k]
     int* ticket;              // zero before the launch
     PermuteArgs perm;         // topk_idx / topk_w above are its inputs
+    // selection from router partial sums (select_permute_kernel): logits = sum over the
+    // nsplit partials [nsplit, T, E] in split order, then + bias
+    const float* part;
+    int nsplit;
 };
+
+// The router GEMM splits K so that small token counts still spread over the SMs; its
+// partial sums are added in split order by the selection.  The split depends only on the
+// shapes (not on the device), so results do not depend on the GPU the call runs on.
+constexpr int kRouterMaxSplit = 16;
+constexpr int kSplitTargetCtas = 148;
+inline int router_splits(int T, int E, int D, int bn) {
+    const long long items = (long long)((T + bn - 1) / bn) * ((E + 127) / 128);
+    long long s = kSplitTargetCtas / (items > 0 ? items : 1);
+    const int nk = D / 64;
+    if (s > kRouterMaxSplit) s = kRouterMaxSplit;
+    if (s > nk) s = nk;
+    return s < 1 ? 1 : (int)s;
+}
 
 struct StreamArgs {
     const uint16_t* x;        // [T, D]
@@ -127,9 +164,15 @@ struct TcArgs {
     const float* row_weight;
     const int32_t* row_dest;
     float* slots;             // [T * S, D] FP32
-    // dense (router) epilogue
-    float* logits;            // [T, E]
-    const float* bias;        // [E] or null
+    // split tail items (narrow tiles): FP32 partial accumulators, one slot of
+    // NA x 128 x BN floats per slice (partial_slots slots), and one zeroed ticket per
+    // (tail item, epilogue warp)
+    float* partial;
+    int* tickets;
+    int partial_slots;
+    // dense (router) epilogue: partial sums over split s of K go to logits + s*T*E
+    float* logits;            // [ksplit, T, E] FP32
+    int ksplit;
     int T;
     int* err;
 };
@@ -142,21 +185,23 @@ cudaError_t ensure_smem_attr(const void* kernel, int bytes, int slot);
 // launch error, cudaSuccess when all kernels were enqueued).  pdl: launch the first kernel
 // as a programmatic dependent of the previous kernel on the stream (set for every launch
 // after the first of an API call; later kernels of one launcher always chain).
-cudaError_t launch_router_small(const uint16_t* x, const uint16_t* W_r, const float* bias, int T,
+cudaError_t launch_router_small(const uint16_t* x, const uint16_t* W_r, int T,
                                 int D, int E, float* logits, bool pdl, cudaStream_t s);
-cudaError_t launch_select(const float* logits, int T, int E, int k, int norm, int32_t* idx,
-                          float* w, bool pdl, cudaStream_t s);
+cudaError_t launch_select(const float* part, int nsplit, const float* bias, int T, int E, int k,
+                          int norm, int32_t* idx, float* w, float* logits_out, bool pdl,
+                          cudaStream_t s);
 cudaError_t launch_permute(const PermuteArgs& a, bool pdl, cudaStream_t s);
 cudaError_t launch_route_fused(const RouteArgs& a, bool pdl, cudaStream_t s);
+cudaError_t launch_select_permute(const RouteArgs& a, bool pdl, cudaStream_t s);
 cudaError_t launch_gather_rows(const uint16_t* x, const int32_t* row_token, int rows, int D,
                                uint16_t* x_perm, bool pdl, cudaStream_t s);
 cudaError_t launch_stream_gate_up(const StreamArgs& a, int max_rows, bool pdl, cudaStream_t s);
 cudaError_t launch_stream_down(const StreamArgs& a, int max_rows, bool pdl, cudaStream_t s);
 cudaError_t launch_tc_router(const TcMaps& maps, const TcArgs& a, int num_sms, bool pdl,
                              cudaStream_t s);
-cudaError_t launch_tc_gate_up(const TcMaps& maps, const TcArgs& a, int num_sms, bool pdl,
+cudaError_t launch_tc_gate_up(const TcMaps& maps, const TcArgs& a, int num_sms, bool narrow, bool pdl,
                               cudaStream_t s);
-cudaError_t launch_tc_down(const TcMaps& maps, const TcArgs& a, int num_sms, bool pdl,
+cudaError_t launch_tc_down(const TcMaps& maps, const TcArgs& a, int num_sms, bool narrow, bool pdl,
                            cudaStream_t s);
 cudaError_t launch_combine(const void* slots, int slots_bf16, int T, int D, int k, int has_shared,
                            const uint16_t* x, const uint16_t* shared_gate,

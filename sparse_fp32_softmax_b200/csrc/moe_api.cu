@@ -15,11 +15,11 @@ namespace moe {
 
 cudaError_t ensure_smem_attr(const void* kernel, int bytes, int slot) {
     static std::mutex mu;
-    static unsigned char done[64][16] = {};
+    static unsigned char done[64][32] = {};
     int dev = 0;
     cudaError_t err = cudaGetDevice(&dev);
     if (err != cudaSuccess) return err;
-    if (dev < 0 || dev >= 64 || slot < 0 || slot >= 16) return cudaErrorInvalidValue;
+    if (dev < 0 || dev >= 64 || slot < 0 || slot >= 32) return cudaErrorInvalidValue;
     std::lock_guard<std::mutex> lock(mu);
     if (done[dev][slot]) return cudaSuccess;
     err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
@@ -40,8 +40,8 @@ bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 
 // Byte offsets of every workspace region.
 struct Plan {
-    int T, D, E, k, I, I_s, has_shared, S, R, ld_h, nchunks, nseg;
-    size_t err, logits, idx, w, counts, offsets, chunk, seg_count, seg_start, gu_items, dn_items,
+    int T, D, E, k, I, I_s, has_shared, S, R, ld_h, nchunks, nseg, rsplit;
+    size_t err, tickets, partial, logits, idx, w, counts, offsets, chunk, seg_count, seg_start, gu_items, dn_items,
         gu_tasks, dn_tasks, row_token, row_weight, row_dest, slot_row, x_perm, h, slots, total;
 };
 
@@ -55,10 +55,14 @@ Plan make_plan(const moe_dims& d, const moe_opts* o) {
     p.ld_h = p.I > p.I_s ? p.I : p.I_s;
     p.nchunks = (int)(((long)p.T * p.k + kPermChunk - 1) / kPermChunk);
     p.nseg = p.E + p.has_shared;
+    p.rsplit = p.T <= kRouterSmallMaxT ? 1 : router_splits(p.T, p.E, p.D, kRtBN);
     size_t off = 0;
     auto take = [&](size_t bytes) { size_t at = off; off += align_up(bytes); return at; };
-    p.err = take(kAlign);
-    p.logits = take((size_t)p.T * p.E * 4);
+    p.err = take(kAlign);                              // [0] error word, [1] routing ticket
+    p.tickets = take((size_t)kSplitTickets * 4);       // split-tail tickets (follow err)
+    p.partial = take(use_narrow_tiles(p.T, p.k, p.E)   // split-tail partial accumulators
+                         ? (size_t)kSplitSlots * 2 * kTcM * kNarrowBN * 4 : 0);
+    p.logits = take((size_t)p.rsplit * p.T * p.E * 4);   // router partial sums (or logits)
     p.idx = take((size_t)p.T * p.k * 4);
     p.w = take((size_t)p.T * p.k * 4);
     p.counts = take((size_t)(p.E + 1) * 4);
@@ -74,7 +78,7 @@ Plan make_plan(const moe_dims& d, const moe_opts* o) {
     p.row_weight = take((size_t)p.R * 4);
     p.row_dest = take((size_t)p.R * 4);
     p.slot_row = take((size_t)p.T * p.k * 4);
-    p.x_perm = take(p.T > kGatherMaxT ? (size_t)p.R * p.D * 2 : 0);
+    p.x_perm = take(p.T <= kGatherMaxT ? 0 : (size_t)p.R * p.D * 2);
     p.h = take((size_t)p.R * p.ld_h * 2);
     p.slots = take((size_t)p.T * p.S * p.D * 4);
     p.total = off;
@@ -209,29 +213,27 @@ SegTables tables_of(const Plan& p, void* ws) {
     return t;
 }
 
-// Router: logits (CUDA-core for small T, tcgen05 GEMM otherwise), then selection.
-// The router's first kernel is launched normally (it reads the caller's x); the selection
-// chains to it.
-moe_status run_route(const moe_bf16* x, const moe_bf16* W_r, const float* bias, const Plan& p,
-                     int norm, float* logits, int32_t* idx, float* w, void* ws,
-                     cudaStream_t s) {
+// Router logits without the bias, as p.rsplit partial sums [rsplit, T, E] at part: CUDA-core
+// kernel for small T (one partial), tcgen05 GEMM with K split in rsplit slices otherwise.
+// Launched without chaining: it reads the caller's x.
+moe_status run_logits(const moe_bf16* x, const moe_bf16* W_r, const Plan& p, float* part, void* ws,
+                      cudaStream_t s) {
     if (p.T <= kRouterSmallMaxT) {
-        MOE_CUDA(launch_router_small(x, W_r, bias, p.T, p.D, p.E, logits, false, s));
-    } else {
-        TcMaps maps;
-        if (!make_map(&maps.A, W_r, p.D, p.E, kTcM)) return MOE_ERR_CUDA;
-        maps.A_shared = maps.A;
-        if (!make_b_maps(maps.B, x, p.D, p.T, kRtBN)) return MOE_ERR_CUDA;
-        TcArgs a{};
-        a.D = p.D; a.E = p.E; a.T = p.T; a.I = p.I; a.nseg = 1;
-        a.logits = logits;
-        a.bias = bias;
-        a.err = at<int>(ws, p.err);
-        const int sms = num_sms_of_current_device();
-        if (sms <= 0) return MOE_ERR_CUDA;
-        MOE_CUDA(launch_tc_router(maps, a, sms, false, s));
+        MOE_CUDA(launch_router_small(x, W_r, p.T, p.D, p.E, part, false, s));
+        return MOE_OK;
     }
-    MOE_CUDA(launch_select(logits, p.T, p.E, p.k, norm, idx, w, true, s));
+    TcMaps maps;
+    if (!make_map(&maps.A, W_r, p.D, p.E, kTcM)) return MOE_ERR_CUDA;
+    maps.A_shared = maps.A;
+    if (!make_b_maps(maps.B, x, p.D, p.T, kRtBN)) return MOE_ERR_CUDA;
+    TcArgs a{};
+    a.D = p.D; a.E = p.E; a.T = p.T; a.I = p.I; a.nseg = 1;
+    a.logits = part;
+    a.ksplit = p.rsplit;
+    a.err = at<int>(ws, p.err);
+    const int sms = num_sms_of_current_device();
+    if (sms <= 0) return MOE_ERR_CUDA;
+    MOE_CUDA(launch_tc_router(maps, a, sms, false, s));
     return MOE_OK;
 }
 
@@ -270,8 +272,12 @@ moe_status moe_route(const moe_bf16* x, const moe_bf16* W_r, const float* bias,
     if (ws_bytes < p.total) return MOE_ERR_WORKSPACE;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     MOE_CUDA(cudaMemsetAsync(at<int>(ws, p.err), 0, sizeof(int), s));
-    float* lg = logits ? logits : at<float>(ws, p.logits);
-    return run_route(x, W_r, bias, p, dims->norm_topk_prob, lg, topk_idx, topk_w, ws, s);
+    float* part = at<float>(ws, p.logits);
+    moe_status st2 = run_logits(x, W_r, p, part, ws, s);
+    if (st2 != MOE_OK) return st2;
+    MOE_CUDA(launch_select(part, p.rsplit, bias, p.T, p.E, p.k, dims->norm_topk_prob, topk_idx,
+                           topk_w, logits, true, s));
+    return MOE_OK;
 }
 
 moe_status moe_permute(const int32_t* topk_idx, const float* topk_w, const moe_bf16* x,
@@ -312,6 +318,8 @@ moe_status moe_permute(const int32_t* topk_idx, const float* topk_w, const moe_b
     a.slot_row = slot_row;
     a.cap = cap;
     a.tables = SegTables{nullptr, nullptr, nullptr, nullptr, nullptr, nullptr};
+    a.gu_bn = kGuBN;
+    a.dn_bn = kDnBN;
     a.err = at<int>(ws, p.err);
     // padding rows are only written per expert segment; rows past offsets[E] stay as given,
     // so mark every row as padding first
@@ -345,7 +353,8 @@ moe_status moe_forward_ex(const moe_bf16* x, const moe_bf16* W_r, const moe_bf16
     if (sms <= 0) return MOE_ERR_CUDA;
 
     int* err = at<int>(ws, p.err);
-    float* logits = (opts && opts->logits_out) ? opts->logits_out : at<float>(ws, p.logits);
+    float* logits_user = opts ? opts->logits_out : nullptr;
+    float* logits = logits_user ? logits_user : at<float>(ws, p.logits);
     int32_t* idx = (opts && opts->topk_idx_out) ? opts->topk_idx_out : at<int32_t>(ws, p.idx);
     float* w = (opts && opts->topk_w_out) ? opts->topk_w_out : at<float>(ws, p.w);
     const float* bias = opts ? opts->router_bias : nullptr;
@@ -356,33 +365,43 @@ moe_status moe_forward_ex(const moe_bf16* x, const moe_bf16* W_r, const moe_bf16
     float* out_f32 = opts ? opts->out_f32 : nullptr;
 
     // tensor maps of the grouped path are encoded before anything is enqueued
-    // gate_up token rows: for T <= kGatherMaxT gathered straight from x (one-row box,
-    // tile::gather4: no permuted copy); above, tiles of a permuted copy.  down reads h tiles.
+    // narrow tiles (deeper pipelines) when experts average few rows; a segment with more
+    // rows than a tile is simply split into several token tiles.  gate_up token rows: for
+    // T <= kGatherMaxT gathered from x (one-row box, tile::gather4), else a permuted copy.
+    const bool narrow = use_narrow_tiles(p.T, p.k, p.E);
     const bool gather = p.T <= kGatherMaxT;
+    const int gu_bn = narrow ? kNarrowBN : kGuBN;
+    const int dn_bn = narrow ? kNarrowBN : kDnBN;
     TcMaps mGu, mDn;
     if (!streaming) {
         uint16_t* h = at<uint16_t>(ws, p.h);
         const bool gu_b_ok = gather ? make_map(&mGu.B[0], x, p.D, p.T, 1)
-                                    : make_b_maps(mGu.B, at<uint16_t>(ws, p.x_perm), p.D, p.R, kGuBN);
+                                    : make_b_maps(mGu.B, at<uint16_t>(ws, p.x_perm), p.D, p.R, gu_bn);
         if (!make_map(&mGu.A, W_gate_up, p.D, (uint64_t)p.E * 2 * p.I, kTcM) ||
             !make_map(&mGu.A_shared, sgu ? sgu : W_gate_up, p.D,
                       sgu ? 2 * (uint64_t)p.I_s : 2 * (uint64_t)p.I, kTcM) ||
             !gu_b_ok ||
             !make_map(&mDn.A, W_down, p.I, (uint64_t)p.E * p.D, kTcM) ||
             !make_map(&mDn.A_shared, sdn ? sdn : W_down, sdn ? p.I_s : p.I, p.D, kTcM) ||
-            !make_b_maps(mDn.B, h, p.ld_h, p.R, kDnBN))
+            !make_b_maps(mDn.B, h, p.ld_h, p.R, dn_bn))
             return MOE_ERR_CUDA;
         if (gather)
             for (int bi = 1; bi < kNumBBoxes; ++bi) mGu.B[bi] = mGu.B[0];
     }
 
-    // the header of the workspace: [0] device error word, [1] routing ticket
-    MOE_CUDA(cudaMemsetAsync(err, 0, 2 * sizeof(int), s));
+    // the header of the workspace: device error word, routing ticket, split-tail tickets
+    MOE_CUDA(cudaMemsetAsync(err, 0, p.tickets - p.err + (size_t)kSplitTickets * 4, s));
     if ((st = record(opts, 0, s)) != MOE_OK) return st;
+    // T <= 32: one kernel routes and permutes.  Above: router partial sums, then selection and
+    // permutation (one kernel while T*k fits a single permutation block).
     const bool fused_route = p.T <= kFusedRouteMaxT;
+    const bool select_permute = !fused_route && (long long)p.T * p.k <= kPermChunk;
+    float* part = at<float>(ws, p.logits);
     if (!fused_route) {
-        if ((st = run_route(x, W_r, bias, p, dims->norm_topk_prob, logits, idx, w, ws, s)) != MOE_OK)
-            return st;
+        if ((st = run_logits(x, W_r, p, part, ws, s)) != MOE_OK) return st;
+        if (!select_permute)
+            MOE_CUDA(launch_select(part, p.rsplit, bias, p.T, p.E, p.k, dims->norm_topk_prob, idx, w,
+                                   logits_user, true, s));
     }
     if ((st = record(opts, 1, s)) != MOE_OK) return st;
 
@@ -403,20 +422,27 @@ moe_status moe_forward_ex(const moe_bf16* x, const moe_bf16* W_r, const moe_bf16
     pa.slot_row = at<int32_t>(ws, p.slot_row);
     pa.cap = p.R;
     pa.tables = tables_of(p, ws);
+    pa.gu_bn = gu_bn;
+    pa.dn_bn = dn_bn;
     pa.err = err;
     // launch chaining between the forward's kernels (not across a stage-event record)
     const bool chain = !(opts && opts->n_stage_events == 6);
+    RouteArgs ra{};
+    ra.x = x; ra.W_r = W_r; ra.bias = bias;
+    ra.T = p.T; ra.D = p.D; ra.E = p.E; ra.k = p.k; ra.norm = dims->norm_topk_prob;
+    ra.topk_idx = idx;
+    ra.topk_w = w;
+    ra.ticket = err + 1;
+    ra.perm = pa;
     if (fused_route) {
         // one kernel: logits, softmax, top-k and (in its last block) the permutation
-        RouteArgs ra{};
-        ra.x = x; ra.W_r = W_r; ra.bias = bias;
-        ra.T = p.T; ra.D = p.D; ra.E = p.E; ra.k = p.k; ra.norm = dims->norm_topk_prob;
         ra.logits_out = logits;
-        ra.topk_idx = idx;
-        ra.topk_w = w;
-        ra.ticket = err + 1;
-        ra.perm = pa;
         MOE_CUDA(launch_route_fused(ra, false, s));
+    } else if (select_permute) {
+        ra.logits_out = logits_user;
+        ra.part = part;
+        ra.nsplit = p.rsplit;
+        MOE_CUDA(launch_select_permute(ra, chain, s));
     } else {
         MOE_CUDA(launch_permute(pa, chain, s));
     }
@@ -453,10 +479,13 @@ moe_status moe_forward_ex(const moe_bf16* x, const moe_bf16* W_r, const moe_bf16
         ta.row_weight = pa.row_weight;
         ta.row_dest = pa.row_dest;
         ta.slots = at<float>(ws, p.slots);
+        ta.partial = narrow ? at<float>(ws, p.partial) : nullptr;
+        ta.tickets = at<int>(ws, p.tickets);
+        ta.partial_slots = narrow ? kSplitSlots : 0;
         ta.err = err;
-        MOE_CUDA(launch_tc_gate_up(mGu, ta, sms, chain, s));
+        MOE_CUDA(launch_tc_gate_up(mGu, ta, sms, narrow, chain, s));
         if ((st = record(opts, 3, s)) != MOE_OK) return st;
-        MOE_CUDA(launch_tc_down(mDn, ta, sms, chain, s));
+        MOE_CUDA(launch_tc_down(mDn, ta, sms, narrow, chain, s));
         if ((st = record(opts, 4, s)) != MOE_OK) return st;
         MOE_CUDA(launch_combine(ta.slots, 0, p.T, p.D, p.k, p.has_shared, x, sg, residual, out,
                                 out_f32, chain, s));

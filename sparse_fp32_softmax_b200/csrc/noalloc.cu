@@ -21,7 +21,7 @@
 
 namespace {
 
-constexpr size_t kNoAllocScratchBytes = 32ull << 20;  // 32 MiB per device
+constexpr size_t kNoAllocScratchBytes = 64ull << 20;  // 64 MiB per device
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 

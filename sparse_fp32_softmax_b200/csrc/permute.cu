@@ -66,7 +66,8 @@ __global__ void __launch_bounds__(kPermThreads) perm_scan_kernel(PermuteArgs a) 
         s_cnt[e] = run;
     }
     __syncthreads();
-    finish_offsets(a, s_cnt, s_off);
+    if (threadIdx.x < 32) finish_offsets_warp(a, s_cnt, s_off);
+    __syncthreads();
     for (int q = threadIdx.x; q < a.nchunks * E; q += blockDim.x)
         a.chunk_counts[q] += s_off[q % E];
 }

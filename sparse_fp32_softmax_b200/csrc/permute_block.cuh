@@ -7,95 +7,89 @@
 
 namespace moe {
 
-// Block-wide exclusive scan of one int per thread (blockDim.x <= 1024, multiple of 32).
-// Returns the exclusive prefix; *total receives the sum.  Contains __syncthreads.
-static __device__ int block_exclusive_scan(int v, int* total) {
-    __shared__ int warp_sums[32];
-    __shared__ int s_total;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int nwarps = blockDim.x >> 5;
+// Warp-wide exclusive scan; *total receives the warp's sum.
+static __device__ __forceinline__ int warp_exclusive_scan(int v, int* total) {
+    const int lane = threadIdx.x & 31;
     int inc = v;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
         const int y = __shfl_up_sync(0xffffffffu, inc, o);
         if (lane >= o) inc += y;
     }
-    if (lane == 31) warp_sums[warp] = inc;
-    __syncthreads();
-    if (warp == 0) {
-        int w = lane < nwarps ? warp_sums[lane] : 0;
-        int winc = w;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, winc, o);
-            if (lane >= o) winc += y;
-        }
-        if (lane < nwarps) warp_sums[lane] = winc - w;  // exclusive warp offsets
-        if (lane == 31) s_total = winc;                 // grand total
-    }
-    __syncthreads();
-    const int res = warp_sums[warp] + inc - v;
-    const int tot = s_total;
-    __syncthreads();
-    if (total) *total = tot;
-    return res;
+    *total = __shfl_sync(0xffffffffu, inc, 31);
+    return inc - v;
 }
 
-// From per-expert totals s_cnt[0..E) (block-visible shared memory): write counts, the
-// tile-padded offsets (also into s_off[0..E]), the segment tables and the work-item prefix
-// sums of the expert kernels.  Whole block (1024 threads, E < 1024).
-static __device__ void finish_offsets(const PermuteArgs& a, const int* s_cnt, int* s_off) {
+// From per-expert totals s_cnt[0..E) (block-visible shared memory), by one whole warp: write
+// counts, the tile-padded offsets (also into s_off[0..E]), the segment tables and the
+// work-item prefix sums of the expert kernels.  Lane L owns a contiguous run of segments;
+// a pass for the lane totals, five warp scans, and a pass that writes.  The caller
+// synchronises the block afterwards.
+static __device__ void finish_offsets_warp(const PermuteArgs& a, const int* s_cnt, int* s_off) {
+    const int lane = threadIdx.x & 31;
     const int E = a.E;
     const int nseg = E + (a.has_shared ? 1 : 0);
-    int total = 0;
-    const int e = threadIdx.x;
-    const int padded = (e < E) ? (s_cnt[e] + a.tile_m - 1) / a.tile_m * a.tile_m : 0;
-    const int off = block_exclusive_scan(padded, &total);
-    if (e < E) {
-        a.counts[e] = s_cnt[e];
-        a.offsets[e] = off;
-        s_off[e] = off;
-        if (a.tables.seg_count) {
-            a.tables.seg_count[e] = s_cnt[e];
-            a.tables.seg_start[e] = off;
+    const int per = (nseg + 31) >> 5;
+    const int s0 = min(nseg, lane * per), s1 = min(nseg, s0 + per);
+    const bool items = a.tables.gu_items != nullptr;
+    struct Seg { int c, pad, gi, di, gt, dt; };
+    auto seg = [&](int s) {
+        Seg g;
+        g.c = (s == E) ? a.T : s_cnt[s];
+        g.pad = (s < E) ? (g.c + a.tile_m - 1) / a.tile_m * a.tile_m : 0;
+        const int Iseg = (s == E) ? a.I_s : a.I;
+        g.gi = g.di = g.gt = g.dt = 0;
+        if (g.c > 0) {
+            g.gi = (g.c + a.gu_bn - 1) / a.gu_bn * (Iseg / kTcM);
+            g.di = (g.c + a.dn_bn - 1) / a.dn_bn * (a.D / kTcM);
+            g.gt = Iseg / 8;    // streaming gate_up: one warp per 8 features
+            g.dt = a.D / 16;    // streaming down: one warp per 16 output rows
         }
+        return g;
+    };
+    int tp = 0, tgi = 0, tdi = 0, tgt = 0, tdt = 0;
+    for (int s = s0; s < s1; ++s) {
+        const Seg g = seg(s);
+        tp += g.pad; tgi += g.gi; tdi += g.di; tgt += g.gt; tdt += g.dt;
     }
-    if (threadIdx.x == 0) {
-        a.offsets[E] = total;
-        s_off[E] = total;
-        if (a.has_shared && a.tables.seg_count) {
-            a.tables.seg_count[E] = a.T;
-            a.tables.seg_start[E] = total;
-        }
-    }
-    if (a.tables.gu_items) {
-        const int s = threadIdx.x;
-        int gi = 0, di = 0, gt = 0, dt = 0;
-        if (s < nseg) {
-            const int c = (s == E) ? a.T : s_cnt[s];
-            const int Iseg = (s == E) ? a.I_s : a.I;
-            if (c > 0) {
-                gi = (c + kGuBN - 1) / kGuBN * (Iseg / kTcM);
-                di = (c + kDnBN - 1) / kDnBN * (a.D / kTcM);
-                gt = Iseg / 8;      // streaming gate_up: one warp per 8 features
-                dt = a.D / 16;      // streaming down: one warp per 16 output rows
+    int Tp, Tgi, Tdi, Tgt, Tdt;
+    int rp = warp_exclusive_scan(tp, &Tp);
+    int rgi = warp_exclusive_scan(tgi, &Tgi);
+    int rdi = warp_exclusive_scan(tdi, &Tdi);
+    int rgt = warp_exclusive_scan(tgt, &Tgt);
+    int rdt = warp_exclusive_scan(tdt, &Tdt);
+    for (int s = s0; s < s1; ++s) {
+        const Seg g = seg(s);
+        if (s < E) {
+            a.counts[s] = g.c;
+            a.offsets[s] = rp;
+            s_off[s] = rp;
+            if (a.tables.seg_count) {
+                a.tables.seg_count[s] = g.c;
+                a.tables.seg_start[s] = rp;
             }
+            rp += g.pad;
+        } else if (a.tables.seg_count) {  // the shared expert: all T rows after the routed ones
+            a.tables.seg_count[E] = a.T;
+            a.tables.seg_start[E] = Tp;
         }
-        int tot;
-        const int pgi = block_exclusive_scan(gi, &tot);
-        if (s < nseg) a.tables.gu_items[s] = pgi;
-        if (s == 0) a.tables.gu_items[nseg] = tot;
-        const int pdi = block_exclusive_scan(di, &tot);
-        if (s < nseg) a.tables.dn_items[s] = pdi;
-        if (s == 0) a.tables.dn_items[nseg] = tot;
-        const int pgt = block_exclusive_scan(gt, &tot);
-        if (s < nseg) a.tables.gu_tasks[s] = pgt;
-        if (s == 0) a.tables.gu_tasks[nseg] = tot;
-        const int pdt = block_exclusive_scan(dt, &tot);
-        if (s < nseg) a.tables.dn_tasks[s] = pdt;
-        if (s == 0) a.tables.dn_tasks[nseg] = tot;
+        if (items) {
+            a.tables.gu_items[s] = rgi; rgi += g.gi;
+            a.tables.dn_items[s] = rdi; rdi += g.di;
+            a.tables.gu_tasks[s] = rgt; rgt += g.gt;
+            a.tables.dn_tasks[s] = rdt; rdt += g.dt;
+        }
     }
-    __syncthreads();
+    if (lane == 0) {
+        a.offsets[E] = Tp;
+        s_off[E] = Tp;
+        if (items) {
+            a.tables.gu_items[nseg] = Tgi;
+            a.tables.dn_items[nseg] = Tdi;
+            a.tables.gu_tasks[nseg] = Tgt;
+            a.tables.dn_tasks[nseg] = Tdt;
+        }
+    }
 }
 
 // Warp w of a block of W warps owns assignments [a0 + w*L, a0 + w*L + L), L = 4096 / W
@@ -225,7 +219,8 @@ static __device__ void permute_one_block(const PermuteArgs& a, int* wb) {
         s_cnt[e] = run;
     }
     __syncthreads();
-    finish_offsets(a, s_cnt, s_off);
+    if (threadIdx.x < 32) finish_offsets_warp(a, s_cnt, s_off);
+    __syncthreads();
     for (int q = threadIdx.x; q < 32 * E; q += blockDim.x) wb[q] += s_off[q % E];
     __syncthreads();
     scatter_warp_slices(a, ws, wb);

@@ -21,7 +21,6 @@ namespace moe {
 // weight read (decode); larger T goes to the tcgen05 router GEMM.
 __global__ void __launch_bounds__(256) router_small_kernel(const uint16_t* __restrict__ x,
                                                            const uint16_t* __restrict__ W_r,
-                                                           const float* __restrict__ bias,
                                                            int T, int D, int E,
                                                            float* __restrict__ logits) {
     pdl_wait();
@@ -68,48 +67,50 @@ __global__ void __launch_bounds__(256) router_small_kernel(const uint16_t* __res
             for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
             if (lane == i) mine = a;
         }
-        if (lane < nt) {
-            float l = mine;
-            if (bias) l = l + bias[e];
-            logits[(size_t)(t0 + lane) * E + e] = l;
-        }
+        if (lane < nt) logits[(size_t)(t0 + lane) * E + e] = mine;  // bias: added by the selection
     }
 }
 
-cudaError_t launch_router_small(const uint16_t* x, const uint16_t* W_r, const float* bias, int T,
-                                int D, int E, float* logits, bool pdl, cudaStream_t s) {
+cudaError_t launch_router_small(const uint16_t* x, const uint16_t* W_r, int T, int D, int E,
+                                float* logits, bool pdl, cudaStream_t s) {
     const long ntask = (long)E * ((T + 7) / 8);
     const int warps_per_block = 8;
     long blocks = (ntask + warps_per_block - 1) / warps_per_block;
     if (blocks > 148 * 16) blocks = 148 * 16;
     return launch_kernel(router_small_kernel, dim3((int)blocks), dim3(warps_per_block * 32), 0, s, pdl,
-                         x, W_r, bias, T, D, E, logits);
+                         x, W_r, T, D, E, logits);
 }
 
 // ------------------------------------------------------------------ softmax / top-k / renorm
 
-// One warp per token over a logits matrix in global memory.
+// One warp per token over the router's partial sums in global memory.
 template <int VPL>
-__global__ void __launch_bounds__(256) select_kernel(const float* __restrict__ logits, int T, int E,
+__global__ void __launch_bounds__(256) select_kernel(const float* __restrict__ part, int nsplit,
+                                                     const float* __restrict__ bias, int T, int E,
                                                      int k, int norm, int32_t* __restrict__ idx,
-                                                     float* __restrict__ w) {
+                                                     float* __restrict__ w,
+                                                     float* __restrict__ logits_out) {
     pdl_wait();
     pdl_launch_dependents();
     const int nwarps = (gridDim.x * blockDim.x) >> 5;
     for (int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < T; t += nwarps)
-        select_token<VPL>(logits + (size_t)t * E, E, k, norm, idx + (size_t)t * k, w + (size_t)t * k);
+        select_token<VPL>(part + (size_t)t * E, nsplit, (size_t)T * E, bias, E, k, norm,
+                          idx + (size_t)t * k, w + (size_t)t * k,
+                          logits_out ? logits_out + (size_t)t * E : nullptr);
 }
 
-cudaError_t launch_select(const float* logits, int T, int E, int k, int norm, int32_t* idx,
-                          float* w, bool pdl, cudaStream_t s) {
+cudaError_t launch_select(const float* part, int nsplit, const float* bias, int T, int E, int k,
+                          int norm, int32_t* idx, float* w, float* logits_out, bool pdl,
+                          cudaStream_t s) {
     const int threads = 256;
     int blocks = (T + 7) / 8;
     if (blocks > 148 * 32) blocks = 148 * 32;
     if (blocks < 1) blocks = 1;
-    void (*k_)(const float*, int, int, int, int, int32_t*, float*) =
+    void (*k_)(const float*, int, const float*, int, int, int, int, int32_t*, float*, float*) =
         E <= 32 ? select_kernel<1> : E <= 64 ? select_kernel<2> : E <= 128 ? select_kernel<4>
         : E <= 256 ? select_kernel<8> : select_kernel<16>;
-    return launch_kernel(k_, dim3(blocks), dim3(threads), 0, s, pdl, logits, T, E, k, norm, idx, w);
+    return launch_kernel(k_, dim3(blocks), dim3(threads), 0, s, pdl, part, nsplit, bias, T, E, k,
+                         norm, idx, w, logits_out);
 }
 
 }  // namespace moe

@@ -42,6 +42,10 @@ def layer(name, T=None):
     return _layers[key]
 
 
+def to_f64(y):
+    return y.double().numpy()
+
+
 def run_forward(cfg, G, path="auto", x=None, residual=None, k=None, norm=None):
     x = G["x"] if x is None else x
     k = cfg.k if k is None else k
@@ -270,18 +274,23 @@ def test_forward_zero_input(path):
 
 @pytest.mark.parametrize("path", ["stream", "grouped"])
 def test_determinism_and_batch_invariance(path):
-    """Bitwise-equal reruns, and a token's output independent of the other tokens in the
-    batch for a given router kernel (T <= 64 runs the CUDA-core router, larger T the
-    tensor-core one; the two sum the logits in different FP32 orders)."""
+    """Bitwise-equal reruns of the same batch.  A token's routing (experts and FP32 weights)
+    does not depend on the other tokens of the batch within a router kernel's range (T <= 64
+    runs the CUDA-core router, larger T the tensor-core one with a K split fixed by the shapes;
+    the two sum the logits in different FP32 orders).  Its output agrees within the output
+    tolerance: the expert GEMMs split the last wave's items along K, and how many items there
+    are depends on the batch, so the FP32 summation order of y can change with it."""
     cfg, L, G = _small_layer(256)
-    y1, *_ = run_forward(cfg, G, path)
-    y2, *_ = run_forward(cfg, G, path)
-    assert torch.equal(y1, y2)
-    y100, *_ = run_forward(cfg, G, path, x=G["x"][:100].contiguous())
-    assert torch.equal(y100, y1[:100])
-    y64, *_ = run_forward(cfg, G, path, x=G["x"][:64].contiguous())
-    y8, *_ = run_forward(cfg, G, path, x=G["x"][:8].contiguous())
-    assert torch.equal(y8, y64[:8])
+    y1, i1, w1, l1 = run_forward(cfg, G, path)
+    y2, i2, w2, l2 = run_forward(cfg, G, path)
+    assert torch.equal(y1, y2) and (i1 == i2).all() and (w1 == w2).all() and (l1 == l2).all()
+    y100, i100, w100, l100 = run_forward(cfg, G, path, x=G["x"][:100].contiguous())
+    assert (l100 == l1[:100]).all() and (i100 == i1[:100]).all() and (w100 == w1[:100]).all()
+    assert_y_close(to_f64(y100), to_f64(y1[:100]), "T=100 vs the first 100 of T=256")
+    y64, i64, w64, l64 = run_forward(cfg, G, path, x=G["x"][:64].contiguous())
+    y8, i8, w8, l8 = run_forward(cfg, G, path, x=G["x"][:8].contiguous())
+    assert (l8 == l64[:8]).all() and (i8 == i64[:8]).all() and (w8 == w64[:8]).all()
+    assert_y_close(to_f64(y8), to_f64(y64[:8]), "T=8 vs the first 8 of T=64")
 
 
 def test_paths_agree_and_status_ok():
