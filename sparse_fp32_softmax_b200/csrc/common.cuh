@@ -174,6 +174,17 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* m
         : "memory");
 }
 
+// 5-D tile load (no L2 hint), coordinates innermost first.
+__device__ __forceinline__ void tma_load_5d(void* smem_dst, const CUtensorMap* map, uint64_t* bar,
+                                            int c0, int c1, int c2, int c3, int c4) {
+    asm volatile(
+        "cp.async.bulk.tensor.5d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3),
+        "r"(c4)
+        : "memory");
+}
+
 // Row gather: four rows (r0..r3) of a 2-D tensor whose map has a one-row box {64 cols, 1},
 // columns [x, x+64), written to shared memory as four consecutive 128-byte rows (the 128-byte
 // swizzle follows the destination address, so consecutive gathers build the same layout a

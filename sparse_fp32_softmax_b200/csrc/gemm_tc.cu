@@ -8,9 +8,15 @@
 //
 // Layout of the work (swap-AB): a tile is 128 weight rows (the MMA's M) by up to BN tokens
 // (its N), so an expert with few tokens costs a narrow N instead of a padded 128-row M.
-//   gate_up: two accumulators per tile, gate rows [f0, f0+128) and the matching up rows
-//            [I+f0, ...), against the same token tile; TMEM lane f holds gate and up of
-//            feature f for every token, and the epilogue writes h = silu(g) * u in bf16.
+//   gate_up, narrow tiles (BN = 64, decode): two accumulators per tile, gate rows
+//            [f0, f0+128) and the matching up rows [I+f0, ...), against the same token tile;
+//            TMEM lane f holds gate and up of feature f, and the epilogue writes
+//            h = silu(g) * u in bf16.
+//   gate_up, wide tiles (BN = 256): one accumulator whose 128 rows interleave gate and up
+//            of 64 features in groups of 16 (fetched by one 5-D TMA load); lane l and lane
+//            l+16 of a lane quarter hold gate and up of one feature and swap halves with a
+//            shuffle.  A tcgen05.mma costs its issuing thread roughly the same whatever N,
+//            so N = 256 halves the instructions of the two-accumulator layout at N = 128.
 //   down:    one accumulator, down rows [d0, d0+128) against a tile of h rows; the epilogue
 //            scales by the routing weight and stores FP32 into the token's slot (a bf16 slot
 //            would add a third bf16 rounding on top of h and the output).
@@ -19,8 +25,8 @@
 //            bias, by the selection), so that a handful of token tiles still fills the SMs.
 //
 // Per CTA (one per SM, persistent over a device-side item list):
-//   warp 0      TMA producer: 4-stage ring of {A tile(s) 128x64, B tile BNx64} bf16 tiles in
-//               the 128-byte swizzle layout, completion counted on an mbarrier;
+//   warp 0      TMA producer: ring of STAGES stages {A tile(s) 128x64, B tile BNx64} of bf16
+//               in the 128-byte swizzle layout, completion counted on an mbarrier;
 //   warp 1      allocates TMEM, and one thread issues tcgen05.mma (M=128, N=tile width,
 //               K=16 x 4 per stage) with FP32 accumulation in TMEM; tcgen05.commit frees a
 //               stage when its MMAs are done and publishes an accumulator when a tile is;
@@ -40,7 +46,10 @@ enum { kModeGateUp = 0, kModeDown = 1, kModeRouter = 2 };
 template <int MODE, int BN_, int STAGES_>
 struct TcCfg {
     static constexpr int BN = BN_, STAGES = STAGES_;
-    static constexpr int NA = MODE == kModeGateUp ? 2 : 1;   // A tiles (accumulators) per stage
+    // gate_up: narrow tiles keep gate and up in two accumulators (two A tiles per stage);
+    // wide tiles interleave them in one A tile and one accumulator
+    static constexpr bool IL = MODE == kModeGateUp && BN > kNarrowBN;
+    static constexpr int NA = (MODE == kModeGateUp && !IL) ? 2 : 1;   // A tiles per stage
     static constexpr int ACC = NA * BN;                       // TMEM columns per accumulator set
     // two accumulator sets, rounded up to the power-of-two allocation unit (>= 32 columns)
     static constexpr int TMEM = 2 * ACC <= 32 ? 32 : 2 * ACC <= 64 ? 64 : 2 * ACC <= 128 ? 128
@@ -61,8 +70,8 @@ constexpr int kTcThreads = (2 + kEpiWarps) * 32;
 struct TileInfo {
     int bi;       // token-operand box: 16 << bi rows
     int shared;   // A comes from the shared-expert tensor map
-    int a_row0;   // first A row (gate rows for gate_up)
-    int a_row1;   // first up row (gate_up only)
+    int a_row0;   // first A row (gate rows for gate_up; interleaved: 16-feature group)
+    int a_row1;   // first up row (gate_up; interleaved: expert)
     int b_row;    // first B (token) row
     int n_valid;  // valid token columns, 1..BN
     int nk;       // K stages
@@ -150,15 +159,21 @@ __device__ __forceinline__ TileInfo tc_decode_item(const TcArgs& a, const SmemTa
     const int local = item - st->prefix[s];
     const int sh = (s == a.E);
     const int Iseg = sh ? a.I_s : a.I;
-    const int mtc = (MODE == kModeGateUp) ? Iseg / kTcM : a.D / kTcM;
+    const int fpt = (MODE == kModeGateUp && BN > kNarrowBN) ? kGuILFeatures : kTcM;  // per tile
+    const int mtc = (MODE == kModeGateUp) ? Iseg / fpt : a.D / kTcM;
     const int tt = local / mtc, mt = local % mtc;
     const int cnt = st->count[s];
     const int start = st->start[s];
     ti.shared = sh;
     ti.b_row = start + tt * BN;
     ti.n_valid = min(BN, cnt - tt * BN);
-    ti.m0 = mt * kTcM;
-    if (MODE == kModeGateUp) {
+    ti.m0 = mt * fpt;
+    if (MODE == kModeGateUp && BN > kNarrowBN) {
+        // interleaved: 64 features [m0, m0+64) of expert s, as four 16-feature groups
+        ti.a_row0 = ti.m0 / 16;
+        ti.a_row1 = sh ? 0 : s;
+        ti.nk = a.D / kTcK;
+    } else if (MODE == kModeGateUp) {
         const int base = sh ? 0 : s * 2 * a.I;
         ti.a_row0 = base + mt * kTcM;
         ti.a_row1 = base + Iseg + mt * kTcM;
@@ -272,6 +287,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         // rows from x by row_token, lane i taking rows 4i..4i+3 of the tile (rows past the
         // segment repeat its last row; their columns are never used); otherwise lane 0 loads
         // a tile of the permuted rows.
+        const int first = blockIdx.x, step = gridDim.x;   // this CTA's units
         int it = 0;
         bool ok = true;
         int last_round[STAGES];
@@ -287,15 +303,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         };
         TileInfo tn{};
         int gn[4] = {0, 0, 0, 0};
-        if ((int)blockIdx.x < total) {
-            tn = tc_decode_unit<MODE, BN>(a, tabs, sc, blockIdx.x);
+        if (first < total) {
+            tn = tc_decode_unit<MODE, BN>(a, tabs, sc, first);
             if (gather) gather_rows(tn, gn);
         }
-        for (int item = blockIdx.x; item < total && ok; item += gridDim.x) {
+        for (int item = first; item < total && ok; item += step) {
             const TileInfo ti = tn;
             const int g0 = gn[0], g1 = gn[1], g2 = gn[2], g3 = gn[3];
-            if (item + (int)gridDim.x < total) {
-                tn = tc_decode_unit<MODE, BN>(a, tabs, sc, item + gridDim.x);
+            if (item + step < total) {
+                tn = tc_decode_unit<MODE, BN>(a, tabs, sc, item + step);
                 if (gather) gather_rows(tn, gn);
             }
             const CUtensorMap* mA = ti.shared ? &maps.A_shared : &maps.A;
@@ -314,7 +330,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 if (lane == 0) {
                     mbar_arrive_expect_tx(full + s, bytes);
                     const int kx = (ti.k0 + kb) * kTcK;
-                    tma_load(st, mA, full + s, kx, ti.a_row0);
+                    if (Tr::IL)
+                        tma_load_5d(st, mA, full + s, kx, 0, 0, ti.a_row0, ti.a_row1);
+                    else
+                        tma_load(st, mA, full + s, kx, ti.a_row0);
                     if (NA == 2) tma_load(st + kATileBytes, mA, full + s, kx, ti.a_row1);
                     if (!gather) tma_load(st + NA * kATileBytes, mB, full + s, kx, ti.b_row);
                 }
@@ -398,7 +417,23 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         float* ep_wt = ep_wt_all + ew * BN;
         // The epilogue of one 32-column chunk: v (and u, the up accumulator) hold row `row`.
         auto finish_chunk = [&](const TileInfo& ti, int c, const float* v, const float* u) {
-            if (MODE == kModeGateUp) {
+            if (Tr::IL) {
+                // lanes 0-15 of the quarter hold gate rows of features m0 + 16*quarter + l,
+                // lanes 16-31 the up rows of the same features: lane l takes the chunk's tokens
+                // 0-15, lane l+16 tokens 16-31, swapping the other half with its partner
+                const bool is_gate = (lane & 16) == 0;
+                const int f = ti.m0 + 16 * quarter + (lane & 15);
+                const int t0 = c * 32 + (is_gate ? 0 : 16);
+                uint16_t* hp = a.h + (size_t)(ti.b_row + t0) * a.ld_h + f;
+#pragma unroll
+                for (int t = 0; t < 16; ++t) {
+                    const float send = is_gate ? v[16 + t] : v[t];
+                    const float recv = __shfl_xor_sync(0xffffffffu, send, 16);
+                    const float g = is_gate ? v[t] : recv;
+                    const float uu = is_gate ? recv : v[16 + t];
+                    if (t0 + t < ti.n_valid) hp[(size_t)t * a.ld_h] = to_bf16_bits(silu(g) * uu);
+                }
+            } else if (MODE == kModeGateUp) {
                 const int f = ti.m0 + row;
                 uint16_t* hp = a.h + (size_t)(ti.b_row + c * 32) * a.ld_h + f;
 #pragma unroll
@@ -467,13 +502,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     float v[32];
                     tmem_ld32(tb + c * 32, v);
                     float u[32];
-                    if (MODE == kModeGateUp) tmem_ld32(tb + BN + c * 32, u);
+                    if (NA == 2) tmem_ld32(tb + BN + c * 32, u);
                     tmem_ld_wait();
                     float4* d0 = reinterpret_cast<float4*>(ps + (size_t)row * BN + c * 32);
 #pragma unroll
                     for (int q = 0; q < 8; ++q)
                         d0[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-                    if (MODE == kModeGateUp) {
+                    if (NA == 2) {
                         float4* d1 = reinterpret_cast<float4*>(ps + (size_t)(kTcM + row) * BN + c * 32);
 #pragma unroll
                         for (int q = 0; q < 8; ++q)
@@ -506,7 +541,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                             if (sp < ti.nsplit) {
                                 const float* pp = p0 + (size_t)sp * (NA * kTcM * BN) + c * 32 + 4 * g;
                                 lv[sp] = __ldcg(reinterpret_cast<const float4*>(pp + (size_t)row * BN));
-                                if (MODE == kModeGateUp)
+                                if (NA == 2)
                                     lu[sp] = __ldcg(reinterpret_cast<const float4*>(pp + (size_t)(kTcM + row) * BN));
                             }
                         }
@@ -515,7 +550,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         for (int sp = 1; sp < kMaxKSplit; ++sp) {
                             if (sp < ti.nsplit) {
                                 sv.x += lv[sp].x; sv.y += lv[sp].y; sv.z += lv[sp].z; sv.w += lv[sp].w;
-                                if (MODE == kModeGateUp) {
+                                if (NA == 2) {
                                     su.x += lu[sp].x; su.y += lu[sp].y; su.z += lu[sp].z; su.w += lu[sp].w;
                                 }
                             }
@@ -528,7 +563,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             for (int c = half; c < nchunks; c += 2) {
                 float v[32], u[32];
                 tmem_ld32(tb + c * 32, v);
-                if (MODE == kModeGateUp) tmem_ld32(tb + BN + c * 32, u);
+                if (NA == 2) tmem_ld32(tb + BN + c * 32, u);
                 tmem_ld_wait();
                 finish_chunk(ti, c, v, u);
             }

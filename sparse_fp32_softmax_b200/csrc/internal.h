@@ -22,7 +22,12 @@ enum : int {
 // Tile geometry of the tcgen05 grouped GEMMs (swap-AB: weights on M, tokens on N).
 constexpr int kTcM = 128;       // weight rows per tile (MMA M)
 constexpr int kTcK = 64;        // K elements per pipeline stage (one 128-byte swizzle row)
-constexpr int kGuBN = 128;      // token columns per gate_up tile (two accumulators per tile)
+// Wide gate_up tiles interleave gate and up rows in the MMA's M (16 gate rows of 16
+// features, then their 16 up rows, four times: 64 features), so one accumulator of up to 256
+// token columns holds both and every MMA has N up to 256 (a tcgen05.mma costs the issuing
+// thread about the same whatever its N, so wider MMAs do more work per instruction).
+constexpr int kGuBN = 256;      // token columns per wide gate_up tile
+constexpr int kGuILFeatures = 64;  // features per wide (interleaved) gate_up tile
 constexpr int kDnBN = 256;      // token columns per down tile
 constexpr int kRtBN = 128;      // token columns per router-logit tile
 constexpr int kStages = 4;      // shared-memory pipeline depth of the wide tiles
@@ -87,6 +92,7 @@ struct PermuteArgs {
     int cap;                  // rows available in row_* arrays
     SegTables tables;         // may be all-null (moe_permute alone)
     int gu_bn, dn_bn;         // token columns per gate_up / down tile (work-item tables)
+    int gu_features;          // features per gate_up tile (128 narrow, 64 interleaved)
     int* err;
 };
 

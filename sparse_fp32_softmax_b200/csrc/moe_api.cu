@@ -165,6 +165,23 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, ui
     return r == CUDA_SUCCESS;
 }
 
+// gate_up [E, 2*Iseg, D] (gate rows, then up rows, per expert) viewed as 5-D {D, 16 rows,
+// gate|up, Iseg/16 groups, E} with box {64, 16, 2, 4, 1}: one load brings 64 columns of four
+// 16-feature groups, each as 16 gate rows followed by the 16 matching up rows -- the
+// interleaved A tile of the wide gate_up kernel (128 rows, 128-byte swizzle).
+bool make_map_gate_up_il(CUtensorMap* m, const void* base, uint64_t D, uint64_t Iseg, uint64_t E) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[5] = {D, 16, 2, Iseg / 16, E};
+    cuuint64_t strides[4] = {D * 2, Iseg * D * 2, 16 * D * 2, 2 * Iseg * D * 2};
+    cuuint32_t box[5] = {(cuuint32_t)kTcK, 16, 2, (cuuint32_t)(kGuILFeatures / 16), 1};
+    cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 // The token-operand map at every box height up to max_rows.
 bool make_b_maps(CUtensorMap* maps, const void* base, uint64_t cols, uint64_t rows, int max_rows) {
     for (int bi = 0; bi < kNumBBoxes; ++bi) {
@@ -320,6 +337,7 @@ moe_status moe_permute(const int32_t* topk_idx, const float* topk_w, const moe_b
     a.tables = SegTables{nullptr, nullptr, nullptr, nullptr, nullptr, nullptr};
     a.gu_bn = kGuBN;
     a.dn_bn = kDnBN;
+    a.gu_features = kGuILFeatures;
     a.err = at<int>(ws, p.err);
     // padding rows are only written per expert segment; rows past offsets[E] stay as given,
     // so mark every row as padding first
@@ -377,9 +395,14 @@ moe_status moe_forward_ex(const moe_bf16* x, const moe_bf16* W_r, const moe_bf16
         uint16_t* h = at<uint16_t>(ws, p.h);
         const bool gu_b_ok = gather ? make_map(&mGu.B[0], x, p.D, p.T, 1)
                                     : make_b_maps(mGu.B, at<uint16_t>(ws, p.x_perm), p.D, p.R, gu_bn);
-        if (!make_map(&mGu.A, W_gate_up, p.D, (uint64_t)p.E * 2 * p.I, kTcM) ||
-            !make_map(&mGu.A_shared, sgu ? sgu : W_gate_up, p.D,
-                      sgu ? 2 * (uint64_t)p.I_s : 2 * (uint64_t)p.I, kTcM) ||
+        const bool gu_a_ok =
+            narrow ? make_map(&mGu.A, W_gate_up, p.D, (uint64_t)p.E * 2 * p.I, kTcM) &&
+                         make_map(&mGu.A_shared, sgu ? sgu : W_gate_up, p.D,
+                                  sgu ? 2 * (uint64_t)p.I_s : 2 * (uint64_t)p.I, kTcM)
+                   : make_map_gate_up_il(&mGu.A, W_gate_up, p.D, p.I, p.E) &&
+                         make_map_gate_up_il(&mGu.A_shared, sgu ? sgu : W_gate_up, p.D,
+                                             sgu ? p.I_s : p.I, 1);
+        if (!gu_a_ok ||
             !gu_b_ok ||
             !make_map(&mDn.A, W_down, p.I, (uint64_t)p.E * p.D, kTcM) ||
             !make_map(&mDn.A_shared, sdn ? sdn : W_down, sdn ? p.I_s : p.I, p.D, kTcM) ||
@@ -424,6 +447,7 @@ moe_status moe_forward_ex(const moe_bf16* x, const moe_bf16* W_r, const moe_bf16
     pa.tables = tables_of(p, ws);
     pa.gu_bn = gu_bn;
     pa.dn_bn = dn_bn;
+    pa.gu_features = narrow ? kTcM : kGuILFeatures;
     pa.err = err;
     // launch chaining between the forward's kernels (not across a stage-event record)
     const bool chain = !(opts && opts->n_stage_events == 6);

@@ -40,7 +40,7 @@ static __device__ void finish_offsets_warp(const PermuteArgs& a, const int* s_cn
         const int Iseg = (s == E) ? a.I_s : a.I;
         g.gi = g.di = g.gt = g.dt = 0;
         if (g.c > 0) {
-            g.gi = (g.c + a.gu_bn - 1) / a.gu_bn * (Iseg / kTcM);
+            g.gi = (g.c + a.gu_bn - 1) / a.gu_bn * (Iseg / a.gu_features);
             g.di = (g.c + a.dn_bn - 1) / a.dn_bn * (a.D / kTcM);
             g.gt = Iseg / 8;    // streaming gate_up: one warp per 8 features
             g.dt = a.D / 16;    // streaming down: one warp per 16 output rows
