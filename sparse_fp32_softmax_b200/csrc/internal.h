@@ -118,7 +118,7 @@ struct RouteArgs {
 // The router GEMM splits K so that small token counts still spread over the SMs; its
 // partial sums are added in split order by the selection.  The split depends only on the
 // shapes (not on the device), so results do not depend on the GPU the call runs on.
-constexpr int kRouterMaxSplit = 16;
+constexpr int kRouterMaxSplit = 8;
 constexpr int kSplitTargetCtas = 148;
 inline int router_splits(int T, int E, int D, int bn) {
     const long long items = (long long)((T + bn - 1) / bn) * ((E + 127) / 128);

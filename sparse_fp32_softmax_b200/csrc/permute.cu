@@ -66,14 +66,13 @@ __global__ void __launch_bounds__(kPermThreads) perm_scan_kernel(PermuteArgs a) 
         s_cnt[e] = run;
     }
     __syncthreads();
-    if (threadIdx.x < 32) finish_offsets_warp(a, s_cnt, s_off);
-    __syncthreads();
+    finish_offsets(a, s_cnt, s_off);
     for (int q = threadIdx.x; q < a.nchunks * E; q += blockDim.x)
         a.chunk_counts[q] += s_off[q % E];
 }
 
 // 3. stable scatter of one chunk per block
-__global__ void __launch_bounds__(kPermThreads) perm_scatter_kernel(PermuteArgs a) {
+__global__ void __launch_bounds__(kPermThreads, 1) perm_scatter_kernel(PermuteArgs a) {
     extern __shared__ int wb[];  // [32][E]: per-warp counts, then per-warp running row bases
     pdl_wait();
     pdl_launch_dependents();

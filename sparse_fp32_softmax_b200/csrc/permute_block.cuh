@@ -7,89 +7,94 @@
 
 namespace moe {
 
-// Warp-wide exclusive scan; *total receives the warp's sum.
-static __device__ __forceinline__ int warp_exclusive_scan(int v, int* total) {
-    const int lane = threadIdx.x & 31;
-    int inc = v;
+// Block-wide exclusive scan of five ints per thread at once (blockDim.x <= 1024, a multiple
+// of 32): v[j] becomes its exclusive prefix over the block, tot[j] the block's sum.  Two
+// __syncthreads.
+static __device__ void block_exclusive_scan5(int (&v)[5], int (&tot)[5]) {
+    __shared__ int wsum[32][5];
+    __shared__ int wtot[5];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int nwarps = blockDim.x >> 5;
+    int inc[5];
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, inc, o);
-        if (lane >= o) inc += y;
+    for (int j = 0; j < 5; ++j) {
+        inc[j] = v[j];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, inc[j], o);
+            if (lane >= o) inc[j] += y;
+        }
+        if (lane == 31) wsum[warp][j] = inc[j];
     }
-    *total = __shfl_sync(0xffffffffu, inc, 31);
-    return inc - v;
+    __syncthreads();
+    if (warp == 0) {
+#pragma unroll
+        for (int j = 0; j < 5; ++j) {
+            const int w = lane < nwarps ? wsum[lane][j] : 0;
+            int winc = w;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, winc, o);
+                if (lane >= o) winc += y;
+            }
+            if (lane < nwarps) wsum[lane][j] = winc - w;  // exclusive warp offsets
+            if (lane == 31) wtot[j] = winc;
+        }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < 5; ++j) {
+        v[j] = wsum[warp][j] + inc[j] - v[j];
+        tot[j] = wtot[j];
+    }
 }
 
-// From per-expert totals s_cnt[0..E) (block-visible shared memory), by one whole warp: write
-// counts, the tile-padded offsets (also into s_off[0..E]), the segment tables and the
-// work-item prefix sums of the expert kernels.  Lane L owns a contiguous run of segments;
-// a pass for the lane totals, five warp scans, and a pass that writes.  The caller
-// synchronises the block afterwards.
-static __device__ void finish_offsets_warp(const PermuteArgs& a, const int* s_cnt, int* s_off) {
-    const int lane = threadIdx.x & 31;
+// From per-expert totals s_cnt[0..E) (block-visible shared memory), by the whole block (one
+// thread per segment, nseg <= blockDim.x): write counts, the tile-padded offsets (also into
+// s_off[0..E]), the segment tables and the work-item prefix sums of the expert kernels.
+// Ends with the block synchronised.
+static __device__ void finish_offsets(const PermuteArgs& a, const int* s_cnt, int* s_off) {
     const int E = a.E;
     const int nseg = E + (a.has_shared ? 1 : 0);
-    const int per = (nseg + 31) >> 5;
-    const int s0 = min(nseg, lane * per), s1 = min(nseg, s0 + per);
-    const bool items = a.tables.gu_items != nullptr;
-    struct Seg { int c, pad, gi, di, gt, dt; };
-    auto seg = [&](int s) {
-        Seg g;
-        g.c = (s == E) ? a.T : s_cnt[s];
-        g.pad = (s < E) ? (g.c + a.tile_m - 1) / a.tile_m * a.tile_m : 0;
-        const int Iseg = (s == E) ? a.I_s : a.I;
-        g.gi = g.di = g.gt = g.dt = 0;
-        if (g.c > 0) {
-            g.gi = (g.c + a.gu_bn - 1) / a.gu_bn * (Iseg / a.gu_features);
-            g.di = (g.c + a.dn_bn - 1) / a.dn_bn * (a.D / kTcM);
-            g.gt = Iseg / 8;    // streaming gate_up: one warp per 8 features
-            g.dt = a.D / 16;    // streaming down: one warp per 16 output rows
+    const int s = threadIdx.x;
+    int v[5] = {0, 0, 0, 0, 0};   // padded rows, gate_up items, down items, gate_up tasks, down tasks
+    int c = 0;
+    if (s < nseg) {
+        c = (s == E) ? a.T : s_cnt[s];
+        if (s < E) v[0] = (c + a.tile_m - 1) / a.tile_m * a.tile_m;
+        if (c > 0) {
+            const int Iseg = (s == E) ? a.I_s : a.I;
+            v[1] = (c + a.gu_bn - 1) / a.gu_bn * (Iseg / a.gu_features);
+            v[2] = (c + a.dn_bn - 1) / a.dn_bn * (a.D / kTcM);
+            v[3] = Iseg / 8;     // streaming gate_up: one warp per 8 features
+            v[4] = a.D / 16;     // streaming down: one warp per 16 output rows
         }
-        return g;
-    };
-    int tp = 0, tgi = 0, tdi = 0, tgt = 0, tdt = 0;
-    for (int s = s0; s < s1; ++s) {
-        const Seg g = seg(s);
-        tp += g.pad; tgi += g.gi; tdi += g.di; tgt += g.gt; tdt += g.dt;
     }
-    int Tp, Tgi, Tdi, Tgt, Tdt;
-    int rp = warp_exclusive_scan(tp, &Tp);
-    int rgi = warp_exclusive_scan(tgi, &Tgi);
-    int rdi = warp_exclusive_scan(tdi, &Tdi);
-    int rgt = warp_exclusive_scan(tgt, &Tgt);
-    int rdt = warp_exclusive_scan(tdt, &Tdt);
-    for (int s = s0; s < s1; ++s) {
-        const Seg g = seg(s);
-        if (s < E) {
-            a.counts[s] = g.c;
-            a.offsets[s] = rp;
-            s_off[s] = rp;
-            if (a.tables.seg_count) {
-                a.tables.seg_count[s] = g.c;
-                a.tables.seg_start[s] = rp;
-            }
-            rp += g.pad;
-        } else if (a.tables.seg_count) {  // the shared expert: all T rows after the routed ones
+    int tot[5];
+    block_exclusive_scan5(v, tot);
+    if (s < E) {
+        a.counts[s] = c;
+        a.offsets[s] = v[0];
+        s_off[s] = v[0];
+        if (a.tables.seg_count) {
+            a.tables.seg_count[s] = c;
+            a.tables.seg_start[s] = v[0];
+        }
+    } else if (s == E) {
+        a.offsets[E] = tot[0];
+        s_off[E] = tot[0];
+        if (a.has_shared && a.tables.seg_count) {   // the shared expert: after the routed rows
             a.tables.seg_count[E] = a.T;
-            a.tables.seg_start[E] = Tp;
-        }
-        if (items) {
-            a.tables.gu_items[s] = rgi; rgi += g.gi;
-            a.tables.dn_items[s] = rdi; rdi += g.di;
-            a.tables.gu_tasks[s] = rgt; rgt += g.gt;
-            a.tables.dn_tasks[s] = rdt; rdt += g.dt;
+            a.tables.seg_start[E] = tot[0];
         }
     }
-    if (lane == 0) {
-        a.offsets[E] = Tp;
-        s_off[E] = Tp;
-        if (items) {
-            a.tables.gu_items[nseg] = Tgi;
-            a.tables.dn_items[nseg] = Tdi;
-            a.tables.gu_tasks[nseg] = Tgt;
-            a.tables.dn_tasks[nseg] = Tdt;
-        }
+    if (a.tables.gu_items && s <= nseg) {
+        a.tables.gu_items[s] = s < nseg ? v[1] : tot[1];
+        a.tables.dn_items[s] = s < nseg ? v[2] : tot[2];
+        a.tables.gu_tasks[s] = s < nseg ? v[3] : tot[3];
+        a.tables.dn_tasks[s] = s < nseg ? v[4] : tot[4];
     }
+    __syncthreads();
 }
 
 // Warp w of a block of W warps owns assignments [a0 + w*L, a0 + w*L + L), L = 4096 / W
@@ -219,8 +224,7 @@ static __device__ void permute_one_block(const PermuteArgs& a, int* wb) {
         s_cnt[e] = run;
     }
     __syncthreads();
-    if (threadIdx.x < 32) finish_offsets_warp(a, s_cnt, s_off);
-    __syncthreads();
+    finish_offsets(a, s_cnt, s_off);
     for (int q = threadIdx.x; q < 32 * E; q += blockDim.x) wb[q] += s_off[q % E];
     __syncthreads();
     scatter_warp_slices(a, ws, wb);
