@@ -365,7 +365,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             const uint32_t idesc0 = umma_idesc_bf16_f32(kTcM, 16) & ~(0x3Fu << 17);
-            int it = 0, tc = 0;
+            // shared-memory descriptors of stage 0; stage s adds s * SB / 16 to the address
+            // field (stages stay below 256 KB, so the 14-bit field does not carry)
+            const uint64_t dA0 = umma_desc_sw128(smem);
+            const uint64_t dA1 = umma_desc_sw128(smem + kATileBytes);
+            const uint64_t dB = umma_desc_sw128(smem + NA * kATileBytes);
+            int s = 0, phase = 0;   // ring position of the next stage
+            int tc = 0;
             bool ok = true;
             for (int item = blockIdx.x; item < total && ok; item += gridDim.x, ++tc) {
                 const TileInfo ti = tc_decode_unit<MODE, BN>(a, tabs, sc, item);
@@ -380,25 +386,26 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 n = n < 16 ? 16 : (n > BN ? BN : n);
                 const uint32_t idesc = idesc0 | ((uint32_t)(n >> 3) << 17);
                 const uint32_t d0 = tmem_base + (uint32_t)(b * ACC);
-                for (int kb = 0; kb < ti.nk; ++kb, ++it) {
-                    const int s = it % STAGES;
-                    const int round = it / STAGES;
-                    if (!mbar_wait(full + s, round & 1, a.err, kErrWaitMma)) {
+                for (int kb = 0; kb < ti.nk; ++kb) {
+                    if (!mbar_wait(full + s, phase, a.err, kErrWaitMma)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    uint8_t* st = smem + s * SB;
-                    const uint64_t da0 = umma_desc_sw128(st);
-                    const uint64_t da1 = umma_desc_sw128(st + kATileBytes);
-                    const uint64_t db = umma_desc_sw128(st + NA * kATileBytes);
+                    const uint64_t off = (uint64_t)(s * (SB >> 4));
+                    const uint64_t da0 = dA0 + off, da1 = dA1 + off, db = dB + off;
+                    umma_bf16(d0, da0, db, idesc, kb);  // the tile's first MMA overwrites D
+                    if (NA == 2) umma_bf16(d0 + BN, da1, db, idesc, kb);
 #pragma unroll
-                    for (int kk = 0; kk < kTcK / 16; ++kk) {
-                        const uint32_t accum = (kb | kk) != 0;
-                        umma_bf16(d0, da0 + 2 * kk, db + 2 * kk, idesc, accum);
-                        if (NA == 2) umma_bf16(d0 + BN, da1 + 2 * kk, db + 2 * kk, idesc, accum);
+                    for (int kk = 1; kk < kTcK / 16; ++kk) {
+                        umma_bf16_acc(d0, da0 + 2 * kk, db + 2 * kk, idesc);
+                        if (NA == 2) umma_bf16_acc(d0 + BN, da1 + 2 * kk, db + 2 * kk, idesc);
                     }
                     umma_commit(empty + s);
+                    if (++s == STAGES) {
+                        s = 0;
+                        phase ^= 1;
+                    }
                 }
                 if (!ok) break;
                 umma_commit(tfull + b);
@@ -476,6 +483,25 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         a.slots[(size_t)ep_dest[col0 + j] * a.D + d] = ep_wt[col0 + j] * v[j];
             }
         };
+        // down, wide tiles: the slot destinations and routing weights of the token columns
+        // this warp stores (its chunks half, half + 2, ...) are loaded one tile ahead into
+        // registers, so their memory latency overlaps the previous tile's epilogue (measured:
+        // it helps the long-K wide tiles and costs the short narrow ones)
+        constexpr bool kAhead = MODE == kModeDown && BN > kNarrowBN;
+        constexpr int kCPW = (BN + 63) / 64;   // chunks per epilogue warp
+        int nd[kCPW];
+        float nw[kCPW];
+        auto fetch_dest = [&](const TileInfo& t) {
+#pragma unroll
+            for (int i = 0; i < kCPW; ++i) {
+                const int col = (half + 2 * i) * 32 + lane;
+                const bool in = col < t.n_valid;
+                nd[i] = in ? __ldg(a.row_dest + t.b_row + col) : 0;
+                nw[i] = in ? __ldg(a.row_weight + t.b_row + col) : 0.f;
+            }
+        };
+        if (kAhead && (int)blockIdx.x < total)
+            fetch_dest(tc_decode_unit<MODE, BN>(a, tabs, sc, blockIdx.x));
         int tc = 0;
         for (int item = blockIdx.x; item < total; item += gridDim.x, ++tc) {
             const TileInfo ti = tc_decode_unit<MODE, BN>(a, tabs, sc, item);
@@ -486,8 +512,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             tc_fence_after();
             const uint32_t tb = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(b * ACC);
             const int nchunks = (ti.n_valid + 31) >> 5;
-            if (MODE == kModeDown) {
+            if (kAhead) {
                 // each epilogue warp keeps its own copy: no barrier across warps
+                __syncwarp();
+#pragma unroll
+                for (int i = 0; i < kCPW; ++i) {
+                    const int col = (half + 2 * i) * 32 + lane;
+                    if (col < BN) {
+                        ep_dest[col] = nd[i];
+                        ep_wt[col] = nw[i];
+                    }
+                }
+                __syncwarp();
+                if (item + (int)gridDim.x < total)
+                    fetch_dest(tc_decode_unit<MODE, BN>(a, tabs, sc, item + gridDim.x));
+            } else if (MODE == kModeDown) {
                 __syncwarp();
                 for (int c = lane; c < ti.n_valid; c += 32) {
                     ep_dest[c] = __ldg(a.row_dest + ti.b_row + c);

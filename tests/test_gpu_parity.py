@@ -261,6 +261,17 @@ def test_forward_shared_expert_and_residual(path):
     compare_block(cfg, L2, G2, range(200), path=path, what=f"ungated/{path}")
 
 
+@pytest.mark.parametrize("T", [2, 5, 9])
+def test_forward_split_tail_with_shared_expert(T):
+    """Decode-sized batches whose expert GEMMs split their last items along K (a few dozen
+    items on 148 SMs): gate_up over D = 512 (8 K stages, split 3 or 4 ways: uneven slices),
+    down over I = 256 and the shared expert's I_s = 128 (the split is bounded by the shared
+    segment's 2 K stages), with the gated shared expert and a residual."""
+    cfg, L, G = _small_layer(T, D=512, E=64, k=4, I=256, I_s=128)
+    res = torch.randn(T, 512, generator=torch.Generator().manual_seed(7)).to(torch.bfloat16)
+    compare_block(cfg, L, G, range(T), path="grouped", residual_cpu=res, what=f"split tail T={T}")
+
+
 @pytest.mark.parametrize("path", ["stream", "grouped"])
 def test_forward_zero_input(path):
     cfg, L, G = _small_layer(40)
