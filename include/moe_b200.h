@@ -171,6 +171,11 @@ moe_status moe_get_device_status(const void *ws, moe_stream_t stream);
 /* Static, human-readable name of a status. */
 const char *moe_status_string(moe_status s);
 
+/* The CUDA runtime error code (a cudaError_t value) of the most recent CUDA call that made a
+ * call of this library on the calling host thread return MOE_ERR_CUDA; 0 if there was none.
+ * For diagnostics only: it is not reset by successful calls. */
+int moe_last_cuda_error(void);
+
 #ifdef __cplusplus
 }
 #endif

@@ -66,6 +66,8 @@ def load():
         lib.moe_get_device_status.argtypes = [_vp, _vp]
         lib.moe_status_string.argtypes = [_c_int]
         lib.moe_status_string.restype = ctypes.c_char_p
+        lib.moe_last_cuda_error.argtypes = []
+        lib.moe_last_cuda_error.restype = _c_int
         for n in ("moe_route", "moe_permute", "moe_forward", "moe_forward_ex", "moe_forward_noalloc",
                   "moe_get_device_status"):
             getattr(lib, n).restype = _c_int
@@ -87,8 +89,14 @@ def status_string(status: int) -> str:
 moe_status_string = status_string
 
 
+def moe_last_cuda_error() -> int:
+    return int(load().moe_last_cuda_error())
+
+
 def _check(status, what):
     if status != MOE_OK:
+        if status == MOE_ERR_CUDA:
+            what = f"{what} (cudaError {moe_last_cuda_error()})"
         raise MoeError(status, what)
 
 

@@ -43,9 +43,13 @@ namespace moe {
 enum { kModeGateUp = 0, kModeDown = 1, kModeRouter = 2 };
 
 // One kernel configuration: mode, token columns per tile and pipeline depth.
-template <int MODE, int BN_, int STAGES_>
+template <int MODE, int BN_, int STAGES_, bool PAIR_ = false>
 struct TcCfg {
     static constexpr int BN = BN_, STAGES = STAGES_;
+    // PAIR: two CTAs of a cluster share M = 256 MMAs; each holds 128 weight rows and half of
+    // the tile's BN token rows (BNC), and its TMEM holds its 128 rows over all BN columns
+    static constexpr bool PAIR = PAIR_;
+    static constexpr int BNC = PAIR ? BN / 2 : BN;
     // gate_up: narrow tiles keep gate and up in two accumulators (two A tiles per stage);
     // wide tiles interleave them in one A tile and one accumulator
     static constexpr bool IL = MODE == kModeGateUp && BN > kNarrowBN;
@@ -56,7 +60,7 @@ struct TcCfg {
                               : 2 * ACC <= 256 ? 256 : 512;
     static_assert(2 * ACC <= 512, "accumulators exceed TMEM");
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "token tile");
-    static constexpr int SB = NA * (kTcM * kTcK * 2) + BN * kTcK * 2;  // bytes per stage
+    static constexpr int SB = NA * (kTcM * kTcK * 2) + BNC * kTcK * 2;  // bytes per stage
     static constexpr int SMEM = STAGES * SB + 1024 + 256 + (int)sizeof(SmemTables) +
                                 (MODE == kModeDown ? 8 * 2 * 4 * BN : 0);
     static_assert(2 * STAGES + 5 <= 31, "barriers exceed their 256-byte region");
@@ -104,9 +108,8 @@ __device__ __forceinline__ int tc_total_items(const TcArgs& a, const SmemTables*
 }
 
 template <int MODE, int BN, bool SPLIT>
-__device__ __forceinline__ Sched tc_schedule(const TcArgs& a, const SmemTables* st) {
+__device__ __forceinline__ Sched tc_schedule(const TcArgs& a, const SmemTables* st, int G) {
     Sched sc;
-    const int G = gridDim.x;
     sc.n = tc_total_items<MODE, BN>(a, st);
     sc.full = sc.n / G * G;
     sc.S = 1;
@@ -130,8 +133,12 @@ __device__ __forceinline__ int box_index(int n) {
     return bi;
 }
 
-template <int MODE, int BN>
-__device__ __forceinline__ TileInfo tc_decode_item(const TcArgs& a, const SmemTables* st, int item) {
+// Work item -> tile.  PAIR: the pair's tile covers 128 features (gate_up) or 256 down rows
+// and up to BN tokens; `rank` selects this CTA's half of the weight rows (its m0 and A rows);
+// b_row and n_valid describe the whole tile, bi the per-CTA token box (half the tile's rows).
+template <int MODE, int BN, bool PAIR = false>
+__device__ __forceinline__ TileInfo tc_decode_item(const TcArgs& a, const SmemTables* st, int item,
+                                                   int rank = 0) {
     TileInfo ti;
     ti.k0 = 0;
     ti.split = 0;
@@ -159,15 +166,16 @@ __device__ __forceinline__ TileInfo tc_decode_item(const TcArgs& a, const SmemTa
     const int local = item - st->prefix[s];
     const int sh = (s == a.E);
     const int Iseg = sh ? a.I_s : a.I;
-    const int fpt = (MODE == kModeGateUp && BN > kNarrowBN) ? kGuILFeatures : kTcM;  // per tile
-    const int mtc = (MODE == kModeGateUp) ? Iseg / fpt : a.D / kTcM;
+    // weight rows per tile: features (gate_up) or down rows; the pair's tile is twice a CTA's
+    const int fpt = (MODE == kModeGateUp && BN > kNarrowBN) ? kGuILFeatures : kTcM;
+    const int mtc = (MODE == kModeGateUp) ? Iseg / (fpt * (PAIR ? 2 : 1)) : a.D / (kTcM * (PAIR ? 2 : 1));
     const int tt = local / mtc, mt = local % mtc;
     const int cnt = st->count[s];
     const int start = st->start[s];
     ti.shared = sh;
     ti.b_row = start + tt * BN;
     ti.n_valid = min(BN, cnt - tt * BN);
-    ti.m0 = mt * fpt;
+    ti.m0 = (MODE == kModeGateUp) ? (mt * (PAIR ? 2 : 1) + rank) * fpt : (mt * (PAIR ? 2 : 1) + rank) * kTcM;
     if (MODE == kModeGateUp && BN > kNarrowBN) {
         // interleaved: 64 features [m0, m0+64) of expert s, as four 16-feature groups
         ti.a_row0 = ti.m0 / 16;
@@ -180,20 +188,20 @@ __device__ __forceinline__ TileInfo tc_decode_item(const TcArgs& a, const SmemTa
         ti.nk = a.D / kTcK;
     } else {
         const int base = sh ? 0 : s * a.D;
-        ti.a_row0 = base + mt * kTcM;
+        ti.a_row0 = base + ti.m0;
         ti.a_row1 = 0;
         ti.nk = Iseg / kTcK;
     }
-    ti.bi = box_index<BN>(ti.n_valid);
+    ti.bi = PAIR ? box_index<BN / 2>((ti.n_valid + 1) / 2) : box_index<BN>(ti.n_valid);
     return ti;
 }
 
-template <int MODE, int BN>
+template <int MODE, int BN, bool PAIR = false>
 __device__ __forceinline__ TileInfo tc_decode_unit(const TcArgs& a, const SmemTables* st,
-                                                   const Sched& sc, int u) {
-    if (sc.S == 1 || u < sc.full) return tc_decode_item<MODE, BN>(a, st, u);
+                                                   const Sched& sc, int u, int rank = 0) {
+    if (sc.S == 1 || u < sc.full) return tc_decode_item<MODE, BN, PAIR>(a, st, u, rank);
     const int tail = (u - sc.full) / sc.S, split = (u - sc.full) % sc.S;
-    TileInfo ti = tc_decode_item<MODE, BN>(a, st, sc.full + tail);
+    TileInfo ti = tc_decode_item<MODE, BN, PAIR>(a, st, sc.full + tail, rank);
     const int nkt = ti.nk;
     ti.k0 = split * nkt / sc.S;
     ti.nk = (split + 1) * nkt / sc.S - ti.k0;
@@ -213,10 +221,10 @@ __device__ __forceinline__ void tma_load(void* dst, const CUtensorMap* map, uint
         : "memory");
 }
 
-template <int MODE, int BN, int STAGES>
+template <int MODE, int BN, int STAGES, bool PAIR = false>
 __global__ void __launch_bounds__(kTcThreads, 1)
     tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
-    using Tr = TcCfg<MODE, BN, STAGES>;
+    using Tr = TcCfg<MODE, BN, STAGES, PAIR>;
     constexpr int NA = Tr::NA, ACC = Tr::ACC;
     constexpr bool SPLIT = MODE != kModeRouter && BN <= kNarrowBN;
     constexpr int SB = Tr::SB;
@@ -235,6 +243,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     float* ep_wt_all = reinterpret_cast<float*>(ep_dest_all + kEpiWarps * BN);  // [8][BN]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // work units are handed to CTAs, or (PAIR) to the clusters of two CTAs, round-robin
+    const int rank = PAIR ? (int)cluster_ctarank() : 0;
+    const int ublk = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+    const int ugrid = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
 
     // prologue: independent of earlier kernels, overlaps them under launch chaining
     if (threadIdx.x == 0) {
@@ -244,7 +256,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(tfull + b, 1);
-            mbar_init(tempty + b, kEpiWarps * 32);
+            mbar_init(tempty + b, (PAIR ? 2 : 1) * kEpiWarps * 32);  // PAIR: both CTAs' epilogues
         }
         mbar_init(drain, 1);
         mbar_fence_init();
@@ -253,7 +265,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const CUtensorMap* m = lane == 0 ? &maps.A : (lane == 1 ? &maps.A_shared : &maps.B[lane - 2]);
         tma_prefetch_desc(m);
     }
-    if (warp == 1) tmem_alloc(tmem_slot, Tr::TMEM);
+    if (warp == 1) {
+        if (PAIR)
+            tmem_alloc_pair(tmem_slot, Tr::TMEM);
+        else
+            tmem_alloc(tmem_slot, Tr::TMEM);
+    }
     if (MODE == kModeDown) {
         // The work tables come from the permutation, two kernels back: it completed before
         // the gate_up kernel (this kernel's predecessor) passed its own dependency wait,
@@ -262,8 +279,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         // depend on gate_up -- is requested into L2 while gate_up finishes.
         load_tables(tabs, a.tables.dn_items, a.tables.seg_count, a.tables.seg_start, a.nseg);
         __syncthreads();
-        if (warp == 0 && lane == 0 && (int)blockIdx.x < tabs->prefix[a.nseg]) {
-            const TileInfo t0 = tc_decode_item<MODE, BN>(a, tabs, blockIdx.x);
+        if (warp == 0 && lane == 0 && ublk < tabs->prefix[a.nseg]) {
+            const TileInfo t0 = tc_decode_item<MODE, BN, PAIR>(a, tabs, ublk, rank);
             const CUtensorMap* mA = t0.shared ? &maps.A_shared : &maps.A;
             for (int kb = 0; kb < t0.nk; ++kb) tma_prefetch_l2(mA, kb * kTcK, t0.a_row0);
         }
@@ -273,13 +290,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (MODE == kModeGateUp)
         load_tables(tabs, a.tables.gu_items, a.tables.seg_count, a.tables.seg_start, a.nseg);
     tc_fence_before();
-    __syncthreads();
+    if (PAIR)
+        cluster_sync_all();   // both CTAs' barriers exist before any cross-CTA arrive or load
+    else
+        __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
-    const Sched sc = tc_schedule<MODE, BN, SPLIT>(a, tabs);
+    const Sched sc = tc_schedule<MODE, BN, SPLIT>(a, tabs, ugrid);
     const int total = sc.units;
 
-    if ((int)blockIdx.x >= total) {
+    if (ublk >= total) {
         // no work for this CTA: nothing was issued; fall through to the TMEM release
     } else if (warp == 0) {
         // ------------------------------------------------------------ TMA producer warp
@@ -287,7 +307,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         // rows from x by row_token, lane i taking rows 4i..4i+3 of the tile (rows past the
         // segment repeat its last row; their columns are never used); otherwise lane 0 loads
         // a tile of the permuted rows.
-        const int first = blockIdx.x, step = gridDim.x;   // this CTA's units
+        const int first = ublk, step = ugrid;   // this CTA's (pair's) units
         int it = 0;
         bool ok = true;
         int last_round[STAGES];
@@ -304,20 +324,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         TileInfo tn{};
         int gn[4] = {0, 0, 0, 0};
         if (first < total) {
-            tn = tc_decode_unit<MODE, BN>(a, tabs, sc, first);
+            tn = tc_decode_unit<MODE, BN, PAIR>(a, tabs, sc, first, rank);
             if (gather) gather_rows(tn, gn);
         }
         for (int item = first; item < total && ok; item += step) {
             const TileInfo ti = tn;
             const int g0 = gn[0], g1 = gn[1], g2 = gn[2], g3 = gn[3];
             if (item + step < total) {
-                tn = tc_decode_unit<MODE, BN>(a, tabs, sc, item + step);
+                tn = tc_decode_unit<MODE, BN, PAIR>(a, tabs, sc, item + step, rank);
                 if (gather) gather_rows(tn, gn);
             }
             const CUtensorMap* mA = ti.shared ? &maps.A_shared : &maps.A;
             const CUtensorMap* mB = &maps.B[ti.bi];
             const int brows = 16 << ti.bi;
-            const uint32_t bytes = NA * kATileBytes + (uint32_t)brows * kTcK * 2;
+            // PAIR: the leader's barrier counts both CTAs' bytes (same geometry in each)
+            const uint32_t bytes = (PAIR ? 2u : 1u) * (NA * kATileBytes + (uint32_t)brows * kTcK * 2);
             for (int kb = 0; kb < ti.nk; ++kb, ++it) {
                 const int s = it % STAGES;
                 const int round = it / STAGES;
@@ -327,7 +348,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     break;
                 }
                 uint8_t* st = smem + s * SB;
-                if (lane == 0) {
+                if (PAIR && lane == 0) {
+                    // both CTAs load their halves; completion is counted by the leader
+                    if (rank == 0) mbar_arrive_expect_tx(full + s, bytes);
+                    const uint32_t fb = mapa_shared(full + s, 0);
+                    const int kx = (ti.k0 + kb) * kTcK;
+                    if (Tr::IL)
+                        tma_load_5d_pair(st, mA, fb, kx, 0, 0, ti.a_row0, ti.a_row1);
+                    else
+                        tma_load_2d_pair(st, mA, fb, kx, ti.a_row0);
+                    tma_load_2d_pair(st + NA * kATileBytes, mB, fb, kx, ti.b_row + rank * brows);
+                } else if (!PAIR && lane == 0) {
                     mbar_arrive_expect_tx(full + s, bytes);
                     const int kx = (ti.k0 + kb) * kTcK;
                     if (Tr::IL)
@@ -358,13 +389,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 if (!__all_sync(0xffffffffu, got)) break;
             }
         }
+        // (PAIR: a released stage implies its loads landed; the full barriers are the leader's)
+        if (!PAIR) {
 #pragma unroll
-        for (int s = 0; s < STAGES; ++s)
-            if (last_round[s] >= 0) mbar_wait(full + s, last_round[s] & 1, a.err, kErrWaitTail);
+            for (int s = 0; s < STAGES; ++s)
+                if (last_round[s] >= 0) mbar_wait(full + s, last_round[s] & 1, a.err, kErrWaitTail);
+        }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            const uint32_t idesc0 = umma_idesc_bf16_f32(kTcM, 16) & ~(0x3Fu << 17);
+        // (PAIR: the leader CTA's thread issues the pair's M = 256 MMAs)
+        if (lane == 0 && rank == 0) {
+            const uint32_t idesc0 = umma_idesc_bf16_f32(PAIR ? 2 * kTcM : kTcM, 16) & ~(0x3Fu << 17);
             // shared-memory descriptors of stage 0; stage s adds s * SB / 16 to the address
             // field (stages stay below 256 KB, so the 14-bit field does not carry)
             const uint64_t dA0 = umma_desc_sw128(smem);
@@ -373,8 +408,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             int s = 0, phase = 0;   // ring position of the next stage
             int tc = 0;
             bool ok = true;
-            for (int item = blockIdx.x; item < total && ok; item += gridDim.x, ++tc) {
-                const TileInfo ti = tc_decode_unit<MODE, BN>(a, tabs, sc, item);
+            for (int item = ublk; item < total && ok; item += ugrid, ++tc) {
+                const TileInfo ti = tc_decode_unit<MODE, BN, PAIR>(a, tabs, sc, item, rank);
                 const int b = tc & 1;
                 const int use = tc >> 1;
                 if (!mbar_wait(tempty + b, (use & 1) ^ 1, a.err, kErrWaitMma)) {
@@ -384,6 +419,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 tc_fence_after();
                 int n = (ti.n_valid + 15) & ~15;
                 n = n < 16 ? 16 : (n > BN ? BN : n);
+                if (PAIR) n = 2 * (16 << ti.bi);   // both CTAs' token boxes
                 const uint32_t idesc = idesc0 | ((uint32_t)(n >> 3) << 17);
                 const uint32_t d0 = tmem_base + (uint32_t)(b * ACC);
                 for (int kb = 0; kb < ti.nk; ++kb) {
@@ -394,24 +430,38 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     tc_fence_after();
                     const uint64_t off = (uint64_t)(s * (SB >> 4));
                     const uint64_t da0 = dA0 + off, da1 = dA1 + off, db = dB + off;
-                    umma_bf16(d0, da0, db, idesc, kb);  // the tile's first MMA overwrites D
-                    if (NA == 2) umma_bf16(d0 + BN, da1, db, idesc, kb);
+                    if (PAIR) {
+                        umma_bf16_pair(d0, da0, db, idesc, kb);
 #pragma unroll
-                    for (int kk = 1; kk < kTcK / 16; ++kk) {
-                        umma_bf16_acc(d0, da0 + 2 * kk, db + 2 * kk, idesc);
-                        if (NA == 2) umma_bf16_acc(d0 + BN, da1 + 2 * kk, db + 2 * kk, idesc);
+                        for (int kk = 1; kk < kTcK / 16; ++kk)
+                            umma_bf16_pair_acc(d0, da0 + 2 * kk, db + 2 * kk, idesc);
+                        umma_commit_pair_both(empty + s);   // frees the stage in both CTAs
+                    } else {
+                        umma_bf16(d0, da0, db, idesc, kb);  // the tile's first MMA overwrites D
+                        if (NA == 2) umma_bf16(d0 + BN, da1, db, idesc, kb);
+#pragma unroll
+                        for (int kk = 1; kk < kTcK / 16; ++kk) {
+                            umma_bf16_acc(d0, da0 + 2 * kk, db + 2 * kk, idesc);
+                            if (NA == 2) umma_bf16_acc(d0 + BN, da1 + 2 * kk, db + 2 * kk, idesc);
+                        }
+                        umma_commit(empty + s);
                     }
-                    umma_commit(empty + s);
                     if (++s == STAGES) {
                         s = 0;
                         phase ^= 1;
                     }
                 }
                 if (!ok) break;
-                umma_commit(tfull + b);
+                if (PAIR)
+                    umma_commit_pair_both(tfull + b);
+                else
+                    umma_commit(tfull + b);
             }
             // every issued MMA must be complete before TMEM is released
-            umma_commit(drain);
+            if (PAIR)
+                umma_commit_pair_local(drain);
+            else
+                umma_commit(drain);
             mbar_wait(drain, 0, a.err, kErrWaitMma);
         }
     } else {
@@ -500,11 +550,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 nw[i] = in ? __ldg(a.row_weight + t.b_row + col) : 0.f;
             }
         };
-        if (kAhead && (int)blockIdx.x < total)
-            fetch_dest(tc_decode_unit<MODE, BN>(a, tabs, sc, blockIdx.x));
+        if (kAhead && ublk < total)
+            fetch_dest(tc_decode_unit<MODE, BN, PAIR>(a, tabs, sc, ublk, rank));
         int tc = 0;
-        for (int item = blockIdx.x; item < total; item += gridDim.x, ++tc) {
-            const TileInfo ti = tc_decode_unit<MODE, BN>(a, tabs, sc, item);
+        // PAIR: the accumulator is released on the leader's barrier by both CTAs
+        const uint32_t tempty_leader0 = PAIR ? mapa_shared(tempty, 0) : 0u;
+        for (int item = ublk; item < total; item += ugrid, ++tc) {
+            const TileInfo ti = tc_decode_unit<MODE, BN, PAIR>(a, tabs, sc, item, rank);
             const int b = tc & 1;
             const int use = tc >> 1;
             const bool got = mbar_wait(tfull + b, use & 1, a.err, kErrWaitEpilogue);
@@ -524,8 +576,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     }
                 }
                 __syncwarp();
-                if (item + (int)gridDim.x < total)
-                    fetch_dest(tc_decode_unit<MODE, BN>(a, tabs, sc, item + gridDim.x));
+                if (item + ugrid < total)
+                    fetch_dest(tc_decode_unit<MODE, BN, PAIR>(a, tabs, sc, item + ugrid, rank));
             } else if (MODE == kModeDown) {
                 __syncwarp();
                 for (int c = lane; c < ti.n_valid; c += 32) {
@@ -607,44 +659,84 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 finish_chunk(ti, c, v, u);
             }
             tc_fence_before();
-            mbar_arrive(tempty + b);
+            if (PAIR)
+                mbar_arrive_cluster(tempty_leader0 + 8u * b);
+            else
+                mbar_arrive(tempty + b);
         }
     }
     tc_fence_before();
-    __syncthreads();
+    if (PAIR)
+        cluster_sync_all();   // the leader's MMAs into the peer's TMEM are complete
+    else
+        __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, Tr::TMEM);
+        if (PAIR)
+            tmem_dealloc_pair(tmem_base, Tr::TMEM);
+        else
+            tmem_dealloc(tmem_base, Tr::TMEM);
     }
 }
 
-template <int MODE, int BN, int STAGES>
-static cudaError_t launch_tc(const TcMaps& maps, const TcArgs& a, int grid, int attr_slot, bool pdl,
+template <int MODE, int BN, int STAGES, bool PAIR = false>
+static cudaError_t launch_tc(const TcMaps& maps, const TcArgs& a, int grid, bool pdl,
                              cudaStream_t s) {
-    constexpr int smem = TcCfg<MODE, BN, STAGES>::SMEM;
-    cudaError_t err = ensure_smem_attr((const void*)tc_gemm_kernel<MODE, BN, STAGES>, smem, attr_slot);
+    constexpr int smem = TcCfg<MODE, BN, STAGES, PAIR>::SMEM;
+    auto kernel = tc_gemm_kernel<MODE, BN, STAGES, PAIR>;
+    cudaError_t err = ensure_smem_attr((const void*)kernel, smem);
     if (err != cudaSuccess) return err;
     if (grid < 1) grid = 1;
-    return launch_kernel(tc_gemm_kernel<MODE, BN, STAGES>, dim3(grid), dim3(kTcThreads), smem, s, pdl,
-                         maps, a);
+    if (!PAIR) return launch_kernel(kernel, dim3(grid), dim3(kTcThreads), smem, s, pdl, maps, a);
+    // pairs: as many clusters of two as can be resident at once (persistent kernel)
+    static int clusters[64] = {0};
+    int dev = 0;
+    if ((err = cudaGetDevice(&dev)) != cudaSuccess) return err;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidValue;
+    if (clusters[dev] == 0) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(grid & ~1);
+        cfg.blockDim = dim3(kTcThreads);
+        cfg.dynamicSmemBytes = smem;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        if ((err = cudaOccupancyMaxActiveClusters(&n, kernel, &cfg)) != cudaSuccess) return err;
+        if (n < 1) return cudaErrorInvalidConfiguration;
+        clusters[dev] = n;
+    }
+    int pairs = grid / 2 < clusters[dev] ? grid / 2 : clusters[dev];
+    if (pairs < 1) pairs = 1;
+    return launch_kernel_cluster(kernel, dim3(2 * pairs), dim3(kTcThreads), smem, s, pdl, 2, maps, a);
 }
 
 cudaError_t launch_tc_router(const TcMaps& maps, const TcArgs& a, int num_sms, bool pdl,
                              cudaStream_t s) {
     const int items = ((a.T + kRtBN - 1) / kRtBN) * ((a.E + kTcM - 1) / kTcM) * a.ksplit;
-    return launch_tc<kModeRouter, kRtBN, kStages>(maps, a, items < num_sms ? items : num_sms, 3, pdl, s);
+    return launch_tc<kModeRouter, kRtBN, kStages>(maps, a, items < num_sms ? items : num_sms, pdl, s);
 }
 
-cudaError_t launch_tc_gate_up(const TcMaps& maps, const TcArgs& a, int num_sms, bool narrow, bool pdl,
+cudaError_t launch_tc_gate_up(const TcMaps& maps, const TcArgs& a, int num_sms, int tiles, bool pdl,
                               cudaStream_t s) {
-    if (narrow) return launch_tc<kModeGateUp, kNarrowBN, kGuNarrowStages>(maps, a, num_sms, 4, pdl, s);
-    return launch_tc<kModeGateUp, kGuBN, kStages>(maps, a, num_sms, 1, pdl, s);
+    if (tiles == kTilesNarrow)
+        return launch_tc<kModeGateUp, kNarrowBN, kGuNarrowStages>(maps, a, num_sms, pdl, s);
+    if (tiles == kTilesPair)
+        return launch_tc<kModeGateUp, kGuBN, kPairStages, true>(maps, a, num_sms, pdl, s);
+    return launch_tc<kModeGateUp, kGuBN, kStages>(maps, a, num_sms, pdl, s);
 }
 
-cudaError_t launch_tc_down(const TcMaps& maps, const TcArgs& a, int num_sms, bool narrow, bool pdl,
+cudaError_t launch_tc_down(const TcMaps& maps, const TcArgs& a, int num_sms, int tiles, bool pdl,
                            cudaStream_t s) {
-    if (narrow) return launch_tc<kModeDown, kNarrowBN, kDnNarrowStages>(maps, a, num_sms, 5, pdl, s);
-    return launch_tc<kModeDown, kDnBN, kStages>(maps, a, num_sms, 2, pdl, s);
+    if (tiles == kTilesNarrow)
+        return launch_tc<kModeDown, kNarrowBN, kDnNarrowStages>(maps, a, num_sms, pdl, s);
+    if (tiles == kTilesPair)
+        return launch_tc<kModeDown, kDnBN, kPairStages, true>(maps, a, num_sms, pdl, s);
+    return launch_tc<kModeDown, kDnBN, kStages>(maps, a, num_sms, pdl, s);
 }
 
 }  // namespace moe

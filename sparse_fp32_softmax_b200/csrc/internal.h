@@ -44,6 +44,13 @@ constexpr int kNarrowMaxMeanRows = 32;
 // rows, 8 gathers per stage.  Above, the TMA engine's cost per gather operation makes the
 // expert GEMM slower by more than a separate copy costs (measured on B200).
 constexpr int kGatherMaxT = 32;
+// Tile families of the expert GEMMs.  Pair tiles (wide shapes, D % 256 == 0): two CTAs of a
+// cluster share each tcgen05.mma of M = 256 (cta_group::2) -- 128 weight rows per SM, half
+// of the 256 token rows per SM -- which halves the shared-memory operand traffic per FLOP
+// of each SM; gate_up pair tiles cover 128 features, down pair tiles 256 output rows.
+enum { kTilesNarrow = 0, kTilesWide = 1, kTilesPair = 2 };
+constexpr int kPairStages = 6;   // 6 x (16 KB weights + 16 KB tokens) per CTA
+
 // Split tail items of the narrow-tile GEMMs: at most this many K slices per item, and
 // partial-sum slots for one wave (a tail is split only when it is at most half a wave, so
 // the tickets of at most kSplitSlots / 2 items x 8 epilogue warps are in use).
@@ -92,7 +99,8 @@ struct PermuteArgs {
     int cap;                  // rows available in row_* arrays
     SegTables tables;         // may be all-null (moe_permute alone)
     int gu_bn, dn_bn;         // token columns per gate_up / down tile (work-item tables)
-    int gu_features;          // features per gate_up tile (128 narrow, 64 interleaved)
+    int gu_features;          // features per gate_up tile (128 narrow or pair, 64 interleaved)
+    int dn_rows;              // output rows per down tile (128, or 256 for pair tiles)
     int* err;
 };
 
@@ -185,7 +193,7 @@ struct TcArgs {
 
 // Raise a kernel's dynamic shared-memory limit once per device (host-side attribute; done
 // outside stream capture by the first call on each device).
-cudaError_t ensure_smem_attr(const void* kernel, int bytes, int slot);
+cudaError_t ensure_smem_attr(const void* kernel, int bytes);
 
 // ---------------------------------------------------------------- launchers (return the
 // launch error, cudaSuccess when all kernels were enqueued).  pdl: launch the first kernel
@@ -205,9 +213,9 @@ cudaError_t launch_stream_gate_up(const StreamArgs& a, int max_rows, bool pdl, c
 cudaError_t launch_stream_down(const StreamArgs& a, int max_rows, bool pdl, cudaStream_t s);
 cudaError_t launch_tc_router(const TcMaps& maps, const TcArgs& a, int num_sms, bool pdl,
                              cudaStream_t s);
-cudaError_t launch_tc_gate_up(const TcMaps& maps, const TcArgs& a, int num_sms, bool narrow, bool pdl,
+cudaError_t launch_tc_gate_up(const TcMaps& maps, const TcArgs& a, int num_sms, int tiles, bool pdl,
                               cudaStream_t s);
-cudaError_t launch_tc_down(const TcMaps& maps, const TcArgs& a, int num_sms, bool narrow, bool pdl,
+cudaError_t launch_tc_down(const TcMaps& maps, const TcArgs& a, int num_sms, int tiles, bool pdl,
                            cudaStream_t s);
 cudaError_t launch_combine(const void* slots, int slots_bf16, int T, int D, int k, int has_shared,
                            const uint16_t* x, const uint16_t* shared_gate,

@@ -13,18 +13,28 @@ using namespace moe;
 
 namespace moe {
 
-cudaError_t ensure_smem_attr(const void* kernel, int bytes, int slot) {
+cudaError_t ensure_smem_attr(const void* kernel, int bytes) {
+    // once per (device, kernel): the attribute is a host-side setting, raised to the largest
+    // size any launch of that kernel asks for
+    struct Entry { int dev; const void* kernel; int bytes; };
     static std::mutex mu;
-    static unsigned char done[64][32] = {};
+    static Entry done[256];
+    static int n = 0;
     int dev = 0;
     cudaError_t err = cudaGetDevice(&dev);
     if (err != cudaSuccess) return err;
-    if (dev < 0 || dev >= 64 || slot < 0 || slot >= 32) return cudaErrorInvalidValue;
     std::lock_guard<std::mutex> lock(mu);
-    if (done[dev][slot]) return cudaSuccess;
+    for (int i = 0; i < n; ++i)
+        if (done[i].dev == dev && done[i].kernel == kernel && done[i].bytes >= bytes) return cudaSuccess;
     err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-    if (err == cudaSuccess) done[dev][slot] = 1;
-    return err;
+    if (err != cudaSuccess) return err;
+    for (int i = 0; i < n; ++i)
+        if (done[i].dev == dev && done[i].kernel == kernel) {
+            done[i].bytes = bytes;
+            return cudaSuccess;
+        }
+    if (n < 256) done[n++] = Entry{dev, kernel, bytes};
+    return cudaSuccess;
 }
 
 }  // namespace moe
@@ -32,6 +42,9 @@ cudaError_t ensure_smem_attr(const void* kernel, int bytes, int slot) {
 namespace {
 
 constexpr size_t kAlign = 256;
+
+// The cudaError_t of the last CUDA failure seen by this host thread (moe_last_cuda_error).
+thread_local int g_last_cuda_error = 0;
 constexpr int kRouterSmallMaxT = 64;     // below: CUDA-core router; above: tcgen05 router GEMM
 
 size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
@@ -126,11 +139,19 @@ moe_status check_opts(const moe_dims* d, const moe_opts* o) {
 int num_sms_of_current_device() {
     static int cache[64] = {0};
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) {
+        g_last_cuda_error = (int)e;
+        return 0;
+    }
     if (dev < 0 || dev >= 64) return 0;
     if (cache[dev] == 0) {
         int n = 0;
-        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+        e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) {
+            g_last_cuda_error = (int)e;
+            return 0;
+        }
         cache[dev] = n;
     }
     return cache[dev];
@@ -162,6 +183,7 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, ui
     CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) g_last_cuda_error = (int)cudaErrorInvalidValue;
     return r == CUDA_SUCCESS;
 }
 
@@ -179,6 +201,7 @@ bool make_map_gate_up_il(CUtensorMap* m, const void* base, uint64_t D, uint64_t 
     CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides,
                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) g_last_cuda_error = (int)cudaErrorInvalidValue;
     return r == CUDA_SUCCESS;
 }
 
@@ -202,7 +225,11 @@ T* at(void* ws, size_t off) {
 
 #define MOE_CUDA(expr)                                       \
     do {                                                     \
-        if ((expr) != cudaSuccess) return MOE_ERR_CUDA;      \
+        const cudaError_t e_ = (expr);                       \
+        if (e_ != cudaSuccess) {                             \
+            g_last_cuda_error = (int)e_;                     \
+            return MOE_ERR_CUDA;                             \
+        }                                                    \
     } while (0)
 
 // Stage events are recorded as external events so that, under stream capture, they become
@@ -262,6 +289,8 @@ size_t moe_workspace_size(const moe_dims* dims, const moe_opts* opts) {
     if (check_dims(dims) != MOE_OK || check_opts(dims, opts) != MOE_OK) return 0;
     return make_plan(*dims, opts).total;
 }
+
+int moe_last_cuda_error(void) { return g_last_cuda_error; }
 
 const char* moe_status_string(moe_status s) {
     switch (s) {
@@ -338,6 +367,7 @@ moe_status moe_permute(const int32_t* topk_idx, const float* topk_w, const moe_b
     a.gu_bn = kGuBN;
     a.dn_bn = kDnBN;
     a.gu_features = kGuILFeatures;
+    a.dn_rows = kTcM;
     a.err = at<int>(ws, p.err);
     // padding rows are only written per expert segment; rows past offsets[E] stay as given,
     // so mark every row as padding first
@@ -388,13 +418,21 @@ moe_status moe_forward_ex(const moe_bf16* x, const moe_bf16* W_r, const moe_bf16
     // T <= kGatherMaxT gathered from x (one-row box, tile::gather4), else a permuted copy.
     const bool narrow = use_narrow_tiles(p.T, p.k, p.E);
     const bool gather = p.T <= kGatherMaxT;
+    // Wide shapes: gate_up on CTA pairs; down on CTA pairs when its rows split into 256-row
+    // tiles and experts average at least 256 rows (measured on B200: with fewer rows the
+    // pair tiles' narrower N and halved item count cost more than the pairs save).
+    const int gu_tiles = narrow ? kTilesNarrow : kTilesPair;
+    const int dn_tiles = narrow ? kTilesNarrow
+                         : (p.D % 256 == 0 && (long long)p.T * p.k >= 256ll * p.E) ? kTilesPair
+                                                                                    : kTilesWide;
     const int gu_bn = narrow ? kNarrowBN : kGuBN;
     const int dn_bn = narrow ? kNarrowBN : kDnBN;
+    const int b_box_max = gu_tiles == kTilesPair ? kGuBN / 2 : gu_bn;   // token rows per CTA
     TcMaps mGu, mDn;
     if (!streaming) {
         uint16_t* h = at<uint16_t>(ws, p.h);
         const bool gu_b_ok = gather ? make_map(&mGu.B[0], x, p.D, p.T, 1)
-                                    : make_b_maps(mGu.B, at<uint16_t>(ws, p.x_perm), p.D, p.R, gu_bn);
+                                    : make_b_maps(mGu.B, at<uint16_t>(ws, p.x_perm), p.D, p.R, b_box_max);
         const bool gu_a_ok =
             narrow ? make_map(&mGu.A, W_gate_up, p.D, (uint64_t)p.E * 2 * p.I, kTcM) &&
                          make_map(&mGu.A_shared, sgu ? sgu : W_gate_up, p.D,
@@ -406,7 +444,7 @@ moe_status moe_forward_ex(const moe_bf16* x, const moe_bf16* W_r, const moe_bf16
             !gu_b_ok ||
             !make_map(&mDn.A, W_down, p.I, (uint64_t)p.E * p.D, kTcM) ||
             !make_map(&mDn.A_shared, sdn ? sdn : W_down, sdn ? p.I_s : p.I, p.D, kTcM) ||
-            !make_b_maps(mDn.B, h, p.ld_h, p.R, dn_bn))
+            !make_b_maps(mDn.B, h, p.ld_h, p.R, dn_tiles == kTilesPair ? kDnBN / 2 : dn_bn))
             return MOE_ERR_CUDA;
         if (gather)
             for (int bi = 1; bi < kNumBBoxes; ++bi) mGu.B[bi] = mGu.B[0];
@@ -447,7 +485,8 @@ moe_status moe_forward_ex(const moe_bf16* x, const moe_bf16* W_r, const moe_bf16
     pa.tables = tables_of(p, ws);
     pa.gu_bn = gu_bn;
     pa.dn_bn = dn_bn;
-    pa.gu_features = narrow ? kTcM : kGuILFeatures;
+    pa.gu_features = gu_tiles == kTilesWide ? kGuILFeatures : kTcM;
+    pa.dn_rows = dn_tiles == kTilesPair ? 2 * kTcM : kTcM;
     pa.err = err;
     // launch chaining between the forward's kernels (not across a stage-event record)
     const bool chain = !(opts && opts->n_stage_events == 6);
@@ -507,9 +546,9 @@ moe_status moe_forward_ex(const moe_bf16* x, const moe_bf16* W_r, const moe_bf16
         ta.tickets = at<int>(ws, p.tickets);
         ta.partial_slots = narrow ? kSplitSlots : 0;
         ta.err = err;
-        MOE_CUDA(launch_tc_gate_up(mGu, ta, sms, narrow, chain, s));
+        MOE_CUDA(launch_tc_gate_up(mGu, ta, sms, gu_tiles, chain, s));
         if ((st = record(opts, 3, s)) != MOE_OK) return st;
-        MOE_CUDA(launch_tc_down(mDn, ta, sms, narrow, chain, s));
+        MOE_CUDA(launch_tc_down(mDn, ta, sms, dn_tiles, chain, s));
         if ((st = record(opts, 4, s)) != MOE_OK) return st;
         MOE_CUDA(launch_combine(ta.slots, 0, p.T, p.D, p.k, p.has_shared, x, sg, residual, out,
                                 out_f32, chain, s));

@@ -101,12 +101,12 @@ cudaError_t launch_permute(const PermuteArgs& a, bool pdl, cudaStream_t s) {
     const size_t wb_bytes = 32 * (size_t)a.E * sizeof(int);
     if (a.nchunks == 1) {
         cudaError_t err = ensure_smem_attr((const void*)perm_fused_kernel,
-                                           32 * kMaxSegments * (int)sizeof(int), 6);
+                                           32 * kMaxSegments * (int)sizeof(int));
         if (err != cudaSuccess) return err;
         return launch_kernel(perm_fused_kernel, dim3(1), dim3(kPermThreads), wb_bytes, s, pdl, a);
     }
     cudaError_t err = ensure_smem_attr((const void*)perm_scatter_kernel,
-                                       32 * kMaxSegments * (int)sizeof(int), 0);
+                                       32 * kMaxSegments * (int)sizeof(int));
     if (err != cudaSuccess) return err;
     err = launch_kernel(perm_hist_kernel, dim3(a.nchunks), dim3(kPermThreads), a.E * sizeof(int), s,
                         pdl, a);

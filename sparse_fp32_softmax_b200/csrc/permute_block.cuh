@@ -65,7 +65,7 @@ static __device__ void finish_offsets(const PermuteArgs& a, const int* s_cnt, in
         if (c > 0) {
             const int Iseg = (s == E) ? a.I_s : a.I;
             v[1] = (c + a.gu_bn - 1) / a.gu_bn * (Iseg / a.gu_features);
-            v[2] = (c + a.dn_bn - 1) / a.dn_bn * (a.D / kTcM);
+            v[2] = (c + a.dn_bn - 1) / a.dn_bn * (a.D / a.dn_rows);
             v[3] = Iseg / 8;     // streaming gate_up: one warp per 8 features
             v[4] = a.D / 16;     // streaming down: one warp per 16 output rows
         }

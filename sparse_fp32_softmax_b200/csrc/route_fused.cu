@@ -81,8 +81,7 @@ cudaError_t launch_route_fused(const RouteArgs& a, bool pdl, cudaStream_t s) {
     void (*k_)(RouteArgs) = a.E <= 32 ? route_fused_kernel<1> : a.E <= 64 ? route_fused_kernel<2>
                           : a.E <= 128 ? route_fused_kernel<4> : a.E <= 256 ? route_fused_kernel<8>
                           : route_fused_kernel<16>;
-    const int slot = a.E <= 32 ? 0 : a.E <= 64 ? 1 : a.E <= 128 ? 2 : a.E <= 256 ? 3 : 4;
-    cudaError_t err = ensure_smem_attr((const void*)k_, (32 + kFusedRouteMaxT) * kMaxE * 4, 8 + slot);
+    cudaError_t err = ensure_smem_attr((const void*)k_, (32 + kFusedRouteMaxT) * kMaxE * 4);
     if (err != cudaSuccess) return err;
     const int blocks = a.E < 148 ? a.E : 148;
     return launch_kernel(k_, dim3(blocks), dim3(1024), smem, s, pdl, a);
@@ -122,8 +121,7 @@ cudaError_t launch_select_permute(const RouteArgs& a, bool pdl, cudaStream_t s) 
     void (*k_)(RouteArgs) = a.E <= 32 ? select_permute_kernel<1> : a.E <= 64 ? select_permute_kernel<2>
                           : a.E <= 128 ? select_permute_kernel<4> : a.E <= 256 ? select_permute_kernel<8>
                           : select_permute_kernel<16>;
-    const int slot = a.E <= 32 ? 0 : a.E <= 64 ? 1 : a.E <= 128 ? 2 : a.E <= 256 ? 3 : 4;
-    cudaError_t err = ensure_smem_attr((const void*)k_, 32 * kMaxE * 4, 16 + slot);
+    cudaError_t err = ensure_smem_attr((const void*)k_, 32 * kMaxE * 4);
     if (err != cudaSuccess) return err;
     return launch_kernel(k_, dim3((a.T + 31) / 32), dim3(1024), smem, s, pdl, a);
 }

@@ -27,7 +27,7 @@ def test_library_exports_every_declared_function(lib):
     declared = B.header_functions()
     assert set(declared) == {"moe_workspace_size", "moe_route", "moe_permute", "moe_forward",
                              "moe_forward_ex", "moe_forward_noalloc", "moe_get_device_status",
-                             "moe_status_string"}
+                             "moe_status_string", "moe_last_cuda_error"}
     out = subprocess.run(["nm", "-D", "--defined-only", LIB], capture_output=True, text=True, check=True).stdout
     exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
     for name in declared:
@@ -104,10 +104,11 @@ def test_forward_rejects_bad_arguments_before_launch(lib):
 
 @no_gpu
 def test_no_cpu_fallback(lib):
-    """With valid arguments and no GPU the library reports a CUDA failure; it never computes
-    anything on the host."""
+    """With valid arguments and no GPU the library reports a CUDA failure (and keeps the
+    CUDA error code for diagnostics); it never computes anything on the host."""
     d = B.make_dims(64, 256, 8, 2, 128)
     assert _fwd(lib, d, B.moe_workspace_size(d)) == B.MOE_ERR_CUDA
+    assert B.moe_last_cuda_error() != 0
     p = ctypes.c_void_p
     assert lib.moe_route(p(FAKE), p(FAKE), None, ctypes.byref(d), None, p(FAKE), p(FAKE),
                          p(FAKE), B.moe_workspace_size(d), None) == B.MOE_ERR_CUDA
