@@ -97,10 +97,12 @@ static __device__ void finish_offsets(const PermuteArgs& a, const int* s_cnt, in
     __syncthreads();
 }
 
-// Warp w of a block of W warps owns assignments [a0 + w*L, a0 + w*L + L), L = 4096 / W
-// (at most 256 = 8 rounds of 32), in rounds of 32 in increasing order.  A lane's experts
-// (and weights) of all rounds are loaded once, up front, so the passes below cost one memory
-// round trip instead of one per round.
+// Warp w of a block of W warps owns assignments [a0 + w*L, a0 + w*L + L) of the chunk's n_c
+// assignments (n_c <= 4096), L = ceil(n_c / W) rounded up to a multiple of 32 (at most 256 =
+// 8 rounds of 32), in rounds of 32 in increasing order: every warp gets a share, so the
+// serial rounds per warp are as few as the chunk allows.  A lane's experts (and weights) of
+// all rounds are loaded once, up front, so the passes below cost one memory round trip
+// instead of one per round.
 constexpr int kMaxRounds = 8;
 struct WarpSlice {
     int e[kMaxRounds];      // expert of the lane's assignment in each round (-1: none)
@@ -112,8 +114,10 @@ struct WarpSlice {
 static __device__ __forceinline__ WarpSlice load_warp_slice(const PermuteArgs& a, long a0) {
     WarpSlice ws;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int slice = kPermChunk / (blockDim.x >> 5);
     const long n = (long)a.T * a.k;
+    const long n_c = n - a0 < kPermChunk ? n - a0 : kPermChunk;   // this chunk's assignments
+    const int nwarps = blockDim.x >> 5;
+    const int slice = (int)((n_c + nwarps - 1) / nwarps + 31) / 32 * 32;
     ws.rounds = slice / 32;
     ws.w0 = a0 + (long)warp * slice;
 #pragma unroll
@@ -131,6 +135,20 @@ static __device__ __forceinline__ WarpSlice load_warp_slice(const PermuteArgs& a
     return ws;
 }
 
+// Lanes of the warp holding the same value as this lane (e in [-1, 1023]; -1 matches -1):
+// one ballot per bit of the 10-bit value.
+static __device__ __forceinline__ uint32_t match_expert(int e) {
+    const uint32_t v = (uint32_t)e & 0x3FFu;
+    uint32_t m = 0xffffffffu;
+#pragma unroll
+    for (int b = 0; b < 10; ++b) {
+        const uint32_t bit = (v >> b) & 1u;
+        const uint32_t bb = __ballot_sync(0xffffffffu, bit);
+        m &= bit ? bb : ~bb;
+    }
+    return m;
+}
+
 // Counting pass: wb[w*E + e] += assignments of e in the warp's slice.
 static __device__ void count_warp_slices(const PermuteArgs& a, const WarpSlice& ws, int* wb) {
     const int E = a.E;
@@ -140,7 +158,7 @@ static __device__ void count_warp_slices(const PermuteArgs& a, const WarpSlice& 
     for (int r = 0; r < kMaxRounds; ++r) {
         if (r >= ws.rounds) break;
         const int e = ws.e[r];
-        const uint32_t m = __match_any_sync(0xffffffffu, e);
+        const uint32_t m = match_expert(e);
         if (e >= 0 && (m & lt_mask) == 0) wb[warp * E + e] += __popc(m);
     }
 }
@@ -156,7 +174,7 @@ static __device__ void scatter_warp_slices(const PermuteArgs& a, const WarpSlice
         if (r >= ws.rounds) break;
         const int e = ws.e[r];
         const long as = ws.w0 + r * 32 + lane;
-        const uint32_t m = __match_any_sync(0xffffffffu, e);
+        const uint32_t m = match_expert(e);
         int base = 0;
         if (e >= 0) base = wb[warp * E + e];
         __syncwarp();
