@@ -83,6 +83,7 @@ struct TileInfo {
     int split;    // K slice index (router slices, or a split tail item's slice)
     int nsplit;   // > 1: tail item split over K, partial sums reduced by the last slice
     int tail;     // index of a split item among the tail items
+    int seg;      // segment (expert; E = the shared expert)
     int m0;       // first output feature of this tile within its segment
 };
 
@@ -144,6 +145,7 @@ __device__ __forceinline__ TileInfo tc_decode_item(const TcArgs& a, const SmemTa
     ti.split = 0;
     ti.nsplit = 1;
     ti.tail = 0;
+    ti.seg = 0;
     if (MODE == kModeRouter) {
         // consecutive items are the K splits of one tile
         const int mtc = (a.E + kTcM - 1) / kTcM;
@@ -164,6 +166,7 @@ __device__ __forceinline__ TileInfo tc_decode_item(const TcArgs& a, const SmemTa
     }
     const int s = find_segment_smem(st->prefix, a.nseg, item);
     const int local = item - st->prefix[s];
+    ti.seg = s;
     const int sh = (s == a.E);
     const int Iseg = sh ? a.I_s : a.I;
     // weight rows per tile: features (gate_up) or down rows; the pair's tile is twice a CTA's
@@ -209,6 +212,47 @@ __device__ __forceinline__ TileInfo tc_decode_unit(const TcArgs& a, const SmemTa
     ti.nsplit = sc.S;
     ti.tail = tail;
     return ti;
+}
+
+// gate_up -> down hand-off per expert (narrow tiles).  The signalling warp has written h
+// with ordinary stores; the down kernel reads h with TMA (the async proxy), hence the proxy
+// fence on both sides.
+__device__ __forceinline__ void signal_segment_done(const TcArgs& a, int seg, int lane) {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+    __threadfence();
+    __syncwarp();
+    if (lane == 0) {
+        atomicAdd(a.seg_done + seg, 1);
+        atomicAdd(a.seg_done + a.nseg, 1);
+    }
+}
+
+__device__ __forceinline__ int ld_acquire(const int* p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Bounded wait of the down producer (one lane) until gate_up has finished segment seg.
+__device__ __forceinline__ bool wait_segment_done(const TcArgs& a, int seg, bool& all_done) {
+    if (all_done) return true;
+    const int all_target = 8 * __ldg(a.gu_prefix + a.nseg);
+    const int target = 8 * (__ldg(a.gu_prefix + seg + 1) - __ldg(a.gu_prefix + seg));
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+        if (ld_acquire(a.seg_done + a.nseg) >= all_target) {
+            all_done = true;
+            break;
+        }
+        if (ld_acquire(a.seg_done + seg) >= target) break;
+        __nanosleep(128);
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            set_error(a.err, kErrWaitProducer);
+            return false;
+        }
+    }
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+    return true;
 }
 
 // Plain 2-D TMA load without an L2 hint.
@@ -285,7 +329,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             for (int kb = 0; kb < t0.nk; ++kb) tma_prefetch_l2(mA, kb * kTcK, t0.a_row0);
         }
     }
-    pdl_wait();
+    // (down with per-expert hand-off: no wait for the whole gate_up grid; everything read
+    // below besides h was complete before this kernel could start -- see above)
+    if (!(MODE == kModeDown && a.dep_wait)) pdl_wait();
     pdl_launch_dependents();
     if (MODE == kModeGateUp)
         load_tables(tabs, a.tables.gu_items, a.tables.seg_count, a.tables.seg_start, a.nseg);
@@ -308,6 +354,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         // segment repeat its last row; their columns are never used); otherwise lane 0 loads
         // a tile of the permuted rows.
         const int first = ublk, step = ugrid;   // this CTA's (pair's) units
+        bool dep_all_done = false;
         int it = 0;
         bool ok = true;
         int last_round[STAGES];
@@ -333,6 +380,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             if (item + step < total) {
                 tn = tc_decode_unit<MODE, BN, PAIR>(a, tabs, sc, item + step, rank);
                 if (gather) gather_rows(tn, gn);
+            }
+            if (MODE == kModeDown && a.dep_wait) {
+                bool got = true;
+                if (lane == 0) got = wait_segment_done(a, ti.seg, dep_all_done);
+                if (!__shfl_sync(0xffffffffu, got, 0)) {
+                    ok = false;
+                    break;
+                }
             }
             const CUtensorMap* mA = ti.shared ? &maps.A_shared : &maps.A;
             const CUtensorMap* mB = &maps.B[ti.bi];
@@ -649,6 +704,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         finish_quad(ti, c, g, sv, su);
                     }
                 }
+                if (MODE == kModeGateUp && a.seg_done) signal_segment_done(a, ti.seg, lane);
                 continue;
             }
             for (int c = half; c < nchunks; c += 2) {
@@ -663,6 +719,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 mbar_arrive_cluster(tempty_leader0 + 8u * b);
             else
                 mbar_arrive(tempty + b);
+            if (MODE == kModeGateUp && !PAIR && a.seg_done) signal_segment_done(a, ti.seg, lane);
         }
     }
     tc_fence_before();

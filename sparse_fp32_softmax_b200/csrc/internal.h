@@ -56,7 +56,7 @@ constexpr int kPairStages = 6;   // 6 x (16 KB weights + 16 KB tokens) per CTA
 // the tickets of at most kSplitSlots / 2 items x 8 epilogue warps are in use).
 constexpr int kMaxKSplit = 8;
 constexpr int kSplitSlots = 148;
-constexpr int kSplitTickets = 1024;
+constexpr int kSplitTickets = 1024;   // per GEMM; the completion counters follow them
 __host__ __device__ inline bool use_narrow_tiles(long long T, int k, int E) {
     return T * k <= (long long)kNarrowMaxMeanRows * E;
 }
@@ -184,6 +184,14 @@ struct TcArgs {
     float* partial;
     int* tickets;
     int partial_slots;
+    // Per-expert completion of gate_up (narrow tiles): gate_up's epilogue warps add 1 to
+    // seg_done[s] (and to seg_done[nseg]) once they have written their part of an item's h
+    // tile; with dep_wait, the down kernel does not wait for the whole gate_up grid but its
+    // producer waits until seg_done[s] reaches 8 x (gate_up items of segment s), read from
+    // gu_prefix, so down starts on finished experts while gate_up's last wave runs.
+    int* seg_done;
+    const int* gu_prefix;
+    int dep_wait;
     // dense (router) epilogue: partial sums over split s of K go to logits + s*T*E
     float* logits;            // [ksplit, T, E] FP32
     int ksplit;

@@ -72,9 +72,12 @@ Plan make_plan(const moe_dims& d, const moe_opts* o) {
     size_t off = 0;
     auto take = [&](size_t bytes) { size_t at = off; off += align_up(bytes); return at; };
     p.err = take(kAlign);                              // [0] error word, [1] routing ticket
-    p.tickets = take((size_t)kSplitTickets * 4);       // split-tail tickets (follow err)
-    p.partial = take(use_narrow_tiles(p.T, p.k, p.E)   // split-tail partial accumulators
-                         ? (size_t)kSplitSlots * 2 * kTcM * kNarrowBN * 4 : 0);
+    // split-tail tickets of gate_up and of down, then the per-expert completion counters
+    // (all follow err, so one memset clears the header)
+    p.tickets = take((size_t)3 * kSplitTickets * 4);
+    // split-tail partial accumulators: gate_up (two accumulators), then down (one)
+    p.partial = take(use_narrow_tiles(p.T, p.k, p.E)
+                         ? (size_t)kSplitSlots * 3 * kTcM * kNarrowBN * 4 : 0);
     p.logits = take((size_t)p.rsplit * p.T * p.E * 4);   // router partial sums (or logits)
     p.idx = take((size_t)p.T * p.k * 4);
     p.w = take((size_t)p.T * p.k * 4);
@@ -451,7 +454,7 @@ moe_status moe_forward_ex(const moe_bf16* x, const moe_bf16* W_r, const moe_bf16
     }
 
     // the header of the workspace: device error word, routing ticket, split-tail tickets
-    MOE_CUDA(cudaMemsetAsync(err, 0, p.tickets - p.err + (size_t)kSplitTickets * 4, s));
+    MOE_CUDA(cudaMemsetAsync(err, 0, p.tickets - p.err + (size_t)3 * kSplitTickets * 4, s));
     if ((st = record(opts, 0, s)) != MOE_OK) return st;
     // T <= 32: one kernel routes and permutes.  Above: router partial sums, then selection and
     // permutation (one kernel while T*k fits a single permutation block).
@@ -545,10 +548,19 @@ moe_status moe_forward_ex(const moe_bf16* x, const moe_bf16* W_r, const moe_bf16
         ta.partial = narrow ? at<float>(ws, p.partial) : nullptr;
         ta.tickets = at<int>(ws, p.tickets);
         ta.partial_slots = narrow ? kSplitSlots : 0;
+        // narrow tiles: gate_up reports each finished expert; down waits per expert
+        ta.seg_done = narrow ? at<int>(ws, p.tickets) + 2 * kSplitTickets : nullptr;
+        ta.gu_prefix = pa.tables.gu_items;
+        TcArgs tdn = ta;
+        tdn.dep_wait = narrow ? 1 : 0;
+        if (narrow) {
+            tdn.partial = at<float>(ws, p.partial) + (size_t)kSplitSlots * 2 * kTcM * kNarrowBN;
+            tdn.tickets = at<int>(ws, p.tickets) + kSplitTickets;
+        }
         ta.err = err;
         MOE_CUDA(launch_tc_gate_up(mGu, ta, sms, gu_tiles, chain, s));
         if ((st = record(opts, 3, s)) != MOE_OK) return st;
-        MOE_CUDA(launch_tc_down(mDn, ta, sms, dn_tiles, chain, s));
+        MOE_CUDA(launch_tc_down(mDn, tdn, sms, dn_tiles, chain, s));
         if ((st = record(opts, 4, s)) != MOE_OK) return st;
         MOE_CUDA(launch_combine(ta.slots, 0, p.T, p.D, p.k, p.has_shared, x, sg, residual, out,
                                 out_f32, chain, s));
