@@ -381,6 +381,9 @@ def run_ours(args, rank, world, device):
     tag = ("stream_gate_up_" if streaming else "tc_gate_up_") + args.workload
     if tag == "tc_gate_up_prefill":
         tag = "tc_gemm_prefill"
+    # DRAM bytes of one launch from the committed ncu summary (null when there is none for
+    # this workload or the kernel source changed since it was taken)
+    roof["traffic"] = profile_traffic(tag)
     blk_time = max(blk_bytes / (peaks["hbm_gbs"] * 1e9), blk_flops / (peaks["bf16_tflops_sustained"] * 1e12))
 
     # end to end through the public API with host buffers (eager, copies inside the region)

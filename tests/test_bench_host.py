@@ -94,3 +94,8 @@ def test_peaks_and_profile_lookup(tmp_path, monkeypatch):
     assert bench.profile_traffic("tag") == 1234.0
     src.write_text("changed kernel")
     assert bench.profile_traffic("tag") is None
+
+
+def test_bench_attaches_traffic_to_the_roofline():
+    text = open(os.path.join(bench.ROOT, "bench.py")).read()
+    assert 'roof["traffic"] = profile_traffic(tag)' in text
