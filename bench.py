@@ -104,6 +104,20 @@ def profile_traffic(kernel_tag):
     return float(m.group(1))
 
 
+def kernels_per_forward(T, k, streaming):
+    """Kernels one moe_forward_ex call launches (the library's launch sequence): T <= 32 one
+    fused routing + permutation kernel; above, the router, then selection + permutation in
+    one kernel while T*k <= 4096 (else selection, histogram, scan and scatter), and the
+    permuted copy of x for the grouped path; then gate_up, down and the combine."""
+    n = 0
+    if T <= 32:
+        n += 1
+    else:
+        n += 1 + (1 if T * k <= 4096 else 4)
+        n += 0 if streaming else 1
+    return n + 3
+
+
 class ClockSampler:
     """Samples the SM clock and clock-event reasons of one GPU through NVML while running."""
 
@@ -325,7 +339,7 @@ def run_ours(args, rank, world, device):
             for j in range(5):
                 stage_ms[n][j] += e[j].elapsed_time(e[j + 1]) / K
     peaks = load_peaks()
-    launches_per_pass = [8 + (0 if (p["streaming"] or p["T"] <= 32) else 1) for p in passes]   # router 2, permute 3 (+ row copy), gate_up, down, combine
+    launches_per_pass = [kernels_per_forward(p["T"], cfg.k, p["streaming"]) for p in passes]
 
     # roofline of the dominant kernel: the gate_up expert kernel (stage 3).  Reported for
     # the workload's largest pass (one launch shape, the one a single ncu capture covers);
