@@ -107,7 +107,11 @@ size_t moe_workspace_size(const moe_dims *dims, const moe_opts *opts);
  *                  when dims->norm_topk_prob.
  * x [T, D] bf16, W_r [E, D] bf16 (nn.Linear layout), bias [E] FP32 or NULL,
  * logits [T, E] FP32 or NULL (then the workspace holds them), topk_idx [T, k] int32,
- * topk_w [T, k] FP32. */
+ * topk_w [T, k] FP32.
+ * Summation order: for T <= 64 each logit is one FP32 sum; above, D is summed in up to 8
+ * slices added in slice order, the number of slices fixed by (T, E, D).  Results are bitwise
+ * reproducible; a token's logits do not depend on the other tokens within one of those
+ * regimes. */
 moe_status moe_route(const moe_bf16 *x, const moe_bf16 *W_r, const float *bias,
                      const moe_dims *dims, float *logits, int32_t *topk_idx, float *topk_w,
                      void *ws, size_t ws_bytes, moe_stream_t stream);
@@ -134,7 +138,11 @@ moe_status moe_permute(const int32_t *topk_idx, const float *topk_w, const moe_b
 /* The whole block: out[t] = sum_j w[t,j] * expert_{idx[t,j]}(x[t]).
  * x [T, D] bf16, W_r [E, D] bf16, W_gate_up [E, 2I, D] bf16 (gate rows 0..I-1, up rows
  * I..2I-1), W_down [E, D, I] bf16, out [T, D] bf16 (fully overwritten; must not alias x).
- * The k weighted outputs are summed in slot order in FP32 and rounded once to bf16. */
+ * The k weighted outputs are summed in slot order in FP32 and rounded once to bf16.
+ * Results are bitwise reproducible for the same inputs.  At decode shapes (T*k <= 32*E) the
+ * expert GEMMs may split the K sums of their last items into slices (added in slice order),
+ * and how many depends on the batch's work, so a token's output can differ in the last bits
+ * between batches (its routing does not, see moe_route). */
 moe_status moe_forward(const moe_bf16 *x, const moe_bf16 *W_r, const moe_bf16 *W_gate_up,
                        const moe_bf16 *W_down, const moe_dims *dims, moe_bf16 *out, void *ws,
                        size_t ws_bytes, moe_stream_t stream);
