@@ -17,13 +17,13 @@ namespace moe {
 // (T <= 32), one warp per (expert, token) pair, with the same exact-product FP32
 // accumulation as the small-T router.  Logits go to global memory; each block then takes an
 // atomic ticket after a fence, and the block that draws the last ticket sees every block's
-// logits: it selects all tokens (one warp per token) and performs the whole permutation.
+// logits (read through L2): it selects all tokens (one warp per token) and performs the whole
+// permutation.
 // One launch replaces the router, the selection and the permutation kernels.
 template <int VPL>
 __global__ void __launch_bounds__(1024) route_fused_kernel(RouteArgs a) {
     extern __shared__ int route_smem[];
     int* wb = route_smem;                                               // [32][E] (last block)
-    float* lg = reinterpret_cast<float*>(route_smem + 32 * a.E);        // [T][E] (last block)
     __shared__ int s_ticket;
     pdl_wait();
     pdl_launch_dependents();
@@ -66,22 +66,20 @@ __global__ void __launch_bounds__(1024) route_fused_kernel(RouteArgs a) {
     __syncthreads();
     if (s_ticket != (int)gridDim.x - 1) return;
     __threadfence();
-    for (int i = threadIdx.x; i < T * E; i += blockDim.x) lg[i] = __ldcg(a.logits_out + i);
-    __syncthreads();
     for (int t = warp; t < T; t += 32)
-        select_token<VPL>(lg + t * E, 1, 0, nullptr, E, a.k, a.norm, a.topk_idx + (size_t)t * a.k,
-                          a.topk_w + (size_t)t * a.k, nullptr);
+        select_token<VPL, true>(a.logits_out + (size_t)t * E, 1, 0, nullptr, E, a.k, a.norm,
+                                a.topk_idx + (size_t)t * a.k, a.topk_w + (size_t)t * a.k, nullptr);
     __syncthreads();
     permute_one_block(a.perm, wb);
 }
 
 cudaError_t launch_route_fused(const RouteArgs& a, bool pdl, cudaStream_t s) {
     if (a.T > kFusedRouteMaxT) return cudaErrorInvalidValue;
-    const int smem = (32 + a.T) * a.E * 4;
+    const int smem = 32 * a.E * 4;
     void (*k_)(RouteArgs) = a.E <= 32 ? route_fused_kernel<1> : a.E <= 64 ? route_fused_kernel<2>
                           : a.E <= 128 ? route_fused_kernel<4> : a.E <= 256 ? route_fused_kernel<8>
                           : route_fused_kernel<16>;
-    cudaError_t err = ensure_smem_attr((const void*)k_, (32 + kFusedRouteMaxT) * kMaxE * 4);
+    cudaError_t err = ensure_smem_attr((const void*)k_, 32 * kMaxE * 4);
     if (err != cudaSuccess) return err;
     const int blocks = a.E < 148 ? a.E : 148;
     return launch_kernel(k_, dim3(blocks), dim3(1024), smem, s, pdl, a);

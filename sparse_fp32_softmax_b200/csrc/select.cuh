@@ -21,7 +21,10 @@ __device__ __forceinline__ float float_from_order_key(uint32_t o) {
 // order-preserving key of their logit; among equal keys the lower index wins: each round,
 // one warp-wide max over the keys, then one over the complemented indices of the lanes
 // holding that key.
-template <int VPL>
+// L2_LOADS: the partial rows were written by other blocks of the running kernel, so they
+// are read through L2 (ld.global.cg); otherwise with generic loads (shared memory, or
+// global memory written by an earlier kernel).
+template <int VPL, bool L2_LOADS = false>
 __device__ __forceinline__ void select_token(const float* part, int nsplit, size_t split_stride,
                                              const float* bias, int E, int k, int norm,
                                              int32_t* idx_out, float* w_out, float* logits_out) {
@@ -30,7 +33,7 @@ __device__ __forceinline__ void select_token(const float* part, int nsplit, size
 #pragma unroll
     for (int i = 0; i < VPL; ++i) {
         const int e = lane + 32 * i;
-        v[i] = e < E ? part[e] : 0.f;  // generic loads: part may be shared or global memory
+        v[i] = e < E ? (L2_LOADS ? __ldcg(part + e) : part[e]) : 0.f;
     }
 #pragma unroll
     for (int sp = 1; sp < kRouterMaxSplit; ++sp) {  // loads of all partials in flight together

@@ -261,6 +261,14 @@ def test_forward_shared_expert_and_residual(path):
     compare_block(cfg, L2, G2, range(200), path=path, what=f"ungated/{path}")
 
 
+@pytest.mark.parametrize("T", [5, 300])
+def test_forward_dims_not_multiple_of_256(T):
+    """D = I = 384: gate_up K and feature tiles of 128 (pair tiles at T = 300), down rows not a
+    multiple of 256 (the one-CTA wide down tiles at T = 300, narrow tiles at T = 5)."""
+    cfg, L, G = _small_layer(T, D=384, E=16, k=4, I=384)
+    compare_block(cfg, L, G, range(T), path="grouped", what=f"D=I=384 T={T}")
+
+
 @pytest.mark.parametrize("T", [2, 5, 9])
 def test_forward_split_tail_with_shared_expert(T):
     """Decode-sized batches whose expert GEMMs split their last items along K (a few dozen
