@@ -139,6 +139,9 @@ moe_status moe_permute(const int32_t *topk_idx, const float *topk_w, const moe_b
  * x [T, D] bf16, W_r [E, D] bf16, W_gate_up [E, 2I, D] bf16 (gate rows 0..I-1, up rows
  * I..2I-1), W_down [E, D, I] bf16, out [T, D] bf16 (fully overwritten; must not alias x).
  * The k weighted outputs are summed in slot order in FP32 and rounded once to bf16.
+ * Wider shapes run their expert GEMMs on pairs of SMs (thread-block clusters); setting the
+ * environment variable MOE_B200_NO_PAIRS selects single-SM tiles instead (same results up to
+ * FP32 summation order).
  * Results are bitwise reproducible for the same inputs.  At decode shapes (T*k <= 32*E) the
  * expert GEMMs may split the K sums of their last items into slices (added in slice order),
  * and how many depends on the batch's work, so a token's output can differ in the last bits

@@ -36,6 +36,8 @@
 //               MMAs overlap this epilogue.
 // All mbarrier waits are bounded (common.cuh); on expiry the kernel records the fact in the
 // device error word and winds down without leaving TMEM allocated.
+#include <cstdlib>
+
 #include "common.cuh"
 
 namespace moe {
@@ -770,6 +772,43 @@ static cudaError_t launch_tc(const TcMaps& maps, const TcArgs& a, int grid, bool
     int pairs = grid / 2 < clusters[dev] ? grid / 2 : clusters[dev];
     if (pairs < 1) pairs = 1;
     return launch_kernel_cluster(kernel, dim3(2 * pairs), dim3(kTcThreads), smem, s, pdl, 2, maps, a);
+}
+
+// Whether clusters of two CTAs of the pair kernels can be resident on this device (queried
+// once per device); without them the forward uses the one-CTA wide tiles.  The environment
+// variable MOE_B200_NO_PAIRS (any value) selects the wide tiles regardless.
+bool pair_tiles_available() {
+    if (getenv("MOE_B200_NO_PAIRS")) return false;
+    static int state[64] = {0};   // 0 unknown, 1 yes, -1 no
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+    if (state[dev] == 0) {
+        bool ok = true;
+        auto probe = [&](const void* kernel, int smem) {
+            if (ensure_smem_attr(kernel, smem) != cudaSuccess) return false;
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3(2);
+            cfg.blockDim = dim3(kTcThreads);
+            cfg.dynamicSmemBytes = smem;
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = 2;
+            attr[0].val.clusterDim.y = 1;
+            attr[0].val.clusterDim.z = 1;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            int n = 0;
+            const cudaError_t e = cudaOccupancyMaxActiveClusters(&n, kernel, &cfg);
+            if (e != cudaSuccess) (void)cudaGetLastError();   // not sticky; clear it
+            return e == cudaSuccess && n > 0;
+        };
+        ok = probe((const void*)tc_gemm_kernel<kModeGateUp, kGuBN, kPairStages, true>,
+                   TcCfg<kModeGateUp, kGuBN, kPairStages, true>::SMEM) &&
+             probe((const void*)tc_gemm_kernel<kModeDown, kDnBN, kPairStages, true>,
+                   TcCfg<kModeDown, kDnBN, kPairStages, true>::SMEM);
+        state[dev] = ok ? 1 : -1;
+    }
+    return state[dev] == 1;
 }
 
 cudaError_t launch_tc_router(const TcMaps& maps, const TcArgs& a, int num_sms, bool pdl,

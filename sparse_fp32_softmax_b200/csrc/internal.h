@@ -219,6 +219,7 @@ cudaError_t launch_gather_rows(const uint16_t* x, const int32_t* row_token, int 
                                uint16_t* x_perm, bool pdl, cudaStream_t s);
 cudaError_t launch_stream_gate_up(const StreamArgs& a, int max_rows, bool pdl, cudaStream_t s);
 cudaError_t launch_stream_down(const StreamArgs& a, int max_rows, bool pdl, cudaStream_t s);
+bool pair_tiles_available();
 cudaError_t launch_tc_router(const TcMaps& maps, const TcArgs& a, int num_sms, bool pdl,
                              cudaStream_t s);
 cudaError_t launch_tc_gate_up(const TcMaps& maps, const TcArgs& a, int num_sms, int tiles, bool pdl,

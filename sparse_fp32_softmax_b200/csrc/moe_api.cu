@@ -424,10 +424,13 @@ moe_status moe_forward_ex(const moe_bf16* x, const moe_bf16* W_r, const moe_bf16
     // Wide shapes: gate_up on CTA pairs; down on CTA pairs when its rows split into 256-row
     // tiles and experts average at least 256 rows (measured on B200: with fewer rows the
     // pair tiles' narrower N and halved item count cost more than the pairs save).
-    const int gu_tiles = narrow ? kTilesNarrow : kTilesPair;
+    // (devices that cannot co-schedule the pairs take the one-CTA wide tiles)
+    const bool pairs = !narrow && !streaming && pair_tiles_available();
+    const int gu_tiles = narrow ? kTilesNarrow : (pairs ? kTilesPair : kTilesWide);
     const int dn_tiles = narrow ? kTilesNarrow
-                         : (p.D % 256 == 0 && (long long)p.T * p.k >= 256ll * p.E) ? kTilesPair
-                                                                                    : kTilesWide;
+                         : (pairs && p.D % 256 == 0 && (long long)p.T * p.k >= 256ll * p.E)
+                               ? kTilesPair
+                               : kTilesWide;
     const int gu_bn = narrow ? kNarrowBN : kGuBN;
     const int dn_bn = narrow ? kNarrowBN : kDnBN;
     const int b_box_max = gu_tiles == kTilesPair ? kGuBN / 2 : gu_bn;   // token rows per CTA

@@ -261,6 +261,14 @@ def test_forward_shared_expert_and_residual(path):
     compare_block(cfg, L2, G2, range(200), path=path, what=f"ungated/{path}")
 
 
+def test_forward_single_sm_wide_tiles(monkeypatch):
+    """The one-CTA wide tiles (used where SM pairs cannot be scheduled) on a wide shape: the
+    interleaved gate_up and the wide down, against the oracle."""
+    monkeypatch.setenv("MOE_B200_NO_PAIRS", "1")
+    cfg, L, G = _small_layer(600, E=8, k=4)
+    compare_block(cfg, L, G, range(600), path="grouped", what="single-SM wide tiles")
+
+
 @pytest.mark.parametrize("T", [5, 300])
 def test_forward_dims_not_multiple_of_256(T):
     """D = I = 384: gate_up K and feature tiles of 128 (pair tiles at T = 300), down rows not a
