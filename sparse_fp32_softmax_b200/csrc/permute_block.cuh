@@ -193,6 +193,48 @@ static __device__ void scatter_warp_slices(const PermuteArgs& a, const WarpSlice
     }
 }
 
+// The same pass for a single block whose routed rows fit kInvRows: rows are recorded in a
+// shared-memory inverse (row -> assignment, and its weight) instead of written to global
+// memory in assignment order; write_rows_from_inverse then writes them in row order.
+constexpr int kInvRows = 4096;
+static __device__ void scatter_warp_slices_inv(const PermuteArgs& a, const WarpSlice& ws, int* wb,
+                                               int* inv, float* winv) {
+    const int E = a.E;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const uint32_t lt_mask = (1u << lane) - 1u;
+#pragma unroll
+    for (int r = 0; r < kMaxRounds; ++r) {
+        if (r >= ws.rounds) break;
+        const int e = ws.e[r];
+        const long as = ws.w0 + r * 32 + lane;
+        const uint32_t m = match_expert(e);
+        int base = 0;
+        if (e >= 0) base = wb[warp * E + e];
+        __syncwarp();
+        if (e >= 0 && (m & lt_mask) == 0) wb[warp * E + e] = base + __popc(m);
+        __syncwarp();
+        if (e >= 0) {
+            const int row = base + __popc(m & lt_mask);
+            a.slot_row[as] = row;
+            inv[row] = (int)as;
+            winv[row] = ws.w[r];
+        }
+    }
+}
+
+// Row metadata of routed rows [0, rows) in row order (coalesced): padding rows (inv < 0) get
+// token -1, weight 0, destination -1.
+static __device__ void write_rows_from_inverse(const PermuteArgs& a, const int* inv,
+                                               const float* winv, int rows) {
+    for (int r = threadIdx.x; r < rows && r < a.cap; r += blockDim.x) {
+        const int as = inv[r];
+        const int t = as >= 0 ? as / a.k : -1;
+        a.row_token[r] = t;
+        if (a.row_weight) a.row_weight[r] = as >= 0 ? winv[r] : 0.0f;
+        if (a.row_dest) a.row_dest[r] = as >= 0 ? t * a.slots_per_token + (as - t * a.k) : -1;
+    }
+}
+
 // Rows of the shared expert (segment E: all tokens in order after the routed rows) and
 // padding rows of each expert segment (tile_m > 1), spread over blocks b0 of nb.
 static __device__ void write_fixed_rows(const PermuteArgs& a, int rows0, const int* offsets,
@@ -244,9 +286,21 @@ static __device__ void permute_one_block(const PermuteArgs& a, int* wb) {
     __syncthreads();
     finish_offsets(a, s_cnt, s_off);
     for (int q = threadIdx.x; q < 32 * E; q += blockDim.x) wb[q] += s_off[q % E];
-    __syncthreads();
-    scatter_warp_slices(a, ws, wb);
-    write_fixed_rows(a, s_off[E], s_off, s_cnt, 0, 1);
+    const int rows = s_off[E];
+    if (rows <= kInvRows) {
+        __shared__ int inv[kInvRows];
+        __shared__ float winv[kInvRows];
+        for (int r = threadIdx.x; r < rows; r += blockDim.x) inv[r] = -1;   // padding rows
+        __syncthreads();
+        scatter_warp_slices_inv(a, ws, wb, inv, winv);
+        __syncthreads();
+        write_rows_from_inverse(a, inv, winv, rows);
+        if (a.has_shared) write_fixed_rows(a, rows, s_off, s_cnt, 0, 1);   // shared rows only
+    } else {
+        __syncthreads();
+        scatter_warp_slices(a, ws, wb);
+        write_fixed_rows(a, rows, s_off, s_cnt, 0, 1);
+    }
 }
 
 }  // namespace moe
