@@ -529,6 +529,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const int row = quarter * 32 + lane;  // TMEM lane = weight row within the tile
         int* ep_dest = ep_dest_all + ew * BN;
         float* ep_wt = ep_wt_all + ew * BN;
+        // down, wide tiles: the slot destinations and routing weights of the token columns
+        // this warp stores (its chunks half, half + 2, ...) are loaded one tile ahead into
+        // registers (nd, nw), so their memory latency overlaps the previous tile's epilogue
+        // (measured: it helps the long-K wide tiles and costs the short narrow ones); the
+        // current tile's copy (cd, cw) stays in registers and reaches the lanes by shuffles,
+        // keeping the per-element work off shared memory, which the MMAs read their
+        // operands from
+        constexpr bool kAhead = MODE == kModeDown && BN > kNarrowBN;
+        constexpr int kCPW = (BN + 63) / 64;   // chunks per epilogue warp
+        int nd[kCPW], cd[kCPW];
+        float nw[kCPW], cw[kCPW];
         // The epilogue of one 32-column chunk: v (and u, the up accumulator) hold row `row`.
         auto finish_chunk = [&](const TileInfo& ti, int c, const float* v, const float* u) {
             if (Tr::IL) {
@@ -555,10 +566,29 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     if (c * 32 + j < ti.n_valid) hp[(size_t)j * a.ld_h] = to_bf16_bits(silu(v[j]) * u[j]);
             } else if (MODE == kModeDown) {
                 const int d = ti.m0 + row;
+                if (kAhead) {
+                    // lane j holds column c*32 + j of this warp's chunk (c - half) / 2
+                    const int i = (c - half) >> 1;
+                    int dsel = cd[0];
+                    float wsel = cw[0];
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const int col = c * 32 + j;
-                    if (col < ti.n_valid) a.slots[(size_t)ep_dest[col] * a.D + d] = ep_wt[col] * v[j];
+                    for (int q = 1; q < kCPW; ++q)
+                        if (q == i) {
+                            dsel = cd[q];
+                            wsel = cw[q];
+                        }
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int dj = __shfl_sync(0xffffffffu, dsel, j);
+                        const float wj = __shfl_sync(0xffffffffu, wsel, j);
+                        if (c * 32 + j < ti.n_valid) a.slots[(size_t)dj * a.D + d] = wj * v[j];
+                    }
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int col = c * 32 + j;
+                        if (col < ti.n_valid) a.slots[(size_t)ep_dest[col] * a.D + d] = ep_wt[col] * v[j];
+                    }
                 }
             } else {
                 const int e = ti.m0 + row;
@@ -590,14 +620,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         a.slots[(size_t)ep_dest[col0 + j] * a.D + d] = ep_wt[col0 + j] * v[j];
             }
         };
-        // down, wide tiles: the slot destinations and routing weights of the token columns
-        // this warp stores (its chunks half, half + 2, ...) are loaded one tile ahead into
-        // registers, so their memory latency overlaps the previous tile's epilogue (measured:
-        // it helps the long-K wide tiles and costs the short narrow ones)
-        constexpr bool kAhead = MODE == kModeDown && BN > kNarrowBN;
-        constexpr int kCPW = (BN + 63) / 64;   // chunks per epilogue warp
-        int nd[kCPW];
-        float nw[kCPW];
         auto fetch_dest = [&](const TileInfo& t) {
 #pragma unroll
             for (int i = 0; i < kCPW; ++i) {
@@ -622,17 +644,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const uint32_t tb = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(b * ACC);
             const int nchunks = (ti.n_valid + 31) >> 5;
             if (kAhead) {
-                // each epilogue warp keeps its own copy: no barrier across warps
-                __syncwarp();
 #pragma unroll
                 for (int i = 0; i < kCPW; ++i) {
-                    const int col = (half + 2 * i) * 32 + lane;
-                    if (col < BN) {
-                        ep_dest[col] = nd[i];
-                        ep_wt[col] = nw[i];
-                    }
+                    cd[i] = nd[i];
+                    cw[i] = nw[i];
                 }
-                __syncwarp();
                 if (item + ugrid < total)
                     fetch_dest(tc_decode_unit<MODE, BN, PAIR>(a, tabs, sc, item + ugrid, rank));
             } else if (MODE == kModeDown) {
@@ -709,12 +725,31 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 if (MODE == kModeGateUp && a.seg_done) signal_segment_done(a, ti.seg, lane);
                 continue;
             }
-            for (int c = half; c < nchunks; c += 2) {
-                float v[32], u[32];
-                tmem_ld32(tb + c * 32, v);
-                if (NA == 2) tmem_ld32(tb + BN + c * 32, u);
-                tmem_ld_wait();
-                finish_chunk(ti, c, v, u);
+            if (NA == 1) {
+                // one accumulator: the TMEM load of the warp's next chunk is in flight while
+                // this chunk is finished (two register buffers, used alternately)
+                float va[32], vb[32];
+                int c = half;
+                if (c < nchunks) tmem_ld32(tb + c * 32, va);
+                while (c < nchunks) {
+                    tmem_ld_wait();
+                    if (c + 2 < nchunks) tmem_ld32(tb + (c + 2) * 32, vb);
+                    finish_chunk(ti, c, va, va);
+                    c += 2;
+                    if (c >= nchunks) break;
+                    tmem_ld_wait();
+                    if (c + 2 < nchunks) tmem_ld32(tb + (c + 2) * 32, va);
+                    finish_chunk(ti, c, vb, vb);
+                    c += 2;
+                }
+            } else {
+                for (int c = half; c < nchunks; c += 2) {
+                    float v[32], u[32];
+                    tmem_ld32(tb + c * 32, v);
+                    tmem_ld32(tb + BN + c * 32, u);
+                    tmem_ld_wait();
+                    finish_chunk(ti, c, v, u);
+                }
             }
             tc_fence_before();
             if (PAIR)
