@@ -10,8 +10,8 @@
 
 namespace moe {
 
-template <typename SlotT>
-__device__ __forceinline__ void load8(const SlotT* p, float (&v)[8]);
+template <typename T>
+__device__ __forceinline__ void load8(const T* p, float (&v)[8]);
 
 template <>
 __device__ __forceinline__ void load8<float>(const float* p, float (&v)[8]) {
@@ -30,9 +30,8 @@ __device__ __forceinline__ void load8<uint16_t>(const uint16_t* p, float (&v)[8]
 
 constexpr int kCombineThreads = 256;
 
-template <typename SlotT>
 __global__ void __launch_bounds__(kCombineThreads) combine_kernel(
-    const SlotT* __restrict__ slots, int T, int D, int k, int has_shared,
+    const float* __restrict__ slots, int T, int D, int k, int has_shared,
     const uint16_t* __restrict__ x, const uint16_t* __restrict__ shared_gate,
     const uint16_t* __restrict__ residual, uint16_t* __restrict__ out, float* __restrict__ out_f32) {
     __shared__ float red[kCombineThreads / 32];
@@ -60,17 +59,17 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(
             __syncthreads();
             gate = 1.0f / (1.0f + expf(-z));
         }
-        const SlotT* base = slots + (size_t)t * S * D;
+        const float* base = slots + (size_t)t * S * D;
         for (int d = threadIdx.x * 8; d < D; d += kCombineThreads * 8) {
             float acc[8], v[8];
-            load8<SlotT>(base + d, acc);
+            load8<float>(base + d, acc);
             // slots j = 1..k-1 in groups of 8: all loads of a group are in flight together,
             // the additions still run in slot order
             for (int j0 = 1; j0 < k; j0 += 8) {
                 float g[8][8];
 #pragma unroll
                 for (int q = 0; q < 8; ++q)
-                    if (j0 + q < k) load8<SlotT>(base + (size_t)(j0 + q) * D + d, g[q]);
+                    if (j0 + q < k) load8<float>(base + (size_t)(j0 + q) * D + d, g[q]);
 #pragma unroll
                 for (int q = 0; q < 8; ++q)
                     if (j0 + q < k) {
@@ -79,7 +78,7 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(
                     }
             }
             if (has_shared) {
-                load8<SlotT>(base + (size_t)k * D + d, v);
+                load8<float>(base + (size_t)k * D + d, v);
 #pragma unroll
                 for (int i = 0; i < 8; ++i) acc[i] = fmaf(gate, v[i], acc[i]);
             }
@@ -103,19 +102,14 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(
     }
 }
 
-cudaError_t launch_combine(const void* slots, int slots_bf16, int T, int D, int k, int has_shared,
+cudaError_t launch_combine(const float* slots, int T, int D, int k, int has_shared,
                            const uint16_t* x, const uint16_t* shared_gate,
                            const uint16_t* residual, uint16_t* out, float* out_f32, bool pdl,
                            cudaStream_t s) {
     if (T <= 0) return cudaSuccess;
     const int blocks = T < 148 * 16 ? T : 148 * 16;
-    if (slots_bf16)
-        return launch_kernel(combine_kernel<uint16_t>, dim3(blocks), dim3(kCombineThreads), 0, s, pdl,
-                             static_cast<const uint16_t*>(slots), T, D, k, has_shared, x, shared_gate,
-                             residual, out, out_f32);
-    return launch_kernel(combine_kernel<float>, dim3(blocks), dim3(kCombineThreads), 0, s, pdl,
-                         static_cast<const float*>(slots), T, D, k, has_shared, x, shared_gate,
-                         residual, out, out_f32);
+    return launch_kernel(combine_kernel, dim3(blocks), dim3(kCombineThreads), 0, s, pdl, slots, T,
+                         D, k, has_shared, x, shared_gate, residual, out, out_f32);
 }
 
 }  // namespace moe

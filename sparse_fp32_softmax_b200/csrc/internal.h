@@ -226,7 +226,7 @@ cudaError_t launch_tc_gate_up(const TcMaps& maps, const TcArgs& a, int num_sms, 
                               cudaStream_t s);
 cudaError_t launch_tc_down(const TcMaps& maps, const TcArgs& a, int num_sms, int tiles, bool pdl,
                            cudaStream_t s);
-cudaError_t launch_combine(const void* slots, int slots_bf16, int T, int D, int k, int has_shared,
+cudaError_t launch_combine(const float* slots, int T, int D, int k, int has_shared,
                            const uint16_t* x, const uint16_t* shared_gate,
                            const uint16_t* residual, uint16_t* out, float* out_f32, bool pdl,
                            cudaStream_t s);

@@ -535,7 +535,7 @@ moe_status moe_forward_ex(const moe_bf16* x, const moe_bf16* W_r, const moe_bf16
         if ((st = record(opts, 3, s)) != MOE_OK) return st;
         MOE_CUDA(launch_stream_down(sa, p.T, chain, s));
         if ((st = record(opts, 4, s)) != MOE_OK) return st;
-        MOE_CUDA(launch_combine(sa.slots, 0, p.T, p.D, p.k, p.has_shared, x, sg, residual, out,
+        MOE_CUDA(launch_combine(sa.slots, p.T, p.D, p.k, p.has_shared, x, sg, residual, out,
                                 out_f32, chain, s));
     } else {
         TcArgs ta{};
@@ -565,7 +565,7 @@ moe_status moe_forward_ex(const moe_bf16* x, const moe_bf16* W_r, const moe_bf16
         if ((st = record(opts, 3, s)) != MOE_OK) return st;
         MOE_CUDA(launch_tc_down(mDn, tdn, sms, dn_tiles, chain, s));
         if ((st = record(opts, 4, s)) != MOE_OK) return st;
-        MOE_CUDA(launch_combine(ta.slots, 0, p.T, p.D, p.k, p.has_shared, x, sg, residual, out,
+        MOE_CUDA(launch_combine(ta.slots, p.T, p.D, p.k, p.has_shared, x, sg, residual, out,
                                 out_f32, chain, s));
     }
     return record(opts, 5, s);
