@@ -3,26 +3,32 @@
 of the HBM / bf16 roofline reached.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode|prefill|keras|zipf|chain]
-                    [--impl ours|reference] [--eager]
+                    [--extra prefill,keras,zipf,chain|none] [--impl ours|reference] [--eager]
 
 Workloads (seeded synthetic inputs of the block's standard configurations):
-  decode   (default) D=2048, E=128, k=8, I=768; one step = one block pass for each of
+  decode   (headline) D=2048, E=128, k=8, I=768; one step = one block pass for each of
            T = 1, 8, 32, 128, 256 tokens (425 tokens per step);
   prefill  same shape, T = 8192;
   keras    D=2048, E=60, k=4, I=1408, T=4096;
   zipf     D=2048, E=512, k=10, I=512 + gated shared expert (I_s=512), Zipf(1.1) router bias;
   chain    48 residual blocks of the keras shape, T=4096 (weights drawn on the GPU).
-Inputs are resident in HBM when the timed region starts.  Decode weights rotate through one
-copy per T so every pass streams its experts from HBM (each copy 1.2 GB > 126 MB L2); the
+The headline workload gives the JSON line's value; the ``--extra`` workloads (by default
+prefill, keras, zipf and chain) are measured in the same run and reported under
+"workloads", each with its own roofline, block fraction and CPU baseline.
+Inputs are resident in HBM when a timed region starts.  Decode weights rotate through one
+copy per pass so every pass streams its experts from HBM (each copy 1.2 GB > 126 MB L2); the
 other workloads' weights and activations exceed L2 by themselves.
 
 Timing: W untimed warm-up steps, then K steps captured as CUDA graphs (one untimed upload
 replay), timed with CUDA events on the launch stream between a barrier and a device
-synchronise on both sides; max over ranks.  That replay gives the headline value.  A second
-timed replay of the same K steps, captured with six stage events per block pass (start,
-routed, permuted, gate_up, down, combined), gives each stage's duration and the dominant
-kernel's roofline (event nodes between kernels cost a little time, so they are kept out of
-the headline replay).  ``--impl reference`` times the CPU oracle instead (rank 0 only).
+synchronise on both sides; max over ranks.  That replay gives the value.  For a sweep,
+each T is also timed alone the same way (K passes, rotating the weight copies).  A second
+timed replay of the K steps, captured with six stage events per block pass (start, routed,
+permuted, gate_up, down, combined), gives each stage's duration and the per-kernel
+rooflines (event nodes between kernels cost a little time, so they are kept out of the
+other timings).  Roofline peaks: the measured burst bf16 figure for timed regions under a
+second, the sustained one for longer regions.  ``--impl reference`` times the CPU oracle
+instead (rank 0 only).
 """
 from __future__ import annotations
 
@@ -48,14 +54,19 @@ WORKLOADS = {
     "zipf": dict(config="zipf", sweep=(4096,), layers=1),
     "chain": dict(config="keras", sweep=(4096,), layers=48),
 }
+DEFAULT_EXTRA = "prefill,keras,zipf,chain"
 
 FALLBACK_PEAKS = dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0)
+SUSTAINED_REGION_S = 1.0     # timed regions at least this long divide by the sustained peak
 
 NVML_REASONS = {
     0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
     0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
     0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
 }
+
+# stage k of the stage events (between event k and k+1)
+STAGES = ("route", "permute", "gate_up", "down", "combine")
 
 
 # ------------------------------------------------------------------ helpers (no GPU needed)
@@ -69,6 +80,14 @@ def load_peaks():
                     bf16_tflops_sustained=float(d["bf16_tflops_sustained"]), source="measured")
     except (OSError, KeyError, ValueError):
         return dict(FALLBACK_PEAKS, source="fallback")
+
+
+def tensor_peak(peaks, region_s):
+    """(TFLOP/s, name) of the bf16 peak a kernel timed inside a region of region_s seconds is
+    held to: the burst figure for short regions, the sustained one for long ones."""
+    if region_s >= SUSTAINED_REGION_S:
+        return peaks["bf16_tflops_sustained"], "bf16_tflops_sustained"
+    return peaks["bf16_tflops"], "bf16_tflops"
 
 
 def aggregate(per_rank_ms, tokens_per_step_per_rank, steps, world):
@@ -104,17 +123,16 @@ def profile_traffic(kernel_tag):
     return float(m.group(1))
 
 
-def kernels_per_forward(T, k, streaming):
+def kernels_per_forward(T, k):
     """Kernels one moe_forward_ex call launches (the library's launch sequence): T <= 32 one
     fused routing + permutation kernel; above, the router, then selection + permutation in
     one kernel while T*k <= 4096 (else selection, histogram, scan and scatter), and the
-    permuted copy of x for the grouped path; then gate_up, down and the combine."""
+    permuted copy of x; then gate_up, down and the combine."""
     n = 0
     if T <= 32:
         n += 1
     else:
-        n += 1 + (1 if T * k <= 4096 else 4)
-        n += 0 if streaming else 1
+        n += 1 + (1 if T * k <= 4096 else 4) + 1
     return n + 3
 
 
@@ -178,16 +196,34 @@ class ClockSampler:
                     sm_max_mhz=self.max_mhz, reasons=names, samples=len(self.samples))
 
 
+def weight_gb(cfg):
+    return (cfg.E * 3 * cfg.D * cfg.I * 2 + cfg.E * cfg.D * 2 + 3 * cfg.D * cfg.I_s * 2) / 1e9
+
+
+def describe(name, cfg, sweep, spec):
+    s = (f"{name}: D={cfg.D}, E={cfg.E}, k={cfg.k}, I={cfg.I}, norm_topk_prob={cfg.norm_topk_prob}, "
+         f"T={'/'.join(str(t) for t in sweep)}")
+    if cfg.I_s:
+        s += f", gated shared expert I_s={cfg.I_s}"
+    if cfg.zipf_s:
+        s += f", Zipf({cfg.zipf_s}) router bias"
+    if spec["layers"] > 1:
+        s += f", {spec['layers']} residual blocks"
+    return s + "; x ~ N(0,1), weights ~ N(0,0.02), bf16, seeded"
+
+
 # ------------------------------------------------------------------ workload
 
-def build_workload(args, device):
+def build_workload(name, device, copies=None):
+    """(cfg, spec, sweep, device weight sets, device x, CPU layer or None)."""
     import torch
     from sparse_fp32_softmax_b200 import inputs
-    spec = WORKLOADS[args.workload]
+    spec = WORKLOADS[name]
     cfg = inputs.CONFIGS[spec["config"]]
     sweep = spec["sweep"]
     Tmax = max(sweep)
     W = []
+    L = None
     if spec["layers"] > 1:
         for l in range(spec["layers"]):
             W.append(inputs.make_layer(cfg, T=Tmax, layer=l, device=device, gen_device=device, with_x=False))
@@ -197,75 +233,64 @@ def build_workload(args, device):
         x0 = L["x"].to(device)
         base = {k: (v.to(device) if v is not None else None) for k, v in L.items() if k != "x"}
         W.append(base)
-        copies = len(sweep) if args.copies is None else max(1, args.copies)
-        for _ in range(1, copies):              # one weight copy per pass of a step
+        n = len(sweep) if copies is None else max(1, copies)
+        for _ in range(1, n):              # one weight copy per pass of a step
             W.append({k: (v.clone() if v is not None else None) for k, v in base.items()})
-    return cfg, spec, sweep, W, x0
+    return cfg, spec, sweep, W, x0, L
 
 
-def passes_of(cfg, spec, sweep, W, x0, torch):
-    """The block passes of one step: (T, x, weights, residual-source index)."""
-    ps = []
-    if spec["layers"] > 1:
-        for l in range(spec["layers"]):
-            ps.append(dict(T=sweep[0], layer=l, w=W[l]))
-    else:
-        for i, T in enumerate(sweep):
-            ps.append(dict(T=T, layer=None, w=W[i % len(W)], x=x0[:T].contiguous()))
-    return ps
-
-
-def run_ours(args, rank, world, device):
+def measure(name, args, rank, world, device, peaks, with_e2e):
+    """Time one workload; returns (result dict, cfg, CPU layer)."""
     import torch
     from sparse_fp32_softmax_b200 import binding as B
     from sparse_fp32_softmax_b200.roofline import algorithmic_bytes, algorithmic_flops
 
-    cfg, spec, sweep, W, x0 = build_workload(args, device)
+    cfg, spec, sweep, W, x0, L_cpu = build_workload(name, device, args.copies if name == args.workload else None)
     chain = spec["layers"] > 1
-    passes = passes_of(cfg, spec, sweep, W, x0, torch)
-    path = args.path
-    stream = torch.cuda.current_stream()
+    K = args.steps
+    if world > 1:
+        import torch.distributed as dist
 
-    # per-pass buffers, workspaces and routing outputs
-    act = [torch.empty_like(x0), torch.empty_like(x0)] if chain else None
+    # the block passes of one step, with their buffers and workspaces
+    passes = []
+    if chain:
+        act = [torch.empty_like(x0), torch.empty_like(x0)]
+        for l in range(spec["layers"]):       # x0 -> A -> B -> A ...; x0 is never written
+            passes.append(dict(T=sweep[0], w=W[l], x=x0 if l == 0 else act[(l - 1) % 2], out=act[l % 2]))
+            passes[-1]["residual"] = passes[-1]["x"]
+    else:
+        for i, T in enumerate(sweep):
+            passes.append(dict(T=T, w=W[i % len(W)], x=x0[:T].contiguous(), residual=None))
+            passes[-1]["out"] = torch.empty_like(passes[-1]["x"])
     shared_ws = None
-    for n, p in enumerate(passes):
-        T = p["T"]
+    for p in passes:
         w = p["w"]
-        p["dims"] = B.make_dims(T, cfg.D, cfg.E, cfg.k, cfg.I, cfg.norm_topk_prob)
-        p["idx"] = torch.empty(T, cfg.k, dtype=torch.int32, device=device)
-        if chain:                               # x0 -> A -> B -> A ...; x0 is never written
-            p["x"] = x0 if n == 0 else act[(n - 1) % 2]
-            p["out"] = act[n % 2]
-            p["residual"] = p["x"]
-        else:
-            p["out"] = torch.empty_like(p["x"])
-            p["residual"] = None
-        opts = B.make_opts(router_bias=w.get("bias"), shared_gate_up=w.get("shared_gate_up"),
-                           shared_down=w.get("shared_down"), shared_gate=w.get("shared_gate"),
-                           residual=p["residual"], topk_idx_out=p["idx"], path=path)
-        p["opts_base"] = opts
-        if chain:                               # passes run one after another: one workspace
+        p["dims"] = B.make_dims(p["T"], cfg.D, cfg.E, cfg.k, cfg.I, cfg.norm_topk_prob)
+        p["idx"] = torch.empty(p["T"], cfg.k, dtype=torch.int32, device=device)
+        p["opts"] = B.make_opts(router_bias=w.get("bias"), shared_gate_up=w.get("shared_gate_up"),
+                                shared_down=w.get("shared_down"), shared_gate=w.get("shared_gate"),
+                                residual=p["residual"], topk_idx_out=p["idx"])
+        if chain:                             # passes run one after another: one workspace
             if shared_ws is None:
-                shared_ws = B.workspace(p["dims"], opts, device=device)
+                shared_ws = B.workspace(p["dims"], p["opts"], device=device)
             p["ws"] = shared_ws
         else:
-            p["ws"] = B.workspace(p["dims"], opts, device=device)
+            p["ws"] = B.workspace(p["dims"], p["opts"], device=device)
 
-    def enqueue(p, events=None):
-        w = p["w"]
-        opts = B.make_opts(router_bias=w.get("bias"), shared_gate_up=w.get("shared_gate_up"),
-                           shared_down=w.get("shared_down"), shared_gate=w.get("shared_gate"),
-                           residual=p["residual"], topk_idx_out=p["idx"], path=path,
-                           stage_events=events)
+    def enqueue(p, w=None, events=None):
+        w = p["w"] if w is None else w
+        opts = p["opts"]
+        if events is not None:
+            opts = B.make_opts(router_bias=w.get("bias"), shared_gate_up=w.get("shared_gate_up"),
+                               shared_down=w.get("shared_down"), shared_gate=w.get("shared_gate"),
+                               residual=p["residual"], topk_idx_out=p["idx"], stage_events=events)
         B.moe_forward_ex(p["x"], w["W_r"], w["W_gate_up"], w["W_down"], cfg.k, cfg.norm_topk_prob,
                          out=p["out"], ws=p["ws"], opts=opts)
 
     def step(events_for_step=None):
         for n, p in enumerate(passes):
-            enqueue(p, events_for_step[n] if events_for_step else None)
+            enqueue(p, events=events_for_step[n] if events_for_step else None)
 
-    # warm-up (also settles routing for the byte accounting)
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
@@ -274,30 +299,26 @@ def run_ours(args, rank, world, device):
         counts = torch.bincount(p["idx"].reshape(-1).long(), minlength=cfg.E)
         p["touched"] = int((counts > 0).sum())
         p["max_load"] = int(counts.max())
-        p["streaming"] = (path == "stream")
 
-    K = args.steps
-    evs = [[B.stage_events(6) for _ in passes] for _ in range(K)]
     use_graph = not args.eager
+    evs = [[B.stage_events(6) for _ in passes] for _ in range(K)]
 
-    def capture(with_events):
+    def capture(body, n):
+        """CUDA graphs of body(s) for s in range(n), in chunks; one untimed upload replay."""
         graphs = []
-        chunk = 25
-        for c0 in range(0, K, chunk):
+        chunk = max(1, 1000 // max(1, len(passes)))
+        for c0 in range(0, n, chunk):
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=torch.cuda.Stream(device=device)):
-                for s in range(c0, min(K, c0 + chunk)):
-                    step(evs[s] if with_events else None)
+                for s in range(c0, min(n, c0 + chunk)):
+                    body(s)
             graphs.append(g)
-        for g in graphs:                       # untimed upload replay
+        for g in graphs:
             g.replay()
         torch.cuda.synchronize()
         return graphs
 
-    if world > 1:
-        import torch.distributed as dist
-
-    def timed(graphs, with_events, sampler=None):
+    def timed(graphs, eager_body, n, sampler=None):
         start = torch.cuda.Event(enable_timing=True)
         end = torch.cuda.Event(enable_timing=True)
         if world > 1:
@@ -310,26 +331,37 @@ def run_ours(args, rank, world, device):
             for g in graphs:
                 g.replay()
         else:
-            for s in range(K):
-                step(evs[s] if with_events else None)
+            for s in range(n):
+                eager_body(s)
         end.record()
         torch.cuda.synchronize()
         if sampler:
             sampler.__exit__(None, None, None)
         if world > 1:
             dist.barrier()
-        return start.elapsed_time(end)
+        ms = start.elapsed_time(end)
+        if world > 1:
+            t = torch.tensor([ms], device=device)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms = float(t.item())
+        return ms
+
+    def run(body, n, sampler=None):
+        graphs = capture(body, n) if use_graph else None
+        ms = timed(graphs, body, n, sampler)
+        del graphs
+        return ms
 
     sampler = ClockSampler(torch.cuda.current_device())
-    ms = timed(capture(False) if use_graph else None, False, sampler)
-    ms_events = timed(capture(True) if use_graph else None, True)
-    per_rank = [ms]
-    if world > 1:
-        t = torch.tensor([ms], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        per_rank = [float(t.item())]
-    tokens_per_step = sum(p["T"] for p in passes) if not chain else sweep[0]
-    agg = aggregate(per_rank, tokens_per_step, K, world)
+    ms = run(lambda s: step(), K, sampler)
+    ms_events = run(lambda s: step(evs[s]), K)
+    tokens_per_step = sweep[0] if chain else sum(p["T"] for p in passes)
+    agg = aggregate([ms], tokens_per_step, K, world)
+    # each T of a sweep alone (K passes, the weight copies in rotation)
+    per_T_ms = {}
+    if len(passes) > 1:
+        for n, p in enumerate(passes):
+            per_T_ms[p["T"]] = run(lambda s, p=p: enqueue(p, w=W[s % len(W)]), K) / K
 
     # stage durations of every pass of every timed step
     stage_ms = [[0.0] * 5 for _ in passes]
@@ -338,71 +370,94 @@ def run_ours(args, rank, world, device):
             e = evs[s][n]
             for j in range(5):
                 stage_ms[n][j] += e[j].elapsed_time(e[j + 1]) / K
-    peaks = load_peaks()
-    launches_per_pass = [kernels_per_forward(p["T"], cfg.k, p["streaming"]) for p in passes]
+    region_s = ms / 1e3
+    tf_peak, tf_name = tensor_peak(peaks, region_s)
+    hbm = peaks["hbm_gbs"]
 
-    # roofline of the dominant kernel: the gate_up expert kernel (stage 3).  Reported for
-    # the workload's largest pass (one launch shape, the one a single ncu capture covers);
-    # every pass's gate_up rate is listed in the sweep entries.
+    def kernel_roof(kname, bytes_, flops, t_ms, launch):
+        """Roofline entry of one kernel: its own bound (weight bytes at HBM peak against
+        FLOPs at the bf16 peak), achieved = algorithmic work / mean launch time."""
+        t_b = bytes_ / (hbm * 1e9)
+        t_f = flops / (tf_peak * 1e12)
+        if t_b >= t_f:
+            a = bytes_ / (t_ms / 1e3) / 1e9
+            return dict(bound="hbm", achieved=round(a, 1), peak=hbm, unit="GB/s", frac=round(a / hbm, 4),
+                        kernel=kname, launch=launch, algorithmic_bytes_per_launch=int(bytes_),
+                        us_per_launch=round(t_ms * 1e3, 2), peak_source=f"{peaks['source']} hbm_gbs")
+        a = flops / (t_ms / 1e3) / 1e12
+        return dict(bound="tensor", achieved=round(a, 1), peak=tf_peak, unit="TFLOP/s",
+                    frac=round(a / tf_peak, 4), kernel=kname, launch=launch,
+                    algorithmic_flops_per_launch=int(flops), us_per_launch=round(t_ms * 1e3, 2),
+                    peak_source=f"{peaks['source']} {tf_name}")
+
     I2 = 2 * cfg.I
     blk_bytes = blk_flops = 0.0
-    per_T = []
-    gu = []
+    sweep_out = []
+    gu_roofs, dn_roofs = [], []
     for n, p in enumerate(passes):
         T = p["T"]
         b_gu = p["touched"] * I2 * cfg.D * 2 + (2 * cfg.I_s * cfg.D * 2 if cfg.I_s else 0)
         f_gu = 2.0 * T * cfg.k * I2 * cfg.D + (2.0 * T * 2 * cfg.I_s * cfg.D if cfg.I_s else 0)
-        gu.append((b_gu, f_gu, stage_ms[n][2]))
+        b_dn = p["touched"] * cfg.I * cfg.D * 2 + (cfg.I_s * cfg.D * 2 if cfg.I_s else 0)
+        f_dn = 2.0 * T * cfg.k * cfg.I * cfg.D + (2.0 * T * cfg.I_s * cfg.D if cfg.I_s else 0)
+        gu_roofs.append((b_gu, f_gu, stage_ms[n][2], T))
+        dn_roofs.append((b_dn, f_dn, stage_ms[n][3], T))
         b = algorithmic_bytes(T, cfg.D, cfg.E, cfg.k, cfg.I, p["touched"], cfg.I_s, cfg.shared_gated,
                               residual=chain)
         f = algorithmic_flops(T, cfg.D, cfg.E, cfg.k, cfg.I, cfg.I_s, cfg.shared_gated)
         blk_bytes += b
         blk_flops += f
-        t_pass = sum(stage_ms[n])
-        t_roof = max(b / (peaks["hbm_gbs"] * 1e9), f / (peaks["bf16_tflops_sustained"] * 1e12))
-        if not chain:
-            per_T.append(dict(T=T, us=round(t_pass * 1e3, 2), tokens_per_s=round(T / (t_pass / 1e3), 1),
-                              roofline_us=round(t_roof * 1e6, 2), roofline_frac=round(t_roof / (t_pass / 1e3), 4),
-                              touched=p["touched"], max_load=p["max_load"],
-                              stages_us=[round(v * 1e3, 2) for v in stage_ms[n]],
-                              gate_up_gbs=round(b_gu / (stage_ms[n][2] / 1e3) / 1e9, 1),
-                              gate_up_tflops=round(f_gu / (stage_ms[n][2] / 1e3) / 1e12, 1),
-                              path="stream" if p["streaming"] else "grouped"))
-    gu_bytes, gu_flops, gu_ms = gu[-1]
-    if chain:   # every layer has the same shape: average them
-        gu_bytes = sum(g[0] for g in gu) / len(gu)
-        gu_flops = sum(g[1] for g in gu) / len(gu)
-        gu_ms = sum(g[2] for g in gu) / len(gu)
-    # the bound follows the kernel's own work: weight bytes at HBM peak against FLOPs at the
-    # sustained bf16 peak (decode is weight-bound, prefill compute-bound)
-    t_bytes = gu_bytes / (peaks["hbm_gbs"] * 1e9)
-    t_flops = gu_flops / (peaks["bf16_tflops_sustained"] * 1e12)
-    streaming = all(p["streaming"] for p in passes)
-    kname = "stream_gate_up_kernel" if streaming else "tc_gemm_kernel<gate_up>"
-    T_dom = passes[-1]["T"]
-    if t_bytes >= t_flops:
-        achieved = gu_bytes / (gu_ms / 1e3) / 1e9
-        roof = dict(bound="hbm", achieved=round(achieved, 1), peak=peaks["hbm_gbs"], unit="GB/s",
-                    frac=round(achieved / peaks["hbm_gbs"], 4), kernel=kname, launch=f"T={T_dom}",
-                    algorithmic_bytes_per_launch=int(gu_bytes),
-                    peak_source=peaks["source"] + " hbm_gbs")
-    else:
-        achieved = gu_flops / (gu_ms / 1e3) / 1e12
-        roof = dict(bound="tensor", achieved=round(achieved, 1), peak=peaks["bf16_tflops_sustained"],
-                    unit="TFLOP/s", frac=round(achieved / peaks["bf16_tflops_sustained"], 4),
-                    kernel=kname, launch=f"T={T_dom}", algorithmic_flops_per_launch=int(gu_flops),
-                    peak_source=peaks["source"] + " bf16_tflops_sustained")
-    tag = ("stream_gate_up_" if streaming else "tc_gate_up_") + args.workload
-    if tag == "tc_gate_up_prefill":
-        tag = "tc_gemm_prefill"
-    # DRAM bytes of one launch from the committed ncu summary (null when there is none for
-    # this workload or the kernel source changed since it was taken)
+        if len(passes) > 1 and not chain:
+            t_ms = per_T_ms[T]
+            t_roof = max(b / (hbm * 1e9), f / (tf_peak * 1e12))
+            sweep_out.append(dict(
+                T=T, us=round(t_ms * 1e3, 2), tokens_per_s=round(T / (t_ms / 1e3), 1),
+                roofline_us=round(t_roof * 1e6, 2), roofline_frac=round(t_roof / (t_ms / 1e3), 4),
+                touched=p["touched"], max_load=p["max_load"],
+                stages_us_with_events=dict(zip(STAGES, [round(v * 1e3, 2) for v in stage_ms[n]])),
+                gate_up_gbs=round(b_gu / (stage_ms[n][2] / 1e3) / 1e9, 1),
+                down_gbs=round(b_dn / (stage_ms[n][3] / 1e3) / 1e9, 1)))
+
+    def dominant(rs, kname):
+        if chain:   # every layer has the same shape: average them
+            b = sum(r[0] for r in rs) / len(rs)
+            f = sum(r[1] for r in rs) / len(rs)
+            t = sum(r[2] for r in rs) / len(rs)
+            return kernel_roof(kname, b, f, t, f"T={rs[0][3]} (mean of {len(rs)} layers)")
+        b, f, t, T = rs[-1]          # the largest pass: one launch shape, one ncu capture
+        return kernel_roof(kname, b, f, t, f"T={T}")
+
+    roof = dominant(gu_roofs, "tc_gemm_kernel<gate_up>")
+    roof_dn = dominant(dn_roofs, "tc_gemm_kernel<down>")
+    tag = {"decode": "tc_gate_up_decode", "prefill": "tc_gemm_prefill"}.get(name, f"tc_gate_up_{name}")
     roof["traffic"] = profile_traffic(tag)
-    blk_time = max(blk_bytes / (peaks["hbm_gbs"] * 1e9), blk_flops / (peaks["bf16_tflops_sustained"] * 1e12))
+    blk_time = max(blk_bytes / (hbm * 1e9), blk_flops / (tf_peak * 1e12))
+    res = dict(
+        workload=describe(name, cfg, sweep, spec), tokens_per_step=tokens_per_step,
+        value=round(agg["value"], 1), unit="tokens/s", ms_per_step=round(agg["ms_per_step"], 5),
+        timing="CUDA graph replay" if use_graph else "eager",
+        stage_timing=f"second timed replay of the {K} steps with stage events: {ms_events / K:.4f} ms/step",
+        l2=("rotating %d weight copies (%.1f GB) > 126 MB L2" % (len(W), len(W) * weight_gb(cfg))
+            if not chain else "48 distinct layers (%.1f GB) > 126 MB L2" % (48 * weight_gb(cfg))),
+        roofline=roof, roofline_down=roof_dn,
+        block_roofline=dict(time_us=round(blk_time * 1e6, 2), measured_us=round(agg["ms_per_step"] * 1e3, 2),
+                            frac=round(blk_time / (agg["ms_per_step"] / 1e3), 4), bytes=int(blk_bytes),
+                            flops=int(blk_flops), bound=("hbm" if blk_bytes / (hbm * 1e9) >=
+                                                         blk_flops / (tf_peak * 1e12) else "tensor"),
+                            peaks=f"hbm_gbs {hbm}, {tf_name} {tf_peak} ({peaks['source']})"),
+        gpu_launches=int(sum(kernels_per_forward(p["T"], cfg.k) for p in passes) * K),
+        clocks=sampler.summary())
+    if not chain:
+        res["stages_us_with_events"] = dict(zip(STAGES, [round(v * 1e3, 2) for v in stage_ms[-1]]))
+        res["touched"], res["max_load"] = passes[-1]["touched"], passes[-1]["max_load"]
+    else:
+        res["stages_us_with_events"] = dict(zip(STAGES, [round(sum(stage_ms[n][j] for n in range(len(passes)))
+                                                               / len(passes) * 1e3, 2) for j in range(5)]))
+    if sweep_out:
+        res["sweep"] = sweep_out
 
     # end to end through the public API with host buffers (eager, copies inside the region)
-    e2e = None
-    if not chain:
+    if with_e2e and not chain:
         hx = [p["x"].cpu().pin_memory() for p in passes]
         hy = [torch.empty(p["out"].shape, dtype=p["out"].dtype).pin_memory() for p in passes]
         dx = [torch.empty_like(p["x"]) for p in passes]
@@ -412,7 +467,7 @@ def run_ours(args, rank, world, device):
                 dx[n].copy_(hx[n], non_blocking=True)
                 w = p["w"]
                 B.moe_forward_ex(dx[n], w["W_r"], w["W_gate_up"], w["W_down"], cfg.k, cfg.norm_topk_prob,
-                                 out=p["out"], ws=p["ws"], opts=p["opts_base"])
+                                 out=p["out"], ws=p["ws"], opts=p["opts"])
                 hy[n].copy_(p["out"], non_blocking=True)
 
         for _ in range(max(1, args.warmup)):
@@ -430,47 +485,12 @@ def run_ours(args, rank, world, device):
             dist.all_reduce(t, op=dist.ReduceOp.MAX)
             e_ms = float(t.item())
         bytes_in = sum(p["x"].numel() * 2 for p in passes)
-        e2e = dict(value=round(world * tokens_per_step * K / (e_ms / 1e3), 1), unit="tokens/s",
-                   h2d_bytes_per_step=bytes_in, d2h_bytes_per_step=bytes_in, timing="eager")
-
-    line = dict(
-        metric=METRIC, value=round(agg["value"], 1), unit="tokens/s", n_gpus=world, steps=K,
-        warmup=args.warmup, ms_per_step=round(agg["ms_per_step"], 5), higher_is_better=True,
-        scaling="weak", vs_baseline=None, dtype="bf16", data="synthetic",
-        config=dict(workload=describe(args.workload, cfg, sweep, spec), tokens_per_step=tokens_per_step,
-                    stage_timing=f"second timed replay of the {K} steps with stage events: "
-                                 f"{ms_events / K:.4f} ms/step",
-                    l2=("rotating %d weight copies (%.1f GB) > 126 MB L2" % (len(W), len(W) * weight_gb(cfg))
-                        if not chain else "48 distinct layers (%.1f GB) > 126 MB L2" % (48 * weight_gb(cfg))),
-                    timing="CUDA graph replay" if use_graph else "eager", path=path,
-                    parallelism=f"replicas x{world}" if world > 1 else "single GPU"),
-        roofline=roof,
-        block_roofline=dict(time_us=round(blk_time * 1e6, 2), measured_us=round(agg["ms_per_step"] * 1e3, 2),
-                            frac=round(blk_time / (agg["ms_per_step"] / 1e3), 4),
-                            bytes=int(blk_bytes), flops=int(blk_flops)),
-        gpu_launches=int(sum(launches_per_pass) * K),
-        clocks=sampler.summary(),
-        e2e=e2e,
-    )
-    if per_T:
-        line["sweep"] = per_T
-    return line, cfg, passes
-
-
-def weight_gb(cfg):
-    return (cfg.E * 3 * cfg.D * cfg.I * 2 + cfg.E * cfg.D * 2 + 3 * cfg.D * cfg.I_s * 2) / 1e9
-
-
-def describe(name, cfg, sweep, spec):
-    s = (f"{name}: D={cfg.D}, E={cfg.E}, k={cfg.k}, I={cfg.I}, norm_topk_prob={cfg.norm_topk_prob}, "
-         f"T={'/'.join(str(t) for t in sweep)}")
-    if cfg.I_s:
-        s += f", gated shared expert I_s={cfg.I_s}"
-    if cfg.zipf_s:
-        s += f", Zipf({cfg.zipf_s}) router bias"
-    if spec["layers"] > 1:
-        s += f", {spec['layers']} residual blocks"
-    return s + "; x ~ N(0,1), weights ~ N(0,0.02), bf16, seeded"
+        res["e2e"] = dict(value=round(world * tokens_per_step * K / (e_ms / 1e3), 1), unit="tokens/s",
+                          h2d_bytes_per_step=bytes_in, d2h_bytes_per_step=bytes_in, timing="eager")
+    del passes, W, x0, evs
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return res, cfg, L_cpu
 
 
 # ------------------------------------------------------------------ CPU oracle legs
@@ -485,20 +505,26 @@ def oracle_sample_rate(cfg, x, w, rows, threads):
     return len(rows) / (time.perf_counter() - t0)
 
 
-def cpu_baseline(cfg, target_cpu_s=10.0, layers=1):
-    """The oracle as it stands on this host's cores, on a bounded sample of the workload."""
+def cpu_baseline(cfg, L=None, target_cpu_s=4.0, layers=1):
+    """The oracle as it stands on this host, on a bounded sample of the workload: on one core
+    and on every core available to the process."""
     from oracle import oracle as O
     from sparse_fp32_softmax_b200 import inputs
-    L = inputs.make_layer(cfg, T=cfg.T)
+    if L is None:
+        L = inputs.make_layer(cfg, T=cfg.T)
     threads = O.cpu_threads_available()
-    one = oracle_sample_rate(cfg, L["x"], L, [0], 1)           # seconds per token on one core
-    n = int(max(threads, min(2048, target_cpu_s * one)))
+    first = oracle_sample_rate(cfg, L["x"], L, [0], 1)            # tokens/s on one core (1 token)
+    n1 = int(max(1, min(cfg.T, target_cpu_s / 2 * first)))
+    one = oracle_sample_rate(cfg, L["x"], L, list(range(n1)), 1)
+    n = int(max(threads, min(2048, target_cpu_s * one * threads / 2)))
     n = min(n, cfg.T)
-    rows = list(range(n))
-    rate = oracle_sample_rate(cfg, L["x"], L, rows, threads) / layers
-    return dict(value=round(rate, 3), unit="tokens/s", cores=threads, kind="oracle",
-                sample=f"first {n} tokens of the T={cfg.T} batch, one FP64 block pass each "
-                       f"(~{n / one:.0f} CPU-seconds)" + (f", rate divided by {layers} layers" if layers > 1 else ""))
+    rate = oracle_sample_rate(cfg, L["x"], L, list(range(n)), threads)
+    per = f", rate divided by {layers} layers" if layers > 1 else ""
+    return dict(value=round(rate / layers, 3), unit="tokens/s", cores=threads, kind="oracle",
+                sample=f"first {n} tokens of the T={cfg.T} batch, one FP64 block pass each, on {threads} "
+                       f"cores{per}",
+                single_core=dict(value=round(one / layers, 3), unit="tokens/s", cores=1,
+                                 sample=f"first {n1} tokens, one core{per}"))
 
 
 def run_reference(args):
@@ -534,8 +560,9 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="decode", choices=sorted(WORKLOADS))
+    ap.add_argument("--extra", default=DEFAULT_EXTRA,
+                    help="comma-separated workloads measured after the headline one, or 'none'")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--path", default="auto", choices=["auto", "stream", "grouped"])
     ap.add_argument("--eager", action="store_true", help="time eager launches instead of CUDA graphs")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--copies", type=int, default=None,
@@ -543,6 +570,10 @@ def main(argv=None):
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    extra = [] if args.extra in ("", "none") else [w for w in args.extra.split(",") if w != args.workload]
+    for w in extra:
+        if w not in WORKLOADS:
+            ap.error(f"unknown workload {w}")
     rank, world, local = dist_env()
 
     if args.impl == "reference":
@@ -562,9 +593,46 @@ def main(argv=None):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=device)
     from sparse_fp32_softmax_b200.build import build
     build()
-    line, cfg, _ = run_ours(args, rank, world, device)
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(cfg, layers=WORKLOADS[args.workload]["layers"])
+    peaks = load_peaks()
+    want_cpu = rank == 0 and world == 1 and not args.no_cpu_baseline
+    res, cfg, L_cpu = measure(args.workload, args, rank, world, device, peaks, with_e2e=True)
+    line = dict(
+        metric=METRIC, value=res["value"], unit="tokens/s", n_gpus=world, steps=args.steps,
+        warmup=args.warmup, ms_per_step=res["ms_per_step"], higher_is_better=True, scaling="weak",
+        vs_baseline=None, dtype="bf16", data="synthetic",
+        config=dict(workload=res["workload"], tokens_per_step=res["tokens_per_step"], l2=res["l2"],
+                    timing=res["timing"], stage_timing=res["stage_timing"],
+                    parallelism=f"replicas x{world}" if world > 1 else "single GPU"),
+        roofline=res["roofline"], roofline_down=res["roofline_down"], block_roofline=res["block_roofline"],
+        gpu_launches=res["gpu_launches"], clocks=res["clocks"], e2e=res.get("e2e"),
+        stages_us_with_events=res["stages_us_with_events"])
+    if "sweep" in res:
+        line["sweep"] = res["sweep"]
+    if want_cpu:
+        line["cpu_baseline"] = cpu_baseline(cfg, L_cpu, layers=WORKLOADS[args.workload]["layers"])
+    del L_cpu
+    if extra:
+        line["workloads"] = {}
+        keras_cpu = None
+        for wname in extra:
+            r, c, Lc = measure(wname, args, rank, world, device, peaks, with_e2e=False)
+            if want_cpu:
+                if WORKLOADS[wname]["layers"] > 1:
+                    if keras_cpu is None:
+                        keras_cpu = cpu_baseline(c, None)
+                    nl = WORKLOADS[wname]["layers"]
+                    cb = dict(keras_cpu)
+                    cb["value"] = round(keras_cpu["value"] / nl, 3)
+                    cb["sample"] = keras_cpu["sample"] + f", rate divided by {nl} layers"
+                    cb["single_core"] = dict(keras_cpu["single_core"])
+                    cb["single_core"]["value"] = round(keras_cpu["single_core"]["value"] / nl, 3)
+                    r["cpu_baseline"] = cb
+                else:
+                    r["cpu_baseline"] = cpu_baseline(c, Lc)
+                    if wname == "keras":
+                        keras_cpu = r["cpu_baseline"]
+            line["workloads"][wname] = r
+            del Lc
     if world > 1:
         import torch.distributed as dist
         dist.barrier()

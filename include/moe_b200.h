@@ -69,10 +69,18 @@ typedef struct {
 
 /* Which expert path moe_forward_ex takes. */
 enum {
-    MOE_PATH_AUTO = 0,    /* the library's choice (currently the grouped path at every T) */
-    MOE_PATH_STREAM = 1,  /* warp-MMA kernels that stream each touched expert's weights once
-                             straight into registers (no permuted copy of x) */
-    MOE_PATH_GROUPED = 2  /* permute + tcgen05 grouped GEMMs, TMA-fed, TMEM accumulators */
+    MOE_PATH_AUTO = 0,    /* the library's choice (the grouped path at every T) */
+    MOE_PATH_GROUPED = 1  /* permute + tcgen05 grouped GEMMs, TMA-fed, TMEM accumulators */
+};
+
+/* Diagnostics of moe_forward_ex (moe_opts.diag); 0 in normal use. */
+enum {
+    /* The down GEMM's per-expert hand-off wait (used when T*k <= 32*E) watches a completion
+     * counter that nothing increments, so each such wait runs until its limit
+     * (moe_opts.wait_limit_us) and the kernels wind down.  The output is then undefined and
+     * moe_get_device_status reports MOE_ERR_DEVICE_TIMEOUT; the device stays usable.  For
+     * testing the watchdog.  Shapes that do not use the hand-off return MOE_ERR_UNSUPPORTED. */
+    MOE_DIAG_UNSIGNALLED_HANDOFF = 1
 };
 
 /* Options of moe_forward_ex.  Zero-initialise and set what is needed. */
@@ -94,6 +102,14 @@ typedef struct {
     int n_stage_events;
     float *out_f32;                  /* [T, D] FP32 block output before its rounding to bf16
                                         (residual and shared expert included), or NULL */
+    int32_t *expert_counts_out;      /* [E] assignments routed to each expert (the per-expert
+                                        load), or NULL */
+    int32_t *slot_row_out;           /* [T, k] row of assignment (t, j) in the expert-sorted
+                                        order: the slot_row of moe_permute with tile_m = 1,
+                                        or NULL */
+    unsigned wait_limit_us;          /* limit of every bounded device wait in microseconds;
+                                        0 = the default of 2 s */
+    int diag;                        /* MOE_DIAG_* or 0 */
 } moe_opts;
 
 /* Bytes of workspace that moe_route, moe_permute and moe_forward(_ex) need for `dims`
@@ -156,11 +172,11 @@ moe_status moe_forward_ex(const moe_bf16 *x, const moe_bf16 *W_r, const moe_bf16
                           const moe_bf16 *W_down, const moe_dims *dims, const moe_opts *opts,
                           moe_bf16 *out, void *ws, size_t ws_bytes, moe_stream_t stream);
 
-/* moe_forward for callers that cannot allocate device memory: code that enqueues work
- * while a stream is being captured into a CUDA graph, plugin hosts that give a kernel only
- * its input and output buffers, runtimes that forbid allocation after start-up.  The pages
- * have no counterpart: this is a deployment variant of moe_forward, same arguments minus
- * the workspace, same results.
+/* moe_forward for callers that cannot allocate device memory: plugin hosts that give a
+ * kernel only its input and output buffers, and runtimes that forbid device allocation once
+ * they have started (their memory is planned up front).  The pages have no counterpart:
+ * this is a deployment variant of moe_forward, same arguments minus the workspace, same
+ * results.
  * Scratch: a 64 MiB array in the library's own device memory (a file-scope device
  * variable), held by every GPU that loads this part of the library until the process
  * exits.  Calls whose moe_workspace_size(dims, NULL) exceeds 64 MiB return
@@ -169,10 +185,18 @@ moe_status moe_forward_ex(const moe_bf16 *x, const moe_bf16 *W_r, const moe_bf16
  * The first call on a device looks up the array's device address (once per device); make
  * that first call before any stream capture.  All calls on a device share the array and it
  * keeps the last call's contents; each call clears what must start at zero.  Calls that can
- * overlap on the GPU (other streams, unordered host threads) race on the array. */
+ * overlap on the GPU (other streams, unordered host threads) race on the array.
+ * Its device error word (bounded waits, bad indices) is read with
+ * moe_get_device_status_noalloc. */
 moe_status moe_forward_noalloc(const moe_bf16 *x, const moe_bf16 *W_r, const moe_bf16 *W_gate_up,
                                const moe_bf16 *W_down, const moe_dims *dims, moe_bf16 *out,
                                moe_stream_t stream);
+
+/* moe_get_device_status for moe_forward_noalloc, whose workspace the caller never sees:
+ * synchronises `stream` and reports the device error word that the last
+ * moe_forward_noalloc call on the current device left in the library's array (MOE_OK
+ * before the first call).  The pages have no counterpart. */
+moe_status moe_get_device_status_noalloc(moe_stream_t stream);
 
 /* Synchronises `stream` and reports the device error word that the last call using `ws`
  * left: MOE_OK, MOE_ERR_DEVICE_TIMEOUT (a bounded wait expired), MOE_ERR_INVALID_ARG (an

@@ -19,8 +19,9 @@ LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
 HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "moe_b200.h")
 
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_DEVICE_TIMEOUT = range(6)
-MOE_PATH_AUTO, MOE_PATH_STREAM, MOE_PATH_GROUPED = range(3)
-PATHS = {"auto": MOE_PATH_AUTO, "stream": MOE_PATH_STREAM, "grouped": MOE_PATH_GROUPED}
+MOE_PATH_AUTO, MOE_PATH_GROUPED = range(2)
+PATHS = {"auto": MOE_PATH_AUTO, "grouped": MOE_PATH_GROUPED}
+MOE_DIAG_UNSIGNALLED_HANDOFF = 1
 
 _c_int, _vp, _sz = ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t
 
@@ -34,7 +35,9 @@ class moe_opts(ctypes.Structure):
     _fields_ = [("router_bias", _vp), ("shared_gate_up", _vp), ("shared_down", _vp),
                 ("shared_gate", _vp), ("I_s", _c_int), ("residual", _vp), ("logits_out", _vp),
                 ("topk_idx_out", _vp), ("topk_w_out", _vp), ("path", _c_int),
-                ("stage_events", _vp), ("n_stage_events", _c_int), ("out_f32", _vp)]
+                ("stage_events", _vp), ("n_stage_events", _c_int), ("out_f32", _vp),
+                ("expert_counts_out", _vp), ("slot_row_out", _vp), ("wait_limit_us", ctypes.c_uint),
+                ("diag", _c_int)]
 
 
 class MoeError(RuntimeError):
@@ -64,12 +67,13 @@ def load():
         lib.moe_forward_ex.argtypes = [_vp, _vp, _vp, _vp, dp, op, _vp, _vp, _sz, _vp]
         lib.moe_forward_noalloc.argtypes = [_vp, _vp, _vp, _vp, dp, _vp, _vp]
         lib.moe_get_device_status.argtypes = [_vp, _vp]
+        lib.moe_get_device_status_noalloc.argtypes = [_vp]
         lib.moe_status_string.argtypes = [_c_int]
         lib.moe_status_string.restype = ctypes.c_char_p
         lib.moe_last_cuda_error.argtypes = []
         lib.moe_last_cuda_error.restype = _c_int
         for n in ("moe_route", "moe_permute", "moe_forward", "moe_forward_ex", "moe_forward_noalloc",
-                  "moe_get_device_status"):
+                  "moe_get_device_status", "moe_get_device_status_noalloc"):
             getattr(lib, n).restype = _c_int
         _lib = lib
     return _lib
@@ -127,7 +131,8 @@ def make_dims(T, D, E, k, I, norm_topk_prob=True, tile_m=1) -> moe_dims:
 
 def make_opts(router_bias=None, shared_gate_up=None, shared_down=None, shared_gate=None,
               residual=None, logits_out=None, topk_idx_out=None, topk_w_out=None, path="auto",
-              stage_events=None, out_f32=None):
+              stage_events=None, out_f32=None, expert_counts_out=None, slot_row_out=None,
+              wait_limit_us=0, diag=0):
     o = moe_opts()
     o.router_bias = _ptr(router_bias)
     o.shared_gate_up = _ptr(shared_gate_up)
@@ -140,6 +145,10 @@ def make_opts(router_bias=None, shared_gate_up=None, shared_down=None, shared_ga
     o.topk_w_out = _ptr(topk_w_out)
     o.path = PATHS[path] if isinstance(path, str) else int(path)
     o.out_f32 = _ptr(out_f32)
+    o.expert_counts_out = _ptr(expert_counts_out)
+    o.slot_row_out = _ptr(slot_row_out)
+    o.wait_limit_us = int(wait_limit_us)
+    o.diag = int(diag)
     o._events_keepalive = None
     if stage_events is not None:
         handles = (ctypes.c_void_p * len(stage_events))(*[ev.cuda_event for ev in stage_events])
@@ -226,7 +235,8 @@ def moe_forward_ex(x, W_r, W_gate_up, W_down, k, norm_topk_prob=True, out=None, 
                    stream=None, opts: moe_opts | None = None, **opt_kwargs):
     """moe_forward with options; pass a prepared ``opts`` or the keyword arguments of
     ``make_opts`` (router_bias, shared_gate_up, shared_down, shared_gate, residual,
-    logits_out, topk_idx_out, topk_w_out, path, stage_events, out_f32)."""
+    logits_out, topk_idx_out, topk_w_out, path, stage_events, out_f32, expert_counts_out,
+    slot_row_out, wait_limit_us, diag)."""
     dims = _dims_of(x, W_r, W_gate_up, W_down, k, norm_topk_prob)
     if opts is None:
         opts = make_opts(**opt_kwargs)
@@ -254,6 +264,10 @@ def moe_forward_noalloc(x, W_r, W_gate_up, W_down, k, norm_topk_prob=True, out=N
 
 def moe_get_device_status(ws, stream=None) -> int:
     return int(load().moe_get_device_status(_ptr(ws), _stream(stream)))
+
+
+def moe_get_device_status_noalloc(stream=None) -> int:
+    return int(load().moe_get_device_status_noalloc(_stream(stream)))
 
 
 def stage_events(n=6):

@@ -33,7 +33,7 @@ constexpr int kCombineThreads = 256;
 __global__ void __launch_bounds__(kCombineThreads) combine_kernel(
     const float* __restrict__ slots, int T, int D, int k, int has_shared,
     const uint16_t* __restrict__ x, const uint16_t* __restrict__ shared_gate,
-    const uint16_t* __restrict__ residual, uint16_t* __restrict__ out, float* __restrict__ out_f32) {
+    const uint16_t* residual, uint16_t* out, float* __restrict__ out_f32) {
     __shared__ float red[kCombineThreads / 32];
     pdl_wait();
     pdl_launch_dependents();
@@ -83,7 +83,12 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(
                 for (int i = 0; i < 8; ++i) acc[i] = fmaf(gate, v[i], acc[i]);
             }
             if (residual) {
-                load8<uint16_t>(residual + (size_t)t * D + d, v);
+                // out may be the residual buffer itself (a residual chain updated in place):
+                // each thread reads its 8 elements here, before it writes them below, with a
+                // coherent load (not the read-only path)
+                const uint4 r = __ldcg(reinterpret_cast<const uint4*>(residual + (size_t)t * D + d));
+                v[0] = bf16_lo(r.x); v[1] = bf16_hi(r.x); v[2] = bf16_lo(r.y); v[3] = bf16_hi(r.y);
+                v[4] = bf16_lo(r.z); v[5] = bf16_hi(r.z); v[6] = bf16_lo(r.w); v[7] = bf16_hi(r.w);
 #pragma unroll
                 for (int i = 0; i < 8; ++i) acc[i] += v[i];
             }
@@ -107,7 +112,9 @@ cudaError_t launch_combine(const float* slots, int T, int D, int k, int has_shar
                            const uint16_t* residual, uint16_t* out, float* out_f32, bool pdl,
                            cudaStream_t s) {
     if (T <= 0) return cudaSuccess;
-    const int blocks = T < 148 * 16 ? T : 148 * 16;
+    const int sms = device_sm_count();
+    if (sms <= 0) return cudaErrorInvalidDevice;
+    const int blocks = T < sms * 16 ? T : sms * 16;
     return launch_kernel(combine_kernel, dim3(blocks), dim3(kCombineThreads), 0, s, pdl, slots, T,
                          D, k, has_shared, x, shared_gate, residual, out, out_f32);
 }

@@ -37,6 +37,7 @@
 // All mbarrier waits are bounded (common.cuh); on expiry the kernel records the fact in the
 // device error word and winds down without leaving TMEM allocated.
 #include <cstdlib>
+#include <mutex>
 
 #include "common.cuh"
 
@@ -248,7 +249,7 @@ __device__ __forceinline__ bool wait_segment_done(const TcArgs& a, int seg, bool
         }
         if (ld_acquire(a.seg_done + seg) >= target) break;
         __nanosleep(128);
-        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        if (globaltimer_ns() - t0 > a.wait_ns) {
             set_error(a.err, kErrWaitProducer);
             return false;
         }
@@ -399,7 +400,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             for (int kb = 0; kb < ti.nk; ++kb, ++it) {
                 const int s = it % STAGES;
                 const int round = it / STAGES;
-                const bool got = mbar_wait(empty + s, (round & 1) ^ 1, a.err, kErrWaitProducer);
+                const bool got = mbar_wait(empty + s, (round & 1) ^ 1, a.err, kErrWaitProducer, a.wait_ns);
                 if (!__all_sync(0xffffffffu, got)) {
                     ok = false;
                     break;
@@ -442,7 +443,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             for (int i = 0; i < STAGES; ++i, ++it) {
                 const int s = it % STAGES;
                 const int round = it / STAGES;
-                const bool got = mbar_wait(empty + s, (round & 1) ^ 1, a.err, kErrWaitTail);
+                const bool got = mbar_wait(empty + s, (round & 1) ^ 1, a.err, kErrWaitTail, a.wait_ns);
                 if (!__all_sync(0xffffffffu, got)) break;
             }
         }
@@ -450,7 +451,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (!PAIR) {
 #pragma unroll
             for (int s = 0; s < STAGES; ++s)
-                if (last_round[s] >= 0) mbar_wait(full + s, last_round[s] & 1, a.err, kErrWaitTail);
+                if (last_round[s] >= 0) mbar_wait(full + s, last_round[s] & 1, a.err, kErrWaitTail, a.wait_ns);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
@@ -469,7 +470,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 const TileInfo ti = tc_decode_unit<MODE, BN, PAIR>(a, tabs, sc, item, rank);
                 const int b = tc & 1;
                 const int use = tc >> 1;
-                if (!mbar_wait(tempty + b, (use & 1) ^ 1, a.err, kErrWaitMma)) {
+                if (!mbar_wait(tempty + b, (use & 1) ^ 1, a.err, kErrWaitMma, a.wait_ns)) {
                     ok = false;
                     break;
                 }
@@ -480,7 +481,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 const uint32_t idesc = idesc0 | ((uint32_t)(n >> 3) << 17);
                 const uint32_t d0 = tmem_base + (uint32_t)(b * ACC);
                 for (int kb = 0; kb < ti.nk; ++kb) {
-                    if (!mbar_wait(full + s, phase, a.err, kErrWaitMma)) {
+                    if (!mbar_wait(full + s, phase, a.err, kErrWaitMma, a.wait_ns)) {
                         ok = false;
                         break;
                     }
@@ -519,7 +520,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 umma_commit_pair_local(drain);
             else
                 umma_commit(drain);
-            mbar_wait(drain, 0, a.err, kErrWaitMma);
+            mbar_wait(drain, 0, a.err, kErrWaitMma, a.wait_ns);
         }
     } else {
         // ------------------------------------------------------------ epilogue warps 2..9
@@ -638,7 +639,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const TileInfo ti = tc_decode_unit<MODE, BN, PAIR>(a, tabs, sc, item, rank);
             const int b = tc & 1;
             const int use = tc >> 1;
-            const bool got = mbar_wait(tfull + b, use & 1, a.err, kErrWaitEpilogue);
+            const bool got = mbar_wait(tfull + b, use & 1, a.err, kErrWaitEpilogue, a.wait_ns);
             if (!__all_sync(0xffffffffu, got)) break;
             tc_fence_after();
             const uint32_t tb = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(b * ACC);
@@ -782,11 +783,14 @@ static cudaError_t launch_tc(const TcMaps& maps, const TcArgs& a, int grid, bool
     if (err != cudaSuccess) return err;
     if (grid < 1) grid = 1;
     if (!PAIR) return launch_kernel(kernel, dim3(grid), dim3(kTcThreads), smem, s, pdl, maps, a);
-    // pairs: as many clusters of two as can be resident at once (persistent kernel)
+    // pairs: as many clusters of two as can be resident at once (persistent kernel), queried
+    // once per device
+    static std::mutex mu;
     static int clusters[64] = {0};
     int dev = 0;
     if ((err = cudaGetDevice(&dev)) != cudaSuccess) return err;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidValue;
+    std::unique_lock<std::mutex> lock(mu);
     if (clusters[dev] == 0) {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(grid & ~1);
@@ -805,6 +809,7 @@ static cudaError_t launch_tc(const TcMaps& maps, const TcArgs& a, int grid, bool
         clusters[dev] = n;
     }
     int pairs = grid / 2 < clusters[dev] ? grid / 2 : clusters[dev];
+    lock.unlock();
     if (pairs < 1) pairs = 1;
     return launch_kernel_cluster(kernel, dim3(2 * pairs), dim3(kTcThreads), smem, s, pdl, 2, maps, a);
 }
@@ -814,9 +819,11 @@ static cudaError_t launch_tc(const TcMaps& maps, const TcArgs& a, int grid, bool
 // variable MOE_B200_NO_PAIRS (any value) selects the wide tiles regardless.
 bool pair_tiles_available() {
     if (getenv("MOE_B200_NO_PAIRS")) return false;
+    static std::mutex mu;
     static int state[64] = {0};   // 0 unknown, 1 yes, -1 no
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+    std::lock_guard<std::mutex> lock(mu);
     if (state[dev] == 0) {
         bool ok = true;
         auto probe = [&](const void* kernel, int smem) {

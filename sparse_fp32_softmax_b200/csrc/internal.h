@@ -7,7 +7,8 @@
 
 namespace moe {
 
-// Every bounded wait gives up after this long and reports it in the device error word.
+// Every bounded wait gives up after this long (unless the call sets a shorter limit) and
+// reports it in the device error word.
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
 
 // Bits of the device error word (first int of the workspace).
@@ -51,12 +52,16 @@ constexpr int kGatherMaxT = 32;
 enum { kTilesNarrow = 0, kTilesWide = 1, kTilesPair = 2 };
 constexpr int kPairStages = 6;   // 6 x (16 KB weights + 16 KB tokens) per CTA
 
-// Split tail items of the narrow-tile GEMMs: at most this many K slices per item, and
-// partial-sum slots for one wave (a tail is split only when it is at most half a wave, so
-// the tickets of at most kSplitSlots / 2 items x 8 epilogue warps are in use).
+// Split tail items of the narrow-tile GEMMs: at most this many K slices per item, and a
+// fixed capacity of FP32 partial-sum slots (slices per item are capped so that the tail's
+// slices fit; a device with fewer SMs splits less).  A tail is split only when it is at most
+// half a wave of the grid, so at most grid / 2 items x 8 epilogue warps hold a ticket; the
+// persistent expert GEMMs therefore run at most kMaxTcGrid CTAs.
 constexpr int kMaxKSplit = 8;
 constexpr int kSplitSlots = 148;
 constexpr int kSplitTickets = 1024;   // per GEMM; the completion counters follow them
+constexpr int kMaxTcGrid = 2 * kSplitTickets / 8;
+static_assert(kMaxTcGrid / 2 * 8 <= kSplitTickets, "split-tail tickets");
 __host__ __device__ inline bool use_narrow_tiles(long long T, int k, int E) {
     return T * k <= (long long)kNarrowMaxMeanRows * E;
 }
@@ -77,8 +82,6 @@ struct SegTables {
     int* seg_start;   // [nseg] first permuted row of each segment
     int* gu_items;    // [nseg + 1] prefix sums of tcgen05 gate_up work items
     int* dn_items;    // [nseg + 1] prefix sums of tcgen05 down work items
-    int* gu_tasks;    // [nseg + 1] prefix sums of streaming gate_up tasks
-    int* dn_tasks;    // [nseg + 1] prefix sums of streaming down tasks
 };
 
 struct PermuteArgs {
@@ -137,23 +140,6 @@ inline int router_splits(int T, int E, int D, int bn) {
     return s < 1 ? 1 : (int)s;
 }
 
-struct StreamArgs {
-    const uint16_t* x;        // [T, D]
-    const uint16_t* W_gu;     // [E, 2I, D]
-    const uint16_t* W_dn;     // [E, D, I]
-    const uint16_t* S_gu;     // [2I_s, D] or null
-    const uint16_t* S_dn;     // [D, I_s] or null
-    int D, I, I_s, E, nseg;
-    SegTables tables;
-    const int32_t* row_token;
-    const float* row_weight;
-    const int32_t* row_dest;
-    uint16_t* h;              // [rows, ld_h] bf16 SwiGLU output
-    int ld_h;
-    float* slots;             // [T * S, D] FP32
-    int* err;
-};
-
 // Tensor maps of one grouped GEMM: the weight operand (routed experts, shared expert) and
 // the token operand encoded at five box heights (16, 32, 64, 128, 256 rows), so that a work
 // item loads only as many token rows as it has (rounded up to the next height).
@@ -197,11 +183,16 @@ struct TcArgs {
     int ksplit;
     int T;
     int* err;
+    unsigned long long wait_ns;   // limit of every bounded wait (kWaitLimitNs by default)
 };
 
 // Raise a kernel's dynamic shared-memory limit once per device (host-side attribute; done
 // outside stream capture by the first call on each device).
 cudaError_t ensure_smem_attr(const void* kernel, int bytes);
+
+// Streaming multiprocessors of the current device (queried once per device; 0 on error).
+// Launchers size their grids from it.
+int device_sm_count();
 
 // ---------------------------------------------------------------- launchers (return the
 // launch error, cudaSuccess when all kernels were enqueued).  pdl: launch the first kernel
@@ -217,8 +208,6 @@ cudaError_t launch_route_fused(const RouteArgs& a, bool pdl, cudaStream_t s);
 cudaError_t launch_select_permute(const RouteArgs& a, bool pdl, cudaStream_t s);
 cudaError_t launch_gather_rows(const uint16_t* x, const int32_t* row_token, int rows, int D,
                                uint16_t* x_perm, bool pdl, cudaStream_t s);
-cudaError_t launch_stream_gate_up(const StreamArgs& a, int max_rows, bool pdl, cudaStream_t s);
-cudaError_t launch_stream_down(const StreamArgs& a, int max_rows, bool pdl, cudaStream_t s);
 bool pair_tiles_available();
 cudaError_t launch_tc_router(const TcMaps& maps, const TcArgs& a, int num_sms, bool pdl,
                              cudaStream_t s);

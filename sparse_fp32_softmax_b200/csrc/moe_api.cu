@@ -37,11 +37,29 @@ cudaError_t ensure_smem_attr(const void* kernel, int bytes) {
     return cudaSuccess;
 }
 
+int device_sm_count() {
+    static std::mutex mu;
+    static int cache[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+    std::lock_guard<std::mutex> lock(mu);
+    if (cache[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+        cache[dev] = n;
+    }
+    return cache[dev];
+}
+
 }  // namespace moe
 
 namespace {
 
 constexpr size_t kAlign = 256;
+// Ints of the ticket region: gate_up split tickets, down split tickets, the per-expert
+// completion counters of gate_up (nseg + 1 <= kMaxSegments + 1), and the same number of
+// counters that stay zero (MOE_DIAG_UNSIGNALLED_HANDOFF points the down GEMM at them).
+constexpr int kTicketInts = 2 * kSplitTickets + 2 * (kMaxSegments + 1);
 
 // The cudaError_t of the last CUDA failure seen by this host thread (moe_last_cuda_error).
 thread_local int g_last_cuda_error = 0;
@@ -55,7 +73,7 @@ bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 struct Plan {
     int T, D, E, k, I, I_s, has_shared, S, R, ld_h, nchunks, nseg, rsplit;
     size_t err, tickets, partial, logits, idx, w, counts, offsets, chunk, seg_count, seg_start, gu_items, dn_items,
-        gu_tasks, dn_tasks, row_token, row_weight, row_dest, slot_row, x_perm, h, slots, total;
+        row_token, row_weight, row_dest, slot_row, x_perm, h, slots, total;
 };
 
 Plan make_plan(const moe_dims& d, const moe_opts* o) {
@@ -72,9 +90,10 @@ Plan make_plan(const moe_dims& d, const moe_opts* o) {
     size_t off = 0;
     auto take = [&](size_t bytes) { size_t at = off; off += align_up(bytes); return at; };
     p.err = take(kAlign);                              // [0] error word, [1] routing ticket
-    // split-tail tickets of gate_up and of down, then the per-expert completion counters
-    // (all follow err, so one memset clears the header)
-    p.tickets = take((size_t)3 * kSplitTickets * 4);
+    // split-tail tickets of gate_up and of down, the per-expert completion counters, and a
+    // block of counters that no kernel increments (the watchdog diagnostic); all follow err,
+    // so one memset clears the header
+    p.tickets = take((size_t)kTicketInts * 4);
     // split-tail partial accumulators: gate_up (two accumulators), then down (one)
     p.partial = take(use_narrow_tiles(p.T, p.k, p.E)
                          ? (size_t)kSplitSlots * 3 * kTcM * kNarrowBN * 4 : 0);
@@ -88,8 +107,6 @@ Plan make_plan(const moe_dims& d, const moe_opts* o) {
     p.seg_start = take((size_t)(p.nseg + 1) * 4);
     p.gu_items = take((size_t)(p.nseg + 2) * 4);
     p.dn_items = take((size_t)(p.nseg + 2) * 4);
-    p.gu_tasks = take((size_t)(p.nseg + 2) * 4);
-    p.dn_tasks = take((size_t)(p.nseg + 2) * 4);
     p.row_token = take((size_t)p.R * 4);
     p.row_weight = take((size_t)p.R * 4);
     p.row_dest = take((size_t)p.R * 4);
@@ -129,35 +146,30 @@ moe_status check_opts(const moe_dims* d, const moe_opts* o) {
     if (o->logits_out && !aligned(o->logits_out, 4)) return MOE_ERR_INVALID_ARG;
     if (o->topk_idx_out && !aligned(o->topk_idx_out, 4)) return MOE_ERR_INVALID_ARG;
     if (o->topk_w_out && !aligned(o->topk_w_out, 4)) return MOE_ERR_INVALID_ARG;
-    if (o->path < MOE_PATH_AUTO || o->path > MOE_PATH_GROUPED) return MOE_ERR_INVALID_ARG;
+    if (o->path != MOE_PATH_AUTO && o->path != MOE_PATH_GROUPED) return MOE_ERR_INVALID_ARG;
+    if (o->expert_counts_out && !aligned(o->expert_counts_out, 4)) return MOE_ERR_INVALID_ARG;
+    if (o->slot_row_out && !aligned(o->slot_row_out, 4)) return MOE_ERR_INVALID_ARG;
+    if (o->diag != 0 && o->diag != MOE_DIAG_UNSIGNALLED_HANDOFF) return MOE_ERR_INVALID_ARG;
+    if (o->diag == MOE_DIAG_UNSIGNALLED_HANDOFF && !use_narrow_tiles(d->T, d->k, d->E))
+        return MOE_ERR_UNSUPPORTED;
     if (o->n_stage_events != 0 && o->n_stage_events != 6) return MOE_ERR_INVALID_ARG;
     if (o->n_stage_events == 6 && !o->stage_events) return MOE_ERR_INVALID_ARG;
     if (o->out_f32 && !aligned(o->out_f32, 16)) return MOE_ERR_INVALID_ARG;
-    (void)d;
     return MOE_OK;
 }
 
 // ------------------------------------------------------------------ device properties / TMA
 
+// SM count of the current device; on failure 0, with the CUDA error kept for
+// moe_last_cuda_error.
 int num_sms_of_current_device() {
-    static int cache[64] = {0};
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) {
-        g_last_cuda_error = (int)e;
-        return 0;
+    const int n = device_sm_count();
+    if (n <= 0) {
+        int dev = 0;
+        const cudaError_t e = cudaGetDevice(&dev);
+        g_last_cuda_error = e != cudaSuccess ? (int)e : (int)cudaErrorInvalidDevice;
     }
-    if (dev < 0 || dev >= 64) return 0;
-    if (cache[dev] == 0) {
-        int n = 0;
-        e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-        if (e != cudaSuccess) {
-            g_last_cuda_error = (int)e;
-            return 0;
-        }
-        cache[dev] = n;
-    }
-    return cache[dev];
+    return n;
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -255,8 +267,6 @@ SegTables tables_of(const Plan& p, void* ws) {
     t.seg_start = at<int>(ws, p.seg_start);
     t.gu_items = at<int>(ws, p.gu_items);
     t.dn_items = at<int>(ws, p.dn_items);
-    t.gu_tasks = at<int>(ws, p.gu_tasks);
-    t.dn_tasks = at<int>(ws, p.dn_tasks);
     return t;
 }
 
@@ -278,6 +288,7 @@ moe_status run_logits(const moe_bf16* x, const moe_bf16* W_r, const Plan& p, flo
     a.logits = part;
     a.ksplit = p.rsplit;
     a.err = at<int>(ws, p.err);
+    a.wait_ns = kWaitLimitNs;
     const int sms = num_sms_of_current_device();
     if (sms <= 0) return MOE_ERR_CUDA;
     MOE_CUDA(launch_tc_router(maps, a, sms, false, s));
@@ -366,7 +377,7 @@ moe_status moe_permute(const int32_t* topk_idx, const float* topk_w, const moe_b
     a.row_dest = nullptr;
     a.slot_row = slot_row;
     a.cap = cap;
-    a.tables = SegTables{nullptr, nullptr, nullptr, nullptr, nullptr, nullptr};
+    a.tables = SegTables{nullptr, nullptr, nullptr, nullptr};
     a.gu_bn = kGuBN;
     a.dn_bn = kDnBN;
     a.gu_features = kGuILFeatures;
@@ -396,10 +407,6 @@ moe_status moe_forward_ex(const moe_bf16* x, const moe_bf16* W_r, const moe_bf16
     const Plan p = make_plan(*dims, opts);
     if (ws_bytes < p.total) return MOE_ERR_WORKSPACE;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    const int path_req = opts ? opts->path : MOE_PATH_AUTO;
-    // AUTO takes the tensor-core grouped path at every T: measured on B200 it beats the
-    // register-streaming path from T = 1 up (its 2-D TMA weight tiles keep HBM busier)
-    const bool streaming = path_req == MOE_PATH_STREAM;
     const int sms = num_sms_of_current_device();
     if (sms <= 0) return MOE_ERR_CUDA;
 
@@ -414,6 +421,8 @@ moe_status moe_forward_ex(const moe_bf16* x, const moe_bf16* W_r, const moe_bf16
     const moe_bf16* sg = opts ? opts->shared_gate : nullptr;
     const moe_bf16* residual = opts ? opts->residual : nullptr;
     float* out_f32 = opts ? opts->out_f32 : nullptr;
+    const unsigned long long wait_ns =
+        (opts && opts->wait_limit_us) ? (unsigned long long)opts->wait_limit_us * 1000ull : kWaitLimitNs;
 
     // tensor maps of the grouped path are encoded before anything is enqueued
     // narrow tiles (deeper pipelines) when experts average few rows; a segment with more
@@ -425,7 +434,7 @@ moe_status moe_forward_ex(const moe_bf16* x, const moe_bf16* W_r, const moe_bf16
     // tiles and experts average at least 256 rows (measured on B200: with fewer rows the
     // pair tiles' narrower N and halved item count cost more than the pairs save).
     // (devices that cannot co-schedule the pairs take the one-CTA wide tiles)
-    const bool pairs = !narrow && !streaming && pair_tiles_available();
+    const bool pairs = !narrow && pair_tiles_available();
     const int gu_tiles = narrow ? kTilesNarrow : (pairs ? kTilesPair : kTilesWide);
     const int dn_tiles = narrow ? kTilesNarrow
                          : (pairs && p.D % 256 == 0 && (long long)p.T * p.k >= 256ll * p.E)
@@ -435,7 +444,7 @@ moe_status moe_forward_ex(const moe_bf16* x, const moe_bf16* W_r, const moe_bf16
     const int dn_bn = narrow ? kNarrowBN : kDnBN;
     const int b_box_max = gu_tiles == kTilesPair ? kGuBN / 2 : gu_bn;   // token rows per CTA
     TcMaps mGu, mDn;
-    if (!streaming) {
+    {
         uint16_t* h = at<uint16_t>(ws, p.h);
         const bool gu_b_ok = gather ? make_map(&mGu.B[0], x, p.D, p.T, 1)
                                     : make_b_maps(mGu.B, at<uint16_t>(ws, p.x_perm), p.D, p.R, b_box_max);
@@ -456,8 +465,8 @@ moe_status moe_forward_ex(const moe_bf16* x, const moe_bf16* W_r, const moe_bf16
             for (int bi = 1; bi < kNumBBoxes; ++bi) mGu.B[bi] = mGu.B[0];
     }
 
-    // the header of the workspace: device error word, routing ticket, split-tail tickets
-    MOE_CUDA(cudaMemsetAsync(err, 0, p.tickets - p.err + (size_t)3 * kSplitTickets * 4, s));
+    // the header of the workspace: device error word, routing ticket, tickets and counters
+    MOE_CUDA(cudaMemsetAsync(err, 0, p.tickets - p.err + (size_t)kTicketInts * 4, s));
     if ((st = record(opts, 0, s)) != MOE_OK) return st;
     // T <= 32: one kernel routes and permutes.  Above: router partial sums, then selection and
     // permutation (one kernel while T*k fits a single permutation block).
@@ -481,12 +490,12 @@ moe_status moe_forward_ex(const moe_bf16* x, const moe_bf16* W_r, const moe_bf16
     pa.D = p.D; pa.I = p.I; pa.I_s = p.I_s;
     pa.chunk_counts = at<int>(ws, p.chunk);
     pa.nchunks = p.nchunks;
-    pa.counts = at<int>(ws, p.counts);
+    pa.counts = (opts && opts->expert_counts_out) ? opts->expert_counts_out : at<int>(ws, p.counts);
     pa.offsets = at<int>(ws, p.offsets);
     pa.row_token = at<int32_t>(ws, p.row_token);
     pa.row_weight = at<float>(ws, p.row_weight);
     pa.row_dest = at<int32_t>(ws, p.row_dest);
-    pa.slot_row = at<int32_t>(ws, p.slot_row);
+    pa.slot_row = (opts && opts->slot_row_out) ? opts->slot_row_out : at<int32_t>(ws, p.slot_row);
     pa.cap = p.R;
     pa.tables = tables_of(p, ws);
     pa.gu_bn = gu_bn;
@@ -515,59 +524,45 @@ moe_status moe_forward_ex(const moe_bf16* x, const moe_bf16* W_r, const moe_bf16
     } else {
         MOE_CUDA(launch_permute(pa, chain, s));
     }
-    if (!streaming && !gather)
+    if (!gather)
         MOE_CUDA(launch_gather_rows(x, pa.row_token, p.R, p.D, at<uint16_t>(ws, p.x_perm), true, s));
     if ((st = record(opts, 2, s)) != MOE_OK) return st;
 
-    if (streaming) {
-        StreamArgs sa{};
-        sa.x = x; sa.W_gu = W_gate_up; sa.W_dn = W_down; sa.S_gu = sgu; sa.S_dn = sdn;
-        sa.D = p.D; sa.I = p.I; sa.I_s = p.I_s; sa.E = p.E; sa.nseg = p.nseg;
-        sa.tables = pa.tables;
-        sa.row_token = pa.row_token;
-        sa.row_weight = pa.row_weight;
-        sa.row_dest = pa.row_dest;
-        sa.h = at<uint16_t>(ws, p.h);
-        sa.ld_h = p.ld_h;
-        sa.slots = at<float>(ws, p.slots);
-        sa.err = err;
-        MOE_CUDA(launch_stream_gate_up(sa, p.T, chain, s));
-        if ((st = record(opts, 3, s)) != MOE_OK) return st;
-        MOE_CUDA(launch_stream_down(sa, p.T, chain, s));
-        if ((st = record(opts, 4, s)) != MOE_OK) return st;
-        MOE_CUDA(launch_combine(sa.slots, p.T, p.D, p.k, p.has_shared, x, sg, residual, out,
-                                out_f32, chain, s));
-    } else {
-        TcArgs ta{};
-        ta.D = p.D; ta.I = p.I; ta.I_s = p.I_s; ta.E = p.E; ta.nseg = p.nseg; ta.T = p.T;
-        ta.tables = pa.tables;
-        ta.row_token = pa.row_token;
-        ta.gather = gather ? 1 : 0;
-        ta.h = at<uint16_t>(ws, p.h);
-        ta.ld_h = p.ld_h;
-        ta.row_weight = pa.row_weight;
-        ta.row_dest = pa.row_dest;
-        ta.slots = at<float>(ws, p.slots);
-        ta.partial = narrow ? at<float>(ws, p.partial) : nullptr;
-        ta.tickets = at<int>(ws, p.tickets);
-        ta.partial_slots = narrow ? kSplitSlots : 0;
-        // narrow tiles: gate_up reports each finished expert; down waits per expert
-        ta.seg_done = narrow ? at<int>(ws, p.tickets) + 2 * kSplitTickets : nullptr;
-        ta.gu_prefix = pa.tables.gu_items;
-        TcArgs tdn = ta;
-        tdn.dep_wait = narrow ? 1 : 0;
-        if (narrow) {
-            tdn.partial = at<float>(ws, p.partial) + (size_t)kSplitSlots * 2 * kTcM * kNarrowBN;
-            tdn.tickets = at<int>(ws, p.tickets) + kSplitTickets;
-        }
-        ta.err = err;
-        MOE_CUDA(launch_tc_gate_up(mGu, ta, sms, gu_tiles, chain, s));
-        if ((st = record(opts, 3, s)) != MOE_OK) return st;
-        MOE_CUDA(launch_tc_down(mDn, tdn, sms, dn_tiles, chain, s));
-        if ((st = record(opts, 4, s)) != MOE_OK) return st;
-        MOE_CUDA(launch_combine(ta.slots, p.T, p.D, p.k, p.has_shared, x, sg, residual, out,
-                                out_f32, chain, s));
+    int* tickets = at<int>(ws, p.tickets);
+    TcArgs ta{};
+    ta.D = p.D; ta.I = p.I; ta.I_s = p.I_s; ta.E = p.E; ta.nseg = p.nseg; ta.T = p.T;
+    ta.tables = pa.tables;
+    ta.row_token = pa.row_token;
+    ta.gather = gather ? 1 : 0;
+    ta.h = at<uint16_t>(ws, p.h);
+    ta.ld_h = p.ld_h;
+    ta.row_weight = pa.row_weight;
+    ta.row_dest = pa.row_dest;
+    ta.slots = at<float>(ws, p.slots);
+    ta.partial = narrow ? at<float>(ws, p.partial) : nullptr;
+    ta.tickets = tickets;
+    ta.partial_slots = narrow ? kSplitSlots : 0;
+    // narrow tiles: gate_up reports each finished expert; down waits per expert
+    ta.seg_done = narrow ? tickets + 2 * kSplitTickets : nullptr;
+    ta.gu_prefix = pa.tables.gu_items;
+    ta.err = err;
+    ta.wait_ns = wait_ns;
+    TcArgs tdn = ta;
+    tdn.dep_wait = narrow ? 1 : 0;
+    if (narrow) {
+        tdn.partial = at<float>(ws, p.partial) + (size_t)kSplitSlots * 2 * kTcM * kNarrowBN;
+        tdn.tickets = tickets + kSplitTickets;
+        // watchdog diagnostic: down watches counters that no kernel increments
+        if (opts && opts->diag == MOE_DIAG_UNSIGNALLED_HANDOFF)
+            tdn.seg_done = tickets + 2 * kSplitTickets + (kMaxSegments + 1);
     }
+    const int grid = sms < kMaxTcGrid ? sms : kMaxTcGrid;
+    MOE_CUDA(launch_tc_gate_up(mGu, ta, grid, gu_tiles, chain, s));
+    if ((st = record(opts, 3, s)) != MOE_OK) return st;
+    MOE_CUDA(launch_tc_down(mDn, tdn, grid, dn_tiles, chain, s));
+    if ((st = record(opts, 4, s)) != MOE_OK) return st;
+    MOE_CUDA(launch_combine(ta.slots, p.T, p.D, p.k, p.has_shared, x, sg, residual, out,
+                            out_f32, chain, s));
     return record(opts, 5, s);
 }
 
@@ -580,9 +575,13 @@ moe_status moe_forward(const moe_bf16* x, const moe_bf16* W_r, const moe_bf16* W
 moe_status moe_get_device_status(const void* ws, moe_stream_t stream) {
     if (!ws || !aligned(ws, kAlign)) return MOE_ERR_INVALID_ARG;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
+    cudaError_t e = cudaStreamSynchronize(s);
     int word = 0;
-    if (cudaMemcpy(&word, ws, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+    if (e == cudaSuccess) e = cudaMemcpy(&word, ws, sizeof(int), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) {
+        g_last_cuda_error = (int)e;
+        return MOE_ERR_CUDA;
+    }
     if (word & kErrBadIndex) return MOE_ERR_INVALID_ARG;
     if (word) return MOE_ERR_DEVICE_TIMEOUT;
     return MOE_OK;

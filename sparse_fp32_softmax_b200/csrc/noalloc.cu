@@ -1,20 +1,21 @@
 // noalloc.cu -- moe_forward for callers that cannot allocate device memory.
 //
 // Some callers cannot call cudaMalloc (or any allocating routine) at the point where they
-// run the block: code that enqueues work while a stream is being captured into a CUDA
-// graph, plugin hosts that hand a kernel only its input and output buffers and no
-// workspace, and runtimes that forbid device allocation after start-up.  For them the
-// scratch memory of the forward pass lives in a fixed array in the library's own device
-// memory, declared below.  Every GPU that loads this part of the library keeps that array
-// until the process exits.
+// run the block: plugin hosts that hand a kernel only its input and output buffers and no
+// workspace, and runtimes that plan all device memory up front and forbid allocation once
+// they have started.  For them the scratch memory of the forward pass lives in a fixed
+// array in the library's own device memory, declared below.  Every GPU that loads this
+// part of the library keeps that array until the process exits.
 //
 // The array holds the same workspace moe_forward uses (routing tables, permutation, the
 // SwiGLU intermediate and the FP32 slot buffer).  Its size bounds the problem: calls whose
 // workspace would exceed it are refused with MOE_ERR_WORKSPACE before anything runs.
 // All calls on a device share the one array and each call leaves its contents behind; the
-// forward pass clears what must start at zero (the device error word) and overwrites the
-// rest before reading it.  Calls whose work can overlap on the GPU (different streams, or
-// different host threads without ordering) race on the array and must not be issued.
+// forward pass clears what must start at zero (the device error word, tickets and counters
+// at the start of the array) and overwrites the rest before reading it.  Calls whose work
+// can overlap on the GPU (different streams, or different host threads without ordering)
+// race on the array and must not be issued.  The error word the last call left stays in
+// the array's first int, where moe_get_device_status_noalloc reads it.
 #include <mutex>
 
 #include "../../include/moe_b200.h"
@@ -57,6 +58,12 @@ moe_status moe_forward_noalloc(const moe_bf16* x, const moe_bf16* W_r, const moe
     void* ws = scratch_address_of_current_device();
     if (!ws) return MOE_ERR_CUDA;
     return moe_forward(x, W_r, W_gate_up, W_down, dims, out, ws, kNoAllocScratchBytes, stream);
+}
+
+moe_status moe_get_device_status_noalloc(moe_stream_t stream) {
+    void* ws = scratch_address_of_current_device();
+    if (!ws) return MOE_ERR_CUDA;
+    return moe_get_device_status(ws, stream);
 }
 
 }  // extern "C"

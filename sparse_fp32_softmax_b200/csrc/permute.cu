@@ -146,7 +146,9 @@ cudaError_t launch_gather_rows(const uint16_t* x, const int32_t* row_token, int 
                                uint16_t* x_perm, bool pdl, cudaStream_t s) {
     if (rows <= 0) return cudaSuccess;
     int blocks = (rows + 7) / 8;
-    if (blocks > 148 * 8) blocks = 148 * 8;
+    const int sms = device_sm_count();
+    if (sms <= 0) return cudaErrorInvalidDevice;
+    if (blocks > sms * 8) blocks = sms * 8;
     return launch_kernel(gather_rows_kernel, dim3(blocks), dim3(256), 0, s, pdl, x, row_token, rows,
                          D, x_perm);
 }

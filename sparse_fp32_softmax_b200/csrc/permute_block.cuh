@@ -7,17 +7,17 @@
 
 namespace moe {
 
-// Block-wide exclusive scan of five ints per thread at once (blockDim.x <= 1024, a multiple
+// Block-wide exclusive scan of three ints per thread at once (blockDim.x <= 1024, a multiple
 // of 32): v[j] becomes its exclusive prefix over the block, tot[j] the block's sum.  Two
 // __syncthreads.
-static __device__ void block_exclusive_scan5(int (&v)[5], int (&tot)[5]) {
-    __shared__ int wsum[32][5];
-    __shared__ int wtot[5];
+static __device__ void block_exclusive_scan3(int (&v)[3], int (&tot)[3]) {
+    __shared__ int wsum[32][3];
+    __shared__ int wtot[3];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int nwarps = blockDim.x >> 5;
-    int inc[5];
+    int inc[3];
 #pragma unroll
-    for (int j = 0; j < 5; ++j) {
+    for (int j = 0; j < 3; ++j) {
         inc[j] = v[j];
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -29,7 +29,7 @@ static __device__ void block_exclusive_scan5(int (&v)[5], int (&tot)[5]) {
     __syncthreads();
     if (warp == 0) {
 #pragma unroll
-        for (int j = 0; j < 5; ++j) {
+        for (int j = 0; j < 3; ++j) {
             const int w = lane < nwarps ? wsum[lane][j] : 0;
             int winc = w;
 #pragma unroll
@@ -43,7 +43,7 @@ static __device__ void block_exclusive_scan5(int (&v)[5], int (&tot)[5]) {
     }
     __syncthreads();
 #pragma unroll
-    for (int j = 0; j < 5; ++j) {
+    for (int j = 0; j < 3; ++j) {
         v[j] = wsum[warp][j] + inc[j] - v[j];
         tot[j] = wtot[j];
     }
@@ -57,7 +57,7 @@ static __device__ void finish_offsets(const PermuteArgs& a, const int* s_cnt, in
     const int E = a.E;
     const int nseg = E + (a.has_shared ? 1 : 0);
     const int s = threadIdx.x;
-    int v[5] = {0, 0, 0, 0, 0};   // padded rows, gate_up items, down items, gate_up tasks, down tasks
+    int v[3] = {0, 0, 0};   // padded rows, gate_up items, down items
     int c = 0;
     if (s < nseg) {
         c = (s == E) ? a.T : s_cnt[s];
@@ -66,12 +66,10 @@ static __device__ void finish_offsets(const PermuteArgs& a, const int* s_cnt, in
             const int Iseg = (s == E) ? a.I_s : a.I;
             v[1] = (c + a.gu_bn - 1) / a.gu_bn * (Iseg / a.gu_features);
             v[2] = (c + a.dn_bn - 1) / a.dn_bn * (a.D / a.dn_rows);
-            v[3] = Iseg / 8;     // streaming gate_up: one warp per 8 features
-            v[4] = a.D / 16;     // streaming down: one warp per 16 output rows
         }
     }
-    int tot[5];
-    block_exclusive_scan5(v, tot);
+    int tot[3];
+    block_exclusive_scan3(v, tot);
     if (s < E) {
         a.counts[s] = c;
         a.offsets[s] = v[0];
@@ -91,8 +89,6 @@ static __device__ void finish_offsets(const PermuteArgs& a, const int* s_cnt, in
     if (a.tables.gu_items && s <= nseg) {
         a.tables.gu_items[s] = s < nseg ? v[1] : tot[1];
         a.tables.dn_items[s] = s < nseg ? v[2] : tot[2];
-        a.tables.gu_tasks[s] = s < nseg ? v[3] : tot[3];
-        a.tables.dn_tasks[s] = s < nseg ? v[4] : tot[4];
     }
     __syncthreads();
 }

@@ -81,7 +81,9 @@ cudaError_t launch_route_fused(const RouteArgs& a, bool pdl, cudaStream_t s) {
                           : route_fused_kernel<16>;
     cudaError_t err = ensure_smem_attr((const void*)k_, 32 * kMaxE * 4);
     if (err != cudaSuccess) return err;
-    const int blocks = a.E < 148 ? a.E : 148;
+    const int sms = device_sm_count();
+    if (sms <= 0) return cudaErrorInvalidDevice;
+    const int blocks = a.E < sms ? a.E : sms;
     return launch_kernel(k_, dim3(blocks), dim3(1024), smem, s, pdl, a);
 }
 

@@ -76,7 +76,9 @@ cudaError_t launch_router_small(const uint16_t* x, const uint16_t* W_r, int T, i
     const long ntask = (long)E * ((T + 7) / 8);
     const int warps_per_block = 8;
     long blocks = (ntask + warps_per_block - 1) / warps_per_block;
-    if (blocks > 148 * 16) blocks = 148 * 16;
+    const int sms = device_sm_count();
+    if (sms <= 0) return cudaErrorInvalidDevice;
+    if (blocks > sms * 16) blocks = sms * 16;
     return launch_kernel(router_small_kernel, dim3((int)blocks), dim3(warps_per_block * 32), 0, s, pdl,
                          x, W_r, T, D, E, logits);
 }
@@ -104,7 +106,9 @@ cudaError_t launch_select(const float* part, int nsplit, const float* bias, int 
                           cudaStream_t s) {
     const int threads = 256;
     int blocks = (T + 7) / 8;
-    if (blocks > 148 * 32) blocks = 148 * 32;
+    const int sms = device_sm_count();
+    if (sms <= 0) return cudaErrorInvalidDevice;
+    if (blocks > sms * 32) blocks = sms * 32;
     if (blocks < 1) blocks = 1;
     void (*k_)(const float*, int, const float*, int, int, int, int, int32_t*, float*, float*) =
         E <= 32 ? select_kernel<1> : E <= 64 ? select_kernel<2> : E <= 128 ? select_kernel<4>

@@ -27,7 +27,7 @@ def test_library_exports_every_declared_function(lib):
     declared = B.header_functions()
     assert set(declared) == {"moe_workspace_size", "moe_route", "moe_permute", "moe_forward",
                              "moe_forward_ex", "moe_forward_noalloc", "moe_get_device_status",
-                             "moe_status_string", "moe_last_cuda_error"}
+                             "moe_get_device_status_noalloc", "moe_status_string", "moe_last_cuda_error"}
     out = subprocess.run(["nm", "-D", "--defined-only", LIB], capture_output=True, text=True, check=True).stdout
     exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
     for name in declared:
@@ -100,6 +100,16 @@ def test_forward_rejects_bad_arguments_before_launch(lib):
     o = B.moe_opts()
     o.n_stage_events = 3
     assert _fwd(lib, d, n, opts=o) == B.MOE_ERR_INVALID_ARG
+    o = B.moe_opts()
+    o.diag = 2                                  # no such diagnostic
+    assert _fwd(lib, d, n, opts=o) == B.MOE_ERR_INVALID_ARG
+    o = B.moe_opts()
+    o.slot_row_out = FAKE + 2                   # misaligned routing-table output
+    assert _fwd(lib, d, n, opts=o) == B.MOE_ERR_INVALID_ARG
+    o = B.moe_opts()
+    o.diag = B.MOE_DIAG_UNSIGNALLED_HANDOFF     # wide shape (T*k > 32*E): no hand-off wait
+    wide = B.make_dims(512, 256, 8, 2, 128)
+    assert _fwd(lib, wide, B.moe_workspace_size(wide), opts=o) == B.MOE_ERR_UNSUPPORTED
 
 
 @no_gpu
@@ -127,6 +137,7 @@ def test_permute_and_route_validation(lib):
     assert lib.moe_route(None, p(FAKE), None, ctypes.byref(d), None, p(FAKE), p(FAKE), p(FAKE), n,
                          None) == B.MOE_ERR_INVALID_ARG
     assert lib.moe_get_device_status(None, None) == B.MOE_ERR_INVALID_ARG
+    assert lib.moe_get_device_status_noalloc(None) == B.MOE_ERR_CUDA     # no device here
 
 
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):

@@ -96,15 +96,8 @@ def test_peaks_and_profile_lookup(tmp_path, monkeypatch):
     assert bench.profile_traffic("tag") is None
 
 
-def test_bench_attaches_traffic_to_the_roofline():
-    text = open(os.path.join(bench.ROOT, "bench.py")).read()
-    assert 'roof["traffic"] = profile_traffic(tag)' in text
-
-
 def test_kernels_per_forward_follows_the_launch_sequence():
     # fused routing (T <= 32); router + select/permute + row copy (T*k <= 4096); full
-    # permutation (4 kernels) above; then gate_up, down, combine.  The streaming path
-    # has no row copy.
-    assert [bench.kernels_per_forward(T, 8, False) for T in (1, 32, 33, 256, 512, 8192)] == \
+    # permutation (4 kernels) above; then gate_up, down, combine.
+    assert [bench.kernels_per_forward(T, 8) for T in (1, 32, 33, 256, 512, 8192)] == \
         [4, 4, 6, 6, 6, 9]
-    assert bench.kernels_per_forward(256, 8, True) == 5

@@ -1,8 +1,9 @@
 """GPU parity of the CUDA path (through the C ABI) against the CPU oracle.
 
-Stage-wise (router, permutation) and end to end (the whole block) on all five standard
-workloads, both expert paths, and the edge cases: T = 1, ragged T, k = 1, k = E, E = 1,
-norm_topk_prob off, all tokens on one expert, zero input, E = 512 with k = 16.
+Stage-wise (router, permutation) and end to end (the whole block) on the standard
+workloads, and the edge cases: T = 1, ragged T, k = 1, k = E, E = 1, norm_topk_prob off,
+all tokens on one expert, zero input, E = 512 with k = 16.  The 48-block residual chain is
+in test_gpu_chain.py, failure detection in test_gpu_failure.py.
 """
 import os
 
@@ -14,7 +15,7 @@ from oracle import oracle as O
 from sparse_fp32_softmax_b200 import binding as B
 from sparse_fp32_softmax_b200 import inputs
 from tests.parity_util import (W_ATOL, assert_block_output, assert_y_close, check_routing,
-                               logit_deltas, y_errors)
+                               logit_deltas)
 
 pytestmark = pytest.mark.gpu
 
@@ -72,7 +73,7 @@ def compare_block(cfg, L, G, rows, path="auto", x_cpu=None, residual_cpu=None, k
     norm = cfg.norm_topk_prob if norm is None else norm
     x_cpu = L["x"] if x_cpu is None else x_cpu
     res_gpu = residual_cpu.cuda() if residual_cpu is not None else None
-    y, idx, w, logits = run_forward(cfg, G, path, x=x_cpu.cuda(), residual=res_gpu, k=k, norm=norm)
+    y, idx, w, logits = run_forward(cfg, G, x=x_cpu.cuda(), residual=res_gpu, k=k, norm=norm)
     y32 = run_forward.last_f32
     rows = np.asarray(sorted(set(int(r) for r in rows)), np.int32)
     # selection from the GPU's own logits is bit-exact; weights within 1e-6
@@ -175,20 +176,18 @@ def test_permute_bit_exact(tile_m, T, k, E):
 
 # ------------------------------------------------------------------ whole block
 
-@pytest.mark.parametrize("path", ["stream", "grouped"])
-def test_forward_tiny(path):
+def test_forward_tiny():
     cfg, L, G = layer("tiny")
-    r = compare_block(cfg, L, G, range(cfg.T), path=path, what=f"tiny/{path}")
+    r = compare_block(cfg, L, G, range(cfg.T), what="tiny")
     for row, (_, _, expect) in inputs.TINY_TIES.items():
         assert tuple(r["idx"][row].tolist()) == expect
     assert (r["y"][63] == 0).all()
 
 
-@pytest.mark.parametrize("path", ["auto", "stream", "grouped"])
 @pytest.mark.parametrize("T", [1, 8, 32, 128, 256])
-def test_forward_decode_sweep(T, path):
+def test_forward_decode_sweep(T):
     cfg, L, G = layer("decode", T)
-    compare_block(cfg, L, G, range(T), path=path, what=f"decode T={T}/{path}")
+    compare_block(cfg, L, G, range(T), what=f"decode T={T}")
 
 
 def _boundary_rows(cfg, L, n_random=256):
@@ -226,39 +225,35 @@ def _small_layer(T, D=256, E=16, k=4, I=256, seed=5, I_s=0, bias=None):
     return cfg, L, G
 
 
-@pytest.mark.parametrize("path", ["stream", "grouped"])
 @pytest.mark.parametrize("T", [1, 7, 65, 129, 300])
-def test_forward_ragged_T(T, path):
+def test_forward_ragged_T(T):
     cfg, L, G = _small_layer(T)
-    compare_block(cfg, L, G, range(T), path=path, what=f"ragged T={T}/{path}")
+    compare_block(cfg, L, G, range(T), what=f"ragged T={T}")
 
 
-@pytest.mark.parametrize("path", ["stream", "grouped"])
 @pytest.mark.parametrize("E,k,norm", [(16, 1, True), (8, 8, True), (16, 4, False), (1, 1, True),
                                       (512, 16, True)])
-def test_forward_k_E_norm(E, k, norm, path):
+def test_forward_k_E_norm(E, k, norm):
     cfg, L, G = _small_layer(96, E=E, k=k)
-    compare_block(cfg, L, G, range(96), path=path, k=k, norm=norm, what=f"E={E} k={k} norm={norm}/{path}")
+    compare_block(cfg, L, G, range(96), k=k, norm=norm, what=f"E={E} k={k} norm={norm}")
 
 
-@pytest.mark.parametrize("path", ["stream", "grouped"])
-def test_forward_all_tokens_one_expert(path):
+def test_forward_all_tokens_one_expert():
     bias = torch.zeros(16)
     bias[3] = 100.0
     cfg, L, G = _small_layer(600, bias=bias)
-    r = compare_block(cfg, L, G, range(0, 600, 3), path=path, what=f"skewed/{path}")
+    r = compare_block(cfg, L, G, range(0, 600, 3), what="skewed")
     assert (r["idx"][:, 0] == 3).all()
 
 
-@pytest.mark.parametrize("path", ["stream", "grouped"])
-def test_forward_shared_expert_and_residual(path):
+def test_forward_shared_expert_and_residual():
     cfg, L, G = _small_layer(200, I_s=384)
     res = torch.randn(200, 256, generator=torch.Generator().manual_seed(3)).to(torch.bfloat16)
-    compare_block(cfg, L, G, range(200), path=path, residual_cpu=res, what=f"shared+res/{path}")
+    compare_block(cfg, L, G, range(200), residual_cpu=res, what="shared+res")
     # ungated shared expert
     L2 = dict(L, shared_gate=None)
     G2 = dict(G, shared_gate=None)
-    compare_block(cfg, L2, G2, range(200), path=path, what=f"ungated/{path}")
+    compare_block(cfg, L2, G2, range(200), what="ungated")
 
 
 def test_forward_single_sm_wide_tiles(monkeypatch):
@@ -288,19 +283,17 @@ def test_forward_split_tail_with_shared_expert(T):
     compare_block(cfg, L, G, range(T), path="grouped", residual_cpu=res, what=f"split tail T={T}")
 
 
-@pytest.mark.parametrize("path", ["stream", "grouped"])
-def test_forward_zero_input(path):
+def test_forward_zero_input():
     cfg, L, G = _small_layer(40)
     x0 = torch.zeros_like(L["x"])
     res = torch.randn(40, 256, generator=torch.Generator().manual_seed(4)).to(torch.bfloat16)
-    y, idx, w, _ = run_forward(cfg, G, path, x=x0.cuda(), residual=res.cuda())
+    y, idx, w, _ = run_forward(cfg, G, x=x0.cuda(), residual=res.cuda())
     assert torch.equal(y, res)                                 # block(0) = 0 exactly
     assert (idx == np.arange(cfg.k)[None, :]).all()           # all logits 0 -> lowest indices
     assert np.abs(w - 1.0 / cfg.k).max() <= W_ATOL
 
 
-@pytest.mark.parametrize("path", ["stream", "grouped"])
-def test_determinism_and_batch_invariance(path):
+def test_determinism_and_batch_invariance():
     """Bitwise-equal reruns of the same batch.  A token's routing (experts and FP32 weights)
     does not depend on the other tokens of the batch within a router kernel's range (T <= 64
     runs the CUDA-core router, larger T the tensor-core one with a K split fixed by the shapes;
@@ -308,25 +301,20 @@ def test_determinism_and_batch_invariance(path):
     tolerance: the expert GEMMs split the last wave's items along K, and how many items there
     are depends on the batch, so the FP32 summation order of y can change with it."""
     cfg, L, G = _small_layer(256)
-    y1, i1, w1, l1 = run_forward(cfg, G, path)
-    y2, i2, w2, l2 = run_forward(cfg, G, path)
+    y1, i1, w1, l1 = run_forward(cfg, G)
+    y2, i2, w2, l2 = run_forward(cfg, G)
     assert torch.equal(y1, y2) and (i1 == i2).all() and (w1 == w2).all() and (l1 == l2).all()
-    y100, i100, w100, l100 = run_forward(cfg, G, path, x=G["x"][:100].contiguous())
+    y100, i100, w100, l100 = run_forward(cfg, G, x=G["x"][:100].contiguous())
     assert (l100 == l1[:100]).all() and (i100 == i1[:100]).all() and (w100 == w1[:100]).all()
     assert_y_close(to_f64(y100), to_f64(y1[:100]), "T=100 vs the first 100 of T=256")
-    y64, i64, w64, l64 = run_forward(cfg, G, path, x=G["x"][:64].contiguous())
-    y8, i8, w8, l8 = run_forward(cfg, G, path, x=G["x"][:8].contiguous())
+    y64, i64, w64, l64 = run_forward(cfg, G, x=G["x"][:64].contiguous())
+    y8, i8, w8, l8 = run_forward(cfg, G, x=G["x"][:8].contiguous())
     assert (l8 == l64[:8]).all() and (i8 == i64[:8]).all() and (w8 == w64[:8]).all()
     assert_y_close(to_f64(y8), to_f64(y64[:8]), "T=8 vs the first 8 of T=64")
 
 
-def test_paths_agree_and_status_ok():
+def test_status_ok_after_a_forward():
     cfg, L, G = layer("decode", 128)
-    run_forward(cfg, G, "stream")
-    ys = run_forward.last_f32
-    run_forward(cfg, G, "grouped")
-    yg = run_forward.last_f32
-    assert_y_close(ys.double().numpy(), yg.double().numpy(), "stream vs grouped")
     dims = B.make_dims(128, cfg.D, cfg.E, cfg.k, cfg.I)
     ws = B.workspace(dims)
     B.moe_forward(G["x"], G["W_r"], G["W_gate_up"], G["W_down"], cfg.k, ws=ws)
@@ -345,34 +333,46 @@ def test_gpu_errors_before_launch():
     assert ei.value.status == B.MOE_ERR_UNSUPPORTED
 
 
-def test_residual_chain_short():
-    """Three residual blocks of the 48-block chain's shape, x_{l+1} = x_l + MoE_l(x_l).
-    Each layer is checked on the oracle's own layer input (teacher forcing: the oracle's
-    bf16 trajectory is fed to the GPU, never the reverse) with the full output criterion;
-    the free-running GPU chain is compared with the oracle trajectory in relative L2 (its
-    max-abs is dominated by one-ulp bf16 flips of the residual stream, ~3% of rms at |x|>4,
-    which no bf16 chain can avoid)."""
-    cfg = inputs.CONFIGS["keras"]
-    T, nl = 256, 3
-    x_o = inputs.make_layer(cfg, T=T, layer=0)["x"]
-    rows = list(range(T))
-    x_free = x_o.cuda()
-    for l in range(nl):
-        Ll = inputs.make_layer(cfg, T=T, layer=l, with_x=False)
-        Gl = {k: (v.cuda() if v is not None else None) for k, v in Ll.items()}
-        x_in = x_o.cuda()
-        y32 = torch.empty(x_in.shape, dtype=torch.float32, device="cuda")
-        out = B.moe_forward_ex(x_in, Gl["W_r"], Gl["W_gate_up"], Gl["W_down"], cfg.k, True,
-                               residual=x_in, out_f32=y32)
-        free = torch.empty_like(x_free)
-        B.moe_forward_ex(x_free, Gl["W_r"], Gl["W_gate_up"], Gl["W_down"], cfg.k, True, out=free,
-                         residual=x_free)
-        x_free = free
-        y, *_ = O.forward_rows(x_o, Ll["W_r"], Ll["W_gate_up"], Ll["W_down"], cfg.k, rows,
-                               residual=x_o, threads=THREADS)
-        torch.cuda.synchronize()
-        assert_block_output(out.cpu(), y32.cpu(), y, f"chain layer {l}")
-        x_o = torch.from_numpy(y).to(torch.bfloat16)
-    rel, _, _ = y_errors(x_free.cpu().double().numpy(), x_o.double().numpy())
-    print(f"free-running chain vs oracle trajectory after {nl} layers: relative L2 {rel:.2e}")
-    assert rel <= 5e-2, rel     # divergence diagnostic: near-tie routing flips compound
+# ------------------------------------------------------------------ permutation at the
+# workloads' own routing (the forward's internal tables and moe_permute)
+
+@pytest.mark.parametrize("name,T", [("decode", 8), ("decode", 256), ("prefill", None), ("keras", None),
+                                    ("zipf", None)])
+def test_permutation_at_workload_routing(name, T):
+    """The expert-sorted layout the forward builds from its own routing (per-expert counts and
+    the row of every assignment, read back through expert_counts_out / slot_row_out), and
+    moe_permute on the same routing with tile_m = 128, both bit-exact against the oracle's
+    stable counting sort.  zipf's routing is heavily skewed (one expert takes almost every
+    token, across many 4096-assignment chunks of the multi-block permutation)."""
+    cfg, L, G = layer(name, T)
+    x = G["x"]
+    Tn = x.shape[0]
+    idx = torch.empty(Tn, cfg.k, dtype=torch.int32, device="cuda")
+    w = torch.empty(Tn, cfg.k, dtype=torch.float32, device="cuda")
+    counts = torch.empty(cfg.E, dtype=torch.int32, device="cuda")
+    slot_row = torch.empty(Tn, cfg.k, dtype=torch.int32, device="cuda")
+    B.moe_forward_ex(x, G["W_r"], G["W_gate_up"], G["W_down"], cfg.k, cfg.norm_topk_prob,
+                     router_bias=G.get("bias"), shared_gate_up=G.get("shared_gate_up"),
+                     shared_down=G.get("shared_down"), shared_gate=G.get("shared_gate"),
+                     topk_idx_out=idx, topk_w_out=w, expert_counts_out=counts, slot_row_out=slot_row)
+    torch.cuda.synchronize()
+    idx_h = idx.cpu().numpy()
+    o_counts, o_offsets, o_row_token, o_slot_row = O.permute(idx_h, cfg.E, 1)
+    assert np.array_equal(counts.cpu().numpy(), o_counts)
+    assert np.array_equal(slot_row.cpu().numpy().reshape(-1), o_slot_row)
+    # moe_permute on the same routing, tile-padded
+    out = B.moe_permute(idx, cfg.E, 128, topk_w=w, x=x, want_x_perm=True)
+    torch.cuda.synchronize()
+    c, off, rt, sr = O.permute(idx_h, cfg.E, 128)
+    assert np.array_equal(out["counts"].cpu().numpy(), c)
+    assert np.array_equal(out["offsets"].cpu().numpy(), off)
+    assert np.array_equal(out["row_token"].cpu().numpy(), rt)
+    assert np.array_equal(out["slot_row"].cpu().numpy(), sr)
+    rw = out["row_weight"].cpu().numpy()
+    assert np.array_equal(rw[sr], w.cpu().numpy().reshape(-1))
+    xp = out["x_perm"].cpu()
+    valid = torch.from_numpy(rt >= 0)
+    assert torch.equal(xp[valid], L["x"][torch.from_numpy(rt[rt >= 0]).long()])
+    assert (xp[~valid] == 0).all()
+    print(f"{name}: T={Tn} assignments={Tn * cfg.k} touched={(o_counts > 0).sum()} "
+          f"max_load={o_counts.max()} chunks={(Tn * cfg.k + 4095) // 4096}")

@@ -200,8 +200,8 @@ def test_dense_bruteforce_bmm_formulation(oracle_mod):
 
 
 def test_loop_dispatch_equals_per_token(oracle_mod):
-    g = golden("loop_vs_grouped.json")                      # the pages' invariant
-    assert g["checksum_loop"] == g["checksum_grouped"]
+    # the pages' invariant (the loop and grouped dispatches give the same result): the
+    # oracle's loop dispatch against its per-token definition
     x, W_r, W_gu, W_dn = _small_layer(T=20, E=7)
     _, idx, w = oracle_mod.route(x, W_r, 3)
     y_loop = oracle_mod.loop_dispatch(x, idx, w, W_gu, W_dn)

@@ -1,10 +1,11 @@
 """moe_forward_noalloc: the forward pass for callers that cannot allocate device memory
-(work enqueued during CUDA-graph stream capture, plugin hosts that pass only input and
-output buffers, runtimes without device allocation after start-up).  Its scratch is a fixed
-64 MiB array inside the library.
+(plugin hosts that pass only input and output buffers, runtimes that plan device memory up
+front and forbid allocation once started).  Its scratch is a fixed 64 MiB array inside the
+library.
 
 Checked through the C ABI against moe_forward with a caller-owned workspace, on two calls
-in a row (the second one runs on the scratch the first left behind), plus the refusal of a
+in a row (the second one runs on the scratch the first left behind), with the device error
+word of those calls read back through moe_get_device_status_noalloc, plus the refusal of a
 problem whose workspace does not fit.  Kept in a file that is collected last so a failure
 here never hides the other tests; it passes alone in a fresh process as well.
 """
@@ -38,6 +39,7 @@ def test_noalloc_matches_forward_on_two_calls():
         torch.cuda.synchronize()
         assert_y_close(got.double().cpu().numpy(), ref.double().cpu().numpy(), f"noalloc T={T}")
         assert torch.equal(got, ref)          # same kernels, same order: bitwise equal
+        assert B.moe_get_device_status_noalloc() == B.MOE_OK
 
 
 def test_noalloc_refuses_problems_larger_than_its_scratch():
