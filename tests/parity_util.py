@@ -113,6 +113,28 @@ def assert_block_output(y_bf16, y_f32, y_ref, what=""):
     return assert_y_close(y_f32.double().numpy(), y_ref, what)
 
 
+def assert_block_output_rowwise(y_bf16, y_f32, y_ref, what=""):
+    """The output criterion with max-abs read per token row: max_d |err[t, d]| <= 2e-2 *
+    rms(y[t, :]) for every row t, besides relative L2 <= 5e-3 over all rows (bf16 and FP32)
+    and the bf16 output being the RNE rounding of the FP32 value.  For a batch whose rows
+    differ in scale by orders of magnitude (a residual chain whose rows grow at different
+    rates), a tensor-wide rms would measure small rows against large rows' scale.
+    Returns (relative L2 of the FP32 value, largest per-row max-abs / row rms)."""
+    assert torch.equal(y_f32.to(torch.bfloat16), y_bf16), f"{what}: bf16 output is not RNE of its FP32 value"
+    rel_b, _, _ = y_errors(y_bf16.double().numpy(), y_ref)
+    assert rel_b <= Y_REL_L2, f"{what}: bf16 output relative L2 error {rel_b:.3e} > {Y_REL_L2}"
+    yf = y_f32.double().numpy()
+    rel, _, _ = y_errors(yf, y_ref)
+    assert rel <= Y_REL_L2, f"{what}: relative L2 error {rel:.3e} > {Y_REL_L2}"
+    row_rms = np.sqrt(np.mean(np.asarray(y_ref, np.float64) ** 2, axis=1))
+    row_max = np.abs(yf - y_ref).max(axis=1)
+    worst = row_max / np.maximum(row_rms, 1e-300)
+    t = int(worst.argmax())
+    assert (row_max <= Y_MAX_ABS_RMS * row_rms + 1e-30).all(), \
+        f"{what}: row {t}: max-abs error {row_max[t]:.3e} > {Y_MAX_ABS_RMS} * row rms {row_rms[t]:.3e}"
+    return rel, float(worst.max())
+
+
 def assert_y_close(y_gpu, y_ref, what=""):
     rel_l2, max_abs, rms = y_errors(y_gpu, y_ref)
     assert rel_l2 <= Y_REL_L2, f"{what}: relative L2 error {rel_l2:.3e} > {Y_REL_L2}"
