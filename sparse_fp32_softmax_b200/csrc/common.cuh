@@ -89,6 +89,13 @@ __device__ __forceinline__ void set_error(int* err, int bit) {
     if (err) atomicOr(err, bit);
 }
 
+// Load with acquire semantics at GPU scope (pairs with a release by another CTA).
+__device__ __forceinline__ int ld_acquire(const int* p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
 __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
 
@@ -182,6 +189,17 @@ __device__ __forceinline__ void tma_prefetch_l2(const CUtensorMap* map, int x, i
 
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// Plain 2-D TMA tile load (no L2 hint) into this CTA's shared memory, completion counted on
+// the mbarrier `bar`; x is the inner (column) coordinate, y the row.
+__device__ __forceinline__ void tma_load(void* dst, const CUtensorMap* map, uint64_t* bar, int x,
+                                         int y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
+        : "memory");
 }
 
 // 5-D tile load (no L2 hint), coordinates innermost first.
