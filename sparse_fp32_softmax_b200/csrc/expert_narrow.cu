@@ -55,13 +55,19 @@ constexpr int kNwATile = kTcM * kTcK * 2;                      // 16 KB of weigh
 // gate_up does.
 constexpr int kNwSB = 2 * kNwATile + kNwBN * kTcK * 2;         // 40 KB per stage
 constexpr int kNwHalfB = 32 * kTcK * 2;                        // token tile of <= 32 rows
-constexpr int kNwAcc = 2 * kNwBN;                              // TMEM columns per accumulator set
-constexpr int kNwBufs = 4;                                     // accumulator sets (all of TMEM)
-constexpr int kNwTmem = kNwBufs * kNwAcc;
+// Two threads (in warps 1 and 10) issue the MMAs: one takes the even pipeline stages of a
+// unit, the other the odd ones, each into its own accumulators (the issuing thread, not the
+// tensor core, bounds these narrow MMAs); the epilogue adds the two.  An accumulator set is
+// gate | up (64 columns each) for gate_up, or 64 columns for down, per issuer.
+constexpr int kNwHalfAcc = 2 * kNwBN;                          // one issuer's columns
+constexpr int kNwAcc = 2 * kNwHalfAcc;                         // TMEM columns per buffer
+constexpr int kNwBufs = 2;                                     // one buffer per epilogue group
+constexpr int kNwTmem = kNwBufs * kNwAcc;                      // all of TMEM
 constexpr int kNwQD = 8;                                       // unit queue depth
 constexpr int kNwEpiWarps = 8;
 constexpr int kNwGroupWarps = 4;                               // epilogue warps per group
-constexpr int kNwThreads = (2 + kNwEpiWarps) * 32;
+constexpr int kNwMmaWarpB = 2 + kNwEpiWarps;                   // the second MMA issuer's warp
+constexpr int kNwThreads = (3 + kNwEpiWarps) * 32;
 constexpr int kNwCombTok = 4;                                  // tokens per combine unit
 constexpr int kNwMaxAssign = kGatherMaxT * kMaxK;
 
@@ -338,22 +344,21 @@ __device__ void nw_route(const NarrowArgs& a, NwTables* tb, NwRoute* rt) {
 
 // ------------------------------------------------------------------ hand-off and combine
 
-// gate_up -> down hand-off: the signalling warp wrote h with ordinary stores that down reads
-// with TMA (the async proxy), hence the proxy fence.
-__device__ __forceinline__ void nw_signal_done(const NarrowArgs& a, int seg, int lane) {
+// gate_up -> down hand-off: every lane of the finishing warps releases its own h stores
+// (ordinary stores that down reads with TMA, the async proxy, hence the proxy fence) with a
+// non-returning add to its expert's count.
+__device__ __forceinline__ void nw_signal_done(const NarrowArgs& a, int seg) {
     asm volatile("fence.proxy.async.global;" ::: "memory");
-    __threadfence();
-    __syncwarp();
-    if (lane == 0) atomicAdd(a.seg_done + seg, 1);
+    red_release_add(a.seg_done + seg, 1);
 }
 
 // Bounded wait (one lane) until gate_up has finished segment seg: one signal per item from
-// each of the 4 warps of the epilogue group that finished it.  A segment seen finished is
+// each lane of the 4 warps of the epilogue group that finished it.  A segment seen finished is
 // remembered in shared memory (seg_ok), so later units of the same expert do not ask again.
 __device__ bool nw_wait_done(const NarrowArgs& a, const NwTables* tb, uint32_t* seg_ok, int seg) {
     const uint32_t bit = 1u << (seg & 31);
     if (seg_ok[seg >> 5] & bit) return true;
-    const int target = kNwGroupWarps * (tb->gu_prefix[seg + 1] - tb->gu_prefix[seg]);
+    const int target = kNwGroupWarps * 32 * (tb->gu_prefix[seg + 1] - tb->gu_prefix[seg]);
     const uint64_t t0 = globaltimer_ns();
     while (ld_acquire(a.seg_wait + seg) < target) {
         __nanosleep(64);
@@ -410,7 +415,8 @@ __device__ __forceinline__ void nw_combine(const NarrowArgs& a, const NwRoute* r
     *reinterpret_cast<uint2*>(a.out + o) = make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
 }
 
-// Bounded wait (one lane) until every down item's four quarter warps have stored its slots.
+// Bounded wait (one lane) until every lane of every down item's four quarter warps has
+// stored (and released) its slots.
 __device__ bool nw_wait_down(const NarrowArgs& a, int target) {
     const uint64_t t0 = globaltimer_ns();
     while (ld_acquire(a.dn_done) < target) {
@@ -443,14 +449,14 @@ __global__ void __launch_bounds__(kNwThreads, 1)
             mbar_init(bars->empty + s, 1);
         }
         for (int b = 0; b < kNwBufs; ++b) {
-            mbar_init(bars->tfull + b, 1);
+            mbar_init(bars->tfull + b, 2);                     // both MMA issuers
             mbar_init(bars->tempty + b, kNwGroupWarps * 32);   // the epilogue group of the buffer
         }
-        mbar_init(&bars->drain, 1);
+        mbar_init(&bars->drain, 2);
         for (int i = 0; i < (kMaxSegments + 31) / 32; ++i) bars->seg_ok[i] = 0;
         for (int q = 0; q < kNwQD; ++q) {
             mbar_init(bars->qfull + q, 1);
-            mbar_init(bars->qempty + q, 1 + kNwEpiWarps);   // the MMA thread and each epilogue warp
+            mbar_init(bars->qempty + q, 2 + kNwEpiWarps);   // both MMA threads and each epilogue warp
         }
         mbar_fence_init();
     }
@@ -488,8 +494,15 @@ __global__ void __launch_bounds__(kNwThreads, 1)
         int last_round[kNwStages];
 #pragma unroll
         for (int s = 0; s < kNwStages; ++s) last_round[s] = -1;
+        // the next unit is taken once the current one has posted its first stage, so that at
+        // the start every CTA takes one unit before any takes a second
         int next = 0;
         if (lane == 0) next = atomicAdd(a.queue, 1);
+        bool grabbed = false;
+        auto grab_next = [&]() {
+            if (!grabbed && lane == 0) next = atomicAdd(a.queue, 1);
+            grabbed = true;
+        };
         auto stage_begin = [&](uint32_t bytes) -> int {   // wait for a free stage, post its bytes
             const int s = it % kNwStages;
             const int round = it / kNwStages;
@@ -503,11 +516,12 @@ __global__ void __launch_bounds__(kNwThreads, 1)
             for (int q = 0; q < kNwStages; ++q)
                 if (q == s) last_round[q] = round;
             ++it;
+            grab_next();
             return s;
         };
         for (int qi = 0; ok; ++qi) {
             const int u = __shfl_sync(0xffffffffu, next, 0);
-            if (lane == 0 && u < total) next = atomicAdd(a.queue, 1);
+            grabbed = u >= total;
             const int qs = qi % kNwQD;
             const bool gotq = mbar_wait(bars->qempty + qs, ((qi / kNwQD) & 1) ^ 1, a.err, kErrWaitProducer,
                                         a.wait_ns);
@@ -521,7 +535,10 @@ __global__ void __launch_bounds__(kNwThreads, 1)
             }
             if (u >= total) break;
             const NwTile t = nw_decode(a, tb, pg, pd, u);
-            if (t.comb) continue;   // no operands: the epilogue adds the slots
+            if (t.comb) {   // no operands: the epilogue adds the slots
+                grab_next();
+                continue;
+            }
             const int brows = 16 << t.bi;
             if (t.gu) {
                 const CUtensorMap* mA = t.shared ? &maps.gu_A_shared : &maps.gu_A;
@@ -621,8 +638,12 @@ __global__ void __launch_bounds__(kNwThreads, 1)
 #pragma unroll
         for (int s = 0; s < kNwStages; ++s)
             if (last_round[s] >= 0) mbar_wait(bars->full + s, last_round[s] & 1, a.err, kErrWaitTail, a.wait_ns);
-    } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
+    } else if (warp == 1 || warp == kNwMmaWarpB) {
+        // ------------------------------------------------------------ MMA issuers
+        // Issuer X (0: warp 1, 1: warp 10) takes the stages j of each unit with j % 2 == X,
+        // into accumulators at column offset X * kNwHalfAcc of the unit's buffer; both follow
+        // the ring position of every stage (a running count over all units).
+        const int X = warp == 1 ? 0 : 1;
         if (lane == 0) {
             const uint32_t idesc0 = umma_idesc_bf16_f32(kTcM, 16) & ~(0x3Fu << 17);
             const uint64_t dA0 = umma_desc_sw128(smem);
@@ -631,7 +652,7 @@ __global__ void __launch_bounds__(kNwThreads, 1)
             const uint64_t dBd = umma_desc_sw128(smem + kNwATile);       // down h tile
             const uint64_t dBd0 = umma_desc_sw128(smem + 2 * kNwATile);  // two-step down stages
             const uint64_t dBd1 = umma_desc_sw128(smem + 2 * kNwATile + kNwHalfB);
-            int s = 0, phase = 0, tc = 0;
+            int pos = 0, tc = 0;   // ring position of the next unit's first stage
             for (int qi = 0;; ++qi) {
                 const int qs = qi % kNwQD;
                 if (!mbar_wait(bars->qfull + qs, (qi / kNwQD) & 1, a.err, kErrWaitMma, a.wait_ns)) break;
@@ -640,54 +661,65 @@ __global__ void __launch_bounds__(kNwThreads, 1)
                 if (u < 0) break;
                 const NwTile t = nw_decode(a, tb, pg, pd, u);
                 if (t.comb) continue;
-                const int b = tc % kNwBufs, use = tc / kNwBufs;
+                const int b = tc & 1, use = tc >> 1;
                 ++tc;
+                const int base = pos;
+                pos += t.steps;
                 if (!mbar_wait(bars->tempty + b, (use & 1) ^ 1, a.err, kErrWaitMma, a.wait_ns)) break;
                 tc_fence_after();
                 int n = (t.n_valid + 15) & ~15;
                 n = n < 16 ? 16 : n;
                 const uint32_t idesc = idesc0 | ((uint32_t)(n >> 3) << 17);
-                const uint32_t d0 = tmem + (uint32_t)(b * kNwAcc);
+                const uint32_t d0 = tmem + (uint32_t)(b * kNwAcc + X * kNwHalfAcc);
                 bool ok = true;
-                for (int kb = 0; kb < t.steps; ++kb) {
-                    if (!mbar_wait(bars->full + s, phase, a.err, kErrWaitMma, a.wait_ns)) {
+                for (int j = X; j < t.steps; j += 2) {
+                    const int P = base + j;
+                    const int s = P % kNwStages;
+                    const int round = P / kNwStages;
+                    // The other issuer may still hold this slot's previous stage (P - STAGES),
+                    // so its full barrier may not have reached P's phase yet, and a parity wait
+                    // cannot tell two phases apart: first wait until that stage is released
+                    // (the producer's own condition for loading P), then for P's data.
+                    if (round > 0 &&
+                        !mbar_wait(bars->empty + s, (round & 1) ^ 1, a.err, kErrWaitMma, a.wait_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    if (!mbar_wait(bars->full + s, round & 1, a.err, kErrWaitMma, a.wait_ns)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
                     const uint64_t off = (uint64_t)(s * (kNwSB >> 4));
+                    const uint32_t acc = j > X ? 1u : 0u;   // this issuer's first stage overwrites
                     if (t.gu) {
-                        umma_bf16(d0, dA0 + off, dBg + off, idesc, kb);   // the unit's first MMA overwrites
-                        umma_bf16(d0 + kNwBN, dA1 + off, dBg + off, idesc, kb);
+                        umma_bf16(d0, dA0 + off, dBg + off, idesc, acc);
+                        umma_bf16(d0 + kNwBN, dA1 + off, dBg + off, idesc, acc);
 #pragma unroll
                         for (int kk = 1; kk < kTcK / 16; ++kk) {
                             umma_bf16_acc(d0, dA0 + off + 2 * kk, dBg + off + 2 * kk, idesc);
                             umma_bf16_acc(d0 + kNwBN, dA1 + off + 2 * kk, dBg + off + 2 * kk, idesc);
                         }
                     } else if (t.dbl) {
-                        umma_bf16(d0, dA0 + off, dBd0 + off, idesc, kb);
+                        umma_bf16(d0, dA0 + off, dBd0 + off, idesc, acc);
 #pragma unroll
                         for (int kk = 1; kk < kTcK / 16; ++kk)
                             umma_bf16_acc(d0, dA0 + off + 2 * kk, dBd0 + off + 2 * kk, idesc);
-                        if (2 * kb + 1 < t.nk) {
+                        if (2 * j + 1 < t.nk) {
 #pragma unroll
                             for (int kk = 0; kk < kTcK / 16; ++kk)
                                 umma_bf16_acc(d0, dA1 + off + 2 * kk, dBd1 + off + 2 * kk, idesc);
                         }
                     } else {
-                        umma_bf16(d0, dA0 + off, dBd + off, idesc, kb);
+                        umma_bf16(d0, dA0 + off, dBd + off, idesc, acc);
 #pragma unroll
                         for (int kk = 1; kk < kTcK / 16; ++kk)
                             umma_bf16_acc(d0, dA0 + off + 2 * kk, dBd + off + 2 * kk, idesc);
                     }
                     umma_commit(bars->empty + s);
-                    if (++s == kNwStages) {
-                        s = 0;
-                        phase ^= 1;
-                    }
                 }
                 if (!ok) break;
-                umma_commit(bars->tfull + b);
+                umma_commit(bars->tfull + b);   // (with no stages of this issuer: arrives at once)
             }
             // every issued MMA must be complete before TMEM is released
             umma_commit(&bars->drain);
@@ -696,9 +728,10 @@ __global__ void __launch_bounds__(kNwThreads, 1)
     } else {
         // ------------------------------------------------------------ epilogue warps 2..9
         // Two groups of four warps take alternate units (group g: units tc with tc % 2 == g,
-        // in accumulator sets g and g + 2), so one group's stores, fences and tickets overlap
-        // the other's; within a group warp w reads its TMEM lane quarter w % 4 and finishes
-        // both 32-column chunks of the unit.
+        // in TMEM buffer g), so one group's stores and fences overlap the other's; within a
+        // group warp w reads its TMEM lane quarter w % 4 and finishes both 32-column chunks of
+        // the unit.  A unit's value is the first issuer's accumulator plus the second's (when
+        // the unit has a second stage).
         const int quarter = warp & 3;
         const int grp = (warp - 2) >> 2;
         const int row = quarter * 32 + lane;
@@ -720,7 +753,7 @@ __global__ void __launch_bounds__(kNwThreads, 1)
                 if (!mine_c) continue;
                 if (!down_done) {
                     bool ok = true;
-                    if (lane == 0) ok = nw_wait_down(a, kNwGroupWarps * pd.n);
+                    if (lane == 0) ok = nw_wait_down(a, kNwGroupWarps * 32 * pd.n);
                     if (!__shfl_sync(0xffffffffu, ok, 0)) break;
                     down_done = true;
                 }
@@ -737,6 +770,23 @@ __global__ void __launch_bounds__(kNwThreads, 1)
             tc_fence_after();
             const uint32_t tb_addr = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(b * kNwAcc);
             const int nch = (t.n_valid + 31) >> 5;   // 1 or 2 chunks
+            const bool two = t.steps >= 2;           // the second issuer wrote its accumulators
+            // 32 columns of the first issuer's accumulator plus the second's, into dst
+            auto ld_sum = [&](uint32_t addr, float (&dst)[32]) {
+                tmem_ld32(addr, dst);
+                tmem_ld_wait();
+                if (two) {
+                    float tmp[16];
+                    tmem_ld16(addr + kNwHalfAcc, tmp);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) dst[i] += tmp[i];
+                    tmem_ld16(addr + kNwHalfAcc + 16, tmp);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) dst[16 + i] += tmp[i];
+                }
+            };
             // down: the slot and the weight of column c*32 + lane of each chunk
             int dl[2] = {0, 0};
             float wl[2] = {0.f, 0.f};
@@ -773,9 +823,8 @@ __global__ void __launch_bounds__(kNwThreads, 1)
                 float* ps = (t.gu ? a.partial_gu : a.partial_dn) +
                             (size_t)(t.tail * t.nsplit + t.split) * (NA * kTcM * kNwBN);
                 for (int c = 0; c < nch; ++c) {
-                    tmem_ld32(tb_addr + c * 32, v);
-                    if (t.gu) tmem_ld32(tb_addr + kNwBN + c * 32, uu);
-                    tmem_ld_wait();
+                    ld_sum(tb_addr + c * 32, v);
+                    if (t.gu) ld_sum(tb_addr + kNwBN + c * 32, uu);
                     float4* d0 = reinterpret_cast<float4*>(ps + (size_t)row * kNwBN + c * 32);
 #pragma unroll
                     for (int q = 0; q < 8; ++q) d0[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
@@ -825,9 +874,8 @@ __global__ void __launch_bounds__(kNwThreads, 1)
                         uu[4 * g] = su.x; uu[4 * g + 1] = su.y; uu[4 * g + 2] = su.z; uu[4 * g + 3] = su.w;
                     }
                 } else {
-                    tmem_ld32(tb_addr + c * 32, v);
-                    if (t.gu) tmem_ld32(tb_addr + kNwBN + c * 32, uu);
-                    tmem_ld_wait();
+                    ld_sum(tb_addr + c * 32, v);
+                    if (t.gu) ld_sum(tb_addr + kNwBN + c * 32, uu);
                     if (c == nch - 1) {
                         tc_fence_before();
                         mbar_arrive(bars->tempty + b);   // all values are in registers or stored
@@ -851,14 +899,10 @@ __global__ void __launch_bounds__(kNwThreads, 1)
                     }
                 }
             }
-            if (t.gu) {
-                nw_signal_done(a, t.seg, lane);
-            } else {
-                // this quarter of the item's slots is stored
-                __threadfence();
-                __syncwarp();
-                if (lane == 0) atomicAdd(a.dn_done, 1);
-            }
+            if (t.gu)
+                nw_signal_done(a, t.seg);
+            else
+                red_release_add(a.dn_done, 1);   // this lane's slots of the item are stored
         }
     }
     tc_fence_before();
