@@ -123,16 +123,17 @@ def profile_traffic(kernel_tag):
     return float(m.group(1))
 
 
-def kernels_per_forward(T, k, E):
-    """Kernels one moe_forward_ex call launches (the library's launch sequence): T <= 32 the
-    router logits and the fused expert kernel (which routes, permutes, runs both GEMMs and
-    the combine); above, the router, then selection + permutation in one kernel while
-    T*k <= 4096 (else selection, histogram, scan and scatter), and the permuted copy of x;
-    then the fused expert kernel when T*k <= 32*E, else gate_up, down and the combine."""
+def kernels_per_forward(T, k):
+    """Kernels one moe_forward_ex call launches (the library's launch sequence): T <= 32 one
+    fused routing + permutation kernel; above, the router, then selection + permutation in
+    one kernel while T*k <= 4096 (else selection, histogram, scan and scatter), and the
+    permuted copy of x; then gate_up, down and the combine."""
+    n = 0
     if T <= 32:
-        return 2
-    n = 1 + (1 if T * k <= 4096 else 4) + 1
-    return n + (1 if T * k <= 32 * E else 3)
+        n += 1
+    else:
+        n += 1 + (1 if T * k <= 4096 else 4) + 1
+    return n + 3
 
 
 class ClockSampler:
@@ -414,7 +415,8 @@ def measure(name, args, rank, world, device, peaks, with_e2e):
                 roofline_us=round(t_roof * 1e6, 2), roofline_frac=round(t_roof / (t_ms / 1e3), 4),
                 touched=p["touched"], max_load=p["max_load"],
                 stages_us_with_events=dict(zip(STAGES, [round(v * 1e3, 2) for v in stage_ms[n]])),
-                expert_stage_gbs=round((b_gu + b_dn) / ((stage_ms[n][2] + stage_ms[n][3]) / 1e3) / 1e9, 1)))
+                gate_up_gbs=round(b_gu / (stage_ms[n][2] / 1e3) / 1e9, 1),
+                down_gbs=round(b_dn / (stage_ms[n][3] / 1e3) / 1e9, 1)))
 
     def dominant(rs, kname):
         if chain:   # every layer has the same shape: average them
@@ -425,17 +427,9 @@ def measure(name, args, rank, world, device, peaks, with_e2e):
         b, f, t, T = rs[-1]          # the largest pass: one launch shape, one ncu capture
         return kernel_roof(kname, b, f, t, f"T={T}")
 
-    narrow = passes[-1]["T"] * cfg.k <= 32 * cfg.E
-    if narrow:
-        # decode shapes: one fused kernel streams gate_up and down weights and combines
-        # (stage 3 of the events; stages 4 and 5 are empty)
-        ex_roofs = [(g[0] + d[0], g[1] + d[1], g[2], g[3]) for g, d in zip(gu_roofs, dn_roofs)]
-        roof = dominant(ex_roofs, "narrow_expert_kernel")
-        roof_dn = None
-    else:
-        roof = dominant(gu_roofs, "tc_gemm_kernel<gate_up>")
-        roof_dn = dominant(dn_roofs, "tc_gemm_kernel<down>")
-    tag = {"decode": "narrow_expert_decode", "prefill": "tc_gemm_prefill"}.get(name, f"tc_gate_up_{name}")
+    roof = dominant(gu_roofs, "tc_gemm_kernel<gate_up>")
+    roof_dn = dominant(dn_roofs, "tc_gemm_kernel<down>")
+    tag = {"decode": "tc_gate_up_decode", "prefill": "tc_gemm_prefill"}.get(name, f"tc_gate_up_{name}")
     roof["traffic"] = profile_traffic(tag)
     blk_time = max(blk_bytes / (hbm * 1e9), blk_flops / (tf_peak * 1e12))
     res = dict(
@@ -451,7 +445,7 @@ def measure(name, args, rank, world, device, peaks, with_e2e):
                             flops=int(blk_flops), bound=("hbm" if blk_bytes / (hbm * 1e9) >=
                                                          blk_flops / (tf_peak * 1e12) else "tensor"),
                             peaks=f"hbm_gbs {hbm}, {tf_name} {tf_peak} ({peaks['source']})"),
-        gpu_launches=int(sum(kernels_per_forward(p["T"], cfg.k, cfg.E) for p in passes) * K),
+        gpu_launches=int(sum(kernels_per_forward(p["T"], cfg.k) for p in passes) * K),
         clocks=sampler.summary())
     if not chain:
         res["stages_us_with_events"] = dict(zip(STAGES, [round(v * 1e3, 2) for v in stage_ms[-1]]))

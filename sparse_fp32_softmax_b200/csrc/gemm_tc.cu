@@ -6,15 +6,17 @@
 // The expert is down(silu(gate x) * up x) with gate_up [E, 2I, D] (gate rows first) and
 // down [E, D, I].  The router logits x W_r^T are a plain dense GEMM of the same shape class.
 //
-// These kernels serve the shapes with many rows per expert (T*k > 32*E: prefill and wider);
-// decode-sized batches run the fused kernel of expert_narrow.cu instead.
 // Layout of the work (swap-AB): a tile is 128 weight rows (the MMA's M) by up to BN tokens
 // (its N), so an expert with few tokens costs a narrow N instead of a padded 128-row M.
-//   gate_up (BN = 256): one accumulator whose 128 rows interleave gate and up
+//   gate_up, narrow tiles (BN = 64, decode): two accumulators per tile, gate rows
+//            [f0, f0+128) and the matching up rows [I+f0, ...), against the same token tile;
+//            TMEM lane f holds gate and up of feature f, and the epilogue writes
+//            h = silu(g) * u in bf16.
+//   gate_up, wide tiles (BN = 256): one accumulator whose 128 rows interleave gate and up
 //            of 64 features in groups of 16 (fetched by one 5-D TMA load); lane l and lane
 //            l+16 of a lane quarter hold gate and up of one feature and swap halves with a
 //            shuffle.  A tcgen05.mma costs its issuing thread roughly the same whatever N,
-//            so N = 256 halves the instructions of a two-accumulator layout at N = 128.
+//            so N = 256 halves the instructions of the two-accumulator layout at N = 128.
 //   down:    one accumulator, down rows [d0, d0+128) against a tile of h rows; the epilogue
 //            scales by the routing weight and stores FP32 into the token's slot (a bf16 slot
 //            would add a third bf16 rounding on top of h and the output).
@@ -51,16 +53,19 @@ struct TcCfg {
     // the tile's BN token rows (BNC), and its TMEM holds its 128 rows over all BN columns
     static constexpr bool PAIR = PAIR_;
     static constexpr int BNC = PAIR ? BN / 2 : BN;
-    // gate_up interleaves gate and up rows in one A tile and one accumulator
-    static constexpr bool IL = MODE == kModeGateUp;
-    static constexpr int ACC = BN;                            // TMEM columns per accumulator
-    // two accumulators, rounded up to the power-of-two allocation unit (>= 32 columns)
+    // gate_up: narrow tiles keep gate and up in two accumulators (two A tiles per stage);
+    // wide tiles interleave them in one A tile and one accumulator
+    static constexpr bool IL = MODE == kModeGateUp && BN > kNarrowBN;
+    static constexpr int NA = (MODE == kModeGateUp && !IL) ? 2 : 1;   // A tiles per stage
+    static constexpr int ACC = NA * BN;                       // TMEM columns per accumulator set
+    // two accumulator sets, rounded up to the power-of-two allocation unit (>= 32 columns)
     static constexpr int TMEM = 2 * ACC <= 32 ? 32 : 2 * ACC <= 64 ? 64 : 2 * ACC <= 128 ? 128
                               : 2 * ACC <= 256 ? 256 : 512;
     static_assert(2 * ACC <= 512, "accumulators exceed TMEM");
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "token tile");
-    static constexpr int SB = kTcM * kTcK * 2 + BNC * kTcK * 2;  // bytes per stage
-    static constexpr int SMEM = STAGES * SB + 1024 + 256 + (int)sizeof(SmemTables);
+    static constexpr int SB = NA * (kTcM * kTcK * 2) + BNC * kTcK * 2;  // bytes per stage
+    static constexpr int SMEM = STAGES * SB + 1024 + 256 + (int)sizeof(SmemTables) +
+                                (MODE == kModeDown ? 8 * 2 * 4 * BN : 0);
     static_assert(2 * STAGES + 5 <= 31, "barriers exceed their 256-byte region");
     static_assert(SMEM <= 232448, "shared memory per block");
 };
@@ -72,20 +77,56 @@ constexpr int kTcThreads = (2 + kEpiWarps) * 32;
 struct TileInfo {
     int bi;       // token-operand box: 16 << bi rows
     int shared;   // A comes from the shared-expert tensor map
-    int a_row0;   // first A row (interleaved gate_up: 16-feature group)
-    int a_row1;   // interleaved gate_up: expert
+    int a_row0;   // first A row (gate rows for gate_up; interleaved: 16-feature group)
+    int a_row1;   // first up row (gate_up; interleaved: expert)
     int b_row;    // first B (token) row
     int n_valid;  // valid token columns, 1..BN
     int nk;       // K stages
-    int k0;       // first K stage
-    int split;    // router K slice
+    int k0;       // first K stage of this unit
+    int split;    // K slice index (router slices, or a split tail item's slice)
+    int nsplit;   // > 1: tail item split over K, partial sums reduced by the last slice
+    int tail;     // index of a split item among the tail items
+    int seg;      // segment (expert; E = the shared expert)
     int m0;       // first output feature of this tile within its segment
+};
+
+// Work schedule of one launch (identical in every CTA): the first `full` items -- whole
+// waves of G = gridDim.x -- run one item per unit; when the remaining tail is at most half a
+// wave, each tail item is split along K into S slices so that no CTA ends a whole item
+// after the others.  The slices come last (at most one per CTA): their reduction then reads
+// L2 while the SM's TMA engine is idle -- mid-stream, those loads would queue behind the
+// weight traffic.  A slice writes FP32 partial accumulators; the last slice of an item to
+// finish (atomic ticket) adds them in slice order and runs the epilogue, so the sums do not
+// depend on timing.
+struct Sched {
+    int n;      // items
+    int full;   // items in whole waves
+    int S;      // slices per tail item (1: no split)
+    int units;  // work units
 };
 
 template <int MODE, int BN>
 __device__ __forceinline__ int tc_total_items(const TcArgs& a, const SmemTables* st) {
     if (MODE == kModeRouter) return ((a.T + BN - 1) / BN) * ((a.E + kTcM - 1) / kTcM) * a.ksplit;
     return st->prefix[a.nseg];
+}
+
+template <int MODE, int BN, bool SPLIT>
+__device__ __forceinline__ Sched tc_schedule(const TcArgs& a, const SmemTables* st, int G) {
+    Sched sc;
+    sc.n = tc_total_items<MODE, BN>(a, st);
+    sc.full = sc.n / G * G;
+    sc.S = 1;
+    const int tail = sc.n - sc.full;
+    if (SPLIT && tail > 0 && 2 * tail <= G) {
+        const int kmin = MODE == kModeGateUp ? a.D : (a.I_s > 0 ? min(a.I, a.I_s) : a.I);
+        int S = min(G / tail, kMaxKSplit);
+        S = min(S, kmin / kTcK);
+        S = min(S, a.partial_slots / tail);
+        if (S >= 2) sc.S = S;
+    }
+    sc.units = sc.full + tail * sc.S;
+    return sc;
 }
 
 // Smallest token box (16 << bi rows, bi <= log2(BN/16)) that covers n valid rows.
@@ -105,6 +146,9 @@ __device__ __forceinline__ TileInfo tc_decode_item(const TcArgs& a, const SmemTa
     TileInfo ti;
     ti.k0 = 0;
     ti.split = 0;
+    ti.nsplit = 1;
+    ti.tail = 0;
+    ti.seg = 0;
     if (MODE == kModeRouter) {
         // consecutive items are the K splits of one tile
         const int mtc = (a.E + kTcM - 1) / kTcM;
@@ -125,23 +169,32 @@ __device__ __forceinline__ TileInfo tc_decode_item(const TcArgs& a, const SmemTa
     }
     const int s = find_segment_smem(st->prefix, a.nseg, item);
     const int local = item - st->prefix[s];
+    ti.seg = s;
     const int sh = (s == a.E);
     const int Iseg = sh ? a.I_s : a.I;
     // weight rows per tile: features (gate_up) or down rows; the pair's tile is twice a CTA's
-    const int fpt = (MODE == kModeGateUp) ? kGuILFeatures : kTcM;
+    const int fpt = (MODE == kModeGateUp && BN > kNarrowBN) ? kGuILFeatures : kTcM;
     const int mtc = (MODE == kModeGateUp) ? Iseg / (fpt * (PAIR ? 2 : 1)) : a.D / (kTcM * (PAIR ? 2 : 1));
     const int tt = local / mtc, mt = local % mtc;
+    const int cnt = st->count[s];
+    const int start = st->start[s];
     ti.shared = sh;
-    ti.b_row = st->start[s] + tt * BN;
-    ti.n_valid = min(BN, st->count[s] - tt * BN);
-    ti.m0 = (mt * (PAIR ? 2 : 1) + rank) * fpt;
-    if (MODE == kModeGateUp) {
+    ti.b_row = start + tt * BN;
+    ti.n_valid = min(BN, cnt - tt * BN);
+    ti.m0 = (MODE == kModeGateUp) ? (mt * (PAIR ? 2 : 1) + rank) * fpt : (mt * (PAIR ? 2 : 1) + rank) * kTcM;
+    if (MODE == kModeGateUp && BN > kNarrowBN) {
         // interleaved: 64 features [m0, m0+64) of expert s, as four 16-feature groups
         ti.a_row0 = ti.m0 / 16;
         ti.a_row1 = sh ? 0 : s;
         ti.nk = a.D / kTcK;
+    } else if (MODE == kModeGateUp) {
+        const int base = sh ? 0 : s * 2 * a.I;
+        ti.a_row0 = base + mt * kTcM;
+        ti.a_row1 = base + Iseg + mt * kTcM;
+        ti.nk = a.D / kTcK;
     } else {
-        ti.a_row0 = (sh ? 0 : s * a.D) + ti.m0;
+        const int base = sh ? 0 : s * a.D;
+        ti.a_row0 = base + ti.m0;
         ti.a_row1 = 0;
         ti.nk = Iseg / kTcK;
     }
@@ -149,11 +202,78 @@ __device__ __forceinline__ TileInfo tc_decode_item(const TcArgs& a, const SmemTa
     return ti;
 }
 
+template <int MODE, int BN, bool PAIR = false>
+__device__ __forceinline__ TileInfo tc_decode_unit(const TcArgs& a, const SmemTables* st,
+                                                   const Sched& sc, int u, int rank = 0) {
+    if (sc.S == 1 || u < sc.full) return tc_decode_item<MODE, BN, PAIR>(a, st, u, rank);
+    const int tail = (u - sc.full) / sc.S, split = (u - sc.full) % sc.S;
+    TileInfo ti = tc_decode_item<MODE, BN, PAIR>(a, st, sc.full + tail, rank);
+    const int nkt = ti.nk;
+    ti.k0 = split * nkt / sc.S;
+    ti.nk = (split + 1) * nkt / sc.S - ti.k0;
+    ti.split = split;
+    ti.nsplit = sc.S;
+    ti.tail = tail;
+    return ti;
+}
+
+// gate_up -> down hand-off per expert (narrow tiles).  The signalling warp has written h
+// with ordinary stores; the down kernel reads h with TMA (the async proxy), hence the proxy
+// fence on both sides.
+__device__ __forceinline__ void signal_segment_done(const TcArgs& a, int seg, int lane) {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+    __threadfence();
+    __syncwarp();
+    if (lane == 0) {
+        atomicAdd(a.seg_done + seg, 1);
+        atomicAdd(a.seg_done + a.nseg, 1);
+    }
+}
+
+__device__ __forceinline__ int ld_acquire(const int* p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Bounded wait of the down producer (one lane) until gate_up has finished segment seg.
+__device__ __forceinline__ bool wait_segment_done(const TcArgs& a, int seg, bool& all_done) {
+    if (all_done) return true;
+    const int all_target = 8 * __ldg(a.gu_prefix + a.nseg);
+    const int target = 8 * (__ldg(a.gu_prefix + seg + 1) - __ldg(a.gu_prefix + seg));
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+        if (ld_acquire(a.seg_done + a.nseg) >= all_target) {
+            all_done = true;
+            break;
+        }
+        if (ld_acquire(a.seg_done + seg) >= target) break;
+        __nanosleep(128);
+        if (globaltimer_ns() - t0 > a.wait_ns) {
+            set_error(a.err, kErrWaitProducer);
+            return false;
+        }
+    }
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+    return true;
+}
+
+// Plain 2-D TMA load without an L2 hint.
+__device__ __forceinline__ void tma_load(void* dst, const CUtensorMap* map, uint64_t* bar, int x,
+                                         int y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
+        : "memory");
+}
+
 template <int MODE, int BN, int STAGES, bool PAIR = false>
 __global__ void __launch_bounds__(kTcThreads, 1)
     tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
     using Tr = TcCfg<MODE, BN, STAGES, PAIR>;
-    constexpr int ACC = Tr::ACC;
+    constexpr int NA = Tr::NA, ACC = Tr::ACC;
+    constexpr bool SPLIT = MODE != kModeRouter && BN <= kNarrowBN;
     constexpr int SB = Tr::SB;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -165,9 +285,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     uint64_t* drain = tempty + 2;       // [1]
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
     SmemTables* tabs = reinterpret_cast<SmemTables*>(smem + STAGES * SB + 256);
+    // down: per epilogue warp, the current tile's row destinations and weights
+    int* ep_dest_all = reinterpret_cast<int*>(tabs + 1);                       // [8][BN]
+    float* ep_wt_all = reinterpret_cast<float*>(ep_dest_all + kEpiWarps * BN);  // [8][BN]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    // work items are handed to CTAs, or (PAIR) to the clusters of two CTAs, round-robin
+    // work units are handed to CTAs, or (PAIR) to the clusters of two CTAs, round-robin
     const int rank = PAIR ? (int)cluster_ctarank() : 0;
     const int ublk = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
     const int ugrid = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
@@ -209,7 +332,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             for (int kb = 0; kb < t0.nk; ++kb) tma_prefetch_l2(mA, kb * kTcK, t0.a_row0);
         }
     }
-    pdl_wait();
+    // (down with per-expert hand-off: no wait for the whole gate_up grid; everything read
+    // below besides h was complete before this kernel could start -- see above)
+    if (!(MODE == kModeDown && a.dep_wait)) pdl_wait();
     pdl_launch_dependents();
     if (MODE == kModeGateUp)
         load_tables(tabs, a.tables.gu_items, a.tables.seg_count, a.tables.seg_start, a.nseg);
@@ -220,71 +345,113 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
-    const int total = tc_total_items<MODE, BN>(a, tabs);
+    const Sched sc = tc_schedule<MODE, BN, SPLIT>(a, tabs, ugrid);
+    const int total = sc.units;
 
     if (ublk >= total) {
         // no work for this CTA: nothing was issued; fall through to the TMEM release
     } else if (warp == 0) {
         // ------------------------------------------------------------ TMA producer warp
-        if (lane == 0) {
-            int it = 0;
-            bool ok = true;
-            int last_round[STAGES];
+        // Weight tiles are issued by lane 0.  Token tiles: in gather mode gate_up fetches its
+        // rows from x by row_token, lane i taking rows 4i..4i+3 of the tile (rows past the
+        // segment repeat its last row; their columns are never used); otherwise lane 0 loads
+        // a tile of the permuted rows.
+        const int first = ublk, step = ugrid;   // this CTA's (pair's) units
+        bool dep_all_done = false;
+        int it = 0;
+        bool ok = true;
+        int last_round[STAGES];
 #pragma unroll
-            for (int s = 0; s < STAGES; ++s) last_round[s] = -1;
-            for (int item = ublk; item < total && ok; item += ugrid) {
-                const TileInfo ti = tc_decode_item<MODE, BN, PAIR>(a, tabs, item, rank);
-                const CUtensorMap* mA = ti.shared ? &maps.A_shared : &maps.A;
-                const CUtensorMap* mB = &maps.B[ti.bi];
-                const int brows = 16 << ti.bi;
-                // PAIR: the leader's barrier counts both CTAs' bytes (same geometry in each)
-                const uint32_t bytes = (PAIR ? 2u : 1u) * (kATileBytes + (uint32_t)brows * kTcK * 2);
-                for (int kb = 0; kb < ti.nk; ++kb, ++it) {
-                    const int s = it % STAGES;
-                    const int round = it / STAGES;
-                    if (!mbar_wait(empty + s, (round & 1) ^ 1, a.err, kErrWaitProducer, a.wait_ns)) {
-                        ok = false;
-                        break;
-                    }
-                    uint8_t* st = smem + s * SB;
+        for (int s = 0; s < STAGES; ++s) last_round[s] = -1;
+        const bool gather = MODE == kModeGateUp && a.gather;
+        // the next unit's gather rows are loaded while the current unit's stages are issued
+        auto gather_rows = [&](const TileInfo& t, int (&g)[4]) {
+            const int base = t.b_row + 4 * lane;
+            const int last = t.b_row + t.n_valid - 1;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) g[q] = __ldg(a.row_token + min(base + q, last));
+        };
+        TileInfo tn{};
+        int gn[4] = {0, 0, 0, 0};
+        if (first < total) {
+            tn = tc_decode_unit<MODE, BN, PAIR>(a, tabs, sc, first, rank);
+            if (gather) gather_rows(tn, gn);
+        }
+        for (int item = first; item < total && ok; item += step) {
+            const TileInfo ti = tn;
+            const int g0 = gn[0], g1 = gn[1], g2 = gn[2], g3 = gn[3];
+            if (item + step < total) {
+                tn = tc_decode_unit<MODE, BN, PAIR>(a, tabs, sc, item + step, rank);
+                if (gather) gather_rows(tn, gn);
+            }
+            if (MODE == kModeDown && a.dep_wait) {
+                bool got = true;
+                if (lane == 0) got = wait_segment_done(a, ti.seg, dep_all_done);
+                if (!__shfl_sync(0xffffffffu, got, 0)) {
+                    ok = false;
+                    break;
+                }
+            }
+            const CUtensorMap* mA = ti.shared ? &maps.A_shared : &maps.A;
+            const CUtensorMap* mB = &maps.B[ti.bi];
+            const int brows = 16 << ti.bi;
+            // PAIR: the leader's barrier counts both CTAs' bytes (same geometry in each)
+            const uint32_t bytes = (PAIR ? 2u : 1u) * (NA * kATileBytes + (uint32_t)brows * kTcK * 2);
+            for (int kb = 0; kb < ti.nk; ++kb, ++it) {
+                const int s = it % STAGES;
+                const int round = it / STAGES;
+                const bool got = mbar_wait(empty + s, (round & 1) ^ 1, a.err, kErrWaitProducer, a.wait_ns);
+                if (!__all_sync(0xffffffffu, got)) {
+                    ok = false;
+                    break;
+                }
+                uint8_t* st = smem + s * SB;
+                if (PAIR && lane == 0) {
+                    // both CTAs load their halves; completion is counted by the leader
+                    if (rank == 0) mbar_arrive_expect_tx(full + s, bytes);
+                    const uint32_t fb = mapa_shared(full + s, 0);
                     const int kx = (ti.k0 + kb) * kTcK;
-                    if (PAIR) {
-                        // both CTAs load their halves; completion is counted by the leader
-                        if (rank == 0) mbar_arrive_expect_tx(full + s, bytes);
-                        const uint32_t fb = mapa_shared(full + s, 0);
-                        if (Tr::IL)
-                            tma_load_5d_pair(st, mA, fb, kx, 0, 0, ti.a_row0, ti.a_row1);
-                        else
-                            tma_load_2d_pair(st, mA, fb, kx, ti.a_row0);
-                        tma_load_2d_pair(st + kATileBytes, mB, fb, kx, ti.b_row + rank * brows);
-                    } else {
-                        mbar_arrive_expect_tx(full + s, bytes);
-                        if (Tr::IL)
-                            tma_load_5d(st, mA, full + s, kx, 0, 0, ti.a_row0, ti.a_row1);
-                        else
-                            tma_load(st, mA, full + s, kx, ti.a_row0);
-                        tma_load(st + kATileBytes, mB, full + s, kx, ti.b_row);
-                    }
-#pragma unroll
-                    for (int q = 0; q < STAGES; ++q)
-                        if (q == s) last_round[q] = round;
+                    if (Tr::IL)
+                        tma_load_5d_pair(st, mA, fb, kx, 0, 0, ti.a_row0, ti.a_row1);
+                    else
+                        tma_load_2d_pair(st, mA, fb, kx, ti.a_row0);
+                    tma_load_2d_pair(st + NA * kATileBytes, mB, fb, kx, ti.b_row + rank * brows);
+                } else if (!PAIR && lane == 0) {
+                    mbar_arrive_expect_tx(full + s, bytes);
+                    const int kx = (ti.k0 + kb) * kTcK;
+                    if (Tr::IL)
+                        tma_load_5d(st, mA, full + s, kx, 0, 0, ti.a_row0, ti.a_row1);
+                    else
+                        tma_load(st, mA, full + s, kx, ti.a_row0);
+                    if (NA == 2) tma_load(st + kATileBytes, mA, full + s, kx, ti.a_row1);
+                    if (!gather) tma_load(st + NA * kATileBytes, mB, full + s, kx, ti.b_row);
                 }
-            }
-            // wait until the MMA issuer has released every stage, then until every issued
-            // load has landed, so no copy is in flight when the CTA exits
-            if (ok) {
-                for (int i = 0; i < STAGES; ++i, ++it) {
-                    const int s = it % STAGES;
-                    const int round = it / STAGES;
-                    if (!mbar_wait(empty + s, (round & 1) ^ 1, a.err, kErrWaitTail, a.wait_ns)) break;
+                if (gather) {
+                    __syncwarp();  // expect_tx is posted before any gather can complete
+                    if (4 * lane < brows)
+                        tma_gather4(st + NA * kATileBytes + lane * 4 * kTcK * 2, mB, full + s,
+                                    (ti.k0 + kb) * kTcK, g0, g1, g2, g3);
                 }
-            }
-            // (PAIR: a released stage implies its loads landed; the full barriers are the leader's)
-            if (!PAIR) {
 #pragma unroll
-                for (int s = 0; s < STAGES; ++s)
-                    if (last_round[s] >= 0) mbar_wait(full + s, last_round[s] & 1, a.err, kErrWaitTail, a.wait_ns);
+                for (int q = 0; q < STAGES; ++q)
+                    if (q == s) last_round[q] = round;
             }
+        }
+        // wait until the MMA issuer has released every stage, then until every issued
+        // load has landed, so no copy is in flight when the CTA exits
+        if (ok) {
+            for (int i = 0; i < STAGES; ++i, ++it) {
+                const int s = it % STAGES;
+                const int round = it / STAGES;
+                const bool got = mbar_wait(empty + s, (round & 1) ^ 1, a.err, kErrWaitTail, a.wait_ns);
+                if (!__all_sync(0xffffffffu, got)) break;
+            }
+        }
+        // (PAIR: a released stage implies its loads landed; the full barriers are the leader's)
+        if (!PAIR) {
+#pragma unroll
+            for (int s = 0; s < STAGES; ++s)
+                if (last_round[s] >= 0) mbar_wait(full + s, last_round[s] & 1, a.err, kErrWaitTail, a.wait_ns);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
@@ -294,12 +461,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             // shared-memory descriptors of stage 0; stage s adds s * SB / 16 to the address
             // field (stages stay below 256 KB, so the 14-bit field does not carry)
             const uint64_t dA0 = umma_desc_sw128(smem);
-            const uint64_t dB = umma_desc_sw128(smem + kATileBytes);
+            const uint64_t dA1 = umma_desc_sw128(smem + kATileBytes);
+            const uint64_t dB = umma_desc_sw128(smem + NA * kATileBytes);
             int s = 0, phase = 0;   // ring position of the next stage
             int tc = 0;
             bool ok = true;
             for (int item = ublk; item < total && ok; item += ugrid, ++tc) {
-                const TileInfo ti = tc_decode_item<MODE, BN, PAIR>(a, tabs, item, rank);
+                const TileInfo ti = tc_decode_unit<MODE, BN, PAIR>(a, tabs, sc, item, rank);
                 const int b = tc & 1;
                 const int use = tc >> 1;
                 if (!mbar_wait(tempty + b, (use & 1) ^ 1, a.err, kErrWaitMma, a.wait_ns)) {
@@ -319,7 +487,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     }
                     tc_fence_after();
                     const uint64_t off = (uint64_t)(s * (SB >> 4));
-                    const uint64_t da0 = dA0 + off, db = dB + off;
+                    const uint64_t da0 = dA0 + off, da1 = dA1 + off, db = dB + off;
                     if (PAIR) {
                         umma_bf16_pair(d0, da0, db, idesc, kb);
 #pragma unroll
@@ -328,8 +496,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         umma_commit_pair_both(empty + s);   // frees the stage in both CTAs
                     } else {
                         umma_bf16(d0, da0, db, idesc, kb);  // the tile's first MMA overwrites D
+                        if (NA == 2) umma_bf16(d0 + BN, da1, db, idesc, kb);
 #pragma unroll
-                        for (int kk = 1; kk < kTcK / 16; ++kk) umma_bf16_acc(d0, da0 + 2 * kk, db + 2 * kk, idesc);
+                        for (int kk = 1; kk < kTcK / 16; ++kk) {
+                            umma_bf16_acc(d0, da0 + 2 * kk, db + 2 * kk, idesc);
+                            if (NA == 2) umma_bf16_acc(d0 + BN, da1 + 2 * kk, db + 2 * kk, idesc);
+                        }
                         umma_commit(empty + s);
                     }
                     if (++s == STAGES) {
@@ -356,19 +528,22 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const int ew = warp - 2;               // epilogue warp 0..7
         const int half = ew >> 2;              // which alternate chunks this warp takes
         const int row = quarter * 32 + lane;  // TMEM lane = weight row within the tile
-        // down: the slot destinations and routing weights of the token columns this warp
-        // stores (its chunks half, half + 2, ...) are loaded one tile ahead into registers
-        // (nd, nw), so their memory latency overlaps the previous tile's epilogue; the
+        int* ep_dest = ep_dest_all + ew * BN;
+        float* ep_wt = ep_wt_all + ew * BN;
+        // down, wide tiles: the slot destinations and routing weights of the token columns
+        // this warp stores (its chunks half, half + 2, ...) are loaded one tile ahead into
+        // registers (nd, nw), so their memory latency overlaps the previous tile's epilogue
+        // (measured: it helps the long-K wide tiles and costs the short narrow ones); the
         // current tile's copy (cd, cw) stays in registers and reaches the lanes by shuffles,
         // keeping the per-element work off shared memory, which the MMAs read their
         // operands from
-        constexpr bool kAhead = MODE == kModeDown;
+        constexpr bool kAhead = MODE == kModeDown && BN > kNarrowBN;
         constexpr int kCPW = (BN + 63) / 64;   // chunks per epilogue warp
-        int nd[kCPW] = {}, cd[kCPW] = {};
-        float nw[kCPW] = {}, cw[kCPW] = {};
-        // The epilogue of one 32-column chunk: v holds row `row`.
-        auto finish_chunk = [&](const TileInfo& ti, int c, const float* v) {
-            if (MODE == kModeGateUp) {
+        int nd[kCPW], cd[kCPW];
+        float nw[kCPW], cw[kCPW];
+        // The epilogue of one 32-column chunk: v (and u, the up accumulator) hold row `row`.
+        auto finish_chunk = [&](const TileInfo& ti, int c, const float* v, const float* u) {
+            if (Tr::IL) {
                 // lanes 0-15 of the quarter hold gate rows of features m0 + 16*quarter + l,
                 // lanes 16-31 the up rows of the same features: lane l takes the chunk's tokens
                 // 0-15, lane l+16 tokens 16-31, swapping the other half with its partner
@@ -384,23 +559,37 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     const float uu = is_gate ? recv : v[16 + t];
                     if (t0 + t < ti.n_valid) hp[(size_t)t * a.ld_h] = to_bf16_bits(silu(g) * uu);
                 }
+            } else if (MODE == kModeGateUp) {
+                const int f = ti.m0 + row;
+                uint16_t* hp = a.h + (size_t)(ti.b_row + c * 32) * a.ld_h + f;
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                    if (c * 32 + j < ti.n_valid) hp[(size_t)j * a.ld_h] = to_bf16_bits(silu(v[j]) * u[j]);
             } else if (MODE == kModeDown) {
                 const int d = ti.m0 + row;
-                // lane j holds column c*32 + j of this warp's chunk (c - half) / 2
-                const int i = (c - half) >> 1;
-                int dsel = cd[0];
-                float wsel = cw[0];
+                if (kAhead) {
+                    // lane j holds column c*32 + j of this warp's chunk (c - half) / 2
+                    const int i = (c - half) >> 1;
+                    int dsel = cd[0];
+                    float wsel = cw[0];
 #pragma unroll
-                for (int q = 1; q < kCPW; ++q)
-                    if (q == i) {
-                        dsel = cd[q];
-                        wsel = cw[q];
+                    for (int q = 1; q < kCPW; ++q)
+                        if (q == i) {
+                            dsel = cd[q];
+                            wsel = cw[q];
+                        }
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int dj = __shfl_sync(0xffffffffu, dsel, j);
+                        const float wj = __shfl_sync(0xffffffffu, wsel, j);
+                        if (c * 32 + j < ti.n_valid) a.slots[(size_t)dj * a.D + d] = wj * v[j];
                     }
+                } else {
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const int dj = __shfl_sync(0xffffffffu, dsel, j);
-                    const float wj = __shfl_sync(0xffffffffu, wsel, j);
-                    if (c * 32 + j < ti.n_valid) a.slots[(size_t)dj * a.D + d] = wj * v[j];
+                    for (int j = 0; j < 32; ++j) {
+                        const int col = c * 32 + j;
+                        if (col < ti.n_valid) a.slots[(size_t)ep_dest[col] * a.D + d] = ep_wt[col] * v[j];
+                    }
                 }
             } else {
                 const int e = ti.m0 + row;
@@ -414,6 +603,24 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 }
             }
         };
+        // The same for four columns 4g..4g+3 of chunk c (the split-tail reduction).
+        auto finish_quad = [&](const TileInfo& ti, int c, int g, const float4& v4, const float4& u4) {
+            const float v[4] = {v4.x, v4.y, v4.z, v4.w};
+            const float u[4] = {u4.x, u4.y, u4.z, u4.w};
+            const int col0 = c * 32 + 4 * g;
+            if (MODE == kModeGateUp) {
+                uint16_t* hp = a.h + (size_t)(ti.b_row + col0) * a.ld_h + ti.m0 + row;
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    if (col0 + j < ti.n_valid) hp[(size_t)j * a.ld_h] = to_bf16_bits(silu(v[j]) * u[j]);
+            } else if (MODE == kModeDown) {
+                const int d = ti.m0 + row;
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    if (col0 + j < ti.n_valid)
+                        a.slots[(size_t)ep_dest[col0 + j] * a.D + d] = ep_wt[col0 + j] * v[j];
+            }
+        };
         auto fetch_dest = [&](const TileInfo& t) {
 #pragma unroll
             for (int i = 0; i < kCPW; ++i) {
@@ -423,12 +630,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 nw[i] = in ? __ldg(a.row_weight + t.b_row + col) : 0.f;
             }
         };
-        if (kAhead && ublk < total) fetch_dest(tc_decode_item<MODE, BN, PAIR>(a, tabs, ublk, rank));
+        if (kAhead && ublk < total)
+            fetch_dest(tc_decode_unit<MODE, BN, PAIR>(a, tabs, sc, ublk, rank));
         int tc = 0;
         // PAIR: the accumulator is released on the leader's barrier by both CTAs
         const uint32_t tempty_leader0 = PAIR ? mapa_shared(tempty, 0) : 0u;
         for (int item = ublk; item < total; item += ugrid, ++tc) {
-            const TileInfo ti = tc_decode_item<MODE, BN, PAIR>(a, tabs, item, rank);
+            const TileInfo ti = tc_decode_unit<MODE, BN, PAIR>(a, tabs, sc, item, rank);
             const int b = tc & 1;
             const int use = tc >> 1;
             const bool got = mbar_wait(tfull + b, use & 1, a.err, kErrWaitEpilogue, a.wait_ns);
@@ -442,29 +650,114 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     cd[i] = nd[i];
                     cw[i] = nw[i];
                 }
-                if (item + ugrid < total) fetch_dest(tc_decode_item<MODE, BN, PAIR>(a, tabs, item + ugrid, rank));
+                if (item + ugrid < total)
+                    fetch_dest(tc_decode_unit<MODE, BN, PAIR>(a, tabs, sc, item + ugrid, rank));
+            } else if (MODE == kModeDown) {
+                __syncwarp();
+                for (int c = lane; c < ti.n_valid; c += 32) {
+                    ep_dest[c] = __ldg(a.row_dest + ti.b_row + c);
+                    ep_wt[c] = __ldg(a.row_weight + ti.b_row + c);
+                }
+                __syncwarp();
             }
-            // the TMEM load of the warp's next chunk is in flight while this chunk is
-            // finished (two register buffers, used alternately)
-            float va[32], vb[32];
-            int c = half;
-            if (c < nchunks) tmem_ld32(tb + c * 32, va);
-            while (c < nchunks) {
-                tmem_ld_wait();
-                if (c + 2 < nchunks) tmem_ld32(tb + (c + 2) * 32, vb);
-                finish_chunk(ti, c, va);
-                c += 2;
-                if (c >= nchunks) break;
-                tmem_ld_wait();
-                if (c + 2 < nchunks) tmem_ld32(tb + (c + 2) * 32, va);
-                finish_chunk(ti, c, vb);
-                c += 2;
+            if (SPLIT && ti.nsplit > 1) {
+                // 1. this slice's partial accumulators (rows x BN per accumulator, FP32)
+                float* ps = a.partial + (size_t)(ti.tail * ti.nsplit + ti.split) * (NA * kTcM * BN);
+                for (int c = half; c < nchunks; c += 2) {
+                    float v[32];
+                    tmem_ld32(tb + c * 32, v);
+                    float u[32];
+                    if (NA == 2) tmem_ld32(tb + BN + c * 32, u);
+                    tmem_ld_wait();
+                    float4* d0 = reinterpret_cast<float4*>(ps + (size_t)row * BN + c * 32);
+#pragma unroll
+                    for (int q = 0; q < 8; ++q)
+                        d0[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+                    if (NA == 2) {
+                        float4* d1 = reinterpret_cast<float4*>(ps + (size_t)(kTcM + row) * BN + c * 32);
+#pragma unroll
+                        for (int q = 0; q < 8; ++q)
+                            d1[q] = make_float4(u[4 * q], u[4 * q + 1], u[4 * q + 2], u[4 * q + 3]);
+                    }
+                }
+                tc_fence_before();
+                mbar_arrive(tempty + b);  // the accumulator is free for the next tile
+                // 2. publish; the warp that completes this (item, warp) portion reduces it
+                __threadfence();
+                __syncwarp();
+                int old = 0;
+                int* ticket = a.tickets + ti.tail * kEpiWarps + ew;
+                if (lane == 0) old = atomicAdd(ticket, 1);
+                old = __shfl_sync(0xffffffffu, old, 0);
+                if (old != ti.nsplit - 1) continue;
+                __threadfence();
+                if (lane == 0) *ticket = 0;  // ready for the next launch
+                const float* p0 = a.partial + (size_t)(ti.tail * ti.nsplit) * (NA * kTcM * BN);
+                for (int c = half; c < nchunks; c += 2) {
+                    // valid columns only, four at a time; the loads of all slices of a group
+                    // are in flight together and are added in slice order
+                    const int ng = (min(32, ti.n_valid - c * 32) + 3) >> 2;
+#pragma unroll
+                    for (int g = 0; g < 8; ++g) {
+                        if (g >= ng) break;
+                        float4 lv[kMaxKSplit], lu[kMaxKSplit] = {};
+#pragma unroll
+                        for (int sp = 0; sp < kMaxKSplit; ++sp) {
+                            if (sp < ti.nsplit) {
+                                const float* pp = p0 + (size_t)sp * (NA * kTcM * BN) + c * 32 + 4 * g;
+                                lv[sp] = __ldcg(reinterpret_cast<const float4*>(pp + (size_t)row * BN));
+                                if (NA == 2)
+                                    lu[sp] = __ldcg(reinterpret_cast<const float4*>(pp + (size_t)(kTcM + row) * BN));
+                            }
+                        }
+                        float4 sv = lv[0], su = lu[0];
+#pragma unroll
+                        for (int sp = 1; sp < kMaxKSplit; ++sp) {
+                            if (sp < ti.nsplit) {
+                                sv.x += lv[sp].x; sv.y += lv[sp].y; sv.z += lv[sp].z; sv.w += lv[sp].w;
+                                if (NA == 2) {
+                                    su.x += lu[sp].x; su.y += lu[sp].y; su.z += lu[sp].z; su.w += lu[sp].w;
+                                }
+                            }
+                        }
+                        finish_quad(ti, c, g, sv, su);
+                    }
+                }
+                if (MODE == kModeGateUp && a.seg_done) signal_segment_done(a, ti.seg, lane);
+                continue;
+            }
+            if (NA == 1) {
+                // one accumulator: the TMEM load of the warp's next chunk is in flight while
+                // this chunk is finished (two register buffers, used alternately)
+                float va[32], vb[32];
+                int c = half;
+                if (c < nchunks) tmem_ld32(tb + c * 32, va);
+                while (c < nchunks) {
+                    tmem_ld_wait();
+                    if (c + 2 < nchunks) tmem_ld32(tb + (c + 2) * 32, vb);
+                    finish_chunk(ti, c, va, va);
+                    c += 2;
+                    if (c >= nchunks) break;
+                    tmem_ld_wait();
+                    if (c + 2 < nchunks) tmem_ld32(tb + (c + 2) * 32, va);
+                    finish_chunk(ti, c, vb, vb);
+                    c += 2;
+                }
+            } else {
+                for (int c = half; c < nchunks; c += 2) {
+                    float v[32], u[32];
+                    tmem_ld32(tb + c * 32, v);
+                    tmem_ld32(tb + BN + c * 32, u);
+                    tmem_ld_wait();
+                    finish_chunk(ti, c, v, u);
+                }
             }
             tc_fence_before();
             if (PAIR)
                 mbar_arrive_cluster(tempty_leader0 + 8u * b);
             else
                 mbar_arrive(tempty + b);
+            if (MODE == kModeGateUp && !PAIR && a.seg_done) signal_segment_done(a, ti.seg, lane);
         }
     }
     tc_fence_before();
@@ -568,6 +861,8 @@ cudaError_t launch_tc_router(const TcMaps& maps, const TcArgs& a, int num_sms, b
 
 cudaError_t launch_tc_gate_up(const TcMaps& maps, const TcArgs& a, int num_sms, int tiles, bool pdl,
                               cudaStream_t s) {
+    if (tiles == kTilesNarrow)
+        return launch_tc<kModeGateUp, kNarrowBN, kGuNarrowStages>(maps, a, num_sms, pdl, s);
     if (tiles == kTilesPair)
         return launch_tc<kModeGateUp, kGuBN, kPairStages, true>(maps, a, num_sms, pdl, s);
     return launch_tc<kModeGateUp, kGuBN, kStages>(maps, a, num_sms, pdl, s);
@@ -575,6 +870,8 @@ cudaError_t launch_tc_gate_up(const TcMaps& maps, const TcArgs& a, int num_sms, 
 
 cudaError_t launch_tc_down(const TcMaps& maps, const TcArgs& a, int num_sms, int tiles, bool pdl,
                            cudaStream_t s) {
+    if (tiles == kTilesNarrow)
+        return launch_tc<kModeDown, kNarrowBN, kDnNarrowStages>(maps, a, num_sms, pdl, s);
     if (tiles == kTilesPair)
         return launch_tc<kModeDown, kDnBN, kPairStages, true>(maps, a, num_sms, pdl, s);
     return launch_tc<kModeDown, kDnBN, kStages>(maps, a, num_sms, pdl, s);

@@ -36,27 +36,27 @@ constexpr int kStages = 4;      // shared-memory pipeline depth of the wide tile
 // so a stage is mostly weight bytes and the freed shared memory buys a deeper pipeline --
 // more weight bytes in flight per SM, which is what a weight-streaming GEMM is bound by.
 constexpr int kNarrowBN = 64;
-// The forward takes the fused narrow kernel when the mean rows per expert, T*k/E, is at
-// most this.
+constexpr int kGuNarrowStages = 5;   // 5 x (2 x 16 KB + 8 KB)
+constexpr int kDnNarrowStages = 8;   // 8 x (16 KB + 8 KB)
+// The forward takes the narrow tiles when the mean rows per expert, T*k/E, is at most this.
 constexpr int kNarrowMaxMeanRows = 32;
-// Largest T for which the narrow kernel routes in its own prologue and gathers its token
-// rows straight from x (tile::gather4, four rows per TMA operation) instead of reading a
-// permuted copy: a tile then has at most 32 rows, 8 gathers per stage.  Above, the TMA
-// engine's cost per gather operation makes the expert GEMM slower by more than a separate
-// copy costs (measured on B200).
+// Largest T for which gate_up gathers its token rows straight from x (tile::gather4, four
+// rows per TMA operation) instead of reading a permuted copy: a tile then has at most 32
+// rows, 8 gathers per stage.  Above, the TMA engine's cost per gather operation makes the
+// expert GEMM slower by more than a separate copy costs (measured on B200).
 constexpr int kGatherMaxT = 32;
-// Tile families of the wide expert GEMMs.  Pair tiles (D % 256 == 0): two CTAs of a cluster
-// share each tcgen05.mma of M = 256 (cta_group::2) -- 128 weight rows per SM, half of the 256
-// token rows per SM -- which halves the shared-memory operand traffic per FLOP of each SM;
-// gate_up pair tiles cover 128 features, down pair tiles 256 output rows.
-enum { kTilesWide = 1, kTilesPair = 2 };
+// Tile families of the expert GEMMs.  Pair tiles (wide shapes, D % 256 == 0): two CTAs of a
+// cluster share each tcgen05.mma of M = 256 (cta_group::2) -- 128 weight rows per SM, half
+// of the 256 token rows per SM -- which halves the shared-memory operand traffic per FLOP
+// of each SM; gate_up pair tiles cover 128 features, down pair tiles 256 output rows.
+enum { kTilesNarrow = 0, kTilesWide = 1, kTilesPair = 2 };
 constexpr int kPairStages = 6;   // 6 x (16 KB weights + 16 KB tokens) per CTA
 
-// Split tail items of the narrow kernel: at most this many K slices per item, and a fixed
-// capacity of FP32 partial-sum slots per phase (slices per item are capped so that the
-// tail's slices fit; a device with fewer SMs splits less).  A tail is split only when it is
-// at most half a wave of the grid, so at most grid / 2 items x 8 epilogue warps hold a
-// ticket; the persistent expert kernels therefore run at most kMaxTcGrid CTAs.
+// Split tail items of the narrow-tile GEMMs: at most this many K slices per item, and a
+// fixed capacity of FP32 partial-sum slots (slices per item are capped so that the tail's
+// slices fit; a device with fewer SMs splits less).  A tail is split only when it is at most
+// half a wave of the grid, so at most grid / 2 items x 8 epilogue warps hold a ticket; the
+// persistent expert GEMMs therefore run at most kMaxTcGrid CTAs.
 constexpr int kMaxKSplit = 8;
 constexpr int kSplitSlots = 148;
 constexpr int kSplitTickets = 1024;   // per GEMM; the completion counters follow them
@@ -107,8 +107,9 @@ struct PermuteArgs {
     int* err;
 };
 
-// Selection of every token and the permutation in one kernel (T*k <= kPermChunk): blocks
-// select 32 tokens each, the last block to finish performs the permutation.
+// Routing of T <= kFusedRouteMaxT tokens in one kernel: blocks split the experts' logits,
+// the last block to finish selects every token and performs the permutation.
+constexpr int kFusedRouteMaxT = 32;
 struct RouteArgs {
     const uint16_t* x;        // [T, D]
     const uint16_t* W_r;      // [E, D]
@@ -123,9 +124,6 @@ struct RouteArgs {
     // nsplit partials [nsplit, T, E] in split order, then + bias
     const float* part;
     int nsplit;
-    // gated shared expert: gates[t] = sigmoid(w_s . x_t) written by the selection (or null)
-    const uint16_t* shared_gate;
-    float* gates;
 };
 
 // The router GEMM splits K so that small token counts still spread over the SMs; its
@@ -155,6 +153,10 @@ struct alignas(64) TcMaps {
 struct TcArgs {
     int D, I, I_s, E, nseg;
     SegTables tables;
+    // gate_up token rows: gather = 1 -> gathered from x by row_token (map B = x with a
+    // one-row box, four rows per TMA operation); gather = 0 -> tiles of the permuted copy
+    const int32_t* row_token;
+    int gather;
     // gate_up epilogue
     uint16_t* h;              // [rows, ld_h] bf16 SwiGLU output
     int ld_h;
@@ -162,6 +164,20 @@ struct TcArgs {
     const float* row_weight;
     const int32_t* row_dest;
     float* slots;             // [T * S, D] FP32
+    // split tail items (narrow tiles): FP32 partial accumulators, one slot of
+    // NA x 128 x BN floats per slice (partial_slots slots), and one zeroed ticket per
+    // (tail item, epilogue warp)
+    float* partial;
+    int* tickets;
+    int partial_slots;
+    // Per-expert completion of gate_up (narrow tiles): gate_up's epilogue warps add 1 to
+    // seg_done[s] (and to seg_done[nseg]) once they have written their part of an item's h
+    // tile; with dep_wait, the down kernel does not wait for the whole gate_up grid but its
+    // producer waits until seg_done[s] reaches 8 x (gate_up items of segment s), read from
+    // gu_prefix, so down starts on finished experts while gate_up's last wave runs.
+    int* seg_done;
+    const int* gu_prefix;
+    int dep_wait;
     // dense (router) epilogue: partial sums over split s of K go to logits + s*T*E
     float* logits;            // [ksplit, T, E] FP32
     int ksplit;
@@ -169,61 +185,6 @@ struct TcArgs {
     int* err;
     unsigned long long wait_ns;   // limit of every bounded wait (kWaitLimitNs by default)
 };
-
-// ------------------------------------------------------------------ fused narrow expert stage
-//
-// Decode shapes (T*k <= kNarrowMaxMeanRows * E) run the whole expert stage in one persistent
-// kernel: gate_up + SwiGLU, down + routing weight, and the weighted combine back to token
-// order (see expert_narrow.cu).  With route = 1 (T <= kGatherMaxT) its CTAs also compute the
-// selection and the permutation from the router logits themselves.
-struct alignas(64) NarrowMaps {
-    CUtensorMap gu_A, gu_A_shared;  // gate_up weights (routed experts, shared expert), box 128 rows
-    CUtensorMap gu_B[3];            // token rows: x with a one-row box (gather, route = 1), else
-                                    // the permuted copy at box heights 16, 32, 64
-    CUtensorMap dn_A, dn_A_shared;  // down weights, box 128 rows
-    CUtensorMap dn_B[3];            // h at box heights 16, 32, 64
-};
-
-struct NarrowArgs {
-    int T, D, E, k, I, I_s, nseg, S, norm;
-    int route;                  // 1: selection and permutation in the kernel (T <= kGatherMaxT)
-    // route = 1: inputs and the routing outputs (written by CTA 0; each may be null)
-    const float* logits;        // [T, E] router logits without the bias
-    const float* bias;          // [E] or null
-    const uint16_t* x;          // [T, D]
-    float* logits_out;          // [T, E] logits with the bias
-    int32_t* topk_idx_out;      // [T, k]
-    float* topk_w_out;          // [T, k]
-    int32_t* counts_out;        // [E]
-    int32_t* slot_row_out;      // [T * k]
-    // route = 0: tables, per-row destinations and weights, gates from the routing kernels
-    SegTables tables;
-    const int32_t* row_dest;    // [rows] t * S + j
-    const float* row_weight;    // [rows]
-    const float* gates;         // [T] shared-expert gates, or null
-    const uint16_t* shared_gate;  // [D] w_s (route = 1 computes the gates from it), or null
-    // intermediates
-    uint16_t* h;                // [rows, ld_h] bf16 SwiGLU output
-    int ld_h;
-    float* slots;               // [T * S, D] FP32 weighted expert outputs
-    float* partial_gu;          // split-tail partial accumulators of gate_up and of down
-    float* partial_dn;
-    int* tickets_gu;            // split-tail tickets (zeroed)
-    int* tickets_dn;
-    int partial_slots;
-    int* seg_done;              // [nseg + 1] gate_up completion counts (zeroed), signalled
-    const int* seg_wait;        // the counts down waits on (seg_done, or for the watchdog
-                                // diagnostic counters that nothing increments)
-    int* queue;                 // work-unit counter (zeroed)
-    int* dn_done;               // down items x 4 quarter warps whose slots are stored (zeroed)
-    // output
-    const uint16_t* residual;   // [T, D] or null
-    uint16_t* out;              // [T, D]
-    float* out_f32;             // [T, D] or null
-    int* err;
-    unsigned long long wait_ns;
-};
-cudaError_t launch_narrow(const NarrowMaps& maps, const NarrowArgs& a, int grid, bool pdl, cudaStream_t s);
 
 // Raise a kernel's dynamic shared-memory limit once per device (host-side attribute; done
 // outside stream capture by the first call on each device).
@@ -240,10 +201,10 @@ int device_sm_count();
 cudaError_t launch_router_small(const uint16_t* x, const uint16_t* W_r, int T,
                                 int D, int E, float* logits, bool pdl, cudaStream_t s);
 cudaError_t launch_select(const float* part, int nsplit, const float* bias, int T, int E, int k,
-                          int norm, int32_t* idx, float* w, float* logits_out, const uint16_t* x,
-                          int D, const uint16_t* shared_gate, float* gates, bool pdl,
+                          int norm, int32_t* idx, float* w, float* logits_out, bool pdl,
                           cudaStream_t s);
 cudaError_t launch_permute(const PermuteArgs& a, bool pdl, cudaStream_t s);
+cudaError_t launch_route_fused(const RouteArgs& a, bool pdl, cudaStream_t s);
 cudaError_t launch_select_permute(const RouteArgs& a, bool pdl, cudaStream_t s);
 cudaError_t launch_gather_rows(const uint16_t* x, const int32_t* row_token, int rows, int D,
                                uint16_t* x_perm, bool pdl, cudaStream_t s);

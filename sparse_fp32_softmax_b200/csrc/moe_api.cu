@@ -57,14 +57,9 @@ namespace {
 
 constexpr size_t kAlign = 256;
 // Ints of the ticket region: gate_up split tickets, down split tickets, the per-expert
-// completion counters of gate_up (nseg + 1 <= kMaxSegments + 1), the same number of counters
-// that stay zero (MOE_DIAG_UNSIGNALLED_HANDOFF points the down GEMM at them), and the
-// work-unit counter and the finished-down count of the fused decode kernel.
-constexpr int kTicketInts = 2 * kSplitTickets + 2 * (kMaxSegments + 1) + 2;
-constexpr int kSegDoneAt = 2 * kSplitTickets;
-constexpr int kDiagZeroAt = kSegDoneAt + kMaxSegments + 1;
-constexpr int kQueueAt = kDiagZeroAt + kMaxSegments + 1;
-constexpr int kDnDoneAt = kQueueAt + 1;
+// completion counters of gate_up (nseg + 1 <= kMaxSegments + 1), and the same number of
+// counters that stay zero (MOE_DIAG_UNSIGNALLED_HANDOFF points the down GEMM at them).
+constexpr int kTicketInts = 2 * kSplitTickets + 2 * (kMaxSegments + 1);
 
 // The cudaError_t of the last CUDA failure seen by this host thread (moe_last_cuda_error).
 thread_local int g_last_cuda_error = 0;
@@ -77,8 +72,8 @@ bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 // Byte offsets of every workspace region.
 struct Plan {
     int T, D, E, k, I, I_s, has_shared, S, R, ld_h, nchunks, nseg, rsplit;
-    size_t err, tickets, partial, logits, idx, w, gates, counts, offsets, chunk, seg_count, seg_start,
-        gu_items, dn_items, row_token, row_weight, row_dest, slot_row, x_perm, h, slots, total;
+    size_t err, tickets, partial, logits, idx, w, counts, offsets, chunk, seg_count, seg_start, gu_items, dn_items,
+        row_token, row_weight, row_dest, slot_row, x_perm, h, slots, total;
 };
 
 Plan make_plan(const moe_dims& d, const moe_opts* o) {
@@ -105,7 +100,6 @@ Plan make_plan(const moe_dims& d, const moe_opts* o) {
     p.logits = take((size_t)p.rsplit * p.T * p.E * 4);   // router partial sums (or logits)
     p.idx = take((size_t)p.T * p.k * 4);
     p.w = take((size_t)p.T * p.k * 4);
-    p.gates = take(p.has_shared ? (size_t)p.T * 4 : 0);   // shared-expert gates (decode shapes)
     p.counts = take((size_t)(p.E + 1) * 4);
     p.offsets = take((size_t)(p.E + 2) * 4);
     p.chunk = take((size_t)p.nchunks * p.E * 4);
@@ -342,7 +336,7 @@ moe_status moe_route(const moe_bf16* x, const moe_bf16* W_r, const float* bias,
     moe_status st2 = run_logits(x, W_r, p, part, ws, s);
     if (st2 != MOE_OK) return st2;
     MOE_CUDA(launch_select(part, p.rsplit, bias, p.T, p.E, p.k, dims->norm_topk_prob, topk_idx,
-                           topk_w, logits, x, p.D, nullptr, nullptr, true, s));
+                           topk_w, logits, true, s));
     return MOE_OK;
 }
 
@@ -430,57 +424,63 @@ moe_status moe_forward_ex(const moe_bf16* x, const moe_bf16* W_r, const moe_bf16
     const unsigned long long wait_ns =
         (opts && opts->wait_limit_us) ? (unsigned long long)opts->wait_limit_us * 1000ull : kWaitLimitNs;
 
-    // Decode shapes (few rows per expert: T*k <= 32*E) run the whole expert stage in one
-    // fused kernel; for T <= kGatherMaxT that kernel also selects and permutes from the router
-    // logits, and gathers its token rows straight from x (no permuted copy).  Wider shapes
-    // run the grouped GEMMs on CTA pairs (or one-CTA wide tiles) and a combine kernel.
+    // tensor maps of the grouped path are encoded before anything is enqueued
+    // narrow tiles (deeper pipelines) when experts average few rows; a segment with more
+    // rows than a tile is simply split into several token tiles.  gate_up token rows: for
+    // T <= kGatherMaxT gathered from x (one-row box, tile::gather4), else a permuted copy.
     const bool narrow = use_narrow_tiles(p.T, p.k, p.E);
-    const bool route_in_kernel = narrow && p.T <= kGatherMaxT;
+    const bool gather = p.T <= kGatherMaxT;
     // Wide shapes: gate_up on CTA pairs; down on CTA pairs when its rows split into 256-row
     // tiles and experts average at least 256 rows (measured on B200: with fewer rows the
     // pair tiles' narrower N and halved item count cost more than the pairs save).
     // (devices that cannot co-schedule the pairs take the one-CTA wide tiles)
     const bool pairs = !narrow && pair_tiles_available();
-    const int gu_tiles = pairs ? kTilesPair : kTilesWide;
-    const int dn_tiles = (pairs && p.D % 256 == 0 && (long long)p.T * p.k >= 256ll * p.E) ? kTilesPair : kTilesWide;
+    const int gu_tiles = narrow ? kTilesNarrow : (pairs ? kTilesPair : kTilesWide);
+    const int dn_tiles = narrow ? kTilesNarrow
+                         : (pairs && p.D % 256 == 0 && (long long)p.T * p.k >= 256ll * p.E)
+                               ? kTilesPair
+                               : kTilesWide;
     const int gu_bn = narrow ? kNarrowBN : kGuBN;
     const int dn_bn = narrow ? kNarrowBN : kDnBN;
-    uint16_t* h = at<uint16_t>(ws, p.h);
-    uint16_t* x_perm = at<uint16_t>(ws, p.x_perm);
-    // tensor maps are encoded before anything is enqueued
+    const int b_box_max = gu_tiles == kTilesPair ? kGuBN / 2 : gu_bn;   // token rows per CTA
     TcMaps mGu, mDn;
-    NarrowMaps mN;
-    if (narrow) {
-        bool ok = make_map(&mN.gu_A, W_gate_up, p.D, (uint64_t)p.E * 2 * p.I, kTcM) &&
-                  make_map(&mN.gu_A_shared, sgu ? sgu : W_gate_up, p.D,
-                           sgu ? 2 * (uint64_t)p.I_s : 2 * (uint64_t)p.I, kTcM) &&
-                  make_map(&mN.dn_A, W_down, p.I, (uint64_t)p.E * p.D, kTcM) &&
-                  make_map(&mN.dn_A_shared, sdn ? sdn : W_down, sdn ? p.I_s : p.I, p.D, kTcM);
-        for (int bi = 0; ok && bi < 3; ++bi) {
-            ok = make_map(&mN.dn_B[bi], h, p.ld_h, p.R, 16u << bi) &&
-                 (route_in_kernel ? make_map(&mN.gu_B[bi], x, p.D, p.T, 1)
-                                  : make_map(&mN.gu_B[bi], x_perm, p.D, p.R, 16u << bi));
-        }
-        if (!ok) return MOE_ERR_CUDA;
-    } else {
-        const int b_box_max = gu_tiles == kTilesPair ? kGuBN / 2 : gu_bn;   // token rows per CTA
-        const bool ok =
-            make_b_maps(mGu.B, x_perm, p.D, p.R, b_box_max) &&
-            make_map_gate_up_il(&mGu.A, W_gate_up, p.D, p.I, p.E) &&
-            make_map_gate_up_il(&mGu.A_shared, sgu ? sgu : W_gate_up, p.D, sgu ? p.I_s : p.I, 1) &&
-            make_map(&mDn.A, W_down, p.I, (uint64_t)p.E * p.D, kTcM) &&
-            make_map(&mDn.A_shared, sdn ? sdn : W_down, sdn ? p.I_s : p.I, p.D, kTcM) &&
-            make_b_maps(mDn.B, h, p.ld_h, p.R, dn_tiles == kTilesPair ? kDnBN / 2 : dn_bn);
-        if (!ok) return MOE_ERR_CUDA;
+    {
+        uint16_t* h = at<uint16_t>(ws, p.h);
+        const bool gu_b_ok = gather ? make_map(&mGu.B[0], x, p.D, p.T, 1)
+                                    : make_b_maps(mGu.B, at<uint16_t>(ws, p.x_perm), p.D, p.R, b_box_max);
+        const bool gu_a_ok =
+            narrow ? make_map(&mGu.A, W_gate_up, p.D, (uint64_t)p.E * 2 * p.I, kTcM) &&
+                         make_map(&mGu.A_shared, sgu ? sgu : W_gate_up, p.D,
+                                  sgu ? 2 * (uint64_t)p.I_s : 2 * (uint64_t)p.I, kTcM)
+                   : make_map_gate_up_il(&mGu.A, W_gate_up, p.D, p.I, p.E) &&
+                         make_map_gate_up_il(&mGu.A_shared, sgu ? sgu : W_gate_up, p.D,
+                                             sgu ? p.I_s : p.I, 1);
+        if (!gu_a_ok ||
+            !gu_b_ok ||
+            !make_map(&mDn.A, W_down, p.I, (uint64_t)p.E * p.D, kTcM) ||
+            !make_map(&mDn.A_shared, sdn ? sdn : W_down, sdn ? p.I_s : p.I, p.D, kTcM) ||
+            !make_b_maps(mDn.B, h, p.ld_h, p.R, dn_tiles == kTilesPair ? kDnBN / 2 : dn_bn))
+            return MOE_ERR_CUDA;
+        if (gather)
+            for (int bi = 1; bi < kNumBBoxes; ++bi) mGu.B[bi] = mGu.B[0];
     }
 
     // the header of the workspace: device error word, routing ticket, tickets and counters
-    MOE_CUDA(cudaMemsetAsync(err, 0, p.partial - p.err, s));
+    MOE_CUDA(cudaMemsetAsync(err, 0, p.tickets - p.err + (size_t)kTicketInts * 4, s));
     if ((st = record(opts, 0, s)) != MOE_OK) return st;
+    // T <= 32: one kernel routes and permutes.  Above: router partial sums, then selection and
+    // permutation (one kernel while T*k fits a single permutation block).
+    const bool fused_route = p.T <= kFusedRouteMaxT;
+    const bool select_permute = !fused_route && (long long)p.T * p.k <= kPermChunk;
     float* part = at<float>(ws, p.logits);
-    float* gates = (narrow && p.has_shared && sg) ? at<float>(ws, p.gates) : nullptr;
-    // launch chaining between the forward's kernels (not across a stage-event record)
-    const bool chain = !(opts && opts->n_stage_events == 6);
+    if (!fused_route) {
+        if ((st = run_logits(x, W_r, p, part, ws, s)) != MOE_OK) return st;
+        if (!select_permute)
+            MOE_CUDA(launch_select(part, p.rsplit, bias, p.T, p.E, p.k, dims->norm_topk_prob, idx, w,
+                                   logits_user, true, s));
+    }
+    if ((st = record(opts, 1, s)) != MOE_OK) return st;
+
     PermuteArgs pa{};
     pa.topk_idx = idx;
     pa.topk_w = w;
@@ -500,100 +500,66 @@ moe_status moe_forward_ex(const moe_bf16* x, const moe_bf16* W_r, const moe_bf16
     pa.tables = tables_of(p, ws);
     pa.gu_bn = gu_bn;
     pa.dn_bn = dn_bn;
-    pa.gu_features = narrow ? kTcM : (gu_tiles == kTilesWide ? kGuILFeatures : kTcM);
-    pa.dn_rows = (!narrow && dn_tiles == kTilesPair) ? 2 * kTcM : kTcM;
+    pa.gu_features = gu_tiles == kTilesWide ? kGuILFeatures : kTcM;
+    pa.dn_rows = dn_tiles == kTilesPair ? 2 * kTcM : kTcM;
     pa.err = err;
-    if (route_in_kernel) {
-        // router logits only (the bias is added by the selection in the expert kernel)
-        MOE_CUDA(launch_router_small(x, W_r, p.T, p.D, p.E, part, false, s));
-        if ((st = record(opts, 1, s)) != MOE_OK) return st;
-        if ((st = record(opts, 2, s)) != MOE_OK) return st;
+    // launch chaining between the forward's kernels (not across a stage-event record)
+    const bool chain = !(opts && opts->n_stage_events == 6);
+    RouteArgs ra{};
+    ra.x = x; ra.W_r = W_r; ra.bias = bias;
+    ra.T = p.T; ra.D = p.D; ra.E = p.E; ra.k = p.k; ra.norm = dims->norm_topk_prob;
+    ra.topk_idx = idx;
+    ra.topk_w = w;
+    ra.ticket = err + 1;
+    ra.perm = pa;
+    if (fused_route) {
+        // one kernel: logits, softmax, top-k and (in its last block) the permutation
+        ra.logits_out = logits;
+        MOE_CUDA(launch_route_fused(ra, false, s));
+    } else if (select_permute) {
+        ra.logits_out = logits_user;
+        ra.part = part;
+        ra.nsplit = p.rsplit;
+        MOE_CUDA(launch_select_permute(ra, chain, s));
     } else {
-        // router partial sums, then selection and permutation (one kernel while T*k fits a
-        // single permutation block), then the permuted copy of x
-        const bool select_permute = (long long)p.T * p.k <= kPermChunk;
-        if ((st = run_logits(x, W_r, p, part, ws, s)) != MOE_OK) return st;
-        if (!select_permute)
-            MOE_CUDA(launch_select(part, p.rsplit, bias, p.T, p.E, p.k, dims->norm_topk_prob, idx, w,
-                                   logits_user, x, p.D, sg, gates, true, s));
-        if ((st = record(opts, 1, s)) != MOE_OK) return st;
-        if (select_permute) {
-            RouteArgs ra{};
-            ra.x = x; ra.W_r = W_r; ra.bias = bias;
-            ra.T = p.T; ra.D = p.D; ra.E = p.E; ra.k = p.k; ra.norm = dims->norm_topk_prob;
-            ra.topk_idx = idx;
-            ra.topk_w = w;
-            ra.ticket = err + 1;
-            ra.perm = pa;
-            ra.logits_out = logits_user;
-            ra.part = part;
-            ra.nsplit = p.rsplit;
-            ra.shared_gate = sg;
-            ra.gates = gates;
-            MOE_CUDA(launch_select_permute(ra, chain, s));
-        } else {
-            MOE_CUDA(launch_permute(pa, chain, s));
-        }
-        MOE_CUDA(launch_gather_rows(x, pa.row_token, p.R, p.D, x_perm, true, s));
-        if ((st = record(opts, 2, s)) != MOE_OK) return st;
+        MOE_CUDA(launch_permute(pa, chain, s));
     }
+    if (!gather)
+        MOE_CUDA(launch_gather_rows(x, pa.row_token, p.R, p.D, at<uint16_t>(ws, p.x_perm), true, s));
+    if ((st = record(opts, 2, s)) != MOE_OK) return st;
 
     int* tickets = at<int>(ws, p.tickets);
-    const int grid = sms < kMaxTcGrid ? sms : kMaxTcGrid;
-    if (narrow) {
-        NarrowArgs na{};
-        na.T = p.T; na.D = p.D; na.E = p.E; na.k = p.k; na.I = p.I; na.I_s = p.I_s;
-        na.nseg = p.nseg; na.S = p.S; na.norm = dims->norm_topk_prob;
-        na.route = route_in_kernel ? 1 : 0;
-        na.logits = part;
-        na.bias = bias;
-        na.x = x;
-        na.logits_out = logits_user;
-        na.topk_idx_out = opts ? opts->topk_idx_out : nullptr;
-        na.topk_w_out = opts ? opts->topk_w_out : nullptr;
-        na.counts_out = opts ? opts->expert_counts_out : nullptr;
-        na.slot_row_out = opts ? opts->slot_row_out : nullptr;
-        na.tables = pa.tables;
-        na.row_dest = pa.row_dest;
-        na.row_weight = pa.row_weight;
-        na.gates = gates;
-        na.shared_gate = sg;
-        na.h = h;
-        na.ld_h = p.ld_h;
-        na.slots = at<float>(ws, p.slots);
-        na.partial_gu = at<float>(ws, p.partial);
-        na.partial_dn = at<float>(ws, p.partial) + (size_t)kSplitSlots * 2 * kTcM * kNarrowBN;
-        na.tickets_gu = tickets;
-        na.tickets_dn = tickets + kSplitTickets;
-        na.partial_slots = kSplitSlots;
-        // watchdog diagnostic: down watches counters that no kernel increments
-        na.seg_done = tickets + kSegDoneAt;
-        na.seg_wait = tickets + ((opts && opts->diag == MOE_DIAG_UNSIGNALLED_HANDOFF) ? kDiagZeroAt : kSegDoneAt);
-        na.queue = tickets + kQueueAt;
-        na.dn_done = tickets + kDnDoneAt;
-        na.residual = residual;
-        na.out = out;
-        na.out_f32 = out_f32;
-        na.err = err;
-        na.wait_ns = wait_ns;
-        MOE_CUDA(launch_narrow(mN, na, grid, chain, s));
-        if ((st = record(opts, 3, s)) != MOE_OK) return st;
-        if ((st = record(opts, 4, s)) != MOE_OK) return st;
-        return record(opts, 5, s);
-    }
     TcArgs ta{};
     ta.D = p.D; ta.I = p.I; ta.I_s = p.I_s; ta.E = p.E; ta.nseg = p.nseg; ta.T = p.T;
     ta.tables = pa.tables;
-    ta.h = h;
+    ta.row_token = pa.row_token;
+    ta.gather = gather ? 1 : 0;
+    ta.h = at<uint16_t>(ws, p.h);
     ta.ld_h = p.ld_h;
     ta.row_weight = pa.row_weight;
     ta.row_dest = pa.row_dest;
     ta.slots = at<float>(ws, p.slots);
+    ta.partial = narrow ? at<float>(ws, p.partial) : nullptr;
+    ta.tickets = tickets;
+    ta.partial_slots = narrow ? kSplitSlots : 0;
+    // narrow tiles: gate_up reports each finished expert; down waits per expert
+    ta.seg_done = narrow ? tickets + 2 * kSplitTickets : nullptr;
+    ta.gu_prefix = pa.tables.gu_items;
     ta.err = err;
     ta.wait_ns = wait_ns;
+    TcArgs tdn = ta;
+    tdn.dep_wait = narrow ? 1 : 0;
+    if (narrow) {
+        tdn.partial = at<float>(ws, p.partial) + (size_t)kSplitSlots * 2 * kTcM * kNarrowBN;
+        tdn.tickets = tickets + kSplitTickets;
+        // watchdog diagnostic: down watches counters that no kernel increments
+        if (opts && opts->diag == MOE_DIAG_UNSIGNALLED_HANDOFF)
+            tdn.seg_done = tickets + 2 * kSplitTickets + (kMaxSegments + 1);
+    }
+    const int grid = sms < kMaxTcGrid ? sms : kMaxTcGrid;
     MOE_CUDA(launch_tc_gate_up(mGu, ta, grid, gu_tiles, chain, s));
     if ((st = record(opts, 3, s)) != MOE_OK) return st;
-    MOE_CUDA(launch_tc_down(mDn, ta, grid, dn_tiles, chain, s));
+    MOE_CUDA(launch_tc_down(mDn, tdn, grid, dn_tiles, chain, s));
     if ((st = record(opts, 4, s)) != MOE_OK) return st;
     MOE_CUDA(launch_combine(ta.slots, p.T, p.D, p.k, p.has_shared, x, sg, residual, out,
                             out_f32, chain, s));

@@ -15,17 +15,39 @@ __device__ __forceinline__ float float_from_order_key(uint32_t o) {
     return __uint_as_float((o & 0x80000000u) ? (o & 0x7FFFFFFFu) : ~o);
 }
 
-// Selection for one token by one warp from its logits in registers: lane L holds the logits
-// of experts L, L+32, ... (v[i] for expert L + 32 i, before the bias).  The bias is added
-// when given and the logits are written to logits_out when given.  Experts are ranked by the
+// Selection for one token by one warp.  The token's logits are the sum of nsplit partial
+// rows (part + s*split_stride, added in split order) plus the bias when given; lane L holds
+// experts L, L+32, ...  and writes them to logits_out when given.  Experts are ranked by the
 // order-preserving key of their logit; among equal keys the lower index wins: each round,
 // one warp-wide max over the keys, then one over the complemented indices of the lanes
 // holding that key.
-template <int VPL>
-__device__ __forceinline__ void select_values(float (&v)[VPL], const float* bias, int E, int k,
-                                              int norm, int32_t* idx_out, float* w_out,
-                                              float* logits_out) {
+// L2_LOADS: the partial rows were written by other blocks of the running kernel, so they
+// are read through L2 (ld.global.cg); otherwise with generic loads (shared memory, or
+// global memory written by an earlier kernel).
+template <int VPL, bool L2_LOADS = false>
+__device__ __forceinline__ void select_token(const float* part, int nsplit, size_t split_stride,
+                                             const float* bias, int E, int k, int norm,
+                                             int32_t* idx_out, float* w_out, float* logits_out) {
     const int lane = threadIdx.x & 31;
+    float v[VPL];
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+        const int e = lane + 32 * i;
+        v[i] = e < E ? (L2_LOADS ? __ldcg(part + e) : part[e]) : 0.f;
+    }
+#pragma unroll
+    for (int sp = 1; sp < kRouterMaxSplit; ++sp) {  // loads of all partials in flight together
+        if (sp < nsplit) {
+            float q[VPL];
+#pragma unroll
+            for (int i = 0; i < VPL; ++i) {
+                const int e = lane + 32 * i;
+                q[i] = e < E ? part[(size_t)sp * split_stride + e] : 0.f;
+            }
+#pragma unroll
+            for (int i = 0; i < VPL; ++i) v[i] += q[i];  // split order
+        }
+    }
     uint32_t key[VPL];
     uint32_t kmax = 0;
 #pragma unroll
@@ -85,69 +107,6 @@ __device__ __forceinline__ void select_values(float (&v)[VPL], const float* bias
         idx_out[lane] = my_e;
         w_out[lane] = out;
     }
-}
-
-// The logits of one token as the sum of nsplit partial rows (part + s*split_stride, added in
-// split order), into the registers select_values takes.
-// L2_LOADS: the partial rows were written by other blocks of the running kernel, so they
-// are read through L2 (ld.global.cg); otherwise with generic loads (shared memory, or
-// global memory written by an earlier kernel).
-template <int VPL, bool L2_LOADS = false>
-__device__ __forceinline__ void load_logits(const float* part, int nsplit, size_t split_stride, int E,
-                                            float (&v)[VPL]) {
-    const int lane = threadIdx.x & 31;
-#pragma unroll
-    for (int i = 0; i < VPL; ++i) {
-        const int e = lane + 32 * i;
-        v[i] = e < E ? (L2_LOADS ? __ldcg(part + e) : part[e]) : 0.f;
-    }
-#pragma unroll
-    for (int sp = 1; sp < kRouterMaxSplit; ++sp) {  // loads of all partials in flight together
-        if (sp < nsplit) {
-            float q[VPL];
-#pragma unroll
-            for (int i = 0; i < VPL; ++i) {
-                const int e = lane + 32 * i;
-                q[i] = e < E ? part[(size_t)sp * split_stride + e] : 0.f;
-            }
-#pragma unroll
-            for (int i = 0; i < VPL; ++i) v[i] += q[i];  // split order
-        }
-    }
-}
-
-// Selection for one token by one warp from its partial logit rows (see load_logits and
-// select_values).
-template <int VPL, bool L2_LOADS = false>
-__device__ __forceinline__ void select_token(const float* part, int nsplit, size_t split_stride,
-                                             const float* bias, int E, int k, int norm,
-                                             int32_t* idx_out, float* w_out, float* logits_out) {
-    float v[VPL];
-    load_logits<VPL, L2_LOADS>(part, nsplit, split_stride, E, v);
-    select_values<VPL>(v, bias, E, k, norm, idx_out, w_out, logits_out);
-}
-
-// The gate of the shared expert for one token, sigmoid(w_s . x) ("27. Mixture of experts",
-// section "The shared expert"), by one warp: FP32 accumulation of the exact bf16 products,
-// lane L taking elements L*8 .. L*8+7 of every 256-element step in order, then a butterfly.
-__device__ __forceinline__ float shared_gate_value(const uint16_t* x, const uint16_t* w_s, int D) {
-    const int lane = threadIdx.x & 31;
-    float acc = 0.f;
-    for (int c = lane * 8; c < D; c += 256) {
-        const uint4 w = ld_v4(w_s + c);
-        const uint4 v = ld_v4(x + c);
-        acc = fmaf(bf16_lo(w.x), bf16_lo(v.x), acc);
-        acc = fmaf(bf16_hi(w.x), bf16_hi(v.x), acc);
-        acc = fmaf(bf16_lo(w.y), bf16_lo(v.y), acc);
-        acc = fmaf(bf16_hi(w.y), bf16_hi(v.y), acc);
-        acc = fmaf(bf16_lo(w.z), bf16_lo(v.z), acc);
-        acc = fmaf(bf16_hi(w.z), bf16_hi(v.z), acc);
-        acc = fmaf(bf16_lo(w.w), bf16_lo(v.w), acc);
-        acc = fmaf(bf16_hi(w.w), bf16_hi(v.w), acc);
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    return 1.0f / (1.0f + expf(-acc));
 }
 
 }  // namespace moe

@@ -97,9 +97,7 @@ def test_peaks_and_profile_lookup(tmp_path, monkeypatch):
 
 
 def test_kernels_per_forward_follows_the_launch_sequence():
-    # T <= 32: router logits + fused expert kernel; router + select/permute + row copy
-    # (T*k <= 4096) or full permutation (4 kernels) above; then the fused expert kernel
-    # (T*k <= 32*E) or gate_up, down, combine.
-    assert [bench.kernels_per_forward(T, 8, 128) for T in (1, 32, 33, 256, 512, 8192)] == \
-        [2, 2, 4, 4, 4, 9]
-    assert bench.kernels_per_forward(4096, 4, 60) == 9
+    # fused routing (T <= 32); router + select/permute + row copy (T*k <= 4096); full
+    # permutation (4 kernels) above; then gate_up, down, combine.
+    assert [bench.kernels_per_forward(T, 8) for T in (1, 32, 33, 256, 512, 8192)] == \
+        [4, 4, 6, 6, 6, 9]
