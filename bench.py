@@ -124,16 +124,10 @@ def profile_traffic(kernel_tag):
 
 
 def kernels_per_forward(T, k):
-    """Kernels one moe_forward_ex call launches (the library's launch sequence): T <= 32 one
-    fused routing + permutation kernel; above, the router, then selection + permutation in
-    one kernel while T*k <= 4096 (else selection, histogram, scan and scatter), and the
-    permuted copy of x; then gate_up, down and the combine."""
-    n = 0
-    if T <= 32:
-        n += 1
-    else:
-        n += 1 + (1 if T * k <= 4096 else 4) + 1
-    return n + 3
+    """Kernels one moe_forward_ex call launches (the library's launch sequence): the router;
+    selection + permutation in one kernel while T*k <= 4096, else selection, histogram, scan
+    and scatter; for T > 32 the permuted copy of x; then gate_up, down and the combine."""
+    return 1 + (1 if T * k <= 4096 else 4) + (1 if T > 32 else 0) + 3
 
 
 class ClockSampler:

@@ -124,10 +124,10 @@ size_t moe_workspace_size(const moe_dims *dims, const moe_opts *opts);
  * x [T, D] bf16, W_r [E, D] bf16 (nn.Linear layout), bias [E] FP32 or NULL,
  * logits [T, E] FP32 or NULL (then the workspace holds them), topk_idx [T, k] int32,
  * topk_w [T, k] FP32.
- * Summation order: for T <= 64 each logit is one FP32 sum; above, D is summed in up to 8
- * slices added in slice order, the number of slices fixed by (T, E, D).  Results are bitwise
- * reproducible; a token's logits do not depend on the other tokens within one of those
- * regimes. */
+ * Summation order: D is summed in FP32 in slices added in slice order -- for T <= 64 in 8
+ * equal slices, above in up to 8 slices whose number is fixed by (T, E, D).  Results are
+ * bitwise reproducible; a token's logits do not depend on the other tokens within one of
+ * those two regimes. */
 moe_status moe_route(const moe_bf16 *x, const moe_bf16 *W_r, const float *bias,
                      const moe_dims *dims, float *logits, int32_t *topk_idx, float *topk_w,
                      void *ws, size_t ws_bytes, moe_stream_t stream);

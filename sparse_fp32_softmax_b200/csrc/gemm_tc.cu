@@ -539,8 +539,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         // operands from
         constexpr bool kAhead = MODE == kModeDown && BN > kNarrowBN;
         constexpr int kCPW = (BN + 63) / 64;   // chunks per epilogue warp
-        int nd[kCPW], cd[kCPW];
-        float nw[kCPW], cw[kCPW];
+        int nd[kCPW] = {}, cd[kCPW] = {};
+        float nw[kCPW] = {}, cw[kCPW] = {};
         // The epilogue of one 32-column chunk: v (and u, the up accumulator) hold row `row`.
         auto finish_chunk = [&](const TileInfo& ti, int c, const float* v, const float* u) {
             if (Tr::IL) {
@@ -681,7 +681,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     }
                 }
                 tc_fence_before();
-                mbar_arrive(tempty + b);  // the accumulator is free for the next tile
+                mbar_arrive_relaxed(tempty + b);  // the accumulator is free for the next tile
                 // 2. publish; the warp that completes this (item, warp) portion reduces it
                 __threadfence();
                 __syncwarp();
@@ -752,11 +752,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     finish_chunk(ti, c, v, u);
                 }
             }
+            // the accumulator's values are in registers or stored: hand it back to the MMA
+            // (no release: the slot and h stores need not be ordered before the MMA)
             tc_fence_before();
             if (PAIR)
-                mbar_arrive_cluster(tempty_leader0 + 8u * b);
+                mbar_arrive_cluster_relaxed(tempty_leader0 + 8u * b);
             else
-                mbar_arrive(tempty + b);
+                mbar_arrive_relaxed(tempty + b);
             if (MODE == kModeGateUp && !PAIR && a.seg_done) signal_segment_done(a, ti.seg, lane);
         }
     }

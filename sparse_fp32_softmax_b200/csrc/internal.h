@@ -107,14 +107,11 @@ struct PermuteArgs {
     int* err;
 };
 
-// Routing of T <= kFusedRouteMaxT tokens in one kernel: blocks split the experts' logits,
-// the last block to finish selects every token and performs the permutation.
-constexpr int kFusedRouteMaxT = 32;
+// Selection and permutation of T*k <= kPermChunk assignments in one kernel: each block
+// selects 32 tokens, the last block to finish performs the permutation.
 struct RouteArgs {
-    const uint16_t* x;        // [T, D]
-    const uint16_t* W_r;      // [E, D]
     const float* bias;        // [E] or null
-    int T, D, E, k, norm;
+    int T, E, k, norm;
     float* logits_out;        // [T, E] (the caller's or workspace scratch)
     int32_t* topk_idx;        // [T, k]
     float* topk_w;            // [T, k]
@@ -204,7 +201,6 @@ cudaError_t launch_select(const float* part, int nsplit, const float* bias, int 
                           int norm, int32_t* idx, float* w, float* logits_out, bool pdl,
                           cudaStream_t s);
 cudaError_t launch_permute(const PermuteArgs& a, bool pdl, cudaStream_t s);
-cudaError_t launch_route_fused(const RouteArgs& a, bool pdl, cudaStream_t s);
 cudaError_t launch_select_permute(const RouteArgs& a, bool pdl, cudaStream_t s);
 cudaError_t launch_gather_rows(const uint16_t* x, const int32_t* row_token, int rows, int D,
                                uint16_t* x_perm, bool pdl, cudaStream_t s);

@@ -412,7 +412,6 @@ moe_status moe_forward_ex(const moe_bf16* x, const moe_bf16* W_r, const moe_bf16
 
     int* err = at<int>(ws, p.err);
     float* logits_user = opts ? opts->logits_out : nullptr;
-    float* logits = logits_user ? logits_user : at<float>(ws, p.logits);
     int32_t* idx = (opts && opts->topk_idx_out) ? opts->topk_idx_out : at<int32_t>(ws, p.idx);
     float* w = (opts && opts->topk_w_out) ? opts->topk_w_out : at<float>(ws, p.w);
     const float* bias = opts ? opts->router_bias : nullptr;
@@ -468,17 +467,14 @@ moe_status moe_forward_ex(const moe_bf16* x, const moe_bf16* W_r, const moe_bf16
     // the header of the workspace: device error word, routing ticket, tickets and counters
     MOE_CUDA(cudaMemsetAsync(err, 0, p.tickets - p.err + (size_t)kTicketInts * 4, s));
     if ((st = record(opts, 0, s)) != MOE_OK) return st;
-    // T <= 32: one kernel routes and permutes.  Above: router partial sums, then selection and
-    // permutation (one kernel while T*k fits a single permutation block).
-    const bool fused_route = p.T <= kFusedRouteMaxT;
-    const bool select_permute = !fused_route && (long long)p.T * p.k <= kPermChunk;
+    // Router logits (partial sums), then selection and permutation: one kernel while T*k
+    // fits a single permutation block, else selection and the three permutation kernels.
+    const bool select_permute = (long long)p.T * p.k <= kPermChunk;
     float* part = at<float>(ws, p.logits);
-    if (!fused_route) {
-        if ((st = run_logits(x, W_r, p, part, ws, s)) != MOE_OK) return st;
-        if (!select_permute)
-            MOE_CUDA(launch_select(part, p.rsplit, bias, p.T, p.E, p.k, dims->norm_topk_prob, idx, w,
-                                   logits_user, true, s));
-    }
+    if ((st = run_logits(x, W_r, p, part, ws, s)) != MOE_OK) return st;
+    if (!select_permute)
+        MOE_CUDA(launch_select(part, p.rsplit, bias, p.T, p.E, p.k, dims->norm_topk_prob, idx, w,
+                               logits_user, true, s));
     if ((st = record(opts, 1, s)) != MOE_OK) return st;
 
     PermuteArgs pa{};
@@ -506,17 +502,13 @@ moe_status moe_forward_ex(const moe_bf16* x, const moe_bf16* W_r, const moe_bf16
     // launch chaining between the forward's kernels (not across a stage-event record)
     const bool chain = !(opts && opts->n_stage_events == 6);
     RouteArgs ra{};
-    ra.x = x; ra.W_r = W_r; ra.bias = bias;
-    ra.T = p.T; ra.D = p.D; ra.E = p.E; ra.k = p.k; ra.norm = dims->norm_topk_prob;
+    ra.bias = bias;
+    ra.T = p.T; ra.E = p.E; ra.k = p.k; ra.norm = dims->norm_topk_prob;
     ra.topk_idx = idx;
     ra.topk_w = w;
     ra.ticket = err + 1;
     ra.perm = pa;
-    if (fused_route) {
-        // one kernel: logits, softmax, top-k and (in its last block) the permutation
-        ra.logits_out = logits;
-        MOE_CUDA(launch_route_fused(ra, false, s));
-    } else if (select_permute) {
+    if (select_permute) {
         ra.logits_out = logits_user;
         ra.part = part;
         ra.nsplit = p.rsplit;

@@ -15,71 +15,78 @@ namespace moe {
 
 // ------------------------------------------------------------------ small-T router logits
 //
-// One warp computes the logits of one expert for a group of up to 8 tokens: each lane walks
-// the row of W_r in 16-byte pieces (8 bf16), 256 elements per step, and accumulates the
-// exact bf16 products in FP32.  Used when T is small enough that the whole GEMM is a
-// weight read (decode); larger T goes to the tcgen05 router GEMM.
-__global__ void __launch_bounds__(256) router_small_kernel(const uint16_t* __restrict__ x,
-                                                           const uint16_t* __restrict__ W_r,
-                                                           int T, int D, int E,
-                                                           float* __restrict__ logits) {
+// One block of 8 warps computes the logits of one expert for a group of up to 8 tokens; the
+// warps split the row of W_r into 8 consecutive slices.  In its slice, lane L takes the
+// 16-byte pieces (8 bf16) L, L+32, ... and accumulates the exact bf16 products in FP32 in
+// order; a butterfly adds the lanes, and warp 0 adds the 8 slices in slice order.  Every
+// weight load of the block is in flight at once, and the E x ceil(T/8) blocks spread the
+// router's bytes over the SMs, so at decode sizes the logits cost about one memory round
+// trip.  Used for T <= 64; larger T goes to the tcgen05 router GEMM.
+constexpr int kRsWarps = 8;
+__global__ void __launch_bounds__(kRsWarps * 32) router_small_kernel(const uint16_t* __restrict__ x,
+                                                                   const uint16_t* __restrict__ W_r,
+                                                                   int T, int D, int E,
+                                                                   float* __restrict__ logits) {
+    __shared__ float part[kRsWarps][8];
     pdl_wait();
     pdl_launch_dependents();
-    const int lane = threadIdx.x & 31;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int ngroups = (T + 7) >> 3;
-    const long ntask = (long)E * ngroups;
-    const long nwarps = ((long)gridDim.x * blockDim.x) >> 5;
-    for (long task = ((long)blockIdx.x * blockDim.x + threadIdx.x) >> 5; task < ntask;
-         task += nwarps) {
-        const int e = (int)(task / ngroups);
-        const int t0 = (int)(task % ngroups) * 8;
-        const int nt = min(8, T - t0);
-        float acc[8];
+    const int e = blockIdx.x / ngroups;
+    const int t0 = (blockIdx.x % ngroups) * 8;
+    const int nt = min(8, T - t0);
+    const int slice = D / kRsWarps;              // a multiple of 16 elements (D % 128 == 0)
+    const int c0 = warp * slice, c1 = c0 + slice;
+    const uint16_t* wr = W_r + (size_t)e * D;
+    float acc[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-        const uint16_t* wr = W_r + (size_t)e * D;
-        for (int c = lane * 8; c < D; c += 256) {
-            const uint4 w = ld_v4(wr + c);
-            const float w0 = bf16_lo(w.x), w1 = bf16_hi(w.x), w2 = bf16_lo(w.y), w3 = bf16_hi(w.y);
-            const float w4 = bf16_lo(w.z), w5 = bf16_hi(w.z), w6 = bf16_lo(w.w), w7 = bf16_hi(w.w);
+    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+#pragma unroll 4
+    for (int c = c0 + lane * 8; c < c1; c += 256) {
+        const uint4 w = ld_v4(wr + c);
+        uint4 v[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                if (i < nt) {
-                    const uint4 v = ld_v4(x + (size_t)(t0 + i) * D + c);
-                    float a = acc[i];
-                    a = fmaf(w0, bf16_lo(v.x), a);
-                    a = fmaf(w1, bf16_hi(v.x), a);
-                    a = fmaf(w2, bf16_lo(v.y), a);
-                    a = fmaf(w3, bf16_hi(v.y), a);
-                    a = fmaf(w4, bf16_lo(v.z), a);
-                    a = fmaf(w5, bf16_hi(v.z), a);
-                    a = fmaf(w6, bf16_lo(v.w), a);
-                    a = fmaf(w7, bf16_hi(v.w), a);
-                    acc[i] = a;
-                }
-            }
-        }
-        float mine = 0.f;
+        for (int i = 0; i < 8; ++i)
+            if (i < nt) v[i] = ld_v4(x + (size_t)(t0 + i) * D + c);
+        const float w0 = bf16_lo(w.x), w1 = bf16_hi(w.x), w2 = bf16_lo(w.y), w3 = bf16_hi(w.y);
+        const float w4 = bf16_lo(w.z), w5 = bf16_hi(w.z), w6 = bf16_lo(w.w), w7 = bf16_hi(w.w);
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-            float a = acc[i];
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
-            if (lane == i) mine = a;
+            if (i < nt) {
+                float q = acc[i];
+                q = fmaf(w0, bf16_lo(v[i].x), q);
+                q = fmaf(w1, bf16_hi(v[i].x), q);
+                q = fmaf(w2, bf16_lo(v[i].y), q);
+                q = fmaf(w3, bf16_hi(v[i].y), q);
+                q = fmaf(w4, bf16_lo(v[i].z), q);
+                q = fmaf(w5, bf16_hi(v[i].z), q);
+                q = fmaf(w6, bf16_lo(v[i].w), q);
+                q = fmaf(w7, bf16_hi(v[i].w), q);
+                acc[i] = q;
+            }
         }
-        if (lane < nt) logits[(size_t)(t0 + lane) * E + e] = mine;  // bias: added by the selection
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        float q = acc[i];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
+        if (lane == 0) part[warp][i] = q;
+    }
+    __syncthreads();
+    if (warp == 0 && lane < nt) {
+        float l = part[0][lane];
+#pragma unroll
+        for (int w = 1; w < kRsWarps; ++w) l += part[w][lane];   // slice order
+        logits[(size_t)(t0 + lane) * E + e] = l;                  // bias: added by the selection
     }
 }
 
 cudaError_t launch_router_small(const uint16_t* x, const uint16_t* W_r, int T, int D, int E,
                                 float* logits, bool pdl, cudaStream_t s) {
-    const long ntask = (long)E * ((T + 7) / 8);
-    const int warps_per_block = 8;
-    long blocks = (ntask + warps_per_block - 1) / warps_per_block;
-    const int sms = device_sm_count();
-    if (sms <= 0) return cudaErrorInvalidDevice;
-    if (blocks > sms * 16) blocks = sms * 16;
-    return launch_kernel(router_small_kernel, dim3((int)blocks), dim3(warps_per_block * 32), 0, s, pdl,
+    if (D % (kRsWarps * 16) != 0) return cudaErrorInvalidValue;
+    const long blocks = (long)E * ((T + 7) / 8);
+    return launch_kernel(router_small_kernel, dim3((unsigned)blocks), dim3(kRsWarps * 32), 0, s, pdl,
                          x, W_r, T, D, E, logits);
 }
 

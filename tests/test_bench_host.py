@@ -97,7 +97,7 @@ def test_peaks_and_profile_lookup(tmp_path, monkeypatch):
 
 
 def test_kernels_per_forward_follows_the_launch_sequence():
-    # fused routing (T <= 32); router + select/permute + row copy (T*k <= 4096); full
-    # permutation (4 kernels) above; then gate_up, down, combine.
+    # router; select/permute in one kernel (T*k <= 4096) or four; the row copy for T > 32;
+    # then gate_up, down, combine.
     assert [bench.kernels_per_forward(T, 8) for T in (1, 32, 33, 256, 512, 8192)] == \
-        [4, 4, 6, 6, 6, 9]
+        [5, 5, 6, 6, 6, 9]
