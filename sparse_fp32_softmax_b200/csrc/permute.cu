@@ -21,7 +21,7 @@ __global__ void __launch_bounds__(kPermThreads) perm_fused_kernel(PermuteArgs a)
     extern __shared__ int wb[];  // [32][E]
     pdl_wait();
     pdl_launch_dependents();
-    permute_one_block(a, wb);
+    permute_one_block(a, wb, load_warp_slice(a, 0));
 }
 
 // ------------------------------------------------------------------ multi-block path

@@ -107,7 +107,13 @@ struct WarpSlice {
     long w0;                // first assignment of the warp's slice
 };
 
-static __device__ __forceinline__ WarpSlice load_warp_slice(const PermuteArgs& a, long a0) {
+// (FROM_SMEM: the assignments' experts and weights are in shared memory at idx_s / w_s,
+// the block having just selected them itself; otherwise they are read from a.topk_idx /
+// a.topk_w)
+template <bool FROM_SMEM = false>
+static __device__ __forceinline__ WarpSlice load_warp_slice(const PermuteArgs& a, long a0,
+                                                            const int* idx_s = nullptr,
+                                                            const float* w_s = nullptr) {
     WarpSlice ws;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const long n = (long)a.T * a.k;
@@ -120,8 +126,14 @@ static __device__ __forceinline__ WarpSlice load_warp_slice(const PermuteArgs& a
     for (int r = 0; r < kMaxRounds; ++r) {
         const long as = ws.w0 + r * 32 + lane;
         const bool in = r < ws.rounds && as < n;
-        int e = in ? __ldcg(a.topk_idx + as) : -1;
-        ws.w[r] = (in && a.topk_w) ? __ldcg(a.topk_w + as) : 1.0f;
+        int e;
+        if (FROM_SMEM) {
+            e = in ? idx_s[as] : -1;
+            ws.w[r] = in ? w_s[as] : 1.0f;
+        } else {
+            e = in ? __ldcg(a.topk_idx + as) : -1;
+            ws.w[r] = (in && a.topk_w) ? __ldcg(a.topk_w + as) : 1.0f;
+        }
         if (in && (e >= a.E || e < 0)) {
             set_error(a.err, kErrBadIndex);
             e = -1;
@@ -259,13 +271,12 @@ static __device__ void write_fixed_rows(const PermuteArgs& a, int rows0, const i
 
 // ------------------------------------------------------------------ single-block path
 
-// The whole permutation by one block of 1024 threads (T*k <= 4096).  wb: [32][E] ints of
-// shared memory.  Also called by the fused routing kernel's last block.
-static __device__ void permute_one_block(const PermuteArgs& a, int* wb) {
+// The whole permutation by one block of 1024 threads (T*k <= 4096), from the block's warp
+// slices (load_warp_slice with a0 = 0).  wb: [32][E] ints of shared memory.
+static __device__ void permute_one_block(const PermuteArgs& a, int* wb, const WarpSlice& ws) {
     __shared__ int s_cnt[kMaxSegments];
     __shared__ int s_off[kMaxSegments + 1];
     const int E = a.E;
-    const WarpSlice ws = load_warp_slice(a, 0);
     for (int q = threadIdx.x; q < 32 * E; q += blockDim.x) wb[q] = 0;
     __syncthreads();
     count_warp_slices(a, ws, wb);
