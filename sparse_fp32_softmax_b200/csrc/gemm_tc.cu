@@ -72,6 +72,7 @@ struct TcCfg {
 
 constexpr int kATileBytes = kTcM * kTcK * 2;  // 16 KB
 constexpr int kEpiWarps = 8;
+constexpr int kQD = 4;          // entries of the claimed-unit ring (narrow tiles)
 constexpr int kTcThreads = (2 + kEpiWarps) * 32;
 
 struct TileInfo {
@@ -274,6 +275,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     using Tr = TcCfg<MODE, BN, STAGES, PAIR>;
     constexpr int NA = Tr::NA, ACC = Tr::ACC;
     constexpr bool SPLIT = MODE != kModeRouter && BN <= kNarrowBN;
+    // DYN (narrow tiles): CTA b starts with unit b; each further unit is claimed from a
+    // counter in global memory (units grid, grid + 1, ... in claiming order), one ahead, by
+    // the producer, which hands each to the MMA issuer and the epilogue warps through a ring
+    // of kQD entries; CTAs that run faster (or draw lighter units) take more of them.
+    // Otherwise CTA (pair) b takes units b, b + grid, ...
+    constexpr bool DYN = SPLIT;
     constexpr int SB = Tr::SB;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -284,6 +291,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     uint64_t* tempty = tfull + 2;       // [2]
     uint64_t* drain = tempty + 2;       // [1]
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    // narrow tiles: ring of claimed units (see DYN below), after the TMEM slot
+    uint64_t* qfull = drain + 2;                            // [kQD]
+    uint64_t* qempty = qfull + kQD;                         // [kQD]
+    int* qitem = reinterpret_cast<int*>(qempty + kQD);      // [kQD]
+    static_assert((2 * STAGES + 6) * 8 + kQD * 20 <= 256, "barrier region");
     SmemTables* tabs = reinterpret_cast<SmemTables*>(smem + STAGES * SB + 256);
     // down: per epilogue warp, the current tile's row destinations and weights
     int* ep_dest_all = reinterpret_cast<int*>(tabs + 1);                       // [8][BN]
@@ -306,6 +318,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             mbar_init(tempty + b, (PAIR ? 2 : 1) * kEpiWarps * 32);  // PAIR: both CTAs' epilogues
         }
         mbar_init(drain, 1);
+        for (int q = 0; q < kQD; ++q) {
+            mbar_init(qfull + q, 1);
+            mbar_init(qempty + q, 1 + kEpiWarps);   // the MMA thread and each epilogue warp
+        }
         mbar_fence_init();
     }
     if (warp == 0 && lane < 2 + kNumBBoxes) {
@@ -348,7 +364,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const Sched sc = tc_schedule<MODE, BN, SPLIT>(a, tabs, ugrid);
     const int total = sc.units;
 
-    if (ublk >= total) {
+    if (!DYN && ublk >= total) {
         // no work for this CTA: nothing was issued; fall through to the TMEM release
     } else if (warp == 0) {
         // ------------------------------------------------------------ TMA producer warp
@@ -373,14 +389,36 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         };
         TileInfo tn{};
         int gn[4] = {0, 0, 0, 0};
-        if (first < total) {
+        if (!DYN && first < total) {
             tn = tc_decode_unit<MODE, BN, PAIR>(a, tabs, sc, first, rank);
             if (gather) gather_rows(tn, gn);
         }
-        for (int item = first; item < total && ok; item += step) {
+        // DYN: the unit claimed for after the current one; the first is the CTA's own index
+        // (no claim), later ones come from the counter, numbered from the grid size on
+        int next = (int)blockIdx.x;
+        for (int item = first, qi = 0; ok; item += DYN ? 0 : step, ++qi) {
+            if (DYN) {
+                // publish the claimed unit (or the end, -1) to the MMA and epilogue warps
+                item = __shfl_sync(0xffffffffu, next, 0);
+                const int qs = qi % kQD;
+                const bool gq = mbar_wait(qempty + qs, ((qi / kQD) & 1) ^ 1, a.err, kErrWaitProducer, a.wait_ns);
+                if (!__all_sync(0xffffffffu, gq)) {
+                    ok = false;
+                    break;
+                }
+                if (lane == 0) {
+                    qitem[qs] = item < total ? item : -1;
+                    mbar_arrive(qfull + qs);
+                }
+                if (item >= total) break;
+                tn = tc_decode_unit<MODE, BN, PAIR>(a, tabs, sc, item, rank);
+                if (gather) gather_rows(tn, gn);
+            } else if (item >= total) {
+                break;
+            }
             const TileInfo ti = tn;
             const int g0 = gn[0], g1 = gn[1], g2 = gn[2], g3 = gn[3];
-            if (item + step < total) {
+            if (!DYN && item + step < total) {
                 tn = tc_decode_unit<MODE, BN, PAIR>(a, tabs, sc, item + step, rank);
                 if (gather) gather_rows(tn, gn);
             }
@@ -435,6 +473,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
                 for (int q = 0; q < STAGES; ++q)
                     if (q == s) last_round[q] = round;
+                // DYN: the next unit is claimed once this one's first stage is on its way, so
+                // that at the start every CTA holds one unit before any holds two
+                if (DYN && kb == 0 && lane == 0)
+                    next = total <= (int)gridDim.x ? total : (int)gridDim.x + atomicAdd(a.sched, 1);
             }
         }
         // wait until the MMA issuer has released every stage, then until every issued
@@ -466,7 +508,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             int s = 0, phase = 0;   // ring position of the next stage
             int tc = 0;
             bool ok = true;
-            for (int item = ublk; item < total && ok; item += ugrid, ++tc) {
+            for (int item = ublk, qi = 0; ok; item += DYN ? 0 : ugrid, ++tc, ++qi) {
+                if (DYN) {
+                    const int qs = qi % kQD;
+                    if (!mbar_wait(qfull + qs, (qi / kQD) & 1, a.err, kErrWaitMma, a.wait_ns)) break;
+                    item = qitem[qs];
+                    mbar_arrive(qempty + qs);
+                    if (item < 0) break;
+                } else if (item >= total) {
+                    break;
+                }
                 const TileInfo ti = tc_decode_unit<MODE, BN, PAIR>(a, tabs, sc, item, rank);
                 const int b = tc & 1;
                 const int use = tc >> 1;
@@ -635,7 +686,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         int tc = 0;
         // PAIR: the accumulator is released on the leader's barrier by both CTAs
         const uint32_t tempty_leader0 = PAIR ? mapa_shared(tempty, 0) : 0u;
-        for (int item = ublk; item < total; item += ugrid, ++tc) {
+        for (int item = ublk, qi = 0;; item += DYN ? 0 : ugrid, ++tc, ++qi) {
+            if (DYN) {
+                const int qs = qi % kQD;
+                const bool gq = mbar_wait(qfull + qs, (qi / kQD) & 1, a.err, kErrWaitEpilogue, a.wait_ns);
+                if (!__all_sync(0xffffffffu, gq)) break;
+                item = qitem[qs];
+                __syncwarp();
+                if (lane == 0) mbar_arrive(qempty + qs);
+                if (item < 0) break;
+            } else if (item >= total) {
+                break;
+            }
             const TileInfo ti = tc_decode_unit<MODE, BN, PAIR>(a, tabs, sc, item, rank);
             const int b = tc & 1;
             const int use = tc >> 1;

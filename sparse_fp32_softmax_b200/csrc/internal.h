@@ -175,6 +175,8 @@ struct TcArgs {
     int* seg_done;
     const int* gu_prefix;
     int dep_wait;
+    // narrow tiles: counter (zero at launch) from which the CTAs claim their units
+    int* sched;
     // dense (router) epilogue: partial sums over split s of K go to logits + s*T*E
     float* logits;            // [ksplit, T, E] FP32
     int ksplit;

@@ -57,9 +57,11 @@ namespace {
 
 constexpr size_t kAlign = 256;
 // Ints of the ticket region: gate_up split tickets, down split tickets, the per-expert
-// completion counters of gate_up (nseg + 1 <= kMaxSegments + 1), and the same number of
-// counters that stay zero (MOE_DIAG_UNSIGNALLED_HANDOFF points the down GEMM at them).
-constexpr int kTicketInts = 2 * kSplitTickets + 2 * (kMaxSegments + 1);
+// completion counters of gate_up (nseg + 1 <= kMaxSegments + 1), the same number of
+// counters that stay zero (MOE_DIAG_UNSIGNALLED_HANDOFF points the down GEMM at them), and
+// the unit counters of the narrow gate_up and down kernels.
+constexpr int kSchedAt = 2 * kSplitTickets + 2 * (kMaxSegments + 1);
+constexpr int kTicketInts = kSchedAt + 2;
 
 // The cudaError_t of the last CUDA failure seen by this host thread (moe_last_cuda_error).
 thread_local int g_last_cuda_error = 0;
@@ -537,10 +539,12 @@ moe_status moe_forward_ex(const moe_bf16* x, const moe_bf16* W_r, const moe_bf16
     // narrow tiles: gate_up reports each finished expert; down waits per expert
     ta.seg_done = narrow ? tickets + 2 * kSplitTickets : nullptr;
     ta.gu_prefix = pa.tables.gu_items;
+    ta.sched = tickets + kSchedAt;
     ta.err = err;
     ta.wait_ns = wait_ns;
     TcArgs tdn = ta;
     tdn.dep_wait = narrow ? 1 : 0;
+    tdn.sched = tickets + kSchedAt + 1;
     if (narrow) {
         tdn.partial = at<float>(ws, p.partial) + (size_t)kSplitSlots * 2 * kTcM * kNarrowBN;
         tdn.tickets = tickets + kSplitTickets;
