@@ -24,12 +24,16 @@ namespace moe {
 
 // ------------------------------------------------------------------ launch chaining
 //
-// Every kernel of the library starts with pdl_wait(): when it was launched as a
-// programmatic dependent of the previous kernel on the stream, this blocks until that
-// kernel has completed and its memory is visible (otherwise it returns at once).  It then
-// calls pdl_launch_dependents() so the next kernel may be launched and run its prologue
-// while this one works.  The first kernel of each API call is launched normally, so the
-// caller's earlier work on the stream is always complete before the library reads inputs.
+// Every kernel of the library calls pdl_wait() before it reads what earlier kernels wrote:
+// when it was launched as a programmatic dependent of the previous kernel on the stream,
+// this blocks until that kernel has completed and its memory is visible (otherwise it
+// returns at once).  pdl_launch_dependents() lets the next kernel be launched and run its
+// prologue while this one works; kernels call it after their wait, except the copy of the
+// permuted rows, which lets gate_up start its speculative weight prefetch early (a
+// dependent can only launch once every block of this kernel is resident, and it waits for
+// this kernel's completion itself).  The
+// first kernel of each API call is launched normally, so the caller's earlier work on the
+// stream is always complete before the library reads inputs.
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_launch_dependents() {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");

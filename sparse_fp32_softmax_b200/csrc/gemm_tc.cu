@@ -350,6 +350,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     // (down with per-expert hand-off: no wait for the whole gate_up grid; everything read
     // below besides h was complete before this kernel could start -- see above)
+    if (MODE == kModeGateUp && DYN && a.spec_steps > 0 && warp == 0 && lane == 0) {
+        const int mt = a.I / kTcM;
+        const int e = (int)blockIdx.x / mt;
+        if (e < a.E) {
+            const int r0 = e * 2 * a.I + ((int)blockIdx.x % mt) * kTcM;
+            for (int kb = 0; kb < a.spec_steps; ++kb) {
+                tma_prefetch_l2(&maps.A, kb * kTcK, r0);
+                tma_prefetch_l2(&maps.A, kb * kTcK, r0 + a.I);
+            }
+        }
+    }
+    // (gate_up lets down start only after its own wait, which down's early reads of the work
+    // tables rely on -- see above)
     if (!(MODE == kModeDown && a.dep_wait)) pdl_wait();
     pdl_launch_dependents();
     if (MODE == kModeGateUp)

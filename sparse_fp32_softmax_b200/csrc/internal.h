@@ -177,6 +177,11 @@ struct TcArgs {
     int dep_wait;
     // narrow tiles: counter (zero at launch) from which the CTAs claim their units
     int* sched;
+    // narrow gate_up: before its dependency wait, CTA b requests into L2 the first spec_steps
+    // K steps of the weight tiles of the unit it most likely starts with (feature tile
+    // b % (I/128) of expert b / (I/128): the first unit when every expert received 1..64
+    // rows); 0 = none.  Only a cache hint: nothing depends on the guess.
+    int spec_steps;
     // dense (router) epilogue: partial sums over split s of K go to logits + s*T*E
     float* logits;            // [ksplit, T, E] FP32
     int ksplit;

@@ -540,9 +540,14 @@ moe_status moe_forward_ex(const moe_bf16* x, const moe_bf16* W_r, const moe_bf16
     ta.seg_done = narrow ? tickets + 2 * kSplitTickets : nullptr;
     ta.gu_prefix = pa.tables.gu_items;
     ta.sched = tickets + kSchedAt;
+    // every expert very likely has rows (T*k >= 4E): the first wave of gate_up units is known
+    // up to that guess, and its weights start towards L2 while routing runs (12 of the K steps
+    // of each first unit: about 57 MB at D = 2048 on 148 SMs, well inside L2)
+    ta.spec_steps = (narrow && (long long)p.T * p.k >= 4ll * p.E) ? min(12, p.D / kTcK) : 0;
     ta.err = err;
     ta.wait_ns = wait_ns;
     TcArgs tdn = ta;
+    tdn.spec_steps = 0;
     tdn.dep_wait = narrow ? 1 : 0;
     tdn.sched = tickets + kSchedAt + 1;
     if (narrow) {

@@ -125,8 +125,10 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __rest
                                                           const int32_t* __restrict__ row_token,
                                                           int rows, int D,
                                                           uint16_t* __restrict__ x_perm) {
-    pdl_wait();
+    // gate_up (next) may launch now: it issues its speculative weight prefetch while the
+    // routing finishes, and waits for this kernel itself
     pdl_launch_dependents();
+    pdl_wait();
     const int lane = threadIdx.x & 31;
     const int nw = (gridDim.x * blockDim.x) >> 5;
     const int vec = D >> 3;
