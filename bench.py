@@ -4,6 +4,7 @@ of the HBM / bf16 roofline reached.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode|prefill|keras|zipf|chain]
                     [--extra prefill,keras,zipf,chain|none] [--impl ours|reference] [--eager]
+                    [--sweep T[,T...]]
 
 Workloads (seeded synthetic inputs of the block's standard configurations):
   decode   (headline) D=2048, E=128, k=8, I=768; one step = one block pass for each of
@@ -561,9 +562,20 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--copies", type=int, default=None,
                     help="decode weight copies in rotation (default: one per pass of a step)")
+    ap.add_argument("--sweep", default=None,
+                    help="token counts of the headline workload's passes, e.g. 8 or 1,256 "
+                         "(default: the workload's own; used to profile one size)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.sweep:
+        try:
+            sw = tuple(int(t) for t in args.sweep.split(","))
+        except ValueError:
+            ap.error("--sweep takes comma-separated token counts")
+        if not sw or min(sw) < 1:
+            ap.error("--sweep takes positive token counts")
+        WORKLOADS[args.workload] = dict(WORKLOADS[args.workload], sweep=sw)
     extra = [] if args.extra in ("", "none") else [w for w in args.extra.split(",") if w != args.workload]
     for w in extra:
         if w not in WORKLOADS:
