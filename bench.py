@@ -54,8 +54,11 @@ WORKLOADS = {
     "keras": dict(config="keras", sweep=(4096,), layers=1),
     "zipf": dict(config="zipf", sweep=(4096,), layers=1),
     "chain": dict(config="keras", sweep=(4096,), layers=48),
+    # the decode sweep with FP8 E4M3 weight-only experts (per-row scales, quantised by the
+    # library); its roofline counts one byte per expert weight plus the scales
+    "decode_fp8": dict(config="decode", sweep=(1, 8, 32, 128, 256), layers=1, fp8=True),
 }
-DEFAULT_EXTRA = "prefill,keras,zipf,chain"
+DEFAULT_EXTRA = "prefill,keras,zipf,chain,decode_fp8"
 
 FALLBACK_PEAKS = dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0)
 SUSTAINED_REGION_S = 1.0     # timed regions at least this long divide by the sustained peak
@@ -231,6 +234,14 @@ def build_workload(name, device, copies=None):
         n = len(sweep) if copies is None else max(1, copies)
         for _ in range(1, n):              # one weight copy per pass of a step
             W.append({k: (v.clone() if v is not None else None) for k, v in base.items()})
+    if spec.get("fp8"):
+        from sparse_fp32_softmax_b200 import binding as B
+        for w in W:                        # FP8 experts replace the bf16 ones
+            q_gu, s_gu = B.moe_quantize_fp8_rows(w.pop("W_gate_up"))
+            q_dn, s_dn = B.moe_quantize_fp8_rows(w.pop("W_down"))
+            w["W_gate_up"] = w["W_down"] = None
+            w["fp8"] = dict(W_gate_up_fp8=q_gu, gate_up_scale=s_gu, W_down_fp8=q_dn, down_scale=s_dn)
+        torch.cuda.synchronize()
     return cfg, spec, sweep, W, x0, L
 
 
@@ -264,7 +275,7 @@ def measure(name, args, rank, world, device, peaks, with_e2e):
         p["idx"] = torch.empty(p["T"], cfg.k, dtype=torch.int32, device=device)
         p["opts"] = B.make_opts(router_bias=w.get("bias"), shared_gate_up=w.get("shared_gate_up"),
                                 shared_down=w.get("shared_down"), shared_gate=w.get("shared_gate"),
-                                residual=p["residual"], topk_idx_out=p["idx"])
+                                residual=p["residual"], topk_idx_out=p["idx"], **w.get("fp8", {}))
         if chain:                             # passes run one after another: one workspace
             if shared_ws is None:
                 shared_ws = B.workspace(p["dims"], p["opts"], device=device)
@@ -278,7 +289,8 @@ def measure(name, args, rank, world, device, peaks, with_e2e):
         if events is not None:
             opts = B.make_opts(router_bias=w.get("bias"), shared_gate_up=w.get("shared_gate_up"),
                                shared_down=w.get("shared_down"), shared_gate=w.get("shared_gate"),
-                               residual=p["residual"], topk_idx_out=p["idx"], stage_events=events)
+                               residual=p["residual"], topk_idx_out=p["idx"], stage_events=events,
+                               **w.get("fp8", {}))
         B.moe_forward_ex(p["x"], w["W_r"], w["W_gate_up"], w["W_down"], cfg.k, cfg.norm_topk_prob,
                          out=p["out"], ws=p["ws"], opts=opts)
 
@@ -391,14 +403,15 @@ def measure(name, args, rank, world, device, peaks, with_e2e):
     gu_roofs, dn_roofs = [], []
     for n, p in enumerate(passes):
         T = p["T"]
-        b_gu = p["touched"] * I2 * cfg.D * 2 + (2 * cfg.I_s * cfg.D * 2 if cfg.I_s else 0)
+        wb = 1 if spec.get("fp8") else 2   # bytes per expert weight (FP8: + a scale per row)
+        b_gu = p["touched"] * I2 * (cfg.D * wb + (4 if wb == 1 else 0)) + (2 * cfg.I_s * cfg.D * 2 if cfg.I_s else 0)
         f_gu = 2.0 * T * cfg.k * I2 * cfg.D + (2.0 * T * 2 * cfg.I_s * cfg.D if cfg.I_s else 0)
-        b_dn = p["touched"] * cfg.I * cfg.D * 2 + (cfg.I_s * cfg.D * 2 if cfg.I_s else 0)
+        b_dn = p["touched"] * cfg.D * (cfg.I * wb + (4 if wb == 1 else 0)) + (cfg.I_s * cfg.D * 2 if cfg.I_s else 0)
         f_dn = 2.0 * T * cfg.k * cfg.I * cfg.D + (2.0 * T * cfg.I_s * cfg.D if cfg.I_s else 0)
         gu_roofs.append((b_gu, f_gu, stage_ms[n][2], T))
         dn_roofs.append((b_dn, f_dn, stage_ms[n][3], T))
         b = algorithmic_bytes(T, cfg.D, cfg.E, cfg.k, cfg.I, p["touched"], cfg.I_s, cfg.shared_gated,
-                              residual=chain)
+                              residual=chain, fp8_experts=bool(spec.get("fp8")))
         f = algorithmic_flops(T, cfg.D, cfg.E, cfg.k, cfg.I, cfg.I_s, cfg.shared_gated)
         blk_bytes += b
         blk_flops += f

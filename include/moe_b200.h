@@ -110,7 +110,31 @@ typedef struct {
     unsigned wait_limit_us;          /* limit of every bounded device wait in microseconds;
                                         0 = the default of 2 s */
     int diag;                        /* MOE_DIAG_* or 0 */
+    /* FP8 weight-only experts.  When W_gate_up_fp8 is set, the routed experts' weights are
+     * read from W_gate_up_fp8 [E, 2I, D] and W_down_fp8 [E, D, I] (one E4M3 byte per weight,
+     * as written by moe_quantize_fp8_rows) with one FP32 scale per weight row,
+     * gate_up_scale [E * 2I] and down_scale [E * D]; weight (e, r, c) = scale[e, r] *
+     * value(q[e, r, c]).  The bf16 W_gate_up and W_down arguments are then not read and may
+     * be NULL.  Tokens stay bf16; each weight tile is widened to bf16 exactly in shared
+     * memory and the row scale is applied to the FP32 accumulator.  Supported at decode
+     * shapes (T*k <= 32*E) without a shared expert; otherwise MOE_ERR_UNSUPPORTED. */
+    const uint8_t *W_gate_up_fp8;    /* [E, 2I, D] E4M3, or NULL (bf16 weights) */
+    const float *gate_up_scale;      /* [E * 2I] FP32 */
+    const uint8_t *W_down_fp8;       /* [E, D, I] E4M3 */
+    const float *down_scale;         /* [E * D] FP32 */
 } moe_opts;
+
+/* Per-row FP8 quantisation of a bf16 matrix W [rows, cols] (rows of the expert weight
+ * tensors: pass W_gate_up as E*2I rows of D, W_down as E*D rows of I).  No format is fixed
+ * by the pages; this is the plainest per-row (per output channel) E4M3 scheme:
+ *   amax[r]  = max_c |W[r, c]|;
+ *   scale[r] = amax[r] / 448 in FP32 (round to nearest even), or 1 when amax[r] == 0;
+ *   q[r, c]  = E4M3 (OCP "e4m3fn": bias 7, max 448, no infinities) of the FP32 quotient
+ *              W[r, c] / scale[r], rounded to nearest even and saturated to +-448.
+ * Bitwise deterministic.  W [rows, cols] bf16, q [rows, cols] bytes, scale [rows] FP32; cols
+ * a multiple of 16 and all pointers 16-byte aligned.  Enqueued on `stream`. */
+moe_status moe_quantize_fp8_rows(const moe_bf16 *W, int64_t rows, int cols, uint8_t *q, float *scale,
+                                 moe_stream_t stream);
 
 /* Bytes of workspace that moe_route, moe_permute and moe_forward(_ex) need for `dims`
  * (and `opts`, which may be NULL).  Returns 0 for invalid or unsupported arguments. */

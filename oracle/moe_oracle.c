@@ -331,3 +331,116 @@ int oracle_loop_dispatch(const uint16_t *x, const int32_t *idx, const float *w, 
     free(tok); free(slot); free(G); free(H);
     return 0;
 }
+
+/* ---------------------------------------------------------------- FP8 weight-only experts */
+
+/* Low-precision experts ("27. Mixture of experts", section "The economics of MoE
+ * inference"; "Qwen3-VL and Mixture of Experts", section "Deploying it").  The pages fix no
+ * format; the reading taken is per-row E4M3 (OCP "e4m3fn": sign, 4 exponent bits with bias 7,
+ * 3 mantissa bits; no infinities, largest value 448):
+ *   scale[r] = amax_c |W[r, c]| / 448 in FP32 (1 when the row is all zero),
+ *   q[r, c]  = E4M3 of the FP32 quotient W[r, c] / scale[r], nearest-even, saturated to 448,
+ *   weight   = scale[r] * value(q[r, c]).                                                   */
+
+/* The value of an E4M3 code (NaN for the two NaN codes). */
+double oracle_e4m3_value(uint8_t code) {
+    int s = code >> 7, e = (code >> 3) & 15, m = code & 7;
+    double v;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0) v = ldexp((double)m, -9);                 /* subnormal: m / 8 * 2^(1 - 7) */
+    else v = ldexp(1.0 + m / 8.0, e - 7);
+    return s ? -v : v;
+}
+
+/* The E4M3 code of a finite FP32 value: nearest, ties to even mantissa, saturated to 448. */
+static uint8_t e4m3_encode(float f) {
+    uint8_t sign = signbit(f) ? 0x80 : 0x00;
+    double a = fabs((double)f);
+    if (a >= 448.0) return sign | 0x7E;                  /* 448 = 2^8 * 1.75 */
+    if (a < ldexp(1.0, -6)) {                            /* below the smallest normal: steps of 2^-9 */
+        double m = nearbyint(ldexp(a, 9));               /* 0..8; 8 is the smallest normal's code */
+        return sign | (uint8_t)m;
+    }
+    int E;
+    double f2 = frexp(a, &E);                            /* a = f2 * 2^E, f2 in [0.5, 1) */
+    int e = E - 1;                                       /* a = (2 f2) * 2^e, 2 f2 in [1, 2) */
+    double m = nearbyint((2.0 * f2 - 1.0) * 8.0);        /* mantissa step, ties to even */
+    if (m == 8.0) { m = 0.0; e += 1; }
+    if (e > 8 || (e == 8 && m > 6.0)) return sign | 0x7E;
+    return sign | (uint8_t)(((e + 7) << 3) | (int)m);
+}
+
+int oracle_quantize_fp8_rows(const uint16_t *W, long rows, int cols, uint8_t *q, float *scale) {
+    if (!W || !q || !scale || rows < 0 || cols <= 0) return 1;
+    for (long r = 0; r < rows; ++r) {
+        const uint16_t *w = W + (size_t)r * cols;
+        float amax = 0.0f;
+        for (int c = 0; c < cols; ++c) {
+            float a = fabsf((float)bf16_to_double(w[c]));
+            if (a > amax) amax = a;
+        }
+        volatile float s = amax > 0.0f ? amax / 448.0f : 1.0f;   /* one FP32 division */
+        scale[r] = s;
+        for (int c = 0; c < cols; ++c) {
+            volatile float v = (float)bf16_to_double(w[c]) / s;  /* one FP32 division */
+            q[(size_t)r * cols + c] = e4m3_encode(v);
+        }
+    }
+    return 0;
+}
+
+/* One SwiGLU expert with FP8 weights (as swiglu_expert; weight = scale[row] * value(q)). */
+static void swiglu_expert_fp8(const uint16_t *x_row, const uint8_t *q_gu, const float *s_gu,
+                              const uint8_t *q_dn, const float *s_dn, int D, int I, double *h,
+                              double *out) {
+    for (int i = 0; i < I; ++i) {
+        double g = 0.0, u = 0.0;
+        for (int d = 0; d < D; ++d) {
+            double xd = bf16_to_double(x_row[d]);
+            g += oracle_e4m3_value(q_gu[(size_t)i * D + d]) * xd;
+            u += oracle_e4m3_value(q_gu[(size_t)(I + i) * D + d]) * xd;
+        }
+        g *= (double)s_gu[i];
+        u *= (double)s_gu[I + i];
+        h[i] = g / (1.0 + exp(-g)) * u;
+    }
+    for (int d = 0; d < D; ++d) {
+        double s = 0.0;
+        for (int i = 0; i < I; ++i) s += oracle_e4m3_value(q_dn[(size_t)d * I + i]) * h[i];
+        out[d] = s * (double)s_dn[d];
+    }
+}
+
+/* y for the listed token rows with FP8 routed experts (no shared expert):
+ *   y[t] = sum_{j<k} w[t,j] * expert_{idx[t,j]}(x[t]) (+ residual[t]);
+ * q_gu [E, 2I, D], s_gu [E * 2I], q_dn [E, D, I], s_dn [E * D]. */
+int oracle_combine_rows_fp8(const uint16_t *x, const int32_t *idx, const float *w,
+                            const int32_t *rows, int nrows, int T, int D, int E, int k, int I,
+                            const uint8_t *q_gu, const float *s_gu, const uint8_t *q_dn,
+                            const float *s_dn, const uint16_t *residual, double *y_out) {
+    if (!x || !idx || !w || !rows || !q_gu || !s_gu || !q_dn || !s_dn || !y_out || D <= 0 || I <= 0 || k <= 0)
+        return 1;
+    double *h = (double *)malloc(sizeof(double) * (size_t)I);
+    double *o = (double *)malloc(sizeof(double) * (size_t)D);
+    if (!h || !o) { free(h); free(o); return 2; }
+    for (int n = 0; n < nrows; ++n) {
+        int t = rows[n];
+        if (t < 0 || t >= T) { free(h); free(o); return 1; }
+        const uint16_t *xr = x + (size_t)t * D;
+        double *y = y_out + (size_t)n * D;
+        for (int d = 0; d < D; ++d) y[d] = 0.0;
+        for (int j = 0; j < k; ++j) {
+            int e = idx[(size_t)t * k + j];
+            if (e < 0 || e >= E) { free(h); free(o); return 1; }
+            swiglu_expert_fp8(xr, q_gu + (size_t)e * 2 * I * D, s_gu + (size_t)e * 2 * I,
+                              q_dn + (size_t)e * D * I, s_dn + (size_t)e * D, D, I, h, o);
+            double wj = (double)w[(size_t)t * k + j];
+            for (int d = 0; d < D; ++d) y[d] += wj * o[d];
+        }
+        if (residual)
+            for (int d = 0; d < D; ++d) y[d] += bf16_to_double(residual[(size_t)t * D + d]);
+    }
+    free(h);
+    free(o);
+    return 0;
+}

@@ -33,6 +33,7 @@ _i32p = ctypes.POINTER(ctypes.c_int32)
 _u16p = ctypes.POINTER(ctypes.c_uint16)
 _f32p = ctypes.POINTER(ctypes.c_float)
 _f64p = ctypes.POINTER(ctypes.c_double)
+_u8p = ctypes.POINTER(ctypes.c_uint8)
 
 
 def build(force: bool = False) -> str:
@@ -65,8 +66,15 @@ def lib():
                                               _f32p]
             l.oracle_loop_dispatch.argtypes = [_u16p, _i32p, _f32p, c_int, c_int, c_int, c_int,
                                                c_int, _u16p, _u16p, _f64p]
+            l.oracle_e4m3_value.argtypes = [ctypes.c_uint8]
+            l.oracle_e4m3_value.restype = ctypes.c_double
+            l.oracle_quantize_fp8_rows.argtypes = [_u16p, ctypes.c_long, c_int, _u8p, _f32p]
+            l.oracle_combine_rows_fp8.argtypes = [_u16p, _i32p, _f32p, _i32p, c_int, c_int, c_int,
+                                                  c_int, c_int, c_int, _u8p, _f32p, _u8p, _f32p,
+                                                  _u16p, _f64p]
             for name in ("oracle_router_logits", "oracle_select", "oracle_route", "oracle_permute",
-                         "oracle_combine_rows", "oracle_forward_rows", "oracle_loop_dispatch"):
+                         "oracle_combine_rows", "oracle_forward_rows", "oracle_loop_dispatch",
+                         "oracle_quantize_fp8_rows", "oracle_combine_rows_fp8"):
                 getattr(l, name).restype = ctypes.c_int
             _lib = l
     return _lib
@@ -231,6 +239,50 @@ def loop_dispatch(x, idx, w, W_gu, W_dn):
                                       _p(W_gu, _u16p), _p(W_dn, _u16p), _p(y, _f64p)),
            "oracle_loop_dispatch")
     return y
+
+
+def e4m3_value(code: int) -> float:
+    """The value of one E4M3 code (NaN for the NaN codes)."""
+    return float(lib().oracle_e4m3_value(int(code) & 0xFF))
+
+
+def quantize_fp8_rows(W):
+    """Per-row E4M3 quantisation of W viewed as [rows, W.shape[-1]] -> (q uint8 of W's shape,
+    scale float32 [rows])."""
+    W = as_u16(W)
+    cols = W.shape[-1]
+    rows = W.size // cols
+    q = np.empty(W.shape, np.uint8)
+    scale = np.empty(rows, np.float32)
+    _check(lib().oracle_quantize_fp8_rows(_p(W, _u16p), rows, cols, _p(q, _u8p), _p(scale, _f32p)),
+           "oracle_quantize_fp8_rows")
+    return q, scale
+
+
+def combine_rows_fp8(x, idx, w, rows, q_gu, s_gu, q_dn, s_dn, residual=None, threads=1):
+    """y [len(rows), D] (float64) with FP8 routed experts (weight = scale[row] * value(q))."""
+    x, res = as_u16(x), as_u16(residual)
+    q_gu = np.ascontiguousarray(np.asarray(q_gu.cpu() if hasattr(q_gu, "cpu") else q_gu), dtype=np.uint8)
+    q_dn = np.ascontiguousarray(np.asarray(q_dn.cpu() if hasattr(q_dn, "cpu") else q_dn), dtype=np.uint8)
+    s_gu, s_dn = _f32(s_gu), _f32(s_dn)
+    idx, w = _i32(idx), _f32(w)
+    T, D = x.shape
+    k = idx.shape[1]
+    E = q_gu.shape[0]
+    I = q_gu.shape[1] // 2
+    parts = _chunks(rows, threads)
+    outs = [np.empty((len(p), D), np.float64) for p in parts]
+
+    def run(i):
+        p = parts[i]
+        _check(lib().oracle_combine_rows_fp8(_p(x, _u16p), _p(idx, _i32p), _p(w, _f32p), _p(p, _i32p),
+                                             len(p), T, D, E, k, I, _p(q_gu, _u8p), _p(s_gu, _f32p),
+                                             _p(q_dn, _u8p), _p(s_dn, _f32p), _p(res, _u16p),
+                                             _p(outs[i], _f64p)), "oracle_combine_rows_fp8")
+
+    with ThreadPoolExecutor(max_workers=len(parts)) as ex:
+        list(ex.map(run, range(len(parts))))
+    return np.concatenate(outs, axis=0) if outs else np.empty((0, D))
 
 
 def cpu_threads_available() -> int:

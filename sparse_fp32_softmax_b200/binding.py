@@ -37,7 +37,8 @@ class moe_opts(ctypes.Structure):
                 ("topk_idx_out", _vp), ("topk_w_out", _vp), ("path", _c_int),
                 ("stage_events", _vp), ("n_stage_events", _c_int), ("out_f32", _vp),
                 ("expert_counts_out", _vp), ("slot_row_out", _vp), ("wait_limit_us", ctypes.c_uint),
-                ("diag", _c_int)]
+                ("diag", _c_int), ("W_gate_up_fp8", _vp), ("gate_up_scale", _vp),
+                ("W_down_fp8", _vp), ("down_scale", _vp)]
 
 
 class MoeError(RuntimeError):
@@ -72,8 +73,9 @@ def load():
         lib.moe_status_string.restype = ctypes.c_char_p
         lib.moe_last_cuda_error.argtypes = []
         lib.moe_last_cuda_error.restype = _c_int
+        lib.moe_quantize_fp8_rows.argtypes = [_vp, ctypes.c_int64, _c_int, _vp, _vp, _vp]
         for n in ("moe_route", "moe_permute", "moe_forward", "moe_forward_ex", "moe_forward_noalloc",
-                  "moe_get_device_status", "moe_get_device_status_noalloc"):
+                  "moe_get_device_status", "moe_get_device_status_noalloc", "moe_quantize_fp8_rows"):
             getattr(lib, n).restype = _c_int
         _lib = lib
     return _lib
@@ -132,7 +134,8 @@ def make_dims(T, D, E, k, I, norm_topk_prob=True, tile_m=1) -> moe_dims:
 def make_opts(router_bias=None, shared_gate_up=None, shared_down=None, shared_gate=None,
               residual=None, logits_out=None, topk_idx_out=None, topk_w_out=None, path="auto",
               stage_events=None, out_f32=None, expert_counts_out=None, slot_row_out=None,
-              wait_limit_us=0, diag=0):
+              wait_limit_us=0, diag=0, W_gate_up_fp8=None, gate_up_scale=None, W_down_fp8=None,
+              down_scale=None):
     o = moe_opts()
     o.router_bias = _ptr(router_bias)
     o.shared_gate_up = _ptr(shared_gate_up)
@@ -149,6 +152,11 @@ def make_opts(router_bias=None, shared_gate_up=None, shared_down=None, shared_ga
     o.slot_row_out = _ptr(slot_row_out)
     o.wait_limit_us = int(wait_limit_us)
     o.diag = int(diag)
+    o.W_gate_up_fp8 = _ptr(W_gate_up_fp8)
+    o.gate_up_scale = _ptr(gate_up_scale)
+    o.W_down_fp8 = _ptr(W_down_fp8)
+    o.down_scale = _ptr(down_scale)
+    o._fp8 = (W_gate_up_fp8, W_down_fp8)   # shapes for the dims, and kept alive with the options
     o._events_keepalive = None
     if stage_events is not None:
         handles = (ctypes.c_void_p * len(stage_events))(*[ev.cuda_event for ev in stage_events])
@@ -210,11 +218,16 @@ def moe_permute(topk_idx, E, tile_m=1, topk_w=None, x=None, want_x_perm=False, w
     return out
 
 
-def _dims_of(x, W_r, W_gate_up, W_down, k, norm_topk_prob):
+def _dims_of(x, W_r, W_gate_up, W_down, k, norm_topk_prob, W_gate_up_fp8=None, W_down_fp8=None):
     _need(x, "x", torch.bfloat16, 2)
     _need(W_r, "W_r", torch.bfloat16, 2)
-    _need(W_gate_up, "W_gate_up", torch.bfloat16, 3)
-    _need(W_down, "W_down", torch.bfloat16, 3)
+    if W_gate_up is None and W_gate_up_fp8 is not None:   # FP8 experts: shapes from the bytes
+        _need(W_gate_up_fp8, "W_gate_up_fp8", torch.uint8, 3)
+        _need(W_down_fp8, "W_down_fp8", torch.uint8, 3)
+        W_gate_up = W_gate_up_fp8
+    else:
+        _need(W_gate_up, "W_gate_up", torch.bfloat16, 3)
+        _need(W_down, "W_down", torch.bfloat16, 3)
     T, D = x.shape
     E, I2, _ = W_gate_up.shape
     return make_dims(T, D, E, k, I2 // 2, norm_topk_prob)
@@ -236,10 +249,12 @@ def moe_forward_ex(x, W_r, W_gate_up, W_down, k, norm_topk_prob=True, out=None, 
     """moe_forward with options; pass a prepared ``opts`` or the keyword arguments of
     ``make_opts`` (router_bias, shared_gate_up, shared_down, shared_gate, residual,
     logits_out, topk_idx_out, topk_w_out, path, stage_events, out_f32, expert_counts_out,
-    slot_row_out, wait_limit_us, diag)."""
-    dims = _dims_of(x, W_r, W_gate_up, W_down, k, norm_topk_prob)
+    slot_row_out, wait_limit_us, diag, W_gate_up_fp8, gate_up_scale, W_down_fp8, down_scale).
+    With FP8 experts (W_gate_up_fp8 ...), W_gate_up and W_down may be None."""
     if opts is None:
         opts = make_opts(**opt_kwargs)
+    fp8 = getattr(opts, "_fp8", (None, None))
+    dims = _dims_of(x, W_r, W_gate_up, W_down, k, norm_topk_prob, fp8[0], fp8[1])
     if out is None:
         out = torch.empty_like(x)
     if ws is None:
@@ -248,6 +263,23 @@ def moe_forward_ex(x, W_r, W_gate_up, W_down, k, norm_topk_prob=True, out=None, 
                                  ctypes.byref(opts), _ptr(out), _ptr(ws), ws.numel(), _stream(stream)),
            "moe_forward_ex")
     return out
+
+
+def moe_quantize_fp8_rows(W, q=None, scale=None, stream=None):
+    """Per-row FP8 E4M3 quantisation of the bf16 matrix W viewed as [rows, W.shape[-1]]:
+    -> (q uint8 of W's shape, scale FP32 [rows]).  The format is in the header."""
+    _need(W, "W", torch.bfloat16)
+    cols = int(W.shape[-1])
+    rows = W.numel() // cols if cols else 0
+    if q is None:
+        q = torch.empty(W.shape, dtype=torch.uint8, device=W.device)
+    if scale is None:
+        scale = torch.empty(rows, dtype=torch.float32, device=W.device)
+    _need(q, "q", torch.uint8)
+    _need(scale, "scale", torch.float32)
+    _check(load().moe_quantize_fp8_rows(_ptr(W), rows, cols, _ptr(q), _ptr(scale), _stream(stream)),
+           "moe_quantize_fp8_rows")
+    return q, scale
 
 
 def moe_forward_noalloc(x, W_r, W_gate_up, W_down, k, norm_topk_prob=True, out=None, stream=None):

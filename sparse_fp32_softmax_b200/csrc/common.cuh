@@ -9,6 +9,8 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -96,6 +98,27 @@ __device__ __forceinline__ void set_error(int* err, int bit) {
 __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
 
+// FP8 E4M3 -> bf16, exactly: every E4M3 value (at most 4 significant bits, |v| <= 448,
+// >= 2^-9) is an fp16 value and a bf16 value.  Two values (bytes 0 and 1 of `two`, value 0
+// into the low half) through the conversion instructions E4M3 -> fp16 -> FP32 -> bf16.
+// (Measured on B200: an integer-operation widening -- exponent + 120, with a branch for the
+// zero-exponent codes -- ran slower inside the GEMM's converter warps.)
+__device__ __forceinline__ uint32_t widen_e4m3x2(uint32_t two) {
+    const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)two, __NV_E4M3);
+    const float lo = __half2float(__half(__half_raw{h.x}));
+    const float hi = __half2float(__half(__half_raw{h.y}));
+    __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&b);
+}
+// Sixteen values (byte i of v is value i): values 0-7 into lo and 8-15 into hi (value 2m in
+// the low half of word m).
+__device__ __forceinline__ void widen_e4m3x16(const uint4& v, uint4& lo, uint4& hi) {
+    lo.x = widen_e4m3x2(v.x & 0xFFFFu); lo.y = widen_e4m3x2(v.x >> 16);
+    lo.z = widen_e4m3x2(v.y & 0xFFFFu); lo.w = widen_e4m3x2(v.y >> 16);
+    hi.x = widen_e4m3x2(v.z & 0xFFFFu); hi.y = widen_e4m3x2(v.z >> 16);
+    hi.z = widen_e4m3x2(v.w & 0xFFFFu); hi.w = widen_e4m3x2(v.w >> 16);
+}
+
 // Round-to-nearest-even pack of two floats into a bf16x2 word (lo in the low half).
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
@@ -132,6 +155,12 @@ __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
 // Make barrier initialisation visible to the async proxy (TMA, tensor core) and cluster.
 __device__ __forceinline__ void mbar_fence_init() {
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Order this thread's ordinary shared-memory stores before later reads of the async proxy
+// (the tensor core reading operands the thread wrote).
+__device__ __forceinline__ void fence_proxy_async_shared() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 

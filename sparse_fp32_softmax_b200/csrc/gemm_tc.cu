@@ -45,8 +45,14 @@ namespace moe {
 
 enum { kModeGateUp = 0, kModeDown = 1, kModeRouter = 2 };
 
-// One kernel configuration: mode, token columns per tile and pipeline depth.
-template <int MODE, int BN_, int STAGES_, bool PAIR_ = false>
+constexpr int kEpiWarps = 8;
+constexpr int kConvWarps = 4;      // F8: warps that widen FP8 weight tiles to bf16
+constexpr int kQD = 4;             // entries of the claimed-unit ring (narrow tiles)
+constexpr int kBarRegion = 512;    // bytes of mbarriers and small shared state
+
+// One kernel configuration: mode, token columns per tile, pipeline depth, CTA pairs, and
+// whether the weights arrive as FP8 E4M3 with a scale per weight row (F8).
+template <int MODE, int BN_, int STAGES_, bool PAIR_ = false, bool F8_ = false>
 struct TcCfg {
     static constexpr int BN = BN_, STAGES = STAGES_;
     // PAIR: two CTAs of a cluster share M = 256 MMAs; each holds 128 weight rows and half of
@@ -63,17 +69,28 @@ struct TcCfg {
                               : 2 * ACC <= 256 ? 256 : 512;
     static_assert(2 * ACC <= 512, "accumulators exceed TMEM");
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "token tile");
-    static constexpr int SB = NA * (kTcM * kTcK * 2) + BNC * kTcK * 2;  // bytes per stage
-    static constexpr int SMEM = STAGES * SB + 1024 + 256 + (int)sizeof(SmemTables) +
+    // F8: the weight tiles of a stage arrive as FP8 bytes (64 per row per K step, no swizzle)
+    // in the load ring; converter warps widen them (exactly) to bf16 into a ring of CONV
+    // 128-byte-swizzled stages, copy the stage's bf16 token tile next to them and release the
+    // load stage at once, so the loads in flight do not wait for the MMAs; the MMAs read the
+    // bf16 ring.
+    static constexpr bool F8 = F8_;
+    static_assert(!F8 || (!PAIR && !IL && MODE != kModeRouter), "FP8 weights: narrow tiles only");
+    static constexpr int CONV = F8 ? (NA == 2 ? 2 : 3) : 0;
+    static constexpr int A_BYTES = NA * kTcM * kTcK * (F8 ? 1 : 2);   // weight bytes per load stage
+    static constexpr int SB = A_BYTES + BNC * kTcK * 2;              // bytes per load stage
+    static constexpr int CSB = NA * kTcM * kTcK * 2 + BNC * kTcK * 2;   // bf16 stage (F8)
+    static constexpr int CONVB = CONV * CSB;                           // bf16 ring (F8)
+    static constexpr int THREADS = (2 + kEpiWarps + (F8 ? kConvWarps : 0)) * 32;
+    static constexpr int SMEM = STAGES * SB + CONVB + 1024 + kBarRegion + (int)sizeof(SmemTables) +
                                 (MODE == kModeDown ? 8 * 2 * 4 * BN : 0);
-    static_assert(2 * STAGES + 5 <= 31, "barriers exceed their 256-byte region");
+    static_assert(SB % 1024 == 0, "stages keep the 1024-byte alignment of swizzled tiles");
+    static_assert((2 * STAGES + 6) * 8 + kQD * 20 + 2 * CONV * 8 <= kBarRegion, "barrier region");
     static_assert(SMEM <= 232448, "shared memory per block");
 };
 
 constexpr int kATileBytes = kTcM * kTcK * 2;  // 16 KB
-constexpr int kEpiWarps = 8;
-constexpr int kQD = 4;          // entries of the claimed-unit ring (narrow tiles)
-constexpr int kTcThreads = (2 + kEpiWarps) * 32;
+constexpr int kA8TileBytes = kTcM * kTcK;     // 8 KB (FP8)
 
 struct TileInfo {
     int bi;       // token-operand box: 16 << bi rows
@@ -269,10 +286,10 @@ __device__ __forceinline__ void tma_load(void* dst, const CUtensorMap* map, uint
         : "memory");
 }
 
-template <int MODE, int BN, int STAGES, bool PAIR = false>
-__global__ void __launch_bounds__(kTcThreads, 1)
+template <int MODE, int BN, int STAGES, bool PAIR = false, bool F8 = false>
+__global__ void __launch_bounds__((TcCfg<MODE, BN, STAGES, PAIR, F8>::THREADS), 1)
     tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
-    using Tr = TcCfg<MODE, BN, STAGES, PAIR>;
+    using Tr = TcCfg<MODE, BN, STAGES, PAIR, F8>;
     constexpr int NA = Tr::NA, ACC = Tr::ACC;
     constexpr bool SPLIT = MODE != kModeRouter && BN <= kNarrowBN;
     // DYN (narrow tiles): CTA b starts with unit b; each further unit is claimed from a
@@ -282,10 +299,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // Otherwise CTA (pair) b takes units b, b + grid, ...
     constexpr bool DYN = SPLIT;
     constexpr int SB = Tr::SB;
+    constexpr int CONVD = Tr::CONV > 0 ? Tr::CONV : 1;   // the bf16 ring's size as a divisor
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * SB);
+    uint8_t* convs = smem + STAGES * SB;   // F8: CONV bf16 stages (NA weight tiles, token tile)
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * SB + Tr::CONVB);
     uint64_t* empty = full + STAGES;
     uint64_t* tfull = empty + STAGES;  // [2]
     uint64_t* tempty = tfull + 2;       // [2]
@@ -295,8 +314,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     uint64_t* qfull = drain + 2;                            // [kQD]
     uint64_t* qempty = qfull + kQD;                         // [kQD]
     int* qitem = reinterpret_cast<int*>(qempty + kQD);      // [kQD]
-    static_assert((2 * STAGES + 6) * 8 + kQD * 20 <= 256, "barrier region");
-    SmemTables* tabs = reinterpret_cast<SmemTables*>(smem + STAGES * SB + 256);
+    uint64_t* conv = reinterpret_cast<uint64_t*>(qitem + kQD);   // [CONV] (F8)
+    uint64_t* cempty = conv + Tr::CONV;                          // [CONV] (F8)
+    SmemTables* tabs = reinterpret_cast<SmemTables*>(smem + STAGES * SB + Tr::CONVB + kBarRegion);
     // down: per epilogue warp, the current tile's row destinations and weights
     int* ep_dest_all = reinterpret_cast<int*>(tabs + 1);                       // [8][BN]
     float* ep_wt_all = reinterpret_cast<float*>(ep_dest_all + kEpiWarps * BN);  // [8][BN]
@@ -311,7 +331,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(full + s, 1);
-            mbar_init(empty + s, 1);
+            mbar_init(empty + s, F8 ? kConvWarps : 1);   // F8: released by the converter warps
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(tfull + b, 1);
@@ -320,12 +340,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         mbar_init(drain, 1);
         for (int q = 0; q < kQD; ++q) {
             mbar_init(qfull + q, 1);
-            mbar_init(qempty + q, 1 + kEpiWarps);   // the MMA thread and each epilogue warp
+            // the MMA thread, each epilogue warp and (F8) each converter warp
+            mbar_init(qempty + q, 1 + kEpiWarps + (F8 ? kConvWarps : 0));
+        }
+        for (int c = 0; c < Tr::CONV; ++c) {
+            mbar_init(conv + c, kConvWarps);   // a converted tile: one arrival per converter warp
+            mbar_init(cempty + c, 1);          // its MMAs are complete (commit)
         }
         mbar_fence_init();
     }
     if (warp == 0 && lane < 2 + kNumBBoxes) {
-        const CUtensorMap* m = lane == 0 ? &maps.A : (lane == 1 ? &maps.A_shared : &maps.B[lane - 2]);
+        const CUtensorMap* m = lane == 0 ? (F8 ? &maps.A8 : &maps.A)
+                                         : (lane == 1 ? &maps.A_shared : &maps.B[lane - 2]);
         tma_prefetch_desc(m);
     }
     if (warp == 1) {
@@ -344,7 +370,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         __syncthreads();
         if (warp == 0 && lane == 0 && ublk < tabs->prefix[a.nseg]) {
             const TileInfo t0 = tc_decode_item<MODE, BN, PAIR>(a, tabs, ublk, rank);
-            const CUtensorMap* mA = t0.shared ? &maps.A_shared : &maps.A;
+            const CUtensorMap* mA = t0.shared ? &maps.A_shared : (F8 ? &maps.A8 : &maps.A);
             for (int kb = 0; kb < t0.nk; ++kb) tma_prefetch_l2(mA, kb * kTcK, t0.a_row0);
         }
     }
@@ -356,8 +382,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (e < a.E) {
             const int r0 = e * 2 * a.I + ((int)blockIdx.x % mt) * kTcM;
             for (int kb = 0; kb < a.spec_steps; ++kb) {
-                tma_prefetch_l2(&maps.A, kb * kTcK, r0);
-                tma_prefetch_l2(&maps.A, kb * kTcK, r0 + a.I);
+                tma_prefetch_l2(F8 ? &maps.A8 : &maps.A, kb * kTcK, r0);
+                tma_prefetch_l2(F8 ? &maps.A8 : &maps.A, kb * kTcK, r0 + a.I);
             }
         }
     }
@@ -443,11 +469,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     break;
                 }
             }
-            const CUtensorMap* mA = ti.shared ? &maps.A_shared : &maps.A;
+            const CUtensorMap* mA = ti.shared ? &maps.A_shared : (F8 ? &maps.A8 : &maps.A);
             const CUtensorMap* mB = &maps.B[ti.bi];
             const int brows = 16 << ti.bi;
             // PAIR: the leader's barrier counts both CTAs' bytes (same geometry in each)
-            const uint32_t bytes = (PAIR ? 2u : 1u) * (NA * kATileBytes + (uint32_t)brows * kTcK * 2);
+            const uint32_t bytes = (PAIR ? 2u : 1u) * (Tr::A_BYTES + (uint32_t)brows * kTcK * 2);
             for (int kb = 0; kb < ti.nk; ++kb, ++it) {
                 const int s = it % STAGES;
                 const int round = it / STAGES;
@@ -466,7 +492,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         tma_load_5d_pair(st, mA, fb, kx, 0, 0, ti.a_row0, ti.a_row1);
                     else
                         tma_load_2d_pair(st, mA, fb, kx, ti.a_row0);
-                    tma_load_2d_pair(st + NA * kATileBytes, mB, fb, kx, ti.b_row + rank * brows);
+                    tma_load_2d_pair(st + Tr::A_BYTES, mB, fb, kx, ti.b_row + rank * brows);
                 } else if (!PAIR && lane == 0) {
                     mbar_arrive_expect_tx(full + s, bytes);
                     const int kx = (ti.k0 + kb) * kTcK;
@@ -474,13 +500,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         tma_load_5d(st, mA, full + s, kx, 0, 0, ti.a_row0, ti.a_row1);
                     else
                         tma_load(st, mA, full + s, kx, ti.a_row0);
-                    if (NA == 2) tma_load(st + kATileBytes, mA, full + s, kx, ti.a_row1);
-                    if (!gather) tma_load(st + NA * kATileBytes, mB, full + s, kx, ti.b_row);
+                    if (NA == 2) tma_load(st + Tr::A_BYTES / 2, mA, full + s, kx, ti.a_row1);
+                    if (!gather) tma_load(st + Tr::A_BYTES, mB, full + s, kx, ti.b_row);
                 }
                 if (gather) {
                     __syncwarp();  // expect_tx is posted before any gather can complete
                     if (4 * lane < brows)
-                        tma_gather4(st + NA * kATileBytes + lane * 4 * kTcK * 2, mB, full + s,
+                        tma_gather4(st + Tr::A_BYTES + lane * 4 * kTcK * 2, mB, full + s,
                                     (ti.k0 + kb) * kTcK, g0, g1, g2, g3);
                 }
 #pragma unroll
@@ -515,10 +541,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const uint32_t idesc0 = umma_idesc_bf16_f32(PAIR ? 2 * kTcM : kTcM, 16) & ~(0x3Fu << 17);
             // shared-memory descriptors of stage 0; stage s adds s * SB / 16 to the address
             // field (stages stay below 256 KB, so the 14-bit field does not carry)
-            const uint64_t dA0 = umma_desc_sw128(smem);
-            const uint64_t dA1 = umma_desc_sw128(smem + kATileBytes);
-            const uint64_t dB = umma_desc_sw128(smem + NA * kATileBytes);
+            // (F8: both operands are read from the bf16 ring, slot c adds c * CSB / 16)
+            const uint64_t dA0 = umma_desc_sw128(F8 ? convs : smem);
+            const uint64_t dA1 = umma_desc_sw128((F8 ? convs : smem) + kATileBytes);
+            const uint64_t dB = umma_desc_sw128(F8 ? convs + NA * kATileBytes : smem + Tr::A_BYTES);
             int s = 0, phase = 0;   // ring position of the next stage
+            int pos = 0;            // F8: stages consumed so far (the bf16 ring follows them)
             int tc = 0;
             bool ok = true;
             for (int item = ublk, qi = 0; ok; item += DYN ? 0 : ugrid, ++tc, ++qi) {
@@ -545,12 +573,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 const uint32_t idesc = idesc0 | ((uint32_t)(n >> 3) << 17);
                 const uint32_t d0 = tmem_base + (uint32_t)(b * ACC);
                 for (int kb = 0; kb < ti.nk; ++kb) {
-                    if (!mbar_wait(full + s, phase, a.err, kErrWaitMma, a.wait_ns)) {
+                    // (F8: the converted stage holds both operands; the load stage may already
+                    // hold a later stage, so its barrier is not looked at)
+                    const int cs = F8 ? pos % CONVD : 0;
+                    if (!(F8 ? mbar_wait(conv + cs, (pos / CONVD) & 1, a.err, kErrWaitMma, a.wait_ns)
+                             : mbar_wait(full + s, phase, a.err, kErrWaitMma, a.wait_ns))) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint64_t off = (uint64_t)(s * (SB >> 4));
+                    const uint64_t off = F8 ? (uint64_t)(cs * (Tr::CSB >> 4)) : (uint64_t)(s * (SB >> 4));
                     const uint64_t da0 = dA0 + off, da1 = dA1 + off, db = dB + off;
                     if (PAIR) {
                         umma_bf16_pair(d0, da0, db, idesc, kb);
@@ -566,8 +598,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                             umma_bf16_acc(d0, da0 + 2 * kk, db + 2 * kk, idesc);
                             if (NA == 2) umma_bf16_acc(d0 + BN, da1 + 2 * kk, db + 2 * kk, idesc);
                         }
-                        umma_commit(empty + s);
+                        if (F8)
+                            umma_commit(cempty + cs);   // the bf16 stage is free again
+                        else
+                            umma_commit(empty + s);
                     }
+                    if (F8) ++pos;
                     if (++s == STAGES) {
                         s = 0;
                         phase ^= 1;
@@ -585,6 +621,67 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             else
                 umma_commit(drain);
             mbar_wait(drain, 0, a.err, kErrWaitMma, a.wait_ns);
+        }
+    } else if (F8 && warp >= 2 + kEpiWarps) {
+        // ------------------------------------------------------------ converter warps (F8)
+        // Each stage's FP8 weight tiles (NA x 128 rows x 64 bytes, row-major) become bf16
+        // tiles in the 128-byte-swizzled K-major layout the MMAs read (the layout a TMA load
+        // with 128-byte swizzle writes: 16-byte chunk c of row r at r * 128 + ((c ^ (r % 8))
+        // * 16)).  Converter thread t takes the 16-byte pieces t, t + 32 * kConvWarps, ... of the stage
+        // (piece = row * 4 + j within a tile), widens its 16 values and stores them as the
+        // row's chunks 2j and 2j + 1.  Units come from the ring like the epilogue's.
+        static_assert(512 % (kConvWarps * 32) == 0, "converter threads divide a tile's pieces");
+        const int ct = (warp - 2 - kEpiWarps) * 32 + lane;   // 0 .. kConvWarps * 32 - 1
+        int pos = 0;
+        bool ok = true;
+        for (int qi = 0; ok; ++qi) {
+            const int qs = qi % kQD;
+            const bool gq = mbar_wait(qfull + qs, (qi / kQD) & 1, a.err, kErrWaitEpilogue, a.wait_ns);
+            if (!__all_sync(0xffffffffu, gq)) break;
+            const int item = qitem[qs];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(qempty + qs);
+            if (item < 0) break;
+            const TileInfo ti = tc_decode_unit<MODE, BN, PAIR>(a, tabs, sc, item, rank);
+            for (int kb = 0; kb < ti.nk; ++kb, ++pos) {
+                const int s = pos % STAGES, cs = pos % CONVD;
+                bool got = mbar_wait(full + s, (pos / STAGES) & 1, a.err, kErrWaitEpilogue, a.wait_ns);
+                if (got)
+                    got = mbar_wait(cempty + cs, ((pos / CONVD) & 1) ^ 1, a.err, kErrWaitEpilogue, a.wait_ns);
+                if (!__all_sync(0xffffffffu, got)) {
+                    ok = false;
+                    break;
+                }
+                const uint8_t* src = smem + s * SB;
+                uint8_t* dst = convs + cs * Tr::CSB;
+#pragma unroll
+                for (int q = 0; q < NA * 512 / (kConvWarps * 32); ++q) {
+                    const int piece = q * (kConvWarps * 32) + ct;
+                    const int at = piece >> 9, pr = piece & 511;
+                    const int row = pr >> 2, j = pr & 3;
+                    const uint4 v = *reinterpret_cast<const uint4*>(src + at * kA8TileBytes + row * 64 + j * 16);
+                    uint4 lo, hi;
+                    widen_e4m3x16(v, lo, hi);
+                    uint8_t* drow = dst + at * kATileBytes + row * 128;
+                    *reinterpret_cast<uint4*>(drow + (((2 * j) ^ (row & 7)) << 4)) = lo;
+                    *reinterpret_cast<uint4*>(drow + (((2 * j + 1) ^ (row & 7)) << 4)) = hi;
+                }
+                // the token tile (bf16, already in its swizzled layout, which depends only on
+                // the 1024-byte-aligned position) is copied next to the widened weights
+                {
+                    const uint4* bsrc = reinterpret_cast<const uint4*>(src + Tr::A_BYTES);
+                    uint4* bdst = reinterpret_cast<uint4*>(dst + NA * kATileBytes);
+                    constexpr int kBChunks = BN * kTcK * 2 / 16;
+#pragma unroll
+                    for (int i = ct; i < kBChunks; i += kConvWarps * 32) bdst[i] = bsrc[i];
+                }
+                fence_proxy_async_shared();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(empty + s);   // the load stage has been read
+                    mbar_arrive(conv + cs);
+                }
+            }
         }
     } else {
         // ------------------------------------------------------------ epilogue warps 2..9
@@ -626,9 +723,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             } else if (MODE == kModeGateUp) {
                 const int f = ti.m0 + row;
                 uint16_t* hp = a.h + (size_t)(ti.b_row + c * 32) * a.ld_h + f;
+                // F8: the accumulators hold sums of q * x; the row scales make them g and u
+                const float sg = F8 ? __ldg(a.a_scale + ti.a_row0 + row) : 1.0f;
+                const float su = F8 ? __ldg(a.a_scale + ti.a_row1 + row) : 1.0f;
 #pragma unroll
                 for (int j = 0; j < 32; ++j)
-                    if (c * 32 + j < ti.n_valid) hp[(size_t)j * a.ld_h] = to_bf16_bits(silu(v[j]) * u[j]);
+                    if (c * 32 + j < ti.n_valid)
+                        hp[(size_t)j * a.ld_h] = F8 ? to_bf16_bits(silu(v[j] * sg) * (u[j] * su))
+                                                    : to_bf16_bits(silu(v[j]) * u[j]);
             } else if (MODE == kModeDown) {
                 const int d = ti.m0 + row;
                 if (kAhead) {
@@ -649,10 +751,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         if (c * 32 + j < ti.n_valid) a.slots[(size_t)dj * a.D + d] = wj * v[j];
                     }
                 } else {
+                    const float sd = F8 ? __ldg(a.a_scale + ti.a_row0 + row) : 1.0f;   // F8 row scale
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
                         const int col = c * 32 + j;
-                        if (col < ti.n_valid) a.slots[(size_t)ep_dest[col] * a.D + d] = ep_wt[col] * v[j];
+                        if (col < ti.n_valid)
+                            a.slots[(size_t)ep_dest[col] * a.D + d] = ep_wt[col] * (F8 ? v[j] * sd : v[j]);
                     }
                 }
             } else {
@@ -674,15 +778,20 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const int col0 = c * 32 + 4 * g;
             if (MODE == kModeGateUp) {
                 uint16_t* hp = a.h + (size_t)(ti.b_row + col0) * a.ld_h + ti.m0 + row;
-#pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    if (col0 + j < ti.n_valid) hp[(size_t)j * a.ld_h] = to_bf16_bits(silu(v[j]) * u[j]);
-            } else if (MODE == kModeDown) {
-                const int d = ti.m0 + row;
+                const float sg = F8 ? __ldg(a.a_scale + ti.a_row0 + row) : 1.0f;
+                const float su = F8 ? __ldg(a.a_scale + ti.a_row1 + row) : 1.0f;
 #pragma unroll
                 for (int j = 0; j < 4; ++j)
                     if (col0 + j < ti.n_valid)
-                        a.slots[(size_t)ep_dest[col0 + j] * a.D + d] = ep_wt[col0 + j] * v[j];
+                        hp[(size_t)j * a.ld_h] = F8 ? to_bf16_bits(silu(v[j] * sg) * (u[j] * su))
+                                                    : to_bf16_bits(silu(v[j]) * u[j]);
+            } else if (MODE == kModeDown) {
+                const int d = ti.m0 + row;
+                const float sd = F8 ? __ldg(a.a_scale + ti.a_row0 + row) : 1.0f;
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    if (col0 + j < ti.n_valid)
+                        a.slots[(size_t)ep_dest[col0 + j] * a.D + d] = ep_wt[col0 + j] * (F8 ? v[j] * sd : v[j]);
             }
         };
         auto fetch_dest = [&](const TileInfo& t) {
@@ -851,11 +960,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
 }
 
-template <int MODE, int BN, int STAGES, bool PAIR = false>
+template <int MODE, int BN, int STAGES, bool PAIR = false, bool F8 = false>
 static cudaError_t launch_tc(const TcMaps& maps, const TcArgs& a, int grid, bool pdl,
                              cudaStream_t s) {
-    constexpr int smem = TcCfg<MODE, BN, STAGES, PAIR>::SMEM;
-    auto kernel = tc_gemm_kernel<MODE, BN, STAGES, PAIR>;
+    constexpr int smem = TcCfg<MODE, BN, STAGES, PAIR, F8>::SMEM;
+    constexpr int kTcThreads = TcCfg<MODE, BN, STAGES, PAIR, F8>::THREADS;
+    auto kernel = tc_gemm_kernel<MODE, BN, STAGES, PAIR, F8>;
     cudaError_t err = ensure_smem_attr((const void*)kernel, smem);
     if (err != cudaSuccess) return err;
     if (grid < 1) grid = 1;
@@ -907,7 +1017,7 @@ bool pair_tiles_available() {
             if (ensure_smem_attr(kernel, smem) != cudaSuccess) return false;
             cudaLaunchConfig_t cfg = {};
             cfg.gridDim = dim3(2);
-            cfg.blockDim = dim3(kTcThreads);
+            cfg.blockDim = dim3(TcCfg<kModeGateUp, kGuBN, kPairStages, true>::THREADS);
             cfg.dynamicSmemBytes = smem;
             cudaLaunchAttribute attr[1];
             attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -936,8 +1046,11 @@ cudaError_t launch_tc_router(const TcMaps& maps, const TcArgs& a, int num_sms, b
     return launch_tc<kModeRouter, kRtBN, kStages>(maps, a, items < num_sms ? items : num_sms, pdl, s);
 }
 
-cudaError_t launch_tc_gate_up(const TcMaps& maps, const TcArgs& a, int num_sms, int tiles, bool pdl,
-                              cudaStream_t s) {
+cudaError_t launch_tc_gate_up(const TcMaps& maps, const TcArgs& a, int num_sms, int tiles, bool f8,
+                              bool pdl, cudaStream_t s) {
+    if (tiles == kTilesNarrow && f8)
+        return launch_tc<kModeGateUp, kNarrowBN, kGuNarrowStagesF8, false, true>(maps, a, num_sms, pdl, s);
+    if (f8) return cudaErrorInvalidValue;
     if (tiles == kTilesNarrow)
         return launch_tc<kModeGateUp, kNarrowBN, kGuNarrowStages>(maps, a, num_sms, pdl, s);
     if (tiles == kTilesPair)
@@ -945,8 +1058,11 @@ cudaError_t launch_tc_gate_up(const TcMaps& maps, const TcArgs& a, int num_sms, 
     return launch_tc<kModeGateUp, kGuBN, kStages>(maps, a, num_sms, pdl, s);
 }
 
-cudaError_t launch_tc_down(const TcMaps& maps, const TcArgs& a, int num_sms, int tiles, bool pdl,
-                           cudaStream_t s) {
+cudaError_t launch_tc_down(const TcMaps& maps, const TcArgs& a, int num_sms, int tiles, bool f8,
+                           bool pdl, cudaStream_t s) {
+    if (tiles == kTilesNarrow && f8)
+        return launch_tc<kModeDown, kNarrowBN, kDnNarrowStagesF8, false, true>(maps, a, num_sms, pdl, s);
+    if (f8) return cudaErrorInvalidValue;
     if (tiles == kTilesNarrow)
         return launch_tc<kModeDown, kNarrowBN, kDnNarrowStages>(maps, a, num_sms, pdl, s);
     if (tiles == kTilesPair)

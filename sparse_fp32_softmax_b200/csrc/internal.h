@@ -38,6 +38,10 @@ constexpr int kStages = 4;      // shared-memory pipeline depth of the wide tile
 constexpr int kNarrowBN = 64;
 constexpr int kGuNarrowStages = 5;   // 5 x (2 x 16 KB + 8 KB)
 constexpr int kDnNarrowStages = 8;   // 8 x (16 KB + 8 KB)
+// FP8 weights (narrow tiles): load stages of 8 KB per weight tile + 8 KB of tokens, plus a
+// ring of three widened bf16 tiles
+constexpr int kGuNarrowStagesF8 = 5;   // 5 x (2 x 8 KB + 8 KB) + 3 x 32 KB
+constexpr int kDnNarrowStagesF8 = 8;   // 8 x (8 KB + 8 KB) + 3 x 16 KB
 // The forward takes the narrow tiles when the mean rows per expert, T*k/E, is at most this.
 constexpr int kNarrowMaxMeanRows = 32;
 // Largest T for which gate_up gathers its token rows straight from x (tile::gather4, four
@@ -145,6 +149,7 @@ struct alignas(64) TcMaps {
     CUtensorMap A;
     CUtensorMap A_shared;
     CUtensorMap B[kNumBBoxes];
+    CUtensorMap A8;   // FP8 weights: [rows, K] bytes, 64 x 128 boxes, no swizzle (F8 kernels)
 };
 
 struct TcArgs {
@@ -177,6 +182,8 @@ struct TcArgs {
     int dep_wait;
     // narrow tiles: counter (zero at launch) from which the CTAs claim their units
     int* sched;
+    // FP8 weights (F8 kernels): FP32 scale of every weight row (A row), [E * rows per expert]
+    const float* a_scale;
     // narrow gate_up: before its dependency wait, CTA b requests into L2 the first spec_steps
     // K steps of the weight tiles of the unit it most likely starts with (feature tile
     // b % (I/128) of expert b / (I/128): the first unit when every expert received 1..64
@@ -214,10 +221,10 @@ cudaError_t launch_gather_rows(const uint16_t* x, const int32_t* row_token, int 
 bool pair_tiles_available();
 cudaError_t launch_tc_router(const TcMaps& maps, const TcArgs& a, int num_sms, bool pdl,
                              cudaStream_t s);
-cudaError_t launch_tc_gate_up(const TcMaps& maps, const TcArgs& a, int num_sms, int tiles, bool pdl,
-                              cudaStream_t s);
-cudaError_t launch_tc_down(const TcMaps& maps, const TcArgs& a, int num_sms, int tiles, bool pdl,
-                           cudaStream_t s);
+cudaError_t launch_tc_gate_up(const TcMaps& maps, const TcArgs& a, int num_sms, int tiles, bool f8,
+                              bool pdl, cudaStream_t s);
+cudaError_t launch_tc_down(const TcMaps& maps, const TcArgs& a, int num_sms, int tiles, bool f8,
+                           bool pdl, cudaStream_t s);
 cudaError_t launch_combine(const float* slots, int T, int D, int k, int has_shared,
                            const uint16_t* x, const uint16_t* shared_gate,
                            const uint16_t* residual, uint16_t* out, float* out_f32, bool pdl,

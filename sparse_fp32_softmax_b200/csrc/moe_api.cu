@@ -157,6 +157,14 @@ moe_status check_opts(const moe_dims* d, const moe_opts* o) {
     if (o->n_stage_events != 0 && o->n_stage_events != 6) return MOE_ERR_INVALID_ARG;
     if (o->n_stage_events == 6 && !o->stage_events) return MOE_ERR_INVALID_ARG;
     if (o->out_f32 && !aligned(o->out_f32, 16)) return MOE_ERR_INVALID_ARG;
+    if (o->W_gate_up_fp8 || o->W_down_fp8 || o->gate_up_scale || o->down_scale) {
+        if (!o->W_gate_up_fp8 || !o->W_down_fp8 || !o->gate_up_scale || !o->down_scale)
+            return MOE_ERR_INVALID_ARG;
+        if (!aligned(o->W_gate_up_fp8, 16) || !aligned(o->W_down_fp8, 16) ||
+            !aligned(o->gate_up_scale, 4) || !aligned(o->down_scale, 4))
+            return MOE_ERR_INVALID_ARG;
+        if (o->shared_gate_up || !use_narrow_tiles(d->T, d->k, d->E)) return MOE_ERR_UNSUPPORTED;
+    }
     return MOE_OK;
 }
 
@@ -199,6 +207,22 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, ui
     cuuint32_t estr[2] = {1, 1};
     CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) g_last_cuda_error = (int)cudaErrorInvalidValue;
+    return r == CUDA_SUCCESS;
+}
+
+// FP8 weights [rows, cols] bytes: boxes of 64 columns (one K step) x 128 rows, unswizzled
+// (the converter warps read them row by row).
+bool make_map8(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols};
+    cuuint32_t box[2] = {(cuuint32_t)kTcK, (cuuint32_t)kTcM};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) g_last_cuda_error = (int)cudaErrorInvalidValue;
     return r == CUDA_SUCCESS;
@@ -401,7 +425,9 @@ moe_status moe_forward_ex(const moe_bf16* x, const moe_bf16* W_r, const moe_bf16
     if (st != MOE_OK) return st;
     st = check_opts(dims, opts);
     if (st != MOE_OK) return st;
-    if (!x || !W_r || !W_gate_up || !W_down || !out || !ws) return MOE_ERR_INVALID_ARG;
+    // FP8 weights replace the bf16 expert tensors (which may then be NULL)
+    const bool f8 = opts && opts->W_gate_up_fp8;
+    if (!x || !W_r || (!f8 && (!W_gate_up || !W_down)) || !out || !ws) return MOE_ERR_INVALID_ARG;
     if (!aligned(x, 16) || !aligned(W_r, 16) || !aligned(W_gate_up, 16) || !aligned(W_down, 16) ||
         !aligned(out, 16) || !aligned(ws, kAlign))
         return MOE_ERR_INVALID_ARG;
@@ -449,17 +475,27 @@ moe_status moe_forward_ex(const moe_bf16* x, const moe_bf16* W_r, const moe_bf16
         uint16_t* h = at<uint16_t>(ws, p.h);
         const bool gu_b_ok = gather ? make_map(&mGu.B[0], x, p.D, p.T, 1)
                                     : make_b_maps(mGu.B, at<uint16_t>(ws, p.x_perm), p.D, p.R, b_box_max);
-        const bool gu_a_ok =
-            narrow ? make_map(&mGu.A, W_gate_up, p.D, (uint64_t)p.E * 2 * p.I, kTcM) &&
-                         make_map(&mGu.A_shared, sgu ? sgu : W_gate_up, p.D,
-                                  sgu ? 2 * (uint64_t)p.I_s : 2 * (uint64_t)p.I, kTcM)
-                   : make_map_gate_up_il(&mGu.A, W_gate_up, p.D, p.I, p.E) &&
-                         make_map_gate_up_il(&mGu.A_shared, sgu ? sgu : W_gate_up, p.D,
-                                             sgu ? p.I_s : p.I, 1);
-        if (!gu_a_ok ||
-            !gu_b_ok ||
-            !make_map(&mDn.A, W_down, p.I, (uint64_t)p.E * p.D, kTcM) ||
-            !make_map(&mDn.A_shared, sdn ? sdn : W_down, sdn ? p.I_s : p.I, p.D, kTcM) ||
+        // weight maps: bf16, or (FP8 weights) the byte maps, with the bf16 slots holding copies
+        // of those (the F8 kernels read only A8; every descriptor passed stays valid)
+        bool a_ok;
+        if (f8) {
+            a_ok = make_map8(&mGu.A8, opts->W_gate_up_fp8, p.D, (uint64_t)p.E * 2 * p.I) &&
+                   make_map8(&mDn.A8, opts->W_down_fp8, p.I, (uint64_t)p.E * p.D);
+            mGu.A = mGu.A_shared = mGu.A8;
+            mDn.A = mDn.A_shared = mDn.A8;
+        } else {
+            a_ok = (narrow ? make_map(&mGu.A, W_gate_up, p.D, (uint64_t)p.E * 2 * p.I, kTcM) &&
+                                 make_map(&mGu.A_shared, sgu ? sgu : W_gate_up, p.D,
+                                          sgu ? 2 * (uint64_t)p.I_s : 2 * (uint64_t)p.I, kTcM)
+                           : make_map_gate_up_il(&mGu.A, W_gate_up, p.D, p.I, p.E) &&
+                                 make_map_gate_up_il(&mGu.A_shared, sgu ? sgu : W_gate_up, p.D,
+                                                     sgu ? p.I_s : p.I, 1)) &&
+                   make_map(&mDn.A, W_down, p.I, (uint64_t)p.E * p.D, kTcM) &&
+                   make_map(&mDn.A_shared, sdn ? sdn : W_down, sdn ? p.I_s : p.I, p.D, kTcM);
+            mGu.A8 = mGu.A;
+            mDn.A8 = mDn.A;
+        }
+        if (!a_ok || !gu_b_ok ||
             !make_b_maps(mDn.B, h, p.ld_h, p.R, dn_tiles == kTilesPair ? kDnBN / 2 : dn_bn))
             return MOE_ERR_CUDA;
         if (gather)
@@ -558,9 +594,13 @@ moe_status moe_forward_ex(const moe_bf16* x, const moe_bf16* W_r, const moe_bf16
             tdn.seg_done = tickets + 2 * kSplitTickets + (kMaxSegments + 1);
     }
     const int grid = sms < kMaxTcGrid ? sms : kMaxTcGrid;
-    MOE_CUDA(launch_tc_gate_up(mGu, ta, grid, gu_tiles, chain, s));
+    if (f8) {
+        ta.a_scale = opts->gate_up_scale;
+        tdn.a_scale = opts->down_scale;
+    }
+    MOE_CUDA(launch_tc_gate_up(mGu, ta, grid, gu_tiles, f8, chain, s));
     if ((st = record(opts, 3, s)) != MOE_OK) return st;
-    MOE_CUDA(launch_tc_down(mDn, tdn, grid, dn_tiles, chain, s));
+    MOE_CUDA(launch_tc_down(mDn, tdn, grid, dn_tiles, f8, chain, s));
     if ((st = record(opts, 4, s)) != MOE_OK) return st;
     MOE_CUDA(launch_combine(ta.slots, p.T, p.D, p.k, p.has_shared, x, sg, residual, out,
                             out_f32, chain, s));

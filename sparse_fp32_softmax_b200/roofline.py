@@ -30,10 +30,15 @@ def expected_touched(E, k, T):
     return E * (1.0 - (1.0 - k / E) ** T)
 
 
-def algorithmic_bytes(T, D, E, k, I, touched, I_s=0, shared_gated=False, residual=False):
+def algorithmic_bytes(T, D, E, k, I, touched, I_s=0, shared_gated=False, residual=False,
+                      fp8_experts=False):
     """HBM bytes the block cannot avoid: each touched expert's weights once, the router,
-    the shared expert (+ its gate vector), x in and y out (+ the residual in)."""
-    b = touched * 3 * D * I * BF16 + E * D * BF16
+    the shared expert (+ its gate vector), x in and y out (+ the residual in).  FP8 experts:
+    one byte per weight plus an FP32 scale per weight row (2I + D rows per expert)."""
+    if fp8_experts:
+        b = touched * (3 * D * I + 4 * (2 * I + D)) + E * D * BF16
+    else:
+        b = touched * 3 * D * I * BF16 + E * D * BF16
     if I_s:
         b += 3 * D * I_s * BF16 + (D * BF16 if shared_gated else 0)
     b += 2 * T * D * BF16

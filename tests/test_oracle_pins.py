@@ -288,3 +288,75 @@ def test_parameter_split_matches_page():
     assert round(stored / 1e9, 1) == p["expert_params_stored_B"]
     assert round(active / 1e9, 2) == p["expert_params_active_B"]
     assert round(active / stored, 3) == p["active_fraction"]
+
+
+# ------------------------------------------------------------------ FP8 weight-only experts
+
+def test_e4m3_values_match_library_decoding(oracle_mod):
+    # every code against torch's float8_e4m3fn decoding, and the format's landmarks
+    codes = np.arange(256, dtype=np.uint8)
+    vals = np.array([oracle_mod.e4m3_value(c) for c in codes])
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    assert np.array_equal(np.isnan(vals), np.isnan(ref))
+    assert np.array_equal(vals[~np.isnan(vals)], ref[~np.isnan(ref)])
+    assert oracle_mod.e4m3_value(0x7E) == 448.0 and oracle_mod.e4m3_value(0x38) == 1.0
+    assert oracle_mod.e4m3_value(0x01) == 2.0 ** -9 and oracle_mod.e4m3_value(0x08) == 2.0 ** -6
+    assert np.isnan(oracle_mod.e4m3_value(0x7F)) and oracle_mod.e4m3_value(0xFE) == -448.0
+
+
+def test_fp8_quantizer_matches_library_rounding(oracle_mod):
+    g = torch.Generator().manual_seed(3)
+    W = torch.randn(96, 384, generator=g) * 0.02
+    W[0] = 0
+    W[1, 5] = 50.0                                  # one large value: most of the row underflows
+    W[2] *= 1e-3
+    W[3, :4] = torch.tensor([448.0, -448.0, 1.0, 2.0 ** -9])
+    Wb = W.to(torch.bfloat16)
+    q, s = oracle_mod.quantize_fp8_rows(Wb)
+    Wf = Wb.float()
+    amax = Wf.abs().amax(dim=1)
+    s_ref = torch.where(amax > 0, amax / 448.0, torch.ones_like(amax))        # FP32 division
+    assert np.array_equal(s.view(np.uint32), s_ref.numpy().view(np.uint32))
+    quot = (Wf / s_ref[:, None]).clamp(-448.0, 448.0)                           # FP32 quotient
+    q_ref = quot.to(torch.float8_e4m3fn).view(torch.uint8).numpy()              # nearest-even
+    assert np.array_equal(q, q_ref)
+
+
+def test_fp8_dequantisation_error_bound(oracle_mod):
+    # |w / s - value(q)| is at most half a step of E4M3 at that magnitude: 2^-4 of the value for
+    # normal values, 2^-10 in the subnormal range
+    g = torch.Generator().manual_seed(4)
+    Wb = (torch.randn(64, 256, generator=g) * 0.05).to(torch.bfloat16)
+    q, s = oracle_mod.quantize_fp8_rows(Wb)
+    table = np.array([oracle_mod.e4m3_value(c) for c in range(256)])
+    v = (Wb.float() / torch.from_numpy(s)[:, None]).double().numpy()
+    err = np.abs(v - table[q])
+    assert (err <= np.maximum(np.abs(v) * 2.0 ** -4, 2.0 ** -10) * (1 + 1e-12)).all()
+
+
+def test_fp8_experts_equal_bf16_experts_on_exact_weights(oracle_mod):
+    # weights on the E4M3 grid times a power of two (each row reaching 448 * 2^n), so that
+    # the row scale is exactly 2^n and the dequantised weights equal the bf16 weights: the FP8
+    # evaluation must then equal the bf16 one bit for bit
+    rng = np.random.default_rng(6)
+    E, I, D, T, k = 3, 16, 32, 5, 2
+    finite = np.array([c for c in range(256) if c not in (0x7F, 0xFF)], np.uint8)
+    table = np.array([oracle_mod.e4m3_value(c) for c in range(256)])
+
+    def grid(rows, cols, n):
+        c = rng.choice(finite, size=(rows, cols))
+        c[:, 0] = 0x7E                               # 448 in every row
+        return torch.from_numpy(table[c] * 2.0 ** n).to(torch.bfloat16)
+
+    W_gu = grid(E * 2 * I, D, -12).reshape(E, 2 * I, D)
+    W_dn = grid(E * D, I, -11).reshape(E, D, I)
+    x = torch.from_numpy(rng.standard_normal((T, D))).to(torch.bfloat16)
+    idx = np.array([[0, 2], [1, 0], [2, 1], [0, 1], [2, 0]], np.int32)
+    w = np.array([[0.7, 0.3], [0.5, 0.5], [0.25, 0.75], [0.9, 0.1], [0.6, 0.4]], np.float32)
+    q_gu, s_gu = oracle_mod.quantize_fp8_rows(W_gu)
+    q_dn, s_dn = oracle_mod.quantize_fp8_rows(W_dn)
+    assert (s_gu == 2.0 ** -12).all() and (s_dn == 2.0 ** -11).all()
+    rows = np.arange(T, dtype=np.int32)
+    y8 = oracle_mod.combine_rows_fp8(x, idx, w, rows, q_gu, s_gu, q_dn, s_dn)
+    y16 = oracle_mod.combine_rows(x, idx, w, rows, W_gu, W_dn)
+    assert np.array_equal(y8, y16)
