@@ -127,10 +127,13 @@ def profile_traffic(kernel_tag):
     return float(m.group(1))
 
 
-def kernels_per_forward(T, k):
-    """Kernels one moe_forward_ex call launches (the library's launch sequence): the router;
-    selection + permutation in one kernel while T*k <= 4096, else selection, histogram, scan
-    and scatter; for T > 32 the permuted copy of x; then gate_up, down and the combine."""
+def kernels_per_forward(T, k, path="grouped"):
+    """Kernels one moe_forward_ex call launches (the library's launch sequence): on the decode
+    path one; on the grouped path the router; selection + permutation in one kernel while
+    T*k <= 4096, else selection, histogram, scan and scatter; for T > 32 the permuted copy of
+    x; then gate_up, down and the combine."""
+    if path == "decode":
+        return 1
     return 1 + (1 if T * k <= 4096 else 4) + (1 if T > 32 else 0) + 3
 
 
@@ -276,6 +279,7 @@ def measure(name, args, rank, world, device, peaks, with_e2e):
         p["opts"] = B.make_opts(router_bias=w.get("bias"), shared_gate_up=w.get("shared_gate_up"),
                                 shared_down=w.get("shared_down"), shared_gate=w.get("shared_gate"),
                                 residual=p["residual"], topk_idx_out=p["idx"], **w.get("fp8", {}))
+        p["path"] = B.moe_forward_path(p["dims"], p["opts"])
         if chain:                             # passes run one after another: one workspace
             if shared_ws is None:
                 shared_ws = B.workspace(p["dims"], p["opts"], device=device)
@@ -418,13 +422,18 @@ def measure(name, args, rank, world, device, peaks, with_e2e):
         if len(passes) > 1 and not chain:
             t_ms = per_T_ms[T]
             t_roof = max(b / (hbm * 1e9), f / (tf_peak * 1e12))
-            sweep_out.append(dict(
-                T=T, us=round(t_ms * 1e3, 2), tokens_per_s=round(T / (t_ms / 1e3), 1),
+            entry = dict(
+                T=T, path=p["path"], us=round(t_ms * 1e3, 2), tokens_per_s=round(T / (t_ms / 1e3), 1),
                 roofline_us=round(t_roof * 1e6, 2), roofline_frac=round(t_roof / (t_ms / 1e3), 4),
-                touched=p["touched"], max_load=p["max_load"],
-                stages_us_with_events=dict(zip(STAGES, [round(v * 1e3, 2) for v in stage_ms[n]])),
-                gate_up_gbs=round(b_gu / (stage_ms[n][2] / 1e3) / 1e9, 1),
-                down_gbs=round(b_dn / (stage_ms[n][3] / 1e3) / 1e9, 1)))
+                touched=p["touched"], max_load=p["max_load"])
+            if p["path"] == "decode":   # one kernel: the whole block between the first two events
+                entry["kernel_us_with_events"] = round(stage_ms[n][0] * 1e3, 2)
+                entry["kernel_gbs"] = round(b / (stage_ms[n][0] / 1e3) / 1e9, 1)
+            else:
+                entry["stages_us_with_events"] = dict(zip(STAGES, [round(v * 1e3, 2) for v in stage_ms[n]]))
+                entry["gate_up_gbs"] = round(b_gu / (stage_ms[n][2] / 1e3) / 1e9, 1)
+                entry["down_gbs"] = round(b_dn / (stage_ms[n][3] / 1e3) / 1e9, 1)
+            sweep_out.append(entry)
 
     def dominant(rs, kname):
         if chain:   # every layer has the same shape: average them
@@ -435,9 +444,20 @@ def measure(name, args, rank, world, device, peaks, with_e2e):
         b, f, t, T = rs[-1]          # the largest pass: one launch shape, one ncu capture
         return kernel_roof(kname, b, f, t, f"T={T}")
 
-    roof = dominant(gu_roofs, "tc_gemm_kernel<gate_up>")
-    roof_dn = dominant(dn_roofs, "tc_gemm_kernel<down>")
+    if passes[-1]["path"] == "decode":
+        # one kernel for the whole block: its roofline is the block's bytes over its duration
+        T = passes[-1]["T"]
+        b = algorithmic_bytes(T, cfg.D, cfg.E, cfg.k, cfg.I, passes[-1]["touched"], cfg.I_s, cfg.shared_gated,
+                              residual=chain, fp8_experts=bool(spec.get("fp8")))
+        f = algorithmic_flops(T, cfg.D, cfg.E, cfg.k, cfg.I, cfg.I_s, cfg.shared_gated)
+        roof = kernel_roof("decode_block_kernel", b, f, stage_ms[-1][0], f"T={T}")
+        roof_dn = None
+    else:
+        roof = dominant(gu_roofs, "tc_gemm_kernel<gate_up>")
+        roof_dn = dominant(dn_roofs, "tc_gemm_kernel<down>")
     tag = {"decode": "tc_gate_up_decode", "prefill": "tc_gemm_prefill"}.get(name, f"tc_gate_up_{name}")
+    if passes[-1]["path"] == "decode":
+        tag = "decode_block_t1"
     roof["traffic"] = profile_traffic(tag)
     blk_time = max(blk_bytes / (hbm * 1e9), blk_flops / (tf_peak * 1e12))
     res = dict(
@@ -453,7 +473,7 @@ def measure(name, args, rank, world, device, peaks, with_e2e):
                             flops=int(blk_flops), bound=("hbm" if blk_bytes / (hbm * 1e9) >=
                                                          blk_flops / (tf_peak * 1e12) else "tensor"),
                             peaks=f"hbm_gbs {hbm}, {tf_name} {tf_peak} ({peaks['source']})"),
-        gpu_launches=int(sum(kernels_per_forward(p["T"], cfg.k) for p in passes) * K),
+        gpu_launches=int(sum(kernels_per_forward(p["T"], cfg.k, p["path"]) for p in passes) * K),
         clocks=sampler.summary())
     if not chain:
         res["stages_us_with_events"] = dict(zip(STAGES, [round(v * 1e3, 2) for v in stage_ms[-1]]))

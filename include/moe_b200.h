@@ -69,8 +69,17 @@ typedef struct {
 
 /* Which expert path moe_forward_ex takes. */
 enum {
-    MOE_PATH_AUTO = 0,    /* the library's choice (the grouped path at every T) */
-    MOE_PATH_GROUPED = 1  /* permute + tcgen05 grouped GEMMs, TMA-fed, TMEM accumulators */
+    MOE_PATH_AUTO = 0,    /* the library's choice: MOE_PATH_DECODE where it applies, else
+                             MOE_PATH_GROUPED (moe_forward_path tells which) */
+    MOE_PATH_GROUPED = 1, /* permute + tcgen05 grouped GEMMs, TMA-fed, TMEM accumulators */
+    MOE_PATH_DECODE = 2   /* the whole block in one kernel for one token (T = 1, D <= 2048,
+                             I <= 1536, and two blocks of ceil(D / SMs) down rows of I fit in
+                             an SM's shared memory beside its buffers): one block per SM, all resident
+                             at once (a call needs the whole GPU; other work running on it
+                             delays the call, up to the wait limit, after which it reports
+                             MOE_ERR_DEVICE_TIMEOUT).  Not with a shared expert, FP8 experts,
+                             expert_counts_out, slot_row_out or MOE_DIAG_UNSIGNALLED_HANDOFF;
+                             asking for it then returns MOE_ERR_UNSUPPORTED */
 };
 
 /* Diagnostics of moe_forward_ex (moe_opts.diag); 0 in normal use. */
@@ -80,7 +89,13 @@ enum {
      * (moe_opts.wait_limit_us) and the kernels wind down.  The output is then undefined and
      * moe_get_device_status reports MOE_ERR_DEVICE_TIMEOUT; the device stays usable.  For
      * testing the watchdog.  Shapes that do not use the hand-off return MOE_ERR_UNSUPPORTED. */
-    MOE_DIAG_UNSIGNALLED_HANDOFF = 1
+    MOE_DIAG_UNSIGNALLED_HANDOFF = 1,
+    /* The decode kernel's grid-wide barrier waits for one block more than the grid has, so it
+     * runs until its limit (moe_opts.wait_limit_us); the output is then undefined and
+     * moe_get_device_status reports MOE_ERR_DEVICE_TIMEOUT; the device stays usable.  For
+     * testing the watchdog of MOE_PATH_DECODE; where that path does not apply,
+     * MOE_ERR_UNSUPPORTED. */
+    MOE_DIAG_DECODE_BARRIER = 2
 };
 
 /* Options of moe_forward_ex.  Zero-initialise and set what is needed. */
@@ -185,16 +200,26 @@ moe_status moe_permute(const int32_t *topk_idx, const float *topk_w, const moe_b
  * Results are bitwise reproducible for the same inputs.  At decode shapes (T*k <= 32*E) the
  * expert GEMMs may split the K sums of their last items into slices (added in slice order),
  * and how many depends on the batch's work, so a token's output can differ in the last bits
- * between batches (its routing does not, see moe_route). */
+ * between batches (its routing does not, see moe_route).  For T = 1 the decode kernel
+ * (MOE_PATH_DECODE) computes every dot product in a fixed order that does not depend on the
+ * GPU's SM count. */
 moe_status moe_forward(const moe_bf16 *x, const moe_bf16 *W_r, const moe_bf16 *W_gate_up,
                        const moe_bf16 *W_down, const moe_dims *dims, moe_bf16 *out, void *ws,
                        size_t ws_bytes, moe_stream_t stream);
 
 /* moe_forward with options (router bias, gated shared expert, residual, routing outputs,
- * path choice, stage events).  out may alias opts->residual but not x. */
+ * path choice, stage events).  out may alias opts->residual but not x.  On MOE_PATH_DECODE
+ * the stage events after routing .. after the combine are all recorded after its one
+ * kernel. */
 moe_status moe_forward_ex(const moe_bf16 *x, const moe_bf16 *W_r, const moe_bf16 *W_gate_up,
                           const moe_bf16 *W_down, const moe_dims *dims, const moe_opts *opts,
                           moe_bf16 *out, void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/* The path (MOE_PATH_DECODE or MOE_PATH_GROUPED) that moe_forward_ex takes for these
+ * arguments, in *path_out; the status moe_forward_ex would return for an invalid or
+ * unsupported request, or MOE_ERR_CUDA without a device (the choice depends on the device's
+ * SM count).  Enqueues nothing. */
+moe_status moe_forward_path(const moe_dims *dims, const moe_opts *opts, int *path_out);
 
 /* moe_forward for callers that cannot allocate device memory: plugin hosts that give a
  * kernel only its input and output buffers, and runtimes that forbid device allocation once

@@ -19,9 +19,10 @@ LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
 HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "moe_b200.h")
 
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_DEVICE_TIMEOUT = range(6)
-MOE_PATH_AUTO, MOE_PATH_GROUPED = range(2)
-PATHS = {"auto": MOE_PATH_AUTO, "grouped": MOE_PATH_GROUPED}
+MOE_PATH_AUTO, MOE_PATH_GROUPED, MOE_PATH_DECODE = range(3)
+PATHS = {"auto": MOE_PATH_AUTO, "grouped": MOE_PATH_GROUPED, "decode": MOE_PATH_DECODE}
 MOE_DIAG_UNSIGNALLED_HANDOFF = 1
+MOE_DIAG_DECODE_BARRIER = 2
 
 _c_int, _vp, _sz = ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t
 
@@ -74,8 +75,10 @@ def load():
         lib.moe_last_cuda_error.argtypes = []
         lib.moe_last_cuda_error.restype = _c_int
         lib.moe_quantize_fp8_rows.argtypes = [_vp, ctypes.c_int64, _c_int, _vp, _vp, _vp]
+        lib.moe_forward_path.argtypes = [dp, op, ctypes.POINTER(_c_int)]
         for n in ("moe_route", "moe_permute", "moe_forward", "moe_forward_ex", "moe_forward_noalloc",
-                  "moe_get_device_status", "moe_get_device_status_noalloc", "moe_quantize_fp8_rows"):
+                  "moe_get_device_status", "moe_get_device_status_noalloc", "moe_quantize_fp8_rows",
+                  "moe_forward_path"):
             getattr(lib, n).restype = _c_int
         _lib = lib
     return _lib
@@ -85,7 +88,7 @@ def header_functions():
     """Names of the functions ``include/moe_b200.h`` declares."""
     with open(HEADER_PATH) as f:
         text = f.read()
-    return sorted(set(re.findall(r"^\s*(?:const\s+)?[a-z_]+\s*\*?\s*(moe_[a-z_]+)\s*\(", text, re.M)))
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[a-z_]+\s*\*?\s*(moe_[a-z0-9_]+)\s*\(", text, re.M)))
 
 
 def status_string(status: int) -> str:
@@ -168,6 +171,14 @@ def make_opts(router_bias=None, shared_gate_up=None, shared_down=None, shared_ga
 
 def moe_workspace_size(dims: moe_dims, opts: moe_opts | None = None) -> int:
     return int(load().moe_workspace_size(ctypes.byref(dims), ctypes.byref(opts) if opts else None))
+
+
+def moe_forward_path(dims: moe_dims, opts: moe_opts | None = None) -> str:
+    """The path moe_forward_ex takes for these arguments: "decode" or "grouped"."""
+    out = _c_int(-1)
+    _check(load().moe_forward_path(ctypes.byref(dims), ctypes.byref(opts) if opts else None, ctypes.byref(out)),
+           "moe_forward_path")
+    return {MOE_PATH_DECODE: "decode", MOE_PATH_GROUPED: "grouped"}[out.value]
 
 
 def workspace(dims: moe_dims, opts: moe_opts | None = None, device=None) -> torch.Tensor:

@@ -209,6 +209,60 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* e
 
 // ------------------------------------------------------------------ TMA
 
+// Untiled bulk copy of `bytes` contiguous bytes from global memory into this CTA's shared
+// memory, completing on `bar` (both addresses 16-byte aligned, bytes a multiple of 16).
+__device__ __forceinline__ void bulk_load(void* smem_dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(smem_dst)),
+        "l"(src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// Bring `bytes` contiguous bytes into L2 (a hint: same alignment rules as bulk_load).
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
+// Hardware barrier `id` (1..15) among `nthreads` threads (whole warps) of the CTA.
+__device__ __forceinline__ void named_barrier_sync(int id, int nthreads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+__device__ __forceinline__ unsigned long long ld_relaxed_gpu_u64(const unsigned long long* p) {
+    unsigned long long v;
+    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_relaxed_gpu_u64(unsigned long long* p, unsigned long long v) {
+    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Barrier over the blocks of a grid whose blocks are all resident at once, called by one
+// thread per block after a block-wide barrier (which orders the block's earlier writes before
+// this thread's release).  `count` is zero when the launch starts; use n (n = 1, 2, ...) of a
+// launch waits until all blocks have arrived n times: target = n * blocks.  Each block adds 1
+// with release semantics and polls with acquire loads.  Bounded: returns false (and sets
+// kErrWaitGrid) once limit_ns nanoseconds have passed.
+__device__ __forceinline__ bool grid_sync(unsigned* count, unsigned target, int* err, uint64_t limit_ns) {
+    asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(count) : "memory");
+    if (ld_acquire_gpu(count) >= target) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (ld_acquire_gpu(count) < target) {
+        if (globaltimer_ns() - t0 > limit_ns) {
+            set_error(err, kErrWaitGrid);
+            return false;
+        }
+    }
+    return true;
+}
+
 // Bring one tile of a 2-D tensor map into L2 (a hint: no completion, no shared memory).
 __device__ __forceinline__ void tma_prefetch_l2(const CUtensorMap* map, int x, int y) {
     asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
@@ -455,7 +509,15 @@ __device__ __forceinline__ void tmem_ld_wait() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
-// ------------------------------------------------------------------ legacy warp MMA
+// ------------------------------------------------------------------ warp MMA (small tiles)
+
+// Four 8x8 bf16 matrices from shared memory into the mma.sync A-fragment registers: lanes
+// 8m..8m+7 give the 16-byte row addresses of matrix m.
+__device__ __forceinline__ void ldmatrix_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
 
 // D = A * B + D for one m16n8k16 bf16 tile with FP32 accumulators (register operands).
 __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint32_t a1,

@@ -18,6 +18,7 @@ enum : int {
     kErrWaitEpilogue = 4,   // epilogue gave up waiting for an accumulator
     kErrBadIndex = 8,       // an expert index outside [0, E) reached the permute stage
     kErrWaitTail = 16,      // producer gave up draining its last stages
+    kErrWaitGrid = 32,      // a block of the decode kernel gave up waiting for the other blocks
 };
 
 // Tile geometry of the tcgen05 grouped GEMMs (swap-AB: weights on M, tokens on N).
@@ -229,5 +230,75 @@ cudaError_t launch_combine(const float* slots, int T, int D, int k, int has_shar
                            const uint16_t* x, const uint16_t* shared_gate,
                            const uint16_t* residual, uint16_t* out, float* out_f32, bool pdl,
                            cudaStream_t s);
+
+// ---------------------------------------------------------------- the decode kernel
+// The whole block for one token in one persistent kernel (one block per SM, all resident at
+// once): router, selection, gate_up, down and the combine, separated by two grid-wide
+// barriers.  Used for T = 1 when the call needs nothing it does not do.
+constexpr int kDecWarps = 8;           // compute warps (plus one copy warp)
+constexpr int kDecThreads = (kDecWarps + 1) * 32;
+constexpr int kDecMaxStages = 32;
+constexpr int kDecMinStages = 2;
+constexpr int kDecSmemBudget = 220 * 1024;   // dynamic shared memory per block
+constexpr int kDecMaxD = 2048;         // a gate/up row is at most 8 16-byte pieces per lane
+constexpr int kDecChunks = kDecMaxD / 256;
+
+// Shared-memory layout of a decode block: the copy ring (a stage holds one expert's down
+// rows for the block's output rows: nd_max rows of I, padded to whole 16-row MMA tiles, each
+// row at a stride of 2I + 16 bytes so that the 8 rows an ldmatrix reads fall in distinct
+// banks), x as FP32 in two planes, h of every slot, the down results of the block's output
+// rows, then the ring's barriers.
+struct DecodeLayout {
+    int stages, nd_max, rs;
+    size_t sb, ring, xs, hs, val, bars, total;
+};
+__host__ __device__ inline DecodeLayout decode_layout(int D, int k, int I, int nd_max, int stages) {
+    DecodeLayout L;
+    L.stages = stages;
+    L.rs = 2 * I + 16;
+    L.sb = ((size_t)((nd_max + 15) / 16) * 16 * L.rs + 127) / 128 * 128;
+    L.nd_max = nd_max;
+    size_t off = 0;
+    L.ring = off;
+    off += (size_t)stages * L.sb;
+    L.xs = off;
+    off += (size_t)D * 4;
+    L.hs = off;
+    off += (size_t)k * I * 2;
+    L.val = off;
+    off += ((size_t)k * nd_max * 4 + 15) / 16 * 16;
+    L.bars = off;
+    off += (size_t)2 * stages * 8;
+    L.total = off;
+    return L;
+}
+
+struct DecodeArgs {
+    const uint16_t* x;        // [D]
+    const uint16_t* W_r;      // [E, D]
+    const float* bias;        // [E] or null
+    const uint16_t* W_gu;     // [E, 2I, D]
+    const uint16_t* W_dn;     // [E, D, I]
+    const uint16_t* residual; // [D] or null (may alias out)
+    uint16_t* out;            // [D]
+    float* out_f32;           // [D] or null
+    float* logits_out;        // [E] or null
+    int32_t* idx_out;         // [k]
+    float* w_out;             // [k]
+    unsigned long long* lgf;  // workspace [E]: flag (high word) and logit before the bias (low
+                              // word); zero before the launch
+    uint16_t* h;              // workspace [k, I]: h of every slot
+    unsigned* bar;            // workspace: the grid-barrier counter, zeroed before the launch
+    int* err;
+    int D, E, k, I, norm;
+    int stages;
+    unsigned long long wait_ns;
+    int extra_blocks;         // 0; 1 makes every grid barrier wait for a block that does not exist
+};
+
+// Ring depth for this shape on a grid of `blocks` blocks, or 0 when the decode kernel does
+// not apply (T != 1, D or I too wide for its buffers).
+int decode_stages(int T, int D, int E, int k, int I, int blocks);
+cudaError_t launch_decode(const DecodeArgs& a, int blocks, bool pdl, cudaStream_t s);
 
 }  // namespace moe

@@ -58,10 +58,12 @@ namespace {
 constexpr size_t kAlign = 256;
 // Ints of the ticket region: gate_up split tickets, down split tickets, the per-expert
 // completion counters of gate_up (nseg + 1 <= kMaxSegments + 1), the same number of
-// counters that stay zero (MOE_DIAG_UNSIGNALLED_HANDOFF points the down GEMM at them), and
-// the unit counters of the narrow gate_up and down kernels.
+// counters that stay zero (MOE_DIAG_UNSIGNALLED_HANDOFF points the down GEMM at them),
+// the unit counters of the narrow gate_up and down kernels, and the grid-barrier counter of
+// the decode kernel.
 constexpr int kSchedAt = 2 * kSplitTickets + 2 * (kMaxSegments + 1);
-constexpr int kTicketInts = kSchedAt + 2;
+constexpr int kDecBarAt = kSchedAt + 2;
+constexpr int kTicketInts = kDecBarAt + 1;
 
 // The cudaError_t of the last CUDA failure seen by this host thread (moe_last_cuda_error).
 thread_local int g_last_cuda_error = 0;
@@ -91,7 +93,8 @@ Plan make_plan(const moe_dims& d, const moe_opts* o) {
     p.rsplit = p.T <= kRouterSmallMaxT ? 1 : router_splits(p.T, p.E, p.D, kRtBN);
     size_t off = 0;
     auto take = [&](size_t bytes) { size_t at = off; off += align_up(bytes); return at; };
-    p.err = take(kAlign);                              // [0] error word, [1] routing ticket
+    // [0] error word, [1] routing ticket; then (decode kernel) the E flagged logits
+    p.err = take(kAlign + (size_t)p.E * 8);
     // split-tail tickets of gate_up and of down, the per-expert completion counters, and a
     // block of counters that no kernel increments (the watchdog diagnostic); all follow err,
     // so one memset clears the header
@@ -148,10 +151,12 @@ moe_status check_opts(const moe_dims* d, const moe_opts* o) {
     if (o->logits_out && !aligned(o->logits_out, 4)) return MOE_ERR_INVALID_ARG;
     if (o->topk_idx_out && !aligned(o->topk_idx_out, 4)) return MOE_ERR_INVALID_ARG;
     if (o->topk_w_out && !aligned(o->topk_w_out, 4)) return MOE_ERR_INVALID_ARG;
-    if (o->path != MOE_PATH_AUTO && o->path != MOE_PATH_GROUPED) return MOE_ERR_INVALID_ARG;
+    if (o->path != MOE_PATH_AUTO && o->path != MOE_PATH_GROUPED && o->path != MOE_PATH_DECODE)
+        return MOE_ERR_INVALID_ARG;
     if (o->expert_counts_out && !aligned(o->expert_counts_out, 4)) return MOE_ERR_INVALID_ARG;
     if (o->slot_row_out && !aligned(o->slot_row_out, 4)) return MOE_ERR_INVALID_ARG;
-    if (o->diag != 0 && o->diag != MOE_DIAG_UNSIGNALLED_HANDOFF) return MOE_ERR_INVALID_ARG;
+    if (o->diag != 0 && o->diag != MOE_DIAG_UNSIGNALLED_HANDOFF && o->diag != MOE_DIAG_DECODE_BARRIER)
+        return MOE_ERR_INVALID_ARG;
     if (o->diag == MOE_DIAG_UNSIGNALLED_HANDOFF && !use_narrow_tiles(d->T, d->k, d->E))
         return MOE_ERR_UNSUPPORTED;
     if (o->n_stage_events != 0 && o->n_stage_events != 6) return MOE_ERR_INVALID_ARG;
@@ -166,6 +171,25 @@ moe_status check_opts(const moe_dims* d, const moe_opts* o) {
         if (o->shared_gate_up || !use_narrow_tiles(d->T, d->k, d->E)) return MOE_ERR_UNSUPPORTED;
     }
     return MOE_OK;
+}
+
+// Ring depth of the decode kernel for this call on `sms` blocks, 0 when it does not apply:
+// more than one token, or a feature it does not implement (shared expert, FP8
+// experts, the permutation outputs, the grouped path's diagnostic).
+int decode_stages_for(const moe_dims& d, const moe_opts* o, int sms) {
+    if (o && (o->shared_gate_up || o->W_gate_up_fp8 || o->expert_counts_out || o->slot_row_out ||
+              o->diag == MOE_DIAG_UNSIGNALLED_HANDOFF))
+        return 0;
+    return decode_stages(d.T, d.D, d.E, d.k, d.I, sms);
+}
+
+// The path moe_forward_ex takes (arguments already checked).
+int choose_path(const moe_dims& d, const moe_opts* o, int sms, int* dec_stages) {
+    const int want = o ? o->path : MOE_PATH_AUTO;
+    *dec_stages = want == MOE_PATH_GROUPED ? 0 : decode_stages_for(d, o, sms);
+    if (want == MOE_PATH_DECODE || (o && o->diag == MOE_DIAG_DECODE_BARRIER))
+        return *dec_stages > 0 ? MOE_PATH_DECODE : -1;
+    return *dec_stages > 0 ? MOE_PATH_DECODE : MOE_PATH_GROUPED;
 }
 
 // ------------------------------------------------------------------ device properties / TMA
@@ -450,6 +474,32 @@ moe_status moe_forward_ex(const moe_bf16* x, const moe_bf16* W_r, const moe_bf16
     float* out_f32 = opts ? opts->out_f32 : nullptr;
     const unsigned long long wait_ns =
         (opts && opts->wait_limit_us) ? (unsigned long long)opts->wait_limit_us * 1000ull : kWaitLimitNs;
+    const bool chain = !(opts && opts->n_stage_events == 6);
+
+    int dec_stages = 0;
+    const int path = choose_path(*dims, opts, sms, &dec_stages);
+    if (path < 0) return MOE_ERR_UNSUPPORTED;
+    if (path == MOE_PATH_DECODE) {
+        // one kernel: the stage events around it mark routing as the whole block
+        MOE_CUDA(cudaMemsetAsync(err, 0, p.tickets - p.err + (size_t)kTicketInts * 4, s));
+        if ((st = record(opts, 0, s)) != MOE_OK) return st;
+        DecodeArgs da{};
+        da.x = x; da.W_r = W_r; da.bias = bias; da.W_gu = W_gate_up; da.W_dn = W_down;
+        da.residual = residual; da.out = out; da.out_f32 = out_f32;
+        da.logits_out = logits_user; da.idx_out = idx; da.w_out = w;
+        da.lgf = reinterpret_cast<unsigned long long*>(at<char>(ws, p.err) + kAlign);
+        da.h = at<uint16_t>(ws, p.h);
+        da.bar = reinterpret_cast<unsigned*>(at<int>(ws, p.tickets) + kDecBarAt);
+        da.err = err;
+        da.D = p.D; da.E = p.E; da.k = p.k; da.I = p.I; da.norm = dims->norm_topk_prob;
+        da.stages = dec_stages;
+        da.wait_ns = wait_ns;
+        da.extra_blocks = (opts && opts->diag == MOE_DIAG_DECODE_BARRIER) ? 1 : 0;
+        MOE_CUDA(launch_decode(da, sms, chain, s));
+        for (int i = 1; i < 6; ++i)
+            if ((st = record(opts, i, s)) != MOE_OK) return st;
+        return MOE_OK;
+    }
 
     // tensor maps of the grouped path are encoded before anything is enqueued
     // narrow tiles (deeper pipelines) when experts average few rows; a segment with more
@@ -538,7 +588,6 @@ moe_status moe_forward_ex(const moe_bf16* x, const moe_bf16* W_r, const moe_bf16
     pa.dn_rows = dn_tiles == kTilesPair ? 2 * kTcM : kTcM;
     pa.err = err;
     // launch chaining between the forward's kernels (not across a stage-event record)
-    const bool chain = !(opts && opts->n_stage_events == 6);
     RouteArgs ra{};
     ra.bias = bias;
     ra.T = p.T; ra.E = p.E; ra.k = p.k; ra.norm = dims->norm_topk_prob;
@@ -605,6 +654,20 @@ moe_status moe_forward_ex(const moe_bf16* x, const moe_bf16* W_r, const moe_bf16
     MOE_CUDA(launch_combine(ta.slots, p.T, p.D, p.k, p.has_shared, x, sg, residual, out,
                             out_f32, chain, s));
     return record(opts, 5, s);
+}
+
+moe_status moe_forward_path(const moe_dims* dims, const moe_opts* opts, int* path_out) {
+    moe_status st = check_dims(dims);
+    if (st != MOE_OK) return st;
+    if ((st = check_opts(dims, opts)) != MOE_OK) return st;
+    if (!path_out) return MOE_ERR_INVALID_ARG;
+    const int sms = num_sms_of_current_device();
+    if (sms <= 0) return MOE_ERR_CUDA;
+    int dec_stages = 0;
+    const int path = choose_path(*dims, opts, sms, &dec_stages);
+    if (path < 0) return MOE_ERR_UNSUPPORTED;
+    *path_out = path;
+    return MOE_OK;
 }
 
 moe_status moe_forward(const moe_bf16* x, const moe_bf16* W_r, const moe_bf16* W_gate_up,

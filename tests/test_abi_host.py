@@ -27,7 +27,8 @@ def test_library_exports_every_declared_function(lib):
     declared = B.header_functions()
     assert set(declared) == {"moe_workspace_size", "moe_route", "moe_permute", "moe_forward",
                              "moe_forward_ex", "moe_forward_noalloc", "moe_get_device_status",
-                             "moe_get_device_status_noalloc", "moe_status_string", "moe_last_cuda_error"}
+                             "moe_get_device_status_noalloc", "moe_status_string", "moe_last_cuda_error",
+                             "moe_quantize_fp8_rows", "moe_forward_path"}
     out = subprocess.run(["nm", "-D", "--defined-only", LIB], capture_output=True, text=True, check=True).stdout
     exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
     for name in declared:
@@ -101,7 +102,7 @@ def test_forward_rejects_bad_arguments_before_launch(lib):
     o.n_stage_events = 3
     assert _fwd(lib, d, n, opts=o) == B.MOE_ERR_INVALID_ARG
     o = B.moe_opts()
-    o.diag = 2                                  # no such diagnostic
+    o.diag = 3                                  # no such diagnostic
     assert _fwd(lib, d, n, opts=o) == B.MOE_ERR_INVALID_ARG
     o = B.moe_opts()
     o.slot_row_out = FAKE + 2                   # misaligned routing-table output
@@ -110,6 +111,21 @@ def test_forward_rejects_bad_arguments_before_launch(lib):
     o.diag = B.MOE_DIAG_UNSIGNALLED_HANDOFF     # wide shape (T*k > 32*E): no hand-off wait
     wide = B.make_dims(512, 256, 8, 2, 128)
     assert _fwd(lib, wide, B.moe_workspace_size(wide), opts=o) == B.MOE_ERR_UNSUPPORTED
+
+
+@no_gpu
+def test_forward_path_query_without_a_device(lib):
+    """moe_forward_path validates like moe_forward_ex; the choice itself needs the device's SM
+    count, so without a GPU a valid query reports a CUDA failure."""
+    d = B.make_dims(2, 256, 8, 2, 128)
+    out = ctypes.c_int(-1)
+    assert lib.moe_forward_path(ctypes.byref(d), None, ctypes.byref(out)) == B.MOE_ERR_CUDA
+    o = B.moe_opts()
+    o.path = 7
+    assert lib.moe_forward_path(ctypes.byref(d), ctypes.byref(o), ctypes.byref(out)) == B.MOE_ERR_INVALID_ARG
+    assert lib.moe_forward_path(ctypes.byref(B.make_dims(2, 256, 8, 9, 128)), None,
+                                ctypes.byref(out)) == B.MOE_ERR_UNSUPPORTED
+    assert lib.moe_forward_path(ctypes.byref(d), None, None) == B.MOE_ERR_INVALID_ARG
 
 
 @no_gpu

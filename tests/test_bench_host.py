@@ -101,3 +101,5 @@ def test_kernels_per_forward_follows_the_launch_sequence():
     # then gate_up, down, combine.
     assert [bench.kernels_per_forward(T, 8) for T in (1, 32, 33, 256, 512, 8192)] == \
         [5, 5, 6, 6, 6, 9]
+    # the decode path is one kernel
+    assert bench.kernels_per_forward(1, 8, "decode") == 1

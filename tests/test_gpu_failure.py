@@ -8,6 +8,8 @@
   bounds every device wait at 20 ms.  The kernels give up, wind down (TMEM released, no copy
   in flight) and moe_get_device_status reports MOE_ERR_DEVICE_TIMEOUT; a normal call on the
   same workspace then runs correctly, so the context stayed usable.
+* The decode kernel's watchdog: MOE_DIAG_DECODE_BARRIER makes its grid-wide barrier wait
+  for one block more than the grid has; the same report and recovery.
 """
 import time
 
@@ -70,6 +72,34 @@ def test_watchdog_reports_timeout_and_device_stays_usable():
     y = B.moe_forward(G["x"], G["W_r"], G["W_gate_up"], G["W_down"], cfg.k, ws=ws)
     assert B.moe_get_device_status(ws) == B.MOE_OK
     assert torch.equal(y.cpu(), ref)
+
+
+def test_decode_kernel_watchdog():
+    """MOE_DIAG_DECODE_BARRIER: the decode kernel's grid barrier waits for a block that does
+    not exist; every block gives up after the 20 ms limit, the call reports
+    MOE_ERR_DEVICE_TIMEOUT, and the next call on the same workspace is exact again."""
+    cfg = inputs.CONFIGS["decode"]
+    L = inputs.make_layer(cfg, T=1)
+    G = {k_: (v.cuda() if v is not None else None) for k_, v in L.items()}
+    dims = B.make_dims(1, cfg.D, cfg.E, cfg.k, cfg.I)
+    ws = B.workspace(dims)
+    ref = B.moe_forward_ex(G["x"], G["W_r"], G["W_gate_up"], G["W_down"], cfg.k, ws=ws, path="decode")
+    assert B.moe_get_device_status(ws) == B.MOE_OK
+    ref = ref.cpu()
+    t0 = time.perf_counter()
+    B.moe_forward_ex(G["x"], G["W_r"], G["W_gate_up"], G["W_down"], cfg.k, ws=ws,
+                     wait_limit_us=20000, diag=B.MOE_DIAG_DECODE_BARRIER)
+    assert B.moe_get_device_status(ws) == B.MOE_ERR_DEVICE_TIMEOUT
+    assert time.perf_counter() - t0 < 1.9
+    y = B.moe_forward_ex(G["x"], G["W_r"], G["W_gate_up"], G["W_down"], cfg.k, ws=ws, path="decode")
+    assert B.moe_get_device_status(ws) == B.MOE_OK
+    assert torch.equal(y.cpu(), ref)
+    # where the decode kernel does not apply the diagnostic is refused
+    L8 = inputs.make_layer(cfg, T=8)
+    with pytest.raises(B.MoeError) as ei:
+        B.moe_forward_ex(L8["x"].cuda(), G["W_r"], G["W_gate_up"], G["W_down"], cfg.k,
+                         diag=B.MOE_DIAG_DECODE_BARRIER)
+    assert ei.value.status == B.MOE_ERR_UNSUPPORTED
 
 
 def test_watchdog_diagnostic_needs_the_handoff():

@@ -73,7 +73,7 @@ def compare_block(cfg, L, G, rows, path="auto", x_cpu=None, residual_cpu=None, k
     norm = cfg.norm_topk_prob if norm is None else norm
     x_cpu = L["x"] if x_cpu is None else x_cpu
     res_gpu = residual_cpu.cuda() if residual_cpu is not None else None
-    y, idx, w, logits = run_forward(cfg, G, x=x_cpu.cuda(), residual=res_gpu, k=k, norm=norm)
+    y, idx, w, logits = run_forward(cfg, G, path=path, x=x_cpu.cuda(), residual=res_gpu, k=k, norm=norm)
     y32 = run_forward.last_f32
     rows = np.asarray(sorted(set(int(r) for r in rows)), np.int32)
     # selection from the GPU's own logits is bit-exact; weights within 1e-6
