@@ -78,7 +78,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_block_kernel(const Deco
     __shared__ int s_idx[kMaxK];
     __shared__ float s_w[kMaxK];
     __shared__ float s_rpart[kDecWarps][kRouterGroup];
-    __shared__ float s_lg[32 * VPL];
+    __shared__ int s_nsel;   // slots published by the selection
 
     const int D = a.D, E = a.E, k = a.k, I = a.I;
     const int G = gridDim.x, b = blockIdx.x;
@@ -96,7 +96,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_block_kernel(const Deco
     const float4* xlo = reinterpret_cast<const float4*>(xs);
     const float4* xhi = reinterpret_cast<const float4*>(xs + D / 2);
 
+    if (threadIdx.x < kMaxK) s_idx[threadIdx.x] = 0;   // in range until the selection publishes
     if (threadIdx.x == 0) {
+        s_nsel = 0;
         for (int s = 0; s < NS; ++s) {
             mbar_init(full + s, 1);
             mbar_init(empty + s, 1);
@@ -159,59 +161,119 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_block_kernel(const Deco
         }
     }
 
-    // ---- 2. selection (warp 1): it polls the E flagged logits (written by the router blocks
-    // of this launch, zero before it) into shared memory, then selects; block 0 also returns
-    // the logits (bias added) when asked, and the routing
-    if (warp == 1) {
-        const uint64_t t0 = globaltimer_ns();
-        for (int e = lane; e < E; e += 32) {
-            unsigned long long v = ld_relaxed_gpu_u64(a.lgf + e);
-            while ((v >> 32) == 0ull) {
-                if (globaltimer_ns() - t0 > a.wait_ns) {
-                    set_error(a.err, kErrWaitGrid);
-                    break;
-                }
-                v = ld_relaxed_gpu_u64(a.lgf + e);
-            }
-            s_lg[e] = __uint_as_float((uint32_t)v);
-        }
-        __syncwarp();
-        select_token<VPL>(s_lg, 1, 0, a.bias, E, k, a.norm, s_idx, s_w,
-                          (b == 0 && a.logits_out) ? a.logits_out : nullptr);
-        __syncwarp();
-        if (lane < k) {
-            if (s_idx[lane] < 0 || s_idx[lane] >= E) {   // cannot happen for finite logits
-                set_error(a.err, kErrBadIndex);
-                s_idx[lane] = 0;
-            }
-            if (b == 0) {
-                a.idx_out[lane] = s_idx[lane];
-                a.w_out[lane] = s_w[lane];
-            }
-        }
-    }
-    __syncthreads();
-
-    // ---- 3./4. the expert phases
-    const int P = k * I;                                     // (slot, feature) pairs
-    const int p0 = (int)((long long)P * b / G), p1 = (int)((long long)P * (b + 1) / G);
     const int d0 = (int)((long long)D * b / G), d1 = (int)((long long)D * (b + 1) / G);
     const int nd = d1 - d0;                                  // output rows of this block
     const int ND = nd > 0 ? k : 0;                           // down stages: one per slot
 
     if (warp == 0) {
-        // the copy warp: the block's down rows into the ring, from the start of the gate_up
-        // phase (they do not depend on h); stages that find no free slot before the down phase
-        // are requested into L2 first
+        // ---- 2. the copy warp selects.  It polls the E flagged logits (written by the router
+        // blocks of this launch, zero before it) and ranks them with the arithmetic of the
+        // selection kernel (select.cuh: order-preserving keys, -0.0 = +0.0, the lower index
+        // first among equal keys), so the result is the same.  After each round it publishes
+        // the slot's expert (s_idx[j], then s_nsel = j + 1) and starts the copy of that
+        // expert's down rows: the compute warps start on slot 0 while later rounds run.  The
+        // softmax weights are finished after the rounds (only the combine needs them).
+        const uint64_t t0 = globaltimer_ns();
+        float v[VPL];
+        uint32_t key[VPL];
+        uint32_t kmax = 0;
+#pragma unroll
+        for (int i = 0; i < VPL; ++i) {
+            const int e = lane + 32 * i;
+            key[i] = 0u;   // below every finite logit's key
+            v[i] = 0.f;
+            if (e < E) {
+                unsigned long long w = ld_relaxed_gpu_u64(a.lgf + e);
+                while ((w >> 32) == 0ull) {
+                    if (globaltimer_ns() - t0 > a.wait_ns) {
+                        set_error(a.err, kErrWaitGrid);
+                        break;
+                    }
+                    w = ld_relaxed_gpu_u64(a.lgf + e);
+                }
+                v[i] = __uint_as_float((uint32_t)w);
+                if (a.bias) v[i] = v[i] + __ldg(a.bias + e);
+                if (b == 0 && a.logits_out) a.logits_out[e] = v[i];
+                v[i] = v[i] + 0.0f;
+                key[i] = float_order_key(v[i]);
+                kmax = key[i] > kmax ? key[i] : kmax;
+            }
+        }
+        const float mx = float_from_order_key(__reduce_max_sync(0xffffffffu, kmax));
+        const uint32_t bytes = (uint32_t)nd * I * 2;         // rows d0..d1-1 of an expert: contiguous
+        int my_e = 0;
+        float my_l = 0.f;
+        for (int j = 0; j < k; ++j) {
+            uint32_t bk = 0;
+            int bi = 0;
+#pragma unroll
+            for (int i = 0; i < VPL; ++i)
+                if (key[i] > bk) {   // strict: the lane's lowest index among equal keys
+                    bk = key[i];
+                    bi = i;
+                }
+            const uint32_t mk = __reduce_max_sync(0xffffffffu, bk);
+            const uint32_t cand = (bk == mk && bk != 0u) ? 0xFFFFFFFFu - (uint32_t)(lane + 32 * bi) : 0u;
+            int e = (int)(0xFFFFFFFFu - __reduce_max_sync(0xffffffffu, cand));
+            if ((e & 31) == lane) {
+#pragma unroll
+                for (int i = 0; i < VPL; ++i)
+                    if (i == (e >> 5)) key[i] = 0u;
+            }
+            if (lane == j) {
+                my_e = e;
+                my_l = float_from_order_key(mk);
+            }
+            if (e < 0 || e >= E) {   // cannot happen for finite logits
+                if (lane == 0) set_error(a.err, kErrBadIndex);
+                e = 0;
+            }
+            if (lane == 0) {
+                s_idx[j] = e;
+                __threadfence_block();
+                *reinterpret_cast<volatile int*>(&s_nsel) = j + 1;
+            }
+            if (j < NS && nd > 0) {   // the first round of ring slot j: no wait for a free slot
+                if (lane == 0) mbar_arrive_expect_tx(full + j, bytes);
+                __syncwarp();
+                const uint16_t* src = a.W_dn + ((size_t)e * D + d0) * I;
+                for (int rr = lane; rr < nd; rr += 32)   // one copy per row: the padded stride
+                    bulk_load(ring + (size_t)j * L.sb + (size_t)rr * L.rs, src + (size_t)rr * I,
+                              (uint32_t)I * 2, full + j);
+            }
+        }
+        float sum = 0.f;
+#pragma unroll
+        for (int i = 0; i < VPL; ++i)
+            if (lane + 32 * i < E) sum += expf(v[i] - mx);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        const float pr = (lane < k) ? expf(my_l - mx) / sum : 0.f;   // FP32 softmax probability
+        float wv = pr;
+        if (a.norm) {
+            float tot = pr;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
+            wv = pr / tot;
+        }
+        if (lane < k) {
+            s_w[lane] = wv;
+            if (b == 0) {
+                a.idx_out[lane] = my_e;
+                a.w_out[lane] = wv;
+            }
+        }
+        __syncwarp();
+        // the down rows that find no free ring slot before the down phase: into L2 now, into
+        // the ring as the compute warps free slots
         if (lane == 0) {
-            const uint32_t bytes = (uint32_t)nd * I * 2;     // rows d0..d1-1 of an expert: contiguous
             for (int j = NS; j < ND; ++j) bulk_prefetch_l2(a.W_dn + ((size_t)s_idx[j] * D + d0) * I, bytes);
-            int issued = 0, s = 0, r = 0;                    // slot s of round r
-            for (int i = 0; i < ND; ++i) {
-                if (r > 0 && !mbar_wait(empty + s, (r - 1) & 1, a.err, kErrWaitProducer, a.wait_ns)) break;
+            int issued = ND < NS ? ND : NS, s = 0, r = 1;    // slot s of round r
+            for (int i = NS; i < ND; ++i) {
+                if (!mbar_wait(empty + s, (r - 1) & 1, a.err, kErrWaitProducer, a.wait_ns)) break;
                 mbar_arrive_expect_tx(full + s, bytes);
                 const uint16_t* src = a.W_dn + ((size_t)s_idx[i] * D + d0) * I;
-                for (int rr = 0; rr < nd; ++rr)   // one copy per row: rows land at the padded stride
+                for (int rr = 0; rr < nd; ++rr)
                     bulk_load(ring + (size_t)s * L.sb + (size_t)rr * L.rs, src + (size_t)rr * I, (uint32_t)I * 2,
                               full + s);
                 issued = i + 1;
@@ -224,28 +286,53 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_block_kernel(const Deco
             for (int i = issued > NS ? issued - NS : 0; i < issued; ++i)
                 mbar_wait(full + i % NS, (i / NS) & 1, a.err, kErrWaitTail, a.wait_ns);
         }
+        __syncwarp();
+        named_barrier_sync(2, kDecThreads);   // the combine reads s_w
         return;
     }
 
     const int cw = warp - 1;
     const int ct = threadIdx.x - 32;
-    // gate_up: warp cw takes pairs p0 + cw, p0 + cw + 8, ...  Its lanes load the pair's gate
-    // row and up row straight into registers (16-byte pieces lane, lane + 32, ...: the loads
-    // of a warp cover whole rows), the next pair's loads in flight while the current pair is
-    // computed.  (Measured on B200: the copy engine of one SM streams about 30 GB/s of
-    // 4-8 KB bulk copies, below the SM's share of HBM; the load units of 8 warps with two
-    // pairs each in flight do better, and leave the copy engine to the down rows.)
+    // ---- 3. gate_up.  The block's pairs, slot-major: for slot j the features
+    // [floor(I(bk+j)/(Gk)), floor(I((b+1)k+j)/(Gk))) taken mod I -- a share of every slot, the
+    // boundaries shifted by j/k of a block from slot to slot so that block totals stay within a
+    // few pairs of each other -- so every block starts on slot 0 while the selection goes on.  Warp cw takes the block's pairs cw, cw + 8, ...  Its lanes
+    // load the pair's gate row and up row straight into registers (16-byte pieces lane,
+    // lane + 32, ...: the loads of a warp cover whole rows), the next pair's loads in flight
+    // while the current pair is computed.  (Measured on B200: the copy engine of one SM streams
+    // about 30 GB/s of 4-8 KB bulk copies, below the SM's share of HBM; the load units of 8
+    // warps with two pairs each in flight do better, and leave the copy engine to the down rows.)
     {
-        uint4 ga[kDecChunks], ua[kDecChunks], gb[kDecChunks], ub[kDecChunks];
-        // pair p = j * I + f: slot j, feature f, advanced without divisions
-        int lj = (p0 + cw) / I, lf = (p0 + cw) - lj * I;
-        auto load_pair = [&](uint4 (&g)[kDecChunks], uint4 (&v)[kDecChunks]) {
-            const uint16_t* gr = a.W_gu + ((size_t)s_idx[lj] * 2 * I + lf) * D;
-            lf += kDecWarps;
-            if (lf >= I) {
-                lf -= I;
-                ++lj;
+        int qj = 0, qf = 0, qfe = 0;   // the warp's next pair: slot qj, feature qf (range end qfe)
+        auto slot_range = [&](int j) {   // unwrapped feature range; feature = value mod I
+            qf = (int)((long long)I * (b * k + j) / ((long long)G * k));
+            qfe = (int)((long long)I * ((b + 1) * k + j) / ((long long)G * k));
+        };
+        auto advance = [&](int n) {
+            qf += n;
+            while (qj < k && qf >= qfe) {
+                const int over = qf - qfe;
+                if (++qj < k) {
+                    slot_range(qj);
+                    qf += over;
+                }
             }
+        };
+        slot_range(0);
+        advance(cw);
+        uint4 ga[kDecChunks], ua[kDecChunks], gb[kDecChunks], ub[kDecChunks];
+        auto load_pair = [&](int j, int f, uint4 (&g)[kDecChunks], uint4 (&v)[kDecChunks]) {
+            // slot j's expert is published by the copy warp's selection round j
+            if (*reinterpret_cast<volatile int*>(&s_nsel) <= j) {
+                const uint64_t t0 = globaltimer_ns();
+                while (*reinterpret_cast<volatile int*>(&s_nsel) <= j)
+                    if (globaltimer_ns() - t0 > a.wait_ns) {
+                        set_error(a.err, kErrWaitMma);
+                        break;
+                    }
+            }
+            const int e = *reinterpret_cast<volatile int*>(&s_idx[j]);
+            const uint16_t* gr = a.W_gu + ((size_t)e * 2 * I + f) * D;
             const uint16_t* ur = gr + (size_t)I * D;
 #pragma unroll
             for (int m = 0; m < kDecChunks; ++m) {
@@ -256,7 +343,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_block_kernel(const Deco
                 }
             }
         };
-        auto finish_pair = [&](int p, const uint4 (&g)[kDecChunks], const uint4 (&v)[kDecChunks]) {
+        auto finish_pair = [&](int j, int f, const uint4 (&g)[kDecChunks], const uint4 (&v)[kDecChunks]) {
             float ag0 = 0.f, ag1 = 0.f, au0 = 0.f, au1 = 0.f;
 #pragma unroll
             for (int m = 0; m < kDecChunks; ++m) {
@@ -268,19 +355,32 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_block_kernel(const Deco
                 }
             }
             const float gs = warp_sum(ag0 + ag1), us = warp_sum(au0 + au1);
-            if (lane == 0) a.h[p] = to_bf16_bits(silu(gs) * us);   // h[slot, feature] = pair p
+            if (lane == 0) a.h[(size_t)j * I + f] = to_bf16_bits(silu(gs) * us);
         };
-        int p = p0 + cw;
-        if (p < p1) load_pair(ga, ua);
-        while (p < p1) {
-            const int pb = p + kDecWarps;
-            if (pb < p1) load_pair(gb, ub);
-            finish_pair(p, ga, ua);
-            if (pb >= p1) break;
-            const int pc = pb + kDecWarps;
-            if (pc < p1) load_pair(ga, ua);
-            finish_pair(pb, gb, ub);
-            p = pc;
+        auto fmod_i = [&](int x) { return x >= I ? x - I : x; };
+        int ja = qj, fa = fmod_i(qf);
+        bool ha = qj < k;
+        if (ha) {
+            advance(kDecWarps);
+            load_pair(ja, fa, ga, ua);
+        }
+        while (ha) {
+            const int jb = qj, fb = fmod_i(qf);
+            const bool hb = qj < k;
+            if (hb) {
+                advance(kDecWarps);
+                load_pair(jb, fb, gb, ub);
+            }
+            finish_pair(ja, fa, ga, ua);
+            if (!hb) break;
+            ja = qj;
+            fa = fmod_i(qf);
+            ha = qj < k;
+            if (ha) {
+                advance(kDecWarps);
+                load_pair(ja, fa, ga, ua);
+            }
+            finish_pair(jb, fb, gb, ub);
         }
     }
     named_barrier_sync(1, kDecWarps * 32);
@@ -352,7 +452,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_block_kernel(const Deco
             if (lane == 0) mbar_arrive(empty + s);
           }
     }
-    named_barrier_sync(1, kDecWarps * 32);
+    named_barrier_sync(2, kDecThreads);   // with the copy warp: s_w is written
     // combine: the k weighted expert outputs in slot order, then the residual
     for (int dd = ct; dd < nd; dd += kDecWarps * 32) {
         const int d = d0 + dd;
