@@ -61,6 +61,47 @@ __device__ __forceinline__ void dot8_2(const uint4& w, const float4& lo, const f
     acc1 = fmaf(bf16_hi(w.w), hi.w, acc1);
 }
 
+// Two E4M3 values (bytes 0 and 1 of `two`) as FP32, exactly (E4M3 -> fp16 -> FP32).
+__device__ __forceinline__ float2 e4m3x2_float2(uint32_t two) {
+    const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(two & 0xFFFFu), __NV_E4M3);
+    return __half22float2(*reinterpret_cast<const __half2*>(&h));
+}
+
+// Dot product of 16 E4M3 weights (byte i = value i) with 16 x values from the two FP32
+// planes (pieces 2c and 2c + 1), as two half sums.
+__device__ __forceinline__ void dot16_e4m3(const uint4& w, const float4& lo0, const float4& hi0, const float4& lo1,
+                                           const float4& hi1, float& acc0, float& acc1) {
+    float2 a = e4m3x2_float2(w.x), bq = e4m3x2_float2(w.x >> 16);
+    acc0 = fmaf(a.x, lo0.x, acc0); acc0 = fmaf(a.y, lo0.y, acc0);
+    acc0 = fmaf(bq.x, lo0.z, acc0); acc0 = fmaf(bq.y, lo0.w, acc0);
+    a = e4m3x2_float2(w.y); bq = e4m3x2_float2(w.y >> 16);
+    acc1 = fmaf(a.x, hi0.x, acc1); acc1 = fmaf(a.y, hi0.y, acc1);
+    acc1 = fmaf(bq.x, hi0.z, acc1); acc1 = fmaf(bq.y, hi0.w, acc1);
+    a = e4m3x2_float2(w.z); bq = e4m3x2_float2(w.z >> 16);
+    acc0 = fmaf(a.x, lo1.x, acc0); acc0 = fmaf(a.y, lo1.y, acc0);
+    acc0 = fmaf(bq.x, lo1.z, acc0); acc0 = fmaf(bq.y, lo1.w, acc0);
+    a = e4m3x2_float2(w.w); bq = e4m3x2_float2(w.w >> 16);
+    acc1 = fmaf(a.x, hi1.x, acc1); acc1 = fmaf(a.y, hi1.y, acc1);
+    acc1 = fmaf(bq.x, hi1.z, acc1); acc1 = fmaf(bq.y, hi1.w, acc1);
+}
+
+// Dot product of 16 E4M3 weights with 16 bf16 values (h0: values 0-7, h1: values 8-15), as
+// two half sums.
+__device__ __forceinline__ void dot16_e4m3_bf16(const uint4& w, const uint4& h0, const uint4& h1, float& acc0,
+                                                float& acc1) {
+    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+    const uint32_t hh[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const float2 a = e4m3x2_float2(ww[q]), bq = e4m3x2_float2(ww[q] >> 16);
+        float& acc = (q & 1) ? acc1 : acc0;
+        acc = fmaf(a.x, bf16_lo(hh[2 * q]), acc);
+        acc = fmaf(a.y, bf16_hi(hh[2 * q]), acc);
+        acc = fmaf(bq.x, bf16_lo(hh[2 * q + 1]), acc);
+        acc = fmaf(bq.y, bf16_hi(hh[2 * q + 1]), acc);
+    }
+}
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -71,8 +112,9 @@ constexpr int kRouterGroup = 4;   // experts whose router rows one block loads t
 
 }  // namespace
 
-// VPL: logits per lane in the selection (E <= 32 * VPL).
-template <int VPL>
+// VPL: logits per lane in the selection (E <= 32 * VPL); F8: E4M3 expert weights with FP32
+// row scales (applied to the FP32 sums) instead of bf16.
+template <int VPL, bool F8>
 __global__ void __launch_bounds__(kDecThreads, 1) decode_block_kernel(const DecodeArgs a) {
     extern __shared__ __align__(1024) uint8_t smem[];
     __shared__ int s_idx[kMaxK];
@@ -85,7 +127,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_block_kernel(const Deco
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int NS = a.stages;
     const int nd_max = (D + G - 1) / G;
-    const DecodeLayout L = decode_layout(D, k, I, nd_max, NS);
+    const DecodeLayout L = decode_layout(D, k, I, nd_max, NS, F8);
     uint8_t* ring = smem + L.ring;
     float* xs = reinterpret_cast<float*>(smem + L.xs);
     uint16_t* hs = reinterpret_cast<uint16_t*>(smem + L.hs);
@@ -200,7 +242,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_block_kernel(const Deco
             }
         }
         const float mx = float_from_order_key(__reduce_max_sync(0xffffffffu, kmax));
-        const uint32_t bytes = (uint32_t)nd * I * 2;         // rows d0..d1-1 of an expert: contiguous
+        const uint32_t bytes = (uint32_t)nd * I * (F8 ? 1 : 2);   // rows d0..d1-1 of an expert: contiguous
         int my_e = 0;
         float my_l = 0.f;
         for (int j = 0; j < k; ++j) {
@@ -236,10 +278,14 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_block_kernel(const Deco
             if (j < NS && nd > 0) {   // the first round of ring slot j: no wait for a free slot
                 if (lane == 0) mbar_arrive_expect_tx(full + j, bytes);
                 __syncwarp();
-                const uint16_t* src = a.W_dn + ((size_t)e * D + d0) * I;
-                for (int rr = lane; rr < nd; rr += 32)   // one copy per row: the padded stride
-                    bulk_load(ring + (size_t)j * L.sb + (size_t)rr * L.rs, src + (size_t)rr * I,
-                              (uint32_t)I * 2, full + j);
+                if constexpr (F8) {   // packed rows: one copy
+                    if (lane == 0) bulk_load(ring + (size_t)j * L.sb, a.W_dn8 + ((size_t)e * D + d0) * I, bytes, full + j);
+                } else {
+                    const uint16_t* src = a.W_dn + ((size_t)e * D + d0) * I;
+                    for (int rr = lane; rr < nd; rr += 32)   // one copy per row: the padded stride
+                        bulk_load(ring + (size_t)j * L.sb + (size_t)rr * L.rs, src + (size_t)rr * I,
+                                  (uint32_t)I * 2, full + j);
+                }
             }
         }
         float sum = 0.f;
@@ -267,15 +313,22 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_block_kernel(const Deco
         // the down rows that find no free ring slot before the down phase: into L2 now, into
         // the ring as the compute warps free slots
         if (lane == 0) {
-            for (int j = NS; j < ND; ++j) bulk_prefetch_l2(a.W_dn + ((size_t)s_idx[j] * D + d0) * I, bytes);
+            for (int j = NS; j < ND; ++j)
+                bulk_prefetch_l2(F8 ? (const void*)(a.W_dn8 + ((size_t)s_idx[j] * D + d0) * I)
+                                    : (const void*)(a.W_dn + ((size_t)s_idx[j] * D + d0) * I),
+                                 bytes);
             int issued = ND < NS ? ND : NS, s = 0, r = 1;    // slot s of round r
             for (int i = NS; i < ND; ++i) {
                 if (!mbar_wait(empty + s, (r - 1) & 1, a.err, kErrWaitProducer, a.wait_ns)) break;
                 mbar_arrive_expect_tx(full + s, bytes);
-                const uint16_t* src = a.W_dn + ((size_t)s_idx[i] * D + d0) * I;
-                for (int rr = 0; rr < nd; ++rr)
-                    bulk_load(ring + (size_t)s * L.sb + (size_t)rr * L.rs, src + (size_t)rr * I, (uint32_t)I * 2,
-                              full + s);
+                if constexpr (F8) {
+                    bulk_load(ring + (size_t)s * L.sb, a.W_dn8 + ((size_t)s_idx[i] * D + d0) * I, bytes, full + s);
+                } else {
+                    const uint16_t* src = a.W_dn + ((size_t)s_idx[i] * D + d0) * I;
+                    for (int rr = 0; rr < nd; ++rr)
+                        bulk_load(ring + (size_t)s * L.sb + (size_t)rr * L.rs, src + (size_t)rr * I, (uint32_t)I * 2,
+                                  full + s);
+                }
                 issued = i + 1;
                 if (++s == NS) {
                     s = 0;
@@ -320,8 +373,11 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_block_kernel(const Deco
         };
         slot_range(0);
         advance(cw);
-        uint4 ga[kDecChunks], ua[kDecChunks], gb[kDecChunks], ub[kDecChunks];
-        auto load_pair = [&](int j, int f, uint4 (&g)[kDecChunks], uint4 (&v)[kDecChunks]) {
+        // 16-byte pieces of a gate/up row per lane (a bf16 piece is 8 values, an E4M3 piece 16)
+        constexpr int NCH = F8 ? kDecChunks8 : kDecChunks;
+        const int RC = F8 ? D / 16 : DC;   // pieces of a row
+        uint4 ga[NCH], ua[NCH], gb[NCH], ub[NCH];
+        auto load_pair = [&](int j, int f, uint4 (&g)[NCH], uint4 (&v)[NCH]) {
             // slot j's expert is published by the copy warp's selection round j
             if (*reinterpret_cast<volatile int*>(&s_nsel) <= j) {
                 const uint64_t t0 = globaltimer_ns();
@@ -332,29 +388,55 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_block_kernel(const Deco
                     }
             }
             const int e = *reinterpret_cast<volatile int*>(&s_idx[j]);
-            const uint16_t* gr = a.W_gu + ((size_t)e * 2 * I + f) * D;
-            const uint16_t* ur = gr + (size_t)I * D;
+            if constexpr (F8) {   // the gate row; the up row is I rows on
+                const uint8_t* gr = a.W_gu8 + ((size_t)e * 2 * I + f) * D;
+                const uint8_t* ur = gr + (size_t)I * D;
 #pragma unroll
-            for (int m = 0; m < kDecChunks; ++m) {
-                const int c = lane + 32 * m;
-                if (c < DC) {
-                    g[m] = ld_stream_v4(gr + (size_t)c * 8);
-                    v[m] = ld_stream_v4(ur + (size_t)c * 8);
+                for (int m = 0; m < NCH; ++m) {
+                    const int c = lane + 32 * m;
+                    if (c < RC) {
+                        g[m] = ld_stream_v4(gr + (size_t)c * 16);
+                        v[m] = ld_stream_v4(ur + (size_t)c * 16);
+                    }
+                }
+            } else {
+                const uint16_t* gr = a.W_gu + ((size_t)e * 2 * I + f) * D;
+                const uint16_t* ur = gr + (size_t)I * D;
+#pragma unroll
+                for (int m = 0; m < NCH; ++m) {
+                    const int c = lane + 32 * m;
+                    if (c < RC) {
+                        g[m] = ld_stream_v4(gr + (size_t)c * 8);
+                        v[m] = ld_stream_v4(ur + (size_t)c * 8);
+                    }
                 }
             }
         };
-        auto finish_pair = [&](int j, int f, const uint4 (&g)[kDecChunks], const uint4 (&v)[kDecChunks]) {
+        auto finish_pair = [&](int j, int f, const uint4 (&g)[NCH], const uint4 (&v)[NCH]) {
             float ag0 = 0.f, ag1 = 0.f, au0 = 0.f, au1 = 0.f;
 #pragma unroll
-            for (int m = 0; m < kDecChunks; ++m) {
+            for (int m = 0; m < NCH; ++m) {
                 const int c = lane + 32 * m;
-                if (c < DC) {
-                    const float4 lo = xlo[c], hi = xhi[c];
-                    dot8_2(g[m], lo, hi, ag0, ag1);
-                    dot8_2(v[m], lo, hi, au0, au1);
+                if (c < RC) {
+                    if constexpr (F8) {   // values 16c..16c+15: x pieces 2c and 2c + 1
+                        const float4 lo0 = xlo[2 * c], hi0 = xhi[2 * c], lo1 = xlo[2 * c + 1], hi1 = xhi[2 * c + 1];
+                        dot16_e4m3(g[m], lo0, hi0, lo1, hi1, ag0, ag1);
+                        dot16_e4m3(v[m], lo0, hi0, lo1, hi1, au0, au1);
+                    } else {
+                        const float4 lo = xlo[c], hi = xhi[c];
+                        dot8_2(g[m], lo, hi, ag0, ag1);
+                        dot8_2(v[m], lo, hi, au0, au1);
+                    }
                 }
             }
-            const float gs = warp_sum(ag0 + ag1), us = warp_sum(au0 + au1);
+            float gs = warp_sum(ag0 + ag1), us = warp_sum(au0 + au1);
+            if constexpr (F8) {   // the row scales turn the sums of q * x into g and u
+                if (lane == 0) {
+                    const size_t row = (size_t)s_idx[j] * 2 * I + f;
+                    gs *= __ldg(a.gu_scale + row);
+                    us *= __ldg(a.gu_scale + row + I);
+                }
+            }
             if (lane == 0) a.h[(size_t)j * I + f] = to_bf16_bits(silu(gs) * us);
         };
         auto fmod_i = [&](int x) { return x >= I ? x - I : x; };
@@ -401,7 +483,47 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_block_kernel(const Deco
     // (16-row tiles x I x one column): warp MMAs m16n8k16 with the rows as A (ldmatrix from
     // the padded stage) and h_i as column 0 of B (lanes 0-3 hold it, the other columns are 0),
     // FP32 accumulators in four chains over K; column 0 of D is in lanes 0, 4, ..., 28.
-    {
+    if constexpr (F8) {
+        // E4M3 rows (packed, I bytes each) times h_i on CUDA cores: rows four at a time, lanes
+        // 8g..8g+7 on row g + 4q, lane 8g + l8 the 16-byte pieces l8, l8 + 8, ... (16 values
+        // each), then the row scale.  The expert of each slot is read once the selection has
+        // published all k (it has long finished by now).
+        {
+            const uint64_t t0 = globaltimer_ns();
+            while (*reinterpret_cast<volatile int*>(&s_nsel) < k)
+                if (globaltimer_ns() - t0 > a.wait_ns) {
+                    set_error(a.err, kErrWaitMma);
+                    break;
+                }
+        }
+        const int g = lane >> 3, l8 = lane & 7;
+        const int PC = I / 16;
+        bool ok = true;
+        for (int s = cw; s < NS && ok; s += kDecWarps)
+            for (int i = s, r = 0; i < ND; i += NS, ++r) {
+                if (!mbar_wait(full + s, r & 1, a.err, kErrWaitMma, a.wait_ns)) {
+                    ok = false;
+                    break;
+                }
+                const uint4* hrow = reinterpret_cast<const uint4*>(hs + (size_t)i * I);
+                const float* sc = a.dn_scale + (size_t)(*reinterpret_cast<volatile int*>(&s_idx[i])) * D + d0;
+                for (int q = 0; q * 4 < nd; ++q) {
+                    const int rr = q * 4 + g;
+                    float acc0 = 0.f, acc1 = 0.f;
+                    if (rr < nd) {
+                        const uint4* wr = reinterpret_cast<const uint4*>(ring + (size_t)s * L.sb + (size_t)rr * L.rs);
+                        for (int c = l8; c < PC; c += 8) dot16_e4m3_bf16(wr[c], hrow[2 * c], hrow[2 * c + 1], acc0, acc1);
+                    }
+                    float v = acc0 + acc1;
+                    v += __shfl_xor_sync(0xffffffffu, v, 4);
+                    v += __shfl_xor_sync(0xffffffffu, v, 2);
+                    v += __shfl_xor_sync(0xffffffffu, v, 1);
+                    if (rr < nd && l8 == 0) val[(size_t)i * nd_max + rr] = v * __ldg(sc + rr);
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(empty + s);
+            }
+    } else {
         const int grp = lane >> 2, tig = lane & 3;
         const int arow = (lane & 7) + ((lane >> 3) & 1) * 8;   // ldmatrix: this lane's row
         const int akof = (lane >> 4) * 16;                     // and its 16-byte half of the k step
@@ -471,11 +593,11 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_block_kernel(const Deco
     }
 }
 
-int decode_stages(int T, int D, int E, int k, int I, int blocks) {
+int decode_stages(int T, int D, int E, int k, int I, int blocks, bool f8) {
     if (T != 1 || k > kMaxK || D > kDecMaxD || blocks < 1) return 0;
     if (D % 64 != 0 || I % 16 != 0 || E > 512) return 0;
     const int nd_max = (D + blocks - 1) / blocks;
-    const DecodeLayout fixed = decode_layout(D, k, I, nd_max, 0);
+    const DecodeLayout fixed = decode_layout(D, k, I, nd_max, 0, f8);
     const long long room = (long long)kDecSmemBudget - (long long)fixed.total;
     const long long per = (long long)fixed.sb + 16;   // a stage and its two barriers
     long long st = room > 0 ? room / per : 0;
@@ -483,11 +605,11 @@ int decode_stages(int T, int D, int E, int k, int I, int blocks) {
     return st >= kDecMinStages ? (int)st : 0;
 }
 
-template <int VPL>
+template <int VPL, bool F8>
 static cudaError_t launch_decode_t(const DecodeArgs& a, int blocks, bool pdl, cudaStream_t s) {
     const int nd_max = (a.D + blocks - 1) / blocks;
-    const size_t smem = decode_layout(a.D, a.k, a.I, nd_max, a.stages).total;
-    auto kern = decode_block_kernel<VPL>;
+    const size_t smem = decode_layout(a.D, a.k, a.I, nd_max, a.stages, F8).total;
+    auto kern = decode_block_kernel<VPL, F8>;
     cudaError_t e = ensure_smem_attr((const void*)kern, (int)smem);
     if (e != cudaSuccess) return e;
     return launch_kernel(kern, dim3(blocks), dim3(kDecThreads), smem, s, pdl, a);
@@ -495,9 +617,14 @@ static cudaError_t launch_decode_t(const DecodeArgs& a, int blocks, bool pdl, cu
 
 cudaError_t launch_decode(const DecodeArgs& a, int blocks, bool pdl, cudaStream_t s) {
     if (a.stages < kDecMinStages) return cudaErrorInvalidValue;
-    if (a.E <= 128) return launch_decode_t<4>(a, blocks, pdl, s);
-    if (a.E <= 256) return launch_decode_t<8>(a, blocks, pdl, s);
-    return launch_decode_t<16>(a, blocks, pdl, s);
+    if (a.W_gu8) {
+        if (a.E <= 128) return launch_decode_t<4, true>(a, blocks, pdl, s);
+        if (a.E <= 256) return launch_decode_t<8, true>(a, blocks, pdl, s);
+        return launch_decode_t<16, true>(a, blocks, pdl, s);
+    }
+    if (a.E <= 128) return launch_decode_t<4, false>(a, blocks, pdl, s);
+    if (a.E <= 256) return launch_decode_t<8, false>(a, blocks, pdl, s);
+    return launch_decode_t<16, false>(a, blocks, pdl, s);
 }
 
 }  // namespace moe

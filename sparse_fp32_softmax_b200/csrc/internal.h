@@ -241,22 +241,23 @@ constexpr int kDecMaxStages = 32;
 constexpr int kDecMinStages = 2;
 constexpr int kDecSmemBudget = 220 * 1024;   // dynamic shared memory per block
 constexpr int kDecMaxD = 2048;         // a gate/up row is at most 8 16-byte pieces per lane
-constexpr int kDecChunks = kDecMaxD / 256;
+constexpr int kDecChunks = kDecMaxD / 256;      // 16-byte pieces of a bf16 gate/up row per lane
+constexpr int kDecChunks8 = kDecMaxD / 512;     // the same for an E4M3 row
 
 // Shared-memory layout of a decode block: the copy ring (a stage holds one expert's down
-// rows for the block's output rows: nd_max rows of I, padded to whole 16-row MMA tiles, each
-// row at a stride of 2I + 16 bytes so that the 8 rows an ldmatrix reads fall in distinct
-// banks), x as FP32 in two planes, h of every slot, the down results of the block's output
-// rows, then the ring's barriers.
+// rows for the block's output rows: nd_max rows of I; bf16 rows padded to whole 16-row MMA
+// tiles, each row at a stride of 2I + 16 bytes so that the 8 rows an ldmatrix reads fall in
+// distinct banks; E4M3 rows packed at a stride of I bytes), x as FP32 in two planes, h of every
+// slot, the down results of the block's output rows, then the ring's barriers.
 struct DecodeLayout {
     int stages, nd_max, rs;
     size_t sb, ring, xs, hs, val, bars, total;
 };
-__host__ __device__ inline DecodeLayout decode_layout(int D, int k, int I, int nd_max, int stages) {
+__host__ __device__ inline DecodeLayout decode_layout(int D, int k, int I, int nd_max, int stages, bool f8) {
     DecodeLayout L;
     L.stages = stages;
-    L.rs = 2 * I + 16;
-    L.sb = ((size_t)((nd_max + 15) / 16) * 16 * L.rs + 127) / 128 * 128;
+    L.rs = f8 ? I : 2 * I + 16;
+    L.sb = ((f8 ? (size_t)nd_max * L.rs : (size_t)((nd_max + 15) / 16) * 16 * L.rs) + 127) / 128 * 128;
     L.nd_max = nd_max;
     size_t off = 0;
     L.ring = off;
@@ -277,8 +278,12 @@ struct DecodeArgs {
     const uint16_t* x;        // [D]
     const uint16_t* W_r;      // [E, D]
     const float* bias;        // [E] or null
-    const uint16_t* W_gu;     // [E, 2I, D]
+    const uint16_t* W_gu;     // [E, 2I, D] (bf16 weights)
     const uint16_t* W_dn;     // [E, D, I]
+    const uint8_t* W_gu8;     // [E, 2I, D] E4M3, or null (then the bf16 weights above)
+    const uint8_t* W_dn8;     // [E, D, I] E4M3
+    const float* gu_scale;    // [E * 2I] FP32 row scales of W_gu8
+    const float* dn_scale;    // [E * D]
     const uint16_t* residual; // [D] or null (may alias out)
     uint16_t* out;            // [D]
     float* out_f32;           // [D] or null
@@ -298,7 +303,7 @@ struct DecodeArgs {
 
 // Ring depth for this shape on a grid of `blocks` blocks, or 0 when the decode kernel does
 // not apply (T != 1, D or I too wide for its buffers).
-int decode_stages(int T, int D, int E, int k, int I, int blocks);
+int decode_stages(int T, int D, int E, int k, int I, int blocks, bool f8);
 cudaError_t launch_decode(const DecodeArgs& a, int blocks, bool pdl, cudaStream_t s);
 
 }  // namespace moe

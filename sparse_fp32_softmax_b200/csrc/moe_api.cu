@@ -174,13 +174,13 @@ moe_status check_opts(const moe_dims* d, const moe_opts* o) {
 }
 
 // Ring depth of the decode kernel for this call on `sms` blocks, 0 when it does not apply:
-// more than one token, or a feature it does not implement (shared expert, FP8
-// experts, the permutation outputs, the grouped path's diagnostic).
+// more than one token, or a feature it does not implement (shared expert, the
+// permutation outputs, the grouped path's diagnostic).
 int decode_stages_for(const moe_dims& d, const moe_opts* o, int sms) {
-    if (o && (o->shared_gate_up || o->W_gate_up_fp8 || o->expert_counts_out || o->slot_row_out ||
+    if (o && (o->shared_gate_up || o->expert_counts_out || o->slot_row_out ||
               o->diag == MOE_DIAG_UNSIGNALLED_HANDOFF))
         return 0;
-    return decode_stages(d.T, d.D, d.E, d.k, d.I, sms);
+    return decode_stages(d.T, d.D, d.E, d.k, d.I, sms, o && o->W_gate_up_fp8);
 }
 
 // The path moe_forward_ex takes (arguments already checked).
@@ -485,6 +485,10 @@ moe_status moe_forward_ex(const moe_bf16* x, const moe_bf16* W_r, const moe_bf16
         if ((st = record(opts, 0, s)) != MOE_OK) return st;
         DecodeArgs da{};
         da.x = x; da.W_r = W_r; da.bias = bias; da.W_gu = W_gate_up; da.W_dn = W_down;
+        if (f8) {
+            da.W_gu8 = opts->W_gate_up_fp8; da.W_dn8 = opts->W_down_fp8;
+            da.gu_scale = opts->gate_up_scale; da.dn_scale = opts->down_scale;
+        }
         da.residual = residual; da.out = out; da.out_f32 = out_f32;
         da.logits_out = logits_user; da.idx_out = idx; da.w_out = w;
         da.lgf = reinterpret_cast<unsigned long long*>(at<char>(ws, p.err) + kAlign);

@@ -6,6 +6,8 @@
 * moe_forward_ex with FP8 experts: routing as in the bf16 tests (the router stays bf16);
   the output against the oracle evaluating the definition with the dequantised weights
   (weight = scale[row] * value(q)), with the block's output criterion.
+* One token runs on the one-token kernel with FP8 weights: against the oracle (the sweep's
+  T=1) and against the grouped FP8 path on the same token.
 * The cases the FP8 path refuses (a shared expert, wider batches) return MOE_ERR_UNSUPPORTED.
 """
 import numpy as np
@@ -15,7 +17,7 @@ import torch
 from oracle import oracle as O
 from sparse_fp32_softmax_b200 import binding as B
 from sparse_fp32_softmax_b200 import inputs
-from tests.parity_util import W_ATOL, assert_block_output, check_routing, logit_deltas
+from tests.parity_util import W_ATOL, assert_block_output, assert_y_close, check_routing, logit_deltas
 
 pytestmark = pytest.mark.gpu
 
@@ -141,3 +143,22 @@ def test_fp8_refused_where_unsupported():
         B.moe_forward_ex(G["x"][:4].contiguous(), G["W_r"], G["W_gate_up"], G["W_down"], cfg.k, True,
                          ws=ws, W_gate_up_fp8=F["W_gate_up_fp8"])
     assert e.value.status == B.MOE_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("t", [0, 5])
+def test_fp8_one_token_kernel_matches_grouped(t):
+    """One token goes through the one-token kernel (AUTO's choice); the grouped FP8 path on the
+    same token gives the same routing bit for bit and the output within the tolerance."""
+    cfg, L, G, F = decode_fp8()
+    x = G["x"][t:t + 1].contiguous()
+    assert B.moe_forward_path(B.make_dims(1, cfg.D, cfg.E, cfg.k, cfg.I), B.make_opts(**F)) == "decode"
+    outs = {}
+    for path in ("decode", "grouped"):
+        idx = torch.empty(1, cfg.k, dtype=torch.int32, device="cuda")
+        w = torch.empty(1, cfg.k, dtype=torch.float32, device="cuda")
+        y = B.moe_forward_ex(x, G["W_r"], None, None, cfg.k, cfg.norm_topk_prob, topk_idx_out=idx,
+                             topk_w_out=w, path=path, **F)
+        torch.cuda.synchronize()
+        outs[path] = (y.cpu(), idx.cpu().numpy(), w.cpu().numpy())
+    assert (outs["decode"][1] == outs["grouped"][1]).all() and (outs["decode"][2] == outs["grouped"][2]).all()
+    assert_y_close(outs["decode"][0].double().numpy(), outs["grouped"][0].double().numpy(), f"fp8 token {t}")
