@@ -457,7 +457,7 @@ def measure(name, args, rank, world, device, peaks, with_e2e):
         roof_dn = dominant(dn_roofs, "tc_gemm_kernel<down>")
     tag = {"decode": "tc_gate_up_decode", "prefill": "tc_gemm_prefill"}.get(name, f"tc_gate_up_{name}")
     if passes[-1]["path"] == "decode":
-        tag = "decode_block_t1"
+        tag = "decode_block_t1_fp8" if spec.get("fp8") else "decode_block_t1"
     roof["traffic"] = profile_traffic(tag)
     blk_time = max(blk_bytes / (hbm * 1e9), blk_flops / (tf_peak * 1e12))
     res = dict(
