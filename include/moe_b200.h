@@ -73,13 +73,14 @@ enum {
                              MOE_PATH_GROUPED (moe_forward_path tells which) */
     MOE_PATH_GROUPED = 1, /* permute + tcgen05 grouped GEMMs, TMA-fed, TMEM accumulators */
     MOE_PATH_DECODE = 2   /* the whole block in one kernel for one token (T = 1, D <= 2048,
-                             I <= 1536, and two blocks of ceil(D / SMs) down rows of I fit in
-                             an SM's shared memory beside its buffers): one block per SM, all resident
-                             at once (a call needs the whole GPU; other work running on it
-                             delays the call, up to the wait limit, after which it reports
-                             MOE_ERR_DEVICE_TIMEOUT).  Not with a shared expert, FP8 experts,
-                             expert_counts_out, slot_row_out or MOE_DIAG_UNSIGNALLED_HANDOFF;
-                             asking for it then returns MOE_ERR_UNSUPPORTED */
+                             and two blocks of ceil(D / SMs) down rows of I fit in an SM's
+                             shared memory beside its buffers), bf16 or FP8 experts: one
+                             block per SM, all resident at once (a call needs the whole GPU;
+                             other work running on it delays the call, up to the wait limit,
+                             after which it reports MOE_ERR_DEVICE_TIMEOUT).  Not with a
+                             shared expert, expert_counts_out, slot_row_out or
+                             MOE_DIAG_UNSIGNALLED_HANDOFF; asking for it then returns
+                             MOE_ERR_UNSUPPORTED */
 };
 
 /* Diagnostics of moe_forward_ex (moe_opts.diag); 0 in normal use. */
@@ -130,9 +131,10 @@ typedef struct {
      * as written by moe_quantize_fp8_rows) with one FP32 scale per weight row,
      * gate_up_scale [E * 2I] and down_scale [E * D]; weight (e, r, c) = scale[e, r] *
      * value(q[e, r, c]).  The bf16 W_gate_up and W_down arguments are then not read and may
-     * be NULL.  Tokens stay bf16; each weight tile is widened to bf16 exactly in shared
-     * memory and the row scale is applied to the FP32 accumulator.  Supported at decode
-     * shapes (T*k <= 32*E) without a shared expert; otherwise MOE_ERR_UNSUPPORTED. */
+     * be NULL.  Tokens stay bf16; the weights are widened exactly (to bf16 in shared memory on
+     * the grouped path, to FP32 in registers on the one-token kernel) and the row scale is
+     * applied to the FP32 sums.  Supported at decode shapes (T*k <= 32*E) without a shared
+     * expert; otherwise MOE_ERR_UNSUPPORTED. */
     const uint8_t *W_gate_up_fp8;    /* [E, 2I, D] E4M3, or NULL (bf16 weights) */
     const float *gate_up_scale;      /* [E * 2I] FP32 */
     const uint8_t *W_down_fp8;       /* [E, D, I] E4M3 */
