@@ -444,3 +444,55 @@ int oracle_combine_rows_fp8(const uint16_t *x, const int32_t *idx, const float *
     free(o);
     return 0;
 }
+
+/* ---------------------------------------------------------------- Switch balance loss
+ *
+ * "Qwen3-VL and Mixture of Experts" (gopikrishnatummala.com), the list of fixes for expert
+ * collapse, "An auxiliary balance loss": L = alpha * N * sum_i f_i P_i over the N experts,
+ * f_i the fraction of tokens sent to expert i and P_i the router's average probability for
+ * it.  The Qwen3-VL MoE walk-through (agent.csdn.net), "load_balancing_loss_func": the
+ * probabilities are the softmax of the gate logits, f comes from the one-hot of the top-k
+ * selection averaged over tokens (so each token adds 1/T for each of its k experts:
+ * f_i = count_i / T), P_i is the mean probability over tokens, and the sum of their products
+ * is multiplied by the number of experts.
+ * Reading taken: alpha is the caller's coefficient; the selection is the given top-k
+ * (the forward's); the gradient treats f as a constant (the selection is not
+ * differentiable): dL/dl[t, e] = alpha * N / T * p[t, e] * (f_e - sum_i f_i p[t, i]).
+ * Everything in double from the FP32 logits. */
+int oracle_aux_loss(const float *logits, const int32_t *idx, int T, int E, int k, double alpha,
+                    double *loss, double *dlogits) {
+    if (T < 1 || E < 1 || k < 1) return 1;
+    double *f = (double *)calloc((size_t)E, sizeof(double));
+    double *P = (double *)calloc((size_t)E, sizeof(double));
+    double *p = (double *)malloc((size_t)E * sizeof(double));
+    if (!f || !P || !p) { free(f); free(P); free(p); return 1; }
+    for (int t = 0; t < T; ++t) {
+        for (int j = 0; j < k; ++j) {
+            int e = idx[(size_t)t * k + j];
+            if (e < 0 || e >= E) { free(f); free(P); free(p); return 1; }
+            f[e] += 1.0;
+        }
+        softmax_row(logits + (size_t)t * E, E, p);
+        for (int e = 0; e < E; ++e) P[e] += p[e];
+    }
+    double sum = 0.0;
+    for (int e = 0; e < E; ++e) {
+        f[e] /= (double)T;
+        P[e] /= (double)T;
+        sum += f[e] * P[e];
+    }
+    *loss = alpha * (double)E * sum;
+    if (dlogits) {
+        const double c = alpha * (double)E / (double)T;
+        for (int t = 0; t < T; ++t) {
+            softmax_row(logits + (size_t)t * E, E, p);
+            double q = 0.0;
+            for (int i = 0; i < E; ++i) q += f[i] * p[i];
+            for (int e = 0; e < E; ++e) dlogits[(size_t)t * E + e] = c * p[e] * (f[e] - q);
+        }
+    }
+    free(f);
+    free(P);
+    free(p);
+    return 0;
+}

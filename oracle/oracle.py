@@ -66,6 +66,8 @@ def lib():
                                               _f32p]
             l.oracle_loop_dispatch.argtypes = [_u16p, _i32p, _f32p, c_int, c_int, c_int, c_int,
                                                c_int, _u16p, _u16p, _f64p]
+            l.oracle_aux_loss.argtypes = [_f32p, _i32p, c_int, c_int, c_int, ctypes.c_double,
+                                          ctypes.POINTER(ctypes.c_double), ctypes.c_void_p]
             l.oracle_e4m3_value.argtypes = [ctypes.c_uint8]
             l.oracle_e4m3_value.restype = ctypes.c_double
             l.oracle_quantize_fp8_rows.argtypes = [_u16p, ctypes.c_long, c_int, _u8p, _f32p]
@@ -283,6 +285,20 @@ def combine_rows_fp8(x, idx, w, rows, q_gu, s_gu, q_dn, s_dn, residual=None, thr
     with ThreadPoolExecutor(max_workers=len(parts)) as ex:
         list(ex.map(run, range(len(parts))))
     return np.concatenate(outs, axis=0) if outs else np.empty((0, D))
+
+
+def aux_loss(logits, idx, alpha=1.0, with_grad=True):
+    """Switch balance loss alpha * E * sum_e f_e P_e and (f fixed) its gradient with respect to
+    the logits, in double (see oracle_aux_loss).  -> (loss, dlogits [T, E] float64 or None)."""
+    lg = _f32(logits)
+    ix = _i32(idx)
+    T, E = lg.shape
+    k = ix.shape[1]
+    loss = ctypes.c_double(0.0)
+    d = np.zeros((T, E), np.float64) if with_grad else None
+    _check(lib().oracle_aux_loss(_p(lg, _f32p), _p(ix, _i32p), T, E, k, float(alpha), ctypes.byref(loss),
+                                 d.ctypes.data_as(ctypes.c_void_p) if d is not None else None), "oracle_aux_loss")
+    return loss.value, d
 
 
 def cpu_threads_available() -> int:

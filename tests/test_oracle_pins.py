@@ -360,3 +360,63 @@ def test_fp8_experts_equal_bf16_experts_on_exact_weights(oracle_mod):
     y8 = oracle_mod.combine_rows_fp8(x, idx, w, rows, q_gu, s_gu, q_dn, s_dn)
     y16 = oracle_mod.combine_rows(x, idx, w, rows, W_gu, W_dn)
     assert np.array_equal(y8, y16)
+
+
+# ------------------------------------------------------------------ Switch balance loss
+# "Qwen3-VL and Mixture of Experts", "An auxiliary balance loss": L = alpha N sum_i f_i P_i;
+# the Qwen3-VL MoE walk-through's load_balancing_loss_func: f from the top-k one-hot averaged
+# over tokens, P the mean softmax probability, times the number of experts.
+
+def test_aux_loss_uniform_logits_give_alpha_k(oracle_mod):
+    """Equal logits make every P_i = 1/N, so L = alpha * sum_i f_i = alpha * k for ANY routing."""
+    rng = np.random.default_rng(3)
+    T, E, k, alpha = 37, 12, 3, 0.01
+    logits = np.full((T, E), 0.75, np.float32)
+    idx = np.stack([rng.permutation(E)[:k] for _ in range(T)]).astype(np.int32)
+    loss, _ = oracle_mod.aux_loss(logits, idx, alpha)
+    assert abs(loss - alpha * k) <= 1e-15
+
+
+def test_aux_loss_balanced_routing_gives_alpha_k(oracle_mod):
+    """Every expert chosen equally often (f_i = k / N) makes L = alpha * k * sum_i P_i = alpha * k
+    for ANY logits."""
+    rng = np.random.default_rng(4)
+    E, k = 8, 2
+    T = E * 5
+    logits = rng.normal(0, 3, (T, E)).astype(np.float32)
+    idx = np.array([[(t + j) % E for j in range(k)] for t in range(T)], np.int32)   # each expert 2*5 times
+    loss, _ = oracle_mod.aux_loss(logits, idx, 0.5)
+    assert abs(loss - 0.5 * k) <= 1e-12
+
+
+def test_aux_loss_collapse_closed_form(oracle_mod):
+    """N = 2, k = 1, every token sent to expert 0 with logits (l, 0): f = (1, 0), P_0 =
+    sigmoid(l), so L = alpha * 2 * sigmoid(l)."""
+    l, T, alpha = 1.25, 9, 0.3
+    logits = np.tile(np.array([[l, 0.0]], np.float32), (T, 1))
+    idx = np.zeros((T, 1), np.int32)
+    loss, d = oracle_mod.aux_loss(logits, idx, alpha)
+    sig = 1.0 / (1.0 + math.exp(-float(np.float32(l))))
+    assert abs(loss - alpha * 2 * sig) <= 1e-14
+    # dL/dl_0 of each token: alpha * 2 / T * sigmoid' (f_0 - f_1 = 1)
+    assert np.allclose(d[:, 0], alpha * 2 / T * sig * (1 - sig), rtol=0, atol=1e-15)
+
+
+def test_aux_loss_gradient_matches_finite_differences(oracle_mod):
+    """dL/dlogits (selection held fixed) against central differences of the loss."""
+    rng = np.random.default_rng(5)
+    T, E, k, alpha = 3, 5, 2, 0.7
+    logits = rng.normal(0, 1, (T, E)).astype(np.float32)
+    idx = np.stack([rng.permutation(E)[:k] for _ in range(T)]).astype(np.int32)
+    _, d = oracle_mod.aux_loss(logits, idx, alpha)
+    h = 2.0 ** -8   # exact in FP32 around values of order 1
+    for t in range(T):
+        for e in range(E):
+            lp, lm = logits.copy(), logits.copy()
+            lp[t, e] += h
+            lm[t, e] -= h
+            fd = (oracle_mod.aux_loss(lp, idx, alpha, False)[0] - oracle_mod.aux_loss(lm, idx, alpha, False)[0]) / (
+                float(lp[t, e]) - float(lm[t, e]))
+            assert abs(fd - d[t, e]) <= 2e-6, (t, e, fd, d[t, e])
+    # each token's gradient sums to zero (a softmax is shift-invariant)
+    assert np.abs(d.sum(axis=1)).max() <= 1e-15
