@@ -484,6 +484,37 @@ def measure(name, args, rank, world, device, peaks, with_e2e):
     if sweep_out:
         res["sweep"] = sweep_out
 
+    # the router's balance loss and its gradient on this workload's own routing (prefill):
+    # one moe_aux_loss call per step, CUDA events around a graph of K calls
+    if name == "prefill":
+        p = passes[-1]
+        w = p["w"]
+        logits, idx, _ = B.moe_route(p["x"], w["W_r"], cfg.k, cfg.norm_topk_prob, bias=w.get("bias"))
+        aux_ws = torch.empty(int(B.load().moe_aux_loss_workspace_size(p["T"], cfg.E)), dtype=torch.uint8, device=device)
+        for _ in range(3):
+            B.moe_aux_loss(logits, idx, 0.001, ws=aux_ws)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=torch.cuda.Stream(device=device)):
+            for _ in range(K):
+                B.moe_aux_loss(logits, idx, 0.001, ws=aux_ws)
+        g.replay()
+        torch.cuda.synchronize()
+        a_ev, b_ev = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a_ev.record()
+        g.replay()
+        b_ev.record()
+        torch.cuda.synchronize()
+        us = a_ev.elapsed_time(b_ev) * 1e3 / K
+        # logits read twice (statistics, gradient), indices once, the gradient written once
+        nbytes = 3 * p["T"] * cfg.E * 4 + p["T"] * cfg.k * 4
+        res["aux_loss"] = dict(us_per_call=round(us, 2), kernels=3, algorithmic_bytes=nbytes,
+                               achieved_gbs=round(nbytes / (us * 1e-6) / 1e9, 1),
+                               hbm_frac=round(nbytes / (us * 1e-6) / 1e9 / hbm, 4),
+                               note="loss and gradient of the Switch balance loss, T=%d, E=%d, k=%d" % (
+                                   p["T"], cfg.E, cfg.k))
+        del g
+
     # end to end through the public API with host buffers (eager, copies inside the region)
     if with_e2e and not chain:
         hx = [p["x"].cpu().pin_memory() for p in passes]
@@ -647,6 +678,8 @@ def main(argv=None):
         stages_us_with_events=res["stages_us_with_events"])
     if "sweep" in res:
         line["sweep"] = res["sweep"]
+    if "aux_loss" in res:
+        line["aux_loss"] = res["aux_loss"]
     if want_cpu:
         line["cpu_baseline"] = cpu_baseline(cfg, L_cpu, layers=WORKLOADS[args.workload]["layers"])
     del L_cpu

@@ -153,6 +153,24 @@ typedef struct {
 moe_status moe_quantize_fp8_rows(const moe_bf16 *W, int64_t rows, int cols, uint8_t *q, float *scale,
                                  moe_stream_t stream);
 
+/* The Switch balance loss of the router ("Qwen3-VL and Mixture of Experts", the fixes for
+ * expert collapse, "An auxiliary balance loss"; the Qwen3-VL MoE walk-through,
+ * "load_balancing_loss_func") and its gradient with respect to the router logits:
+ *   p[t]   = softmax(logits[t]) in FP32;  P_e = (1/T) sum_t p[t, e];
+ *   f_e    = (1/T) * number of (t, j) with topk_idx[t, j] == e  (entries outside [0, E) are
+ *            not counted);
+ *   loss   = alpha * E * sum_e f_e P_e;
+ *   dlogits[t, e] = alpha * E / T * p[t, e] * (f_e - sum_i f_i p[t, i])  (f held fixed: the
+ *            selection is not differentiable).
+ * logits [T, E] FP32 (as moe_route returns them, bias included when one was given), topk_idx
+ * [T, k] int32, loss: one FP32 value in device memory, dlogits [T, E] FP32 or NULL (loss only).
+ * Workspace of moe_aux_loss_workspace_size(T, E) bytes, 256-byte aligned.  All sums run in a
+ * fixed order: bitwise reproducible.  1 <= E <= 512, 1 <= k <= min(E, 16); enqueued on
+ * `stream`. */
+size_t moe_aux_loss_workspace_size(int T, int E);
+moe_status moe_aux_loss(const float *logits, const int32_t *topk_idx, int T, int E, int k, float alpha,
+                        float *loss, float *dlogits, void *ws, size_t ws_bytes, moe_stream_t stream);
+
 /* Bytes of workspace that moe_route, moe_permute and moe_forward(_ex) need for `dims`
  * (and `opts`, which may be NULL).  Returns 0 for invalid or unsupported arguments. */
 size_t moe_workspace_size(const moe_dims *dims, const moe_opts *opts);

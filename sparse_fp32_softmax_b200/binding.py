@@ -76,9 +76,12 @@ def load():
         lib.moe_last_cuda_error.restype = _c_int
         lib.moe_quantize_fp8_rows.argtypes = [_vp, ctypes.c_int64, _c_int, _vp, _vp, _vp]
         lib.moe_forward_path.argtypes = [dp, op, ctypes.POINTER(_c_int)]
+        lib.moe_aux_loss_workspace_size.argtypes = [_c_int, _c_int]
+        lib.moe_aux_loss_workspace_size.restype = _sz
+        lib.moe_aux_loss.argtypes = [_vp, _vp, _c_int, _c_int, _c_int, ctypes.c_float, _vp, _vp, _vp, _sz, _vp]
         for n in ("moe_route", "moe_permute", "moe_forward", "moe_forward_ex", "moe_forward_noalloc",
                   "moe_get_device_status", "moe_get_device_status_noalloc", "moe_quantize_fp8_rows",
-                  "moe_forward_path"):
+                  "moe_forward_path", "moe_aux_loss"):
             getattr(lib, n).restype = _c_int
         _lib = lib
     return _lib
@@ -179,6 +182,26 @@ def moe_forward_path(dims: moe_dims, opts: moe_opts | None = None) -> str:
     _check(load().moe_forward_path(ctypes.byref(dims), ctypes.byref(opts) if opts else None, ctypes.byref(out)),
            "moe_forward_path")
     return {MOE_PATH_DECODE: "decode", MOE_PATH_GROUPED: "grouped"}[out.value]
+
+
+def moe_aux_loss(logits, topk_idx, alpha=1.0, with_grad=True, ws=None, stream=None):
+    """Switch balance loss (and its gradient with respect to the logits) -> (loss [1] f32,
+    dlogits [T, E] f32 or None)."""
+    _need(logits, "logits", torch.float32, 2)
+    _need(topk_idx, "topk_idx", torch.int32, 2)
+    T, E = logits.shape
+    k = topk_idx.shape[1]
+    lib = load()
+    n = int(lib.moe_aux_loss_workspace_size(T, E))
+    if n == 0:
+        raise MoeError(MOE_ERR_UNSUPPORTED, "moe_aux_loss_workspace_size")
+    if ws is None:
+        ws = torch.empty(n, dtype=torch.uint8, device=logits.device)
+    loss = torch.empty(1, dtype=torch.float32, device=logits.device)
+    d = torch.empty(T, E, dtype=torch.float32, device=logits.device) if with_grad else None
+    _check(lib.moe_aux_loss(_ptr(logits), _ptr(topk_idx), T, E, k, float(alpha), _ptr(loss), _ptr(d), _ptr(ws),
+                            ws.numel(), _stream(stream)), "moe_aux_loss")
+    return loss, d
 
 
 def workspace(dims: moe_dims, opts: moe_opts | None = None, device=None) -> torch.Tensor:

@@ -28,7 +28,8 @@ def test_library_exports_every_declared_function(lib):
     assert set(declared) == {"moe_workspace_size", "moe_route", "moe_permute", "moe_forward",
                              "moe_forward_ex", "moe_forward_noalloc", "moe_get_device_status",
                              "moe_get_device_status_noalloc", "moe_status_string", "moe_last_cuda_error",
-                             "moe_quantize_fp8_rows", "moe_forward_path"}
+                             "moe_quantize_fp8_rows", "moe_forward_path", "moe_aux_loss",
+                             "moe_aux_loss_workspace_size"}
     out = subprocess.run(["nm", "-D", "--defined-only", LIB], capture_output=True, text=True, check=True).stdout
     exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
     for name in declared:
@@ -161,3 +162,21 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(B, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError, match="missing"):
         B.load()
+
+
+@no_gpu
+def test_aux_loss_validation_without_a_device(lib):
+    """moe_aux_loss validates before enqueuing; with valid arguments and no GPU it reports a
+    CUDA failure (no host fallback)."""
+    p = ctypes.c_void_p
+    n = lib.moe_aux_loss_workspace_size(64, 8)
+    assert n > 0 and lib.moe_aux_loss_workspace_size(64, 513) == 0
+    args = lambda T=64, E=8, k=2, ws=FAKE, nb=n, lg=FAKE: (p(lg), p(FAKE), T, E, k, ctypes.c_float(0.01), p(FAKE),
+                                                          None, p(ws), nb, None)
+    assert lib.moe_aux_loss(*args(T=0)) == B.MOE_ERR_INVALID_ARG
+    assert lib.moe_aux_loss(*args(k=9)) == B.MOE_ERR_UNSUPPORTED
+    assert lib.moe_aux_loss(*args(E=513)) == B.MOE_ERR_UNSUPPORTED
+    assert lib.moe_aux_loss(*args(lg=0)) == B.MOE_ERR_INVALID_ARG
+    assert lib.moe_aux_loss(*args(ws=FAKE + 16)) == B.MOE_ERR_INVALID_ARG
+    assert lib.moe_aux_loss(*args(nb=n - 4)) == B.MOE_ERR_WORKSPACE
+    assert lib.moe_aux_loss(*args()) == B.MOE_ERR_CUDA
