@@ -1,6 +1,7 @@
 /*
  * moe_oracle.c -- plain, slow, single-threaded CPU oracle for the forward pass of a
- * Qwen-family sparse MoE FFN block.
+ * Qwen-family sparse MoE FFN block (and, for the training-side entry points, the Switch
+ * balance loss and the block's backward pass).
  *
  * TEST INFRASTRUCTURE ONLY.  Nothing in the product path links, loads or calls this file:
  * only the tests, the package's smoke check and the benchmark's CPU-baseline leg do.  It
@@ -495,4 +496,158 @@ int oracle_aux_loss(const float *logits, const int32_t *idx, int T, int E, int k
     free(P);
     free(p);
     return 0;
+}
+
+/* ---------------------------------------------------------------- backward ----------- */
+
+/* The backward pass of the routed block for a given routing, all in double.
+ * "Qwen3-VL and Mixture of Experts", "How the router and experts learn", "What gets trained":
+ * only the experts a token chose receive its gradient, and the router learns through the
+ * gate weights; the selection itself is held fixed (it is piecewise constant).  The function
+ * differentiated is the plain definition (unrounded logits, double softmax, SwiGLU experts),
+ * with loss sum_t dy[t] . y[t].  Per token t with routing idx[t, 0..k-1]:
+ *   p = softmax(W_r x + b);  S = sum_j p[idx_j];  w_j = p[idx_j] / S  (norm)  or  p[idx_j]
+ *   for each slot j, e = idx_j:   g = W_gate[e] x,  u = W_up[e] x,  s = sigmoid(g),
+ *                                 h = g s u,        y += w_j W_down[e] h
+ *     z   = W_down[e]^T dy            dw_j = h . z           dh = w_j z
+ *     dg  = dh u s (1 + g (1 - s))    du   = dh g s
+ *     dx += W_gate[e]^T dg + W_up[e]^T du
+ *     dW_down[e] += (w_j dy) h^T,  dW_gate[e] += dg x^T,  dW_up[e] += du x^T
+ *   dp_j = (dw_j - sum_m dw_m w_m) / S  (norm)  or  dw_j
+ *   dl_e = p_e (dp_e - sum_j p[idx_j] dp_j)   (dp_e = 0 for experts not chosen)
+ *          (+ dlogits_add[t, e], e.g. the balance loss's gradient)
+ *   dW_r += dl x^T,  db += dl,  dx += W_r^T dl   (+ dy when residual)
+ * Inputs: x [T, D], W_r [E, D], W_gu [E, 2I, D], W_dn [E, D, I], dy [T, D] as bf16 bit
+ * patterns; bias [E] float or NULL; idx [T, k]; dlogits_add [T, E] double or NULL.
+ * Outputs (double, overwritten; any may be NULL): dx [T, D], dW_r [E, D], db [E],
+ * dlogits [T, E], dw [T, k], and the weight gradients of the n_exp experts listed in
+ * experts[]: dW_gu [n_exp, 2I, D], dW_dn [n_exp, D, I]. */
+int oracle_backward(const uint16_t *x, const uint16_t *W_r, const float *bias,
+                    const uint16_t *W_gu, const uint16_t *W_dn, const uint16_t *dy,
+                    const int32_t *idx, int T, int D, int E, int k, int I, int norm, int residual,
+                    const double *dlogits_add, double *dx, double *dW_r, double *db,
+                    double *dlogits, double *dw, const int32_t *experts, int n_exp,
+                    double *dW_gu, double *dW_dn) {
+    if (T < 1 || D < 1 || E < 1 || k < 1 || k > E || I < 1 || n_exp < 0) return 1;
+    double *xd = (double *)malloc((size_t)D * sizeof(double));
+    double *dyd = (double *)malloc((size_t)D * sizeof(double));
+    double *dxt = (double *)malloc((size_t)D * sizeof(double));
+    double *l = (double *)malloc((size_t)E * sizeof(double));
+    double *p = (double *)malloc((size_t)E * sizeof(double));
+    double *dl = (double *)malloc((size_t)E * sizeof(double));
+    double *dpe = (double *)malloc((size_t)E * sizeof(double));
+    double *g = (double *)malloc((size_t)I * sizeof(double));
+    double *u = (double *)malloc((size_t)I * sizeof(double));
+    double *z = (double *)malloc((size_t)I * sizeof(double));
+    double *dg = (double *)malloc((size_t)I * sizeof(double));
+    double *du = (double *)malloc((size_t)I * sizeof(double));
+    double *h = (double *)malloc((size_t)I * sizeof(double));
+    double *wj = (double *)malloc((size_t)k * sizeof(double));
+    double *dwj = (double *)malloc((size_t)k * sizeof(double));
+    int *slot_of = (int *)malloc((size_t)E * sizeof(int));
+    int rc = 0;
+    if (!xd || !dyd || !dxt || !l || !p || !dl || !dpe || !g || !u || !z || !dg || !du || !h || !wj ||
+        !dwj || !slot_of) { rc = 1; goto done; }
+    for (int e = 0; e < E; ++e) slot_of[e] = -1;
+    for (int m = 0; m < n_exp; ++m) {
+        if (experts[m] < 0 || experts[m] >= E) { rc = 1; goto done; }
+        slot_of[experts[m]] = m;
+    }
+    if (dW_r) memset(dW_r, 0, (size_t)E * D * sizeof(double));
+    if (db) memset(db, 0, (size_t)E * sizeof(double));
+    if (dW_gu) memset(dW_gu, 0, (size_t)n_exp * 2 * I * D * sizeof(double));
+    if (dW_dn) memset(dW_dn, 0, (size_t)n_exp * D * I * sizeof(double));
+    for (int t = 0; t < T; ++t) {
+        const int32_t *it = idx + (size_t)t * k;
+        for (int j = 0; j < k; ++j)
+            if (it[j] < 0 || it[j] >= E) { rc = 1; goto done; }
+        for (int d = 0; d < D; ++d) {
+            xd[d] = bf16_to_double(x[(size_t)t * D + d]);
+            dyd[d] = bf16_to_double(dy[(size_t)t * D + d]);
+            dxt[d] = residual ? dyd[d] : 0.0;
+        }
+        /* router: unrounded logits, softmax over all E, the given selection's weights */
+        double mx = -INFINITY;
+        for (int e = 0; e < E; ++e) {
+            double s = 0.0;
+            for (int d = 0; d < D; ++d) s += bf16_to_double(W_r[(size_t)e * D + d]) * xd[d];
+            if (bias) s += (double)bias[e];
+            l[e] = s;
+            if (s > mx) mx = s;
+        }
+        double Z = 0.0;
+        for (int e = 0; e < E; ++e) { p[e] = exp(l[e] - mx); Z += p[e]; }
+        for (int e = 0; e < E; ++e) p[e] /= Z;
+        double S = 0.0;
+        for (int j = 0; j < k; ++j) S += p[it[j]];
+        for (int j = 0; j < k; ++j) wj[j] = norm ? p[it[j]] / S : p[it[j]];
+        /* experts */
+        for (int j = 0; j < k; ++j) {
+            const int e = it[j];
+            const uint16_t *Wg = W_gu + (size_t)e * 2 * I * D, *Wu = Wg + (size_t)I * D;
+            const uint16_t *Wd = W_dn + (size_t)e * D * I;
+            for (int i = 0; i < I; ++i) {
+                double gs = 0.0, us = 0.0;
+                for (int d = 0; d < D; ++d) {
+                    gs += bf16_to_double(Wg[(size_t)i * D + d]) * xd[d];
+                    us += bf16_to_double(Wu[(size_t)i * D + d]) * xd[d];
+                }
+                g[i] = gs;
+                u[i] = us;
+                z[i] = 0.0;
+            }
+            for (int d = 0; d < D; ++d)
+                for (int i = 0; i < I; ++i) z[i] += bf16_to_double(Wd[(size_t)d * I + i]) * dyd[d];
+            double dws = 0.0;
+            for (int i = 0; i < I; ++i) {
+                const double s = 1.0 / (1.0 + exp(-g[i]));
+                h[i] = g[i] * s * u[i];
+                dws += h[i] * z[i];
+                const double dh = wj[j] * z[i];
+                dg[i] = dh * u[i] * s * (1.0 + g[i] * (1.0 - s));
+                du[i] = dh * g[i] * s;
+            }
+            dwj[j] = dws;
+            for (int i = 0; i < I; ++i)
+                for (int d = 0; d < D; ++d)
+                    dxt[d] += bf16_to_double(Wg[(size_t)i * D + d]) * dg[i] +
+                              bf16_to_double(Wu[(size_t)i * D + d]) * du[i];
+            const int m = slot_of[e];
+            if (m >= 0 && dW_gu)
+                for (int i = 0; i < I; ++i)
+                    for (int d = 0; d < D; ++d) {
+                        dW_gu[((size_t)m * 2 * I + i) * D + d] += dg[i] * xd[d];
+                        dW_gu[((size_t)m * 2 * I + I + i) * D + d] += du[i] * xd[d];
+                    }
+            if (m >= 0 && dW_dn)
+                for (int d = 0; d < D; ++d)
+                    for (int i = 0; i < I; ++i) dW_dn[((size_t)m * D + d) * I + i] += wj[j] * dyd[d] * h[i];
+        }
+        if (dw)
+            for (int j = 0; j < k; ++j) dw[(size_t)t * k + j] = dwj[j];
+        /* routing weights -> chosen probabilities -> logits */
+        double sdw = 0.0;
+        for (int j = 0; j < k; ++j) sdw += dwj[j] * wj[j];
+        for (int e = 0; e < E; ++e) dpe[e] = 0.0;
+        for (int j = 0; j < k; ++j) dpe[it[j]] += norm ? (dwj[j] - sdw) / S : dwj[j];
+        double pdp = 0.0;
+        for (int e = 0; e < E; ++e) pdp += p[e] * dpe[e];
+        for (int e = 0; e < E; ++e) {
+            dl[e] = p[e] * (dpe[e] - pdp);
+            if (dlogits_add) dl[e] += dlogits_add[(size_t)t * E + e];
+            if (dlogits) dlogits[(size_t)t * E + e] = dl[e];
+            if (db) db[e] += dl[e];
+        }
+        for (int e = 0; e < E; ++e)
+            for (int d = 0; d < D; ++d) {
+                const double wr = bf16_to_double(W_r[(size_t)e * D + d]);
+                dxt[d] += wr * dl[e];
+                if (dW_r) dW_r[(size_t)e * D + d] += dl[e] * xd[d];
+            }
+        if (dx) memcpy(dx + (size_t)t * D, dxt, (size_t)D * sizeof(double));
+    }
+done:
+    free(xd); free(dyd); free(dxt); free(l); free(p); free(dl); free(dpe); free(g); free(u); free(z);
+    free(dg); free(du); free(h); free(wj); free(dwj); free(slot_of);
+    return rc;
 }

@@ -68,6 +68,9 @@ def lib():
                                                c_int, _u16p, _u16p, _f64p]
             l.oracle_aux_loss.argtypes = [_f32p, _i32p, c_int, c_int, c_int, ctypes.c_double,
                                           ctypes.POINTER(ctypes.c_double), ctypes.c_void_p]
+            l.oracle_backward.argtypes = [_u16p, _u16p, _f32p, _u16p, _u16p, _u16p, _i32p, c_int, c_int,
+                                          c_int, c_int, c_int, c_int, c_int, _f64p, _f64p, _f64p,
+                                          _f64p, _f64p, _f64p, _i32p, c_int, _f64p, _f64p]
             l.oracle_e4m3_value.argtypes = [ctypes.c_uint8]
             l.oracle_e4m3_value.restype = ctypes.c_double
             l.oracle_quantize_fp8_rows.argtypes = [_u16p, ctypes.c_long, c_int, _u8p, _f32p]
@@ -76,7 +79,7 @@ def lib():
                                                   _u16p, _f64p]
             for name in ("oracle_router_logits", "oracle_select", "oracle_route", "oracle_permute",
                          "oracle_combine_rows", "oracle_forward_rows", "oracle_loop_dispatch",
-                         "oracle_quantize_fp8_rows", "oracle_combine_rows_fp8"):
+                         "oracle_quantize_fp8_rows", "oracle_combine_rows_fp8", "oracle_backward"):
                 getattr(l, name).restype = ctypes.c_int
             _lib = l
     return _lib
@@ -299,6 +302,31 @@ def aux_loss(logits, idx, alpha=1.0, with_grad=True):
     _check(lib().oracle_aux_loss(_p(lg, _f32p), _p(ix, _i32p), T, E, k, float(alpha), ctypes.byref(loss),
                                  d.ctypes.data_as(ctypes.c_void_p) if d is not None else None), "oracle_aux_loss")
     return loss.value, d
+
+
+def backward(x, W_r, W_gu, W_dn, dy, idx, norm=True, bias=None, residual=False, dlogits_add=None,
+             experts=()):
+    """Gradients of sum_t dy[t] . y[t] for the given routing idx [T, k] (selection held fixed),
+    in double (see oracle_backward).  -> dict with dx [T, D], dW_r [E, D], db [E],
+    dlogits [T, E], dw [T, k], and dW_gu [n, 2I, D], dW_dn [n, D, I] for the listed experts."""
+    x, W_r, W_gu, W_dn, dy = as_u16(x), as_u16(W_r), as_u16(W_gu), as_u16(W_dn), as_u16(dy)
+    bias, ix = _f32(bias), _i32(idx)
+    T, D = x.shape
+    E, k = W_r.shape[0], ix.shape[1]
+    I = W_gu.shape[1] // 2
+    ex = np.ascontiguousarray(np.asarray(experts, dtype=np.int32).reshape(-1))
+    n = len(ex)
+    add = None if dlogits_add is None else np.ascontiguousarray(dlogits_add, dtype=np.float64)
+    out = dict(dx=np.empty((T, D)), dW_r=np.empty((E, D)), db=np.empty(E), dlogits=np.empty((T, E)),
+               dw=np.empty((T, k)), dW_gu=np.empty((n, 2 * I, D)), dW_dn=np.empty((n, D, I)))
+    _check(lib().oracle_backward(_p(x, _u16p), _p(W_r, _u16p), _p(bias, _f32p), _p(W_gu, _u16p),
+                                 _p(W_dn, _u16p), _p(dy, _u16p), _p(ix, _i32p), T, D, E, k, I,
+                                 int(bool(norm)), int(bool(residual)), _p(add, _f64p),
+                                 _p(out["dx"], _f64p), _p(out["dW_r"], _f64p), _p(out["db"], _f64p),
+                                 _p(out["dlogits"], _f64p), _p(out["dw"], _f64p), _p(ex, _i32p), n,
+                                 _p(out["dW_gu"], _f64p) if n else None,
+                                 _p(out["dW_dn"], _f64p) if n else None), "oracle_backward")
+    return out
 
 
 def cpu_threads_available() -> int:

@@ -1,7 +1,8 @@
 """moe_aux_loss (the Switch balance loss and its gradient with respect to the router logits)
 on the GPU against the oracle's FP64 evaluation of the same definition.
 
-Inputs are each configuration's own routing (logits and top-k from moe_route): decode T=256,
+Inputs are each configuration's own routing, made by the oracle's router and selection from
+the seeded layer (FP32 logits and the top-k indices) and given to both sides: decode T=256,
 prefill T=8192, zipf (E=512, k=10, Zipf router bias), tiny (E=8, tie rows).
 
 Tolerances, from the FP32 arithmetic: P_e is a sum of T probabilities (each a few ulp off)
@@ -33,9 +34,8 @@ def _built():
 
 def routing(name, T=None):
     cfg, L, G = layer(name, T)
-    logits, idx, _ = B.moe_route(G["x"], G["W_r"], cfg.k, cfg.norm_topk_prob, bias=G.get("bias"))
-    torch.cuda.synchronize()
-    return cfg, logits, idx
+    logits, idx, _ = O.route(L["x"], L["W_r"], cfg.k, cfg.norm_topk_prob, bias=L.get("bias"))
+    return cfg, torch.from_numpy(logits).cuda(), torch.from_numpy(idx).cuda()
 
 
 @pytest.mark.parametrize("name,T", [("tiny", None), ("decode", 256), ("prefill", None), ("zipf", None)])

@@ -420,3 +420,111 @@ def test_aux_loss_gradient_matches_finite_differences(oracle_mod):
             assert abs(fd - d[t, e]) <= 2e-6, (t, e, fd, d[t, e])
     # each token's gradient sums to zero (a softmax is shift-invariant)
     assert np.abs(d.sum(axis=1)).max() <= 1e-15
+
+
+# ------------------------------------------------------------------ backward pass
+# "Qwen3-VL and Mixture of Experts", "How the router and experts learn", "What gets trained":
+# a token's gradient reaches only the experts it chose, and the router learns through the
+# gate weights; the selection is held fixed.
+
+def _bwd_problem(seed, T, D, E, k, I, bias=True):
+    g = torch.Generator().manual_seed(seed)
+    bf = lambda *s, sc=1.0: (torch.randn(*s, generator=g) * sc).to(torch.bfloat16)
+    P = dict(x=bf(T, D), W_r=bf(E, D, sc=0.5), W_gu=bf(E, 2 * I, D, sc=0.4), W_dn=bf(E, D, I, sc=0.4),
+             dy=bf(T, D), bias=(torch.randn(E, generator=g) * 0.3) if bias else None)
+    # any distinct experts per token (not necessarily the top k): the gradient formula holds
+    # for a fixed selection whatever it is
+    P["idx"] = torch.stack([torch.randperm(E, generator=g)[:k] for _ in range(T)]).to(torch.int32)
+    return P
+
+
+def _block_loss64(P, norm, residual, dl_add=None, over=None):
+    """sum_t dy[t] . y[t] (+ sum dl_add * logits) of the block in float64 torch ops, routing fixed.
+    `over` replaces some float64 leaves (for finite differences / autograd)."""
+    V = {n: P[n].double() for n in ("x", "W_r", "W_gu", "W_dn", "dy")}
+    V["bias"] = P["bias"].double() if P["bias"] is not None else None
+    V.update(over or {})
+    x, W_r, W_gu, W_dn, dy = V["x"], V["W_r"], V["W_gu"], V["W_dn"], V["dy"]
+    idx = P["idx"].long()
+    I = W_gu.shape[1] // 2
+    logits = x @ W_r.T + (V["bias"] if V["bias"] is not None else 0.0)
+    p = torch.softmax(logits, dim=-1)
+    sel = torch.gather(p, 1, idx)
+    w = sel / sel.sum(1, keepdim=True) if norm else sel
+    g = torch.einsum("tkid,td->tki", W_gu[idx, :I, :], x)
+    u = torch.einsum("tkid,td->tki", W_gu[idx, I:, :], x)
+    o = torch.einsum("tkdi,tki->tkd", W_dn[idx], F.silu(g) * u)
+    y = (w[..., None] * o).sum(1) + (x if residual else 0.0)
+    L = (dy * y).sum()
+    if dl_add is not None:
+        L = L + (torch.as_tensor(dl_add) * logits).sum()
+    return L, logits, w
+
+
+@pytest.mark.parametrize("norm,residual,with_add", [(True, False, False), (False, True, False), (True, True, True)])
+def test_backward_matches_autograd(oracle_mod, norm, residual, with_add):
+    """Every gradient of the oracle's backward against float64 autograd of the forward
+    definition (x, all weights, the bias, the logits and the routing weights)."""
+    T, D, E, k, I = 6, 16, 7, 3, 8
+    P = _bwd_problem(11, T, D, E, k, I)
+    dl_add = np.random.default_rng(1).normal(0, 0.1, (T, E)) if with_add else None
+    leaves = {n: P[n].double().requires_grad_(True) for n in ("x", "W_r", "W_gu", "W_dn")}
+    leaves["bias"] = P["bias"].double().requires_grad_(True)
+    L, logits, w = _block_loss64(P, norm, residual, dl_add, over=leaves)
+    logits.retain_grad()
+    w.retain_grad()
+    L.backward()
+    experts = [0, 3, 5]
+    got = oracle_mod.backward(P["x"], P["W_r"], P["W_gu"], P["W_dn"], P["dy"], P["idx"], norm=norm,
+                              bias=P["bias"], residual=residual, dlogits_add=dl_add, experts=experts)
+    want = dict(dx=leaves["x"].grad, dW_r=leaves["W_r"].grad, db=leaves["bias"].grad, dlogits=logits.grad,
+                dw=w.grad, dW_gu=leaves["W_gu"].grad[experts], dW_dn=leaves["W_dn"].grad[experts])
+    for name, ref in want.items():
+        ref = ref.numpy()
+        assert np.abs(got[name] - ref).max() <= 1e-12 * max(1.0, np.abs(ref).max()), name
+    # experts nobody chose get no gradient
+    unused = sorted(set(range(E)) - set(P["idx"].flatten().tolist()))
+    for e in unused:
+        assert not leaves["W_gu"].grad[e].any()
+
+
+def test_backward_finite_differences(oracle_mod):
+    """Central differences of the float64 forward (no autograd) on entries of x, W_r, W_gate_up,
+    W_down and the bias."""
+    T, D, E, k, I = 4, 8, 5, 2, 4
+    P = _bwd_problem(12, T, D, E, k, I)
+    got = oracle_mod.backward(P["x"], P["W_r"], P["W_gu"], P["W_dn"], P["dy"], P["idx"], norm=True,
+                              bias=P["bias"], experts=list(range(E)))
+    rng = np.random.default_rng(2)
+    cases = [("x", "dx"), ("W_r", "dW_r"), ("W_gu", "dW_gu"), ("W_dn", "dW_dn"), ("bias", "db")]
+    h = 1e-6
+    for leaf, out in cases:
+        base = P[leaf].double()
+        for _ in range(4):
+            pos = tuple(int(rng.integers(0, n)) for n in base.shape)
+            plus, minus = base.clone(), base.clone()
+            plus[pos] += h
+            minus[pos] -= h
+            fd = (_block_loss64(P, True, False, over={leaf: plus})[0] -
+                  _block_loss64(P, True, False, over={leaf: minus})[0]).item() / (2 * h)
+            assert abs(fd - got[out][pos]) <= 1e-7 * max(1.0, abs(fd)), (leaf, pos, fd, got[out][pos])
+
+
+def test_backward_one_expert_is_swiglu_mlp(oracle_mod):
+    """E = 1, k = 1: the weight is 1 whatever the logits, so the router gets no gradient, and dx,
+    dW_gate_up, dW_down are those of a plain SwiGLU MLP y = W_down (silu(W_gate x) * W_up x)
+    (torch.nn.functional, autograd)."""
+    T, D, I = 5, 12, 6
+    P = _bwd_problem(13, T, D, 1, 1, I)
+    got = oracle_mod.backward(P["x"], P["W_r"], P["W_gu"], P["W_dn"], P["dy"], P["idx"], norm=True,
+                              bias=P["bias"], experts=[0])
+    assert not got["dlogits"].any() and not got["dW_r"].any() and not got["db"].any()
+    x = P["x"].double().requires_grad_(True)
+    Wg = P["W_gu"][0, :I].double().requires_grad_(True)
+    Wu = P["W_gu"][0, I:].double().requires_grad_(True)
+    Wd = P["W_dn"][0].double().requires_grad_(True)
+    y = F.linear(F.silu(F.linear(x, Wg)) * F.linear(x, Wu), Wd)
+    (P["dy"].double() * y).sum().backward()
+    assert np.allclose(got["dx"], x.grad.numpy(), rtol=0, atol=1e-12)
+    assert np.allclose(got["dW_gu"][0], torch.cat([Wg.grad, Wu.grad]).numpy(), rtol=0, atol=1e-12)
+    assert np.allclose(got["dW_dn"][0], Wd.grad.numpy(), rtol=0, atol=1e-12)
