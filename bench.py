@@ -250,8 +250,11 @@ def build_workload(name, device, copies=None):
 
 def measure(name, args, rank, world, device, peaks, with_e2e):
     """Time one workload; returns (result dict, cfg, CPU layer)."""
+    import ctypes
+
     import torch
     from sparse_fp32_softmax_b200 import binding as B
+    from sparse_fp32_softmax_b200 import inputs
     from sparse_fp32_softmax_b200.roofline import algorithmic_bytes, algorithmic_flops
 
     cfg, spec, sweep, W, x0, L_cpu = build_workload(name, device, args.copies if name == args.workload else None)
@@ -514,6 +517,32 @@ def measure(name, args, rank, world, device, peaks, with_e2e):
                                note="loss and gradient of the Switch balance loss, T=%d, E=%d, k=%d" % (
                                    p["T"], cfg.E, cfg.k))
         del g
+        # the backward pass for the same routing (all gradients: x, router weights, expert
+        # weights, logits, routing weights), eager calls with CUDA events around K of them
+        dy = inputs.upstream_grad(cfg, p["T"]).to(device)
+        bw_dims = B.make_dims(p["T"], cfg.D, cfg.E, cfg.k, cfg.I, cfg.norm_topk_prob)
+        bw_ws = torch.empty(int(B.load().moe_backward_workspace_size(ctypes.byref(bw_dims))), dtype=torch.uint8,
+                            device=device)
+        call = lambda: B.moe_backward(p["x"], w["W_r"], w["W_gate_up"], w["W_down"], dy, idx, cfg.norm_topk_prob,
+                                      bias=w.get("bias"), ws=bw_ws)
+        for _ in range(3):
+            call()
+        torch.cuda.synchronize()
+        a_ev.record()
+        for _ in range(K):
+            call()
+        b_ev.record()
+        torch.cuda.synchronize()
+        ms = a_ev.elapsed_time(b_ev) / K
+        R = p["T"] * cfg.k
+        flops = 16 * R * cfg.D * cfg.I + 4 * p["T"] * cfg.E * cfg.D   # seven GEMMs
+        tf = flops / (ms * 1e-3) / 1e12
+        res["backward"] = dict(ms_per_call=round(ms, 4), gemm_flops=flops, achieved_tflops=round(tf, 1),
+                               frac_of_bf16=round(tf / peaks["bf16_tflops"], 4),
+                               note="moe_backward, T=%d, E=%d, k=%d, I=%d: recompute g/u, z = W_down^T dy, "
+                                    "dW_down, dX, dW_gate_up, dW_r, router dx (warp-MMA grouped GEMMs)" % (
+                                        p["T"], cfg.E, cfg.k, cfg.I))
+        del bw_ws
 
     # end to end through the public API with host buffers (eager, copies inside the region)
     if with_e2e and not chain:
@@ -680,6 +709,8 @@ def main(argv=None):
         line["sweep"] = res["sweep"]
     if "aux_loss" in res:
         line["aux_loss"] = res["aux_loss"]
+    if "backward" in res:
+        line["backward"] = res["backward"]
     if want_cpu:
         line["cpu_baseline"] = cpu_baseline(cfg, L_cpu, layers=WORKLOADS[args.workload]["layers"])
     del L_cpu

@@ -171,6 +171,35 @@ size_t moe_aux_loss_workspace_size(int T, int E);
 moe_status moe_aux_loss(const float *logits, const int32_t *topk_idx, int T, int E, int k, float alpha,
                         float *loss, float *dlogits, void *ws, size_t ws_bytes, moe_stream_t stream);
 
+/* The backward pass of the routed block for a given routing ("Qwen3-VL and Mixture of
+ * Experts", "How the router and experts learn", "What gets trained": a token's gradient
+ * reaches only the experts it chose, and the router learns through the gate weights; the
+ * selection is held fixed).  For the loss sum_t dy[t] . y[t], y the block's output with the
+ * routing topk_idx (normally the forward's), the gradients with respect to:
+ *   dx [T, D]            the input x (+ dy when residual = 1, i.e. y = x + block(x));
+ *   dW_r [E, D]          the router weights;      dbias [E] the router bias (or NULL);
+ *   dW_gate_up [E,2I,D]  and dW_down [E, D, I]    (zero for experts no token chose);
+ *   dlogits [T, E]       the router logits (or NULL);  dw [T, k] the routing weights (or NULL).
+ * Per token and slot j (expert e, weight w_j, s = sigmoid(g), h = g s u):
+ *   z = W_down[e]^T dy,  dw_j = h . z,  dh = w_j z,  dg = dh u s (1 + g (1 - s)),  du = dh g s;
+ *   dp_j = (dw_j - sum_m dw_m w_m) / sum_m p_m (norm_topk_prob) or dw_j;
+ *   dlogits = p (dp - sum_j p_j dp_j) + dlogits_add (e.g. moe_aux_loss's gradient; or NULL).
+ * x, W_r, W_gate_up, W_down as for moe_forward; bias [E] FP32 or NULL (as given to the
+ * forward); dy [T, D] bf16; topk_idx [T, k] int32 (entries outside [0, E) are skipped and
+ * recorded in the device error word, which moe_get_device_status reads from ws).  Outputs are
+ * FP32 and fully overwritten.  The router logits and g, u are recomputed; h, dg, du, w dy and
+ * dlogits are rounded to bf16 once as GEMM operands; all sums run in a fixed order (bitwise
+ * reproducible).  No shared expert.  Shapes as for moe_forward (dims->tile_m is ignored);
+ * 16-byte aligned bf16/FP32 matrices, workspace of moe_backward_workspace_size(dims) bytes,
+ * 256-byte aligned.  Enqueued on `stream`. */
+size_t moe_backward_workspace_size(const moe_dims *dims);
+moe_status moe_backward(const moe_bf16 *x, const moe_bf16 *W_r, const float *bias,
+                        const moe_bf16 *W_gate_up, const moe_bf16 *W_down, const moe_bf16 *dy,
+                        const int32_t *topk_idx, const float *dlogits_add, int residual,
+                        const moe_dims *dims, float *dx, float *dW_r, float *dbias,
+                        float *dW_gate_up, float *dW_down, float *dlogits, float *dw, void *ws,
+                        size_t ws_bytes, moe_stream_t stream);
+
 /* Bytes of workspace that moe_route, moe_permute and moe_forward(_ex) need for `dims`
  * (and `opts`, which may be NULL).  Returns 0 for invalid or unsupported arguments. */
 size_t moe_workspace_size(const moe_dims *dims, const moe_opts *opts);

@@ -79,9 +79,13 @@ def load():
         lib.moe_aux_loss_workspace_size.argtypes = [_c_int, _c_int]
         lib.moe_aux_loss_workspace_size.restype = _sz
         lib.moe_aux_loss.argtypes = [_vp, _vp, _c_int, _c_int, _c_int, ctypes.c_float, _vp, _vp, _vp, _sz, _vp]
+        lib.moe_backward_workspace_size.argtypes = [dp]
+        lib.moe_backward_workspace_size.restype = _sz
+        lib.moe_backward.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_int, dp, _vp, _vp, _vp, _vp, _vp,
+                                     _vp, _vp, _vp, _sz, _vp]
         for n in ("moe_route", "moe_permute", "moe_forward", "moe_forward_ex", "moe_forward_noalloc",
                   "moe_get_device_status", "moe_get_device_status_noalloc", "moe_quantize_fp8_rows",
-                  "moe_forward_path", "moe_aux_loss"):
+                  "moe_forward_path", "moe_aux_loss", "moe_backward"):
             getattr(lib, n).restype = _c_int
         _lib = lib
     return _lib
@@ -202,6 +206,34 @@ def moe_aux_loss(logits, topk_idx, alpha=1.0, with_grad=True, ws=None, stream=No
     _check(lib.moe_aux_loss(_ptr(logits), _ptr(topk_idx), T, E, k, float(alpha), _ptr(loss), _ptr(d), _ptr(ws),
                             ws.numel(), _stream(stream)), "moe_aux_loss")
     return loss, d
+
+
+def moe_backward(x, W_r, W_gate_up, W_down, dy, topk_idx, norm_topk_prob=True, bias=None, dlogits_add=None,
+                 residual=False, with_dbias=None, ws=None, stream=None):
+    """Gradients of sum(dy * y) for the routing topk_idx -> dict of FP32 tensors dx [T, D],
+    dW_r [E, D], dbias [E] (when a bias is given or with_dbias), dW_gate_up [E, 2I, D],
+    dW_down [E, D, I], dlogits [T, E], dw [T, k]."""
+    dims = _dims_of(x, W_r, W_gate_up, W_down, topk_idx.shape[1], norm_topk_prob)
+    _need(dy, "dy", torch.bfloat16, 2)
+    _need(topk_idx, "topk_idx", torch.int32, 2)
+    T, D, E, k, I = dims.T, dims.D, dims.E, dims.k, dims.I
+    lib = load()
+    n = int(lib.moe_backward_workspace_size(ctypes.byref(dims)))
+    if n == 0:
+        raise MoeError(MOE_ERR_UNSUPPORTED, "moe_backward_workspace_size")
+    dev = x.device
+    if ws is None:
+        ws = torch.empty(n, dtype=torch.uint8, device=dev)
+    f32 = lambda *s: torch.empty(*s, dtype=torch.float32, device=dev)
+    out = dict(dx=f32(T, D), dW_r=f32(E, D), dW_gate_up=f32(E, 2 * I, D), dW_down=f32(E, D, I), dlogits=f32(T, E),
+               dw=f32(T, k))
+    out["dbias"] = f32(E) if (bias is not None or with_dbias) else None
+    _check(lib.moe_backward(_ptr(x), _ptr(W_r), _ptr(bias), _ptr(W_gate_up), _ptr(W_down), _ptr(dy), _ptr(topk_idx),
+                            _ptr(dlogits_add), int(bool(residual)), ctypes.byref(dims), _ptr(out["dx"]),
+                            _ptr(out["dW_r"]), _ptr(out["dbias"]), _ptr(out["dW_gate_up"]), _ptr(out["dW_down"]),
+                            _ptr(out["dlogits"]), _ptr(out["dw"]), _ptr(ws), ws.numel(), _stream(stream)),
+           "moe_backward")
+    return out
 
 
 def workspace(dims: moe_dims, opts: moe_opts | None = None, device=None) -> torch.Tensor:

@@ -205,6 +205,8 @@ cudaError_t ensure_smem_attr(const void* kernel, int bytes);
 // Streaming multiprocessors of the current device (queried once per device; 0 on error).
 // Launchers size their grids from it.
 int device_sm_count();
+// Records the cudaError_t behind a MOE_ERR_CUDA for moe_last_cuda_error (this host thread).
+void note_cuda_error(int e);
 
 // ---------------------------------------------------------------- launchers (return the
 // launch error, cudaSuccess when all kernels were enqueued).  pdl: launch the first kernel

@@ -347,6 +347,10 @@ moe_status run_logits(const moe_bf16* x, const moe_bf16* W_r, const Plan& p, flo
 
 }  // namespace
 
+namespace moe {
+void note_cuda_error(int e) { g_last_cuda_error = e; }
+}  // namespace moe
+
 extern "C" {
 
 size_t moe_workspace_size(const moe_dims* dims, const moe_opts* opts) {

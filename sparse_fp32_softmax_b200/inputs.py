@@ -23,6 +23,7 @@ import torch
 
 # tensor ids inside a configuration's seed space
 TID_X, TID_WR, TID_WGU, TID_WDN, TID_SGU, TID_SDN, TID_SG, TID_BIAS = range(8)
+TID_DY = 8   # the upstream gradient dy of the backward pass
 
 
 @dataclass(frozen=True)
@@ -138,6 +139,12 @@ def make_layer(cfg: MoEConfig, T: int | None = None, layer: int | None = None, d
         _apply_tiny_ties(x, W_r, E)
         out["x"], out["W_r"] = x.to(device), W_r.to(device)
     return out
+
+
+def upstream_grad(cfg: MoEConfig, T: int | None = None, device="cpu") -> torch.Tensor:
+    """dy [T, D] for the backward pass: N(0, 1) rounded to bf16, seeded per configuration."""
+    T = cfg.T if T is None else int(T)
+    return normal_bf16((T, cfg.D), 1.0, 1000 * cfg.seed + TID_DY, device=device)
 
 
 def coverage_rows(T: int, n_random: int, seed: int, extra=()) -> list:

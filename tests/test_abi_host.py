@@ -29,7 +29,7 @@ def test_library_exports_every_declared_function(lib):
                              "moe_forward_ex", "moe_forward_noalloc", "moe_get_device_status",
                              "moe_get_device_status_noalloc", "moe_status_string", "moe_last_cuda_error",
                              "moe_quantize_fp8_rows", "moe_forward_path", "moe_aux_loss",
-                             "moe_aux_loss_workspace_size"}
+                             "moe_aux_loss_workspace_size", "moe_backward", "moe_backward_workspace_size"}
     out = subprocess.run(["nm", "-D", "--defined-only", LIB], capture_output=True, text=True, check=True).stdout
     exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
     for name in declared:
@@ -180,3 +180,27 @@ def test_aux_loss_validation_without_a_device(lib):
     assert lib.moe_aux_loss(*args(ws=FAKE + 16)) == B.MOE_ERR_INVALID_ARG
     assert lib.moe_aux_loss(*args(nb=n - 4)) == B.MOE_ERR_WORKSPACE
     assert lib.moe_aux_loss(*args()) == B.MOE_ERR_CUDA
+
+
+@no_gpu
+def test_backward_validation_without_a_device(lib):
+    """moe_backward validates before enqueuing (shape, pointers, alignment, workspace); with
+    valid arguments and no GPU it reports a CUDA failure (no host fallback)."""
+    p = ctypes.c_void_p
+    dims = B.make_dims(64, 256, 8, 2, 128, True)
+    n = lib.moe_backward_workspace_size(ctypes.byref(dims))
+    assert n > lib.moe_workspace_size(ctypes.byref(dims), None) > 0
+    assert lib.moe_backward_workspace_size(ctypes.byref(B.make_dims(64, 200, 8, 2, 128, True))) == 0
+
+    def call(d=dims, x=FAKE, dx=FAKE, ws=FAKE, nb=n, residual=0, idx=FAKE):
+        return lib.moe_backward(p(x), p(FAKE), None, p(FAKE), p(FAKE), p(FAKE), p(idx), None, residual,
+                                ctypes.byref(d), p(dx), p(FAKE), None, p(FAKE), p(FAKE), None, None, p(ws), nb, None)
+    assert call(d=B.make_dims(0, 256, 8, 2, 128, True)) == B.MOE_ERR_INVALID_ARG
+    assert call(d=B.make_dims(64, 200, 8, 2, 128, True)) == B.MOE_ERR_UNSUPPORTED
+    assert call(x=0) == B.MOE_ERR_INVALID_ARG
+    assert call(idx=0) == B.MOE_ERR_INVALID_ARG
+    assert call(dx=FAKE + 4) == B.MOE_ERR_INVALID_ARG
+    assert call(ws=FAKE + 16) == B.MOE_ERR_INVALID_ARG
+    assert call(residual=2) == B.MOE_ERR_INVALID_ARG
+    assert call(nb=n - 256) == B.MOE_ERR_WORKSPACE
+    assert call() == B.MOE_ERR_CUDA
