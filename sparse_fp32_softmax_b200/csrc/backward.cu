@@ -28,11 +28,21 @@
 
 namespace moe {
 
-constexpr int kBwBM = 128, kBwBN = 128, kBwBK = 32, kBwStages = 3, kBwThreads = 256;
-constexpr int kBwRowK = kBwBK + 8;    // smem row length of a [rows][k] tile (conflict-free ldmatrix)
-constexpr int kBwRowMN = kBwBM + 8;   // smem row length of a [k][rows] tile (kBwBM == kBwBN)
-constexpr int kBwTileElems = kBwBM * kBwRowK > kBwBK * kBwRowMN ? kBwBM * kBwRowK : kBwBK * kBwRowMN;
-constexpr int kBwSmem = kBwStages * 2 * kBwTileElems * 2;
+// CTA tile: 128 rows (M) x BN columns (N), K steps of BK, NS-stage cp.async ring; 8 warps as
+// 2 (M) x 4 (N), each a 64 x BN/4 warp tile.  Shared-memory rows are padded by 8 elements so
+// that the 8 row addresses of every ldmatrix fall in distinct banks.
+constexpr int kBwBM = 128, kBwThreads = 256;
+constexpr int kBwBN = 128, kBwBK = 64, kBwStages = 3;   // the configuration the library launches
+template <int BN, int BK>
+struct BwTile {
+    static constexpr int RowK = BK + 8;           // [rows][k] tiles
+    static constexpr int RowM = kBwBM + 8;        // [k][m] tiles
+    static constexpr int RowN = BN + 8;           // [k][n] tiles
+    static constexpr int A = kBwBM * RowK > BK * RowM ? kBwBM * RowK : BK * RowM;   // elements
+    static constexpr int B = BN * RowK > BK * RowN ? BN * RowK : BK * RowN;
+};
+template <int BN, int BK, int NS>
+constexpr int bw_smem_bytes() { return NS * (BwTile<BN, BK>::A + BwTile<BN, BK>::B) * 2; }
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
     // src-size 0 writes 16 zero bytes and reads nothing
@@ -74,8 +84,10 @@ struct BwGemm {
     const int* tile_start;
 };
 
-template <bool A_K, bool B_K, bool KG>
+template <bool A_K, bool B_K, bool KG, int BN, int BK, int NS>
 __global__ void __launch_bounds__(kBwThreads) bw_gemm_kernel(const BwGemm p) {
+    using TL = BwTile<BN, BK>;
+    constexpr int WN = BN / 4, NI = WN / 8, NJ = WN / 16;   // warp tile columns, n8 tiles, x4 loads
     extern __shared__ __align__(128) uint16_t bw_smem[];
     __shared__ int s_g;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -108,106 +120,111 @@ __global__ void __launch_bounds__(kBwThreads) bw_gemm_kernel(const BwGemm p) {
         if (mvalid <= 0) return;
         kvalid_a = p.K;
         kvalid_b = p.b_rows;
-        KT = (p.K + kBwBK - 1) / kBwBK;
+        KT = (p.K + BK - 1) / BK;
     } else {
         g = blockIdx.z;
         m0 = blockIdx.x * kBwBM;
         mvalid = min(kBwBM, p.M - m0);
         row0 = p.seg_off ? p.seg_off[g] : 0;
         kvalid_a = kvalid_b = p.seg_cnt ? p.seg_cnt[g] : p.K;
-        KT = (kvalid_a + kBwBK - 1) / kBwBK;
+        KT = (kvalid_a + BK - 1) / BK;
     }
-    const int n0 = blockIdx.y * kBwBN;
+    const int n0 = blockIdx.y * BN;
     // operand origins: token rows are offset by row0 (along m for !KG, along k for KG)
     const uint16_t* Ag = KG ? p.A + row0 * p.lda : p.A + (row0 + m0) * p.lda;
     const uint16_t* Bg = KG ? p.B + row0 * p.ldb : p.B + (long long)g * p.b_gs;
     float* Cg = KG ? p.C + (long long)g * p.c_gs + (long long)m0 * p.ldc : p.C + (row0 + m0) * p.ldc;
 
     const uint32_t sbase = smem_u32(bw_smem);
-    auto sA = [&](int st) { return sbase + (uint32_t)(st * 2 * kBwTileElems) * 2u; };
-    auto sB = [&](int st) { return sbase + (uint32_t)((st * 2 + 1) * kBwTileElems) * 2u; };
+    auto sA = [&](int st) { return sbase + (uint32_t)(st * (TL::A + TL::B)) * 2u; };
+    auto sB = [&](int st) { return sbase + (uint32_t)(st * (TL::A + TL::B) + TL::A) * 2u; };
 
     auto load_stage = [&](int st, int kt) {
-        const int k0 = kt * kBwBK;
+        const int k0 = kt * BK;
+        constexpr int KC = BK / 8;   // 16-byte chunks along k
 #pragma unroll
-        for (int it = 0; it < 2; ++it) {
+        for (int it = 0; it < kBwBM * BK / 8 / kBwThreads; ++it) {
             const int c = tid + it * kBwThreads;
-            if (A_K) {   // 128 m rows x 4 chunks of 8 k
-                const int r = c >> 2, col = (c & 3) * 8;
+            if (A_K) {   // 128 m rows x KC chunks of 8 k
+                const int r = c / KC, col = (c % KC) * 8;
                 const bool ok = r < mvalid && k0 + col < kvalid_a;
                 const uint16_t* src = ok ? Ag + (long long)r * p.lda + k0 + col : p.A;
-                cp_async16(sA(st) + (uint32_t)(r * kBwRowK + col) * 2u, src, ok);
-            } else {     // 32 k rows x 16 chunks of 8 m
+                cp_async16(sA(st) + (uint32_t)(r * TL::RowK + col) * 2u, src, ok);
+            } else {     // BK k rows x 16 chunks of 8 m
                 const int r = c >> 4, col = (c & 15) * 8;
                 const bool ok = k0 + r < kvalid_a && m0 + col < p.a_cols;
                 const uint16_t* src = ok ? Ag + (long long)(k0 + r) * p.lda + m0 + col : p.A;
-                cp_async16(sA(st) + (uint32_t)(r * kBwRowMN + col) * 2u, src, ok);
+                cp_async16(sA(st) + (uint32_t)(r * TL::RowM + col) * 2u, src, ok);
             }
-            if (B_K) {   // 128 n rows x 4 chunks of 8 k
-                const int r = c >> 2, col = (c & 3) * 8;
+        }
+#pragma unroll
+        for (int it = 0; it < BN * BK / 8 / kBwThreads; ++it) {
+            const int c = tid + it * kBwThreads;
+            if (B_K) {   // BN n rows x KC chunks of 8 k
+                const int r = c / KC, col = (c % KC) * 8;
                 const bool ok = n0 + r < p.N && k0 + col < p.K;
                 const uint16_t* src = ok ? Bg + (long long)(n0 + r) * p.ldb + k0 + col : p.B;
-                cp_async16(sB(st) + (uint32_t)(r * kBwRowK + col) * 2u, src, ok);
-            } else {     // 32 k rows x 16 chunks of 8 n
-                const int r = c >> 4, col = (c & 15) * 8;
+                cp_async16(sB(st) + (uint32_t)(r * TL::RowK + col) * 2u, src, ok);
+            } else {     // BK k rows x BN/8 chunks of 8 n
+                const int r = c / (BN / 8), col = (c % (BN / 8)) * 8;
                 const bool ok = k0 + r < kvalid_b && n0 + col < p.N;
                 const uint16_t* src = ok ? Bg + (long long)(k0 + r) * p.ldb + n0 + col : p.B;
-                cp_async16(sB(st) + (uint32_t)(r * kBwRowMN + col) * 2u, src, ok);
+                cp_async16(sB(st) + (uint32_t)(r * TL::RowN + col) * 2u, src, ok);
             }
         }
     };
 
-    float acc[4][4][4];
+    float acc[4][NI][4];
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
+        for (int j = 0; j < NI; ++j)
 #pragma unroll
             for (int q = 0; q < 4; ++q) acc[i][j][q] = 0.f;
 
-    const int wm0 = (warp >> 2) * 64, wn0 = (warp & 3) * 32;
+    const int wm0 = (warp >> 2) * 64, wn0 = (warp & 3) * WN;
     const int li = lane >> 3, lr = lane & 7;
 #pragma unroll
-    for (int s = 0; s < kBwStages - 1; ++s) {
+    for (int s = 0; s < NS - 1; ++s) {
         if (s < KT) load_stage(s, s);
         cp_async_commit();
     }
     for (int kt = 0; kt < KT; ++kt) {
-        cp_async_wait<kBwStages - 2>();
+        cp_async_wait<NS - 2>();
         __syncthreads();
-        const int nk = kt + kBwStages - 1;
-        if (nk < KT) load_stage(nk % kBwStages, nk);
+        const int nk = kt + NS - 1;
+        if (nk < KT) load_stage(nk % NS, nk);
         cp_async_commit();
-        const int st = kt % kBwStages;
+        const int st = kt % NS;
 #pragma unroll
-        for (int kk = 0; kk < kBwBK; kk += 16) {
-            uint32_t a[4][4], b[2][4];
+        for (int kk = 0; kk < BK; kk += 16) {
+            uint32_t a[4][4], b[NJ][4];
 #pragma unroll
             for (int mi = 0; mi < 4; ++mi) {
                 if (A_K) {
                     const int row = wm0 + mi * 16 + (lane & 15), col = kk + (lane >> 4) * 8;
-                    ldmatrix_x4(sA(st) + (uint32_t)(row * kBwRowK + col) * 2u, a[mi][0], a[mi][1], a[mi][2], a[mi][3]);
+                    ldmatrix_x4(sA(st) + (uint32_t)(row * TL::RowK + col) * 2u, a[mi][0], a[mi][1], a[mi][2], a[mi][3]);
                 } else {
                     const int krow = kk + lr + (li >> 1) * 8, mcol = wm0 + mi * 16 + (li & 1) * 8;
-                    ldmatrix_x4_trans(sA(st) + (uint32_t)(krow * kBwRowMN + mcol) * 2u, a[mi][0], a[mi][1], a[mi][2],
+                    ldmatrix_x4_trans(sA(st) + (uint32_t)(krow * TL::RowM + mcol) * 2u, a[mi][0], a[mi][1], a[mi][2],
                                       a[mi][3]);
                 }
             }
 #pragma unroll
-            for (int nj = 0; nj < 2; ++nj) {
+            for (int nj = 0; nj < NJ; ++nj) {
                 if (B_K) {
                     const int nrow = wn0 + nj * 16 + lr + (li >> 1) * 8, kcol = kk + (li & 1) * 8;
-                    ldmatrix_x4(sB(st) + (uint32_t)(nrow * kBwRowK + kcol) * 2u, b[nj][0], b[nj][1], b[nj][2], b[nj][3]);
+                    ldmatrix_x4(sB(st) + (uint32_t)(nrow * TL::RowK + kcol) * 2u, b[nj][0], b[nj][1], b[nj][2], b[nj][3]);
                 } else {
                     const int krow = kk + lr + (li & 1) * 8, ncol = wn0 + nj * 16 + (li >> 1) * 8;
-                    ldmatrix_x4_trans(sB(st) + (uint32_t)(krow * kBwRowMN + ncol) * 2u, b[nj][0], b[nj][1], b[nj][2],
+                    ldmatrix_x4_trans(sB(st) + (uint32_t)(krow * TL::RowN + ncol) * 2u, b[nj][0], b[nj][1], b[nj][2],
                                       b[nj][3]);
                 }
             }
 #pragma unroll
             for (int mi = 0; mi < 4; ++mi)
 #pragma unroll
-                for (int ni = 0; ni < 4; ++ni)
+                for (int ni = 0; ni < NI; ++ni)
                     mma_bf16_16816(acc[mi][ni], a[mi][0], a[mi][1], a[mi][2], a[mi][3], b[ni >> 1][(ni & 1) * 2],
                                    b[ni >> 1][(ni & 1) * 2 + 1]);
         }
@@ -216,7 +233,7 @@ __global__ void __launch_bounds__(kBwThreads) bw_gemm_kernel(const BwGemm p) {
 #pragma unroll
     for (int mi = 0; mi < 4; ++mi)
 #pragma unroll
-        for (int ni = 0; ni < 4; ++ni) {
+        for (int ni = 0; ni < NI; ++ni) {
             const int col = n0 + wn0 + ni * 8 + (lane & 3) * 2;
             if (col >= p.N) continue;
 #pragma unroll
@@ -494,11 +511,12 @@ bool bw_aligned(const void* p, size_t a) { return reinterpret_cast<uintptr_t>(p)
 
 template <bool A_K, bool B_K, bool KG>
 cudaError_t bw_gemm(const BwGemm& g, int grid_x, int grid_z, cudaStream_t s) {
-    cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(bw_gemm_kernel<A_K, B_K, KG>), kBwSmem);
+    auto kern = bw_gemm_kernel<A_K, B_K, KG, kBwBN, kBwBK, kBwStages>;
+    constexpr int smem = bw_smem_bytes<kBwBN, kBwBK, kBwStages>();
+    cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), smem);
     if (e != cudaSuccess) return e;
     if (grid_x < 1 || grid_z < 1) return cudaSuccess;
-    return launch_kernel(bw_gemm_kernel<A_K, B_K, KG>, dim3(grid_x, (g.N + kBwBN - 1) / kBwBN, grid_z),
-                         dim3(kBwThreads), kBwSmem, s, false, g);
+    return launch_kernel(kern, dim3(grid_x, (g.N + kBwBN - 1) / kBwBN, grid_z), dim3(kBwThreads), smem, s, false, g);
 }
 
 }  // namespace
