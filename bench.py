@@ -537,7 +537,7 @@ def measure(name, args, rank, world, device, peaks, with_e2e):
         R = p["T"] * cfg.k
         flops = 16 * R * cfg.D * cfg.I + 4 * p["T"] * cfg.E * cfg.D   # seven GEMMs
         tf = flops / (ms * 1e-3) / 1e12
-        res["backward"] = dict(ms_per_call=round(ms, 4), kernels=19, gemm_flops=flops, achieved_tflops=round(tf, 1),
+        res["backward"] = dict(ms_per_call=round(ms, 4), kernels=20, gemm_flops=flops, achieved_tflops=round(tf, 1),
                                frac_of_bf16=round(tf / peaks["bf16_tflops"], 4),
                                note="moe_backward, T=%d, E=%d, k=%d, I=%d: recompute g/u, z = W_down^T dy, "
                                     "dW_down, dX, dW_gate_up, dW_r, router dx (warp-MMA grouped GEMMs)" % (

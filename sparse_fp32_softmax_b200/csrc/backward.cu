@@ -246,8 +246,11 @@ __global__ void __launch_bounds__(kBwThreads) bw_gemm_kernel(const BwGemm p) {
         }
 }
 
-// First 128-row tile of each group: tile_start[g] = sum_{g' < g} ceil(cnt[g'] / 128).
-__global__ void bw_tile_table_kernel(const int* __restrict__ cnt, int groups, int* __restrict__ tile_start) {
+// First 128-row tile of each group: tile_start[g] = sum_{g' < g} ceil(cnt[g'] / 128); and the
+// S token slices of the router-weight gradient: slices[s] = floor(s T / S), slices[S + s] =
+// its row count.
+__global__ void bw_tile_table_kernel(const int* __restrict__ cnt, int groups, int* __restrict__ tile_start, int T,
+                                     int S, int* __restrict__ slices) {
     if (threadIdx.x == 0) {
         int acc = 0;
         for (int g = 0; g < groups; ++g) {
@@ -255,6 +258,24 @@ __global__ void bw_tile_table_kernel(const int* __restrict__ cnt, int groups, in
             acc += (cnt[g] + kBwBM - 1) / kBwBM;
         }
         tile_start[groups] = acc;
+        for (int q = 0; q < S; ++q) {
+            const int a = (int)((long long)q * T / S), b = (int)((long long)(q + 1) * T / S);
+            slices[q] = a;
+            slices[S + q] = b - a;
+        }
+    }
+}
+
+// out[i] = sum_s part[s][i] in slice order (the router-weight gradient's K slices).
+__global__ void bw_slice_sum_kernel(const float* __restrict__ part, int S, long long n, float* __restrict__ out) {
+    for (long long i = 4 * (blockIdx.x * (long long)blockDim.x + threadIdx.x); i < n;
+         i += 4 * (long long)gridDim.x * blockDim.x) {
+        float4 acc = *reinterpret_cast<const float4*>(part + i);
+        for (int q = 1; q < S; ++q) {
+            const float4 v = *reinterpret_cast<const float4*>(part + (long long)q * n + i);
+            acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+        }
+        *reinterpret_cast<float4*>(out + i) = acc;
     }
 }
 
@@ -456,10 +477,14 @@ namespace {
 // Workspace of moe_backward: the forward's workspace (router and permutation scratch, and
 // the device error word at its start), then the backward's own buffers.  R = T k rows.
 struct BwPlan {
-    size_t sub, sub_bytes, logits, idx, w, counts, offsets, tiles, row_token, slot_row, row_w, dw_row, xp, dyp, gu, z,
-        h, dgu, dout, dxr_rows, dlog, dl16, dxr, total;
-    int R, Epad;
+    size_t sub, sub_bytes, logits, idx, w, counts, offsets, tiles, slices, row_token, slot_row, row_w, dw_row, xp, dyp,
+        gu, z, h, dgu, dout, dxr_rows, dlog, dl16, dxr, dwr_part, total;
+    int R, Epad, S;
 };
+
+// Token slices of the router-weight gradient dW_r = dl^T x (its K is T): one per 512 tokens,
+// at most 16, a function of T only (so the summation order does not depend on the GPU).
+inline int bw_router_slices(int T) { return std::max(1, std::min(16, T / 512)); }
 
 size_t bw_align(size_t v) { return (v + 255) / 256 * 256; }
 
@@ -467,6 +492,7 @@ BwPlan bw_plan(const moe_dims& d, size_t sub_bytes) {
     BwPlan p;
     p.R = d.T * d.k;
     p.Epad = (d.E + 7) / 8 * 8;
+    p.S = bw_router_slices(d.T);
     const size_t T = d.T, D = d.D, E = d.E, k = d.k, I = d.I, R = p.R;
     size_t off = 0;
     auto take = [&](size_t bytes) {
@@ -482,6 +508,7 @@ BwPlan bw_plan(const moe_dims& d, size_t sub_bytes) {
     p.counts = take(E * 4);
     p.offsets = take((E + 1) * 4);
     p.tiles = take((E + 1) * 4);
+    p.slices = take((size_t)2 * p.S * 4);
     p.row_token = take(R * 4);
     p.slot_row = take(R * 4);
     p.row_w = take(R * 4);
@@ -497,6 +524,7 @@ BwPlan bw_plan(const moe_dims& d, size_t sub_bytes) {
     p.dlog = take(T * E * 4);
     p.dl16 = take(T * p.Epad * 2);
     p.dxr = take(T * D * 4);
+    p.dwr_part = take(p.S > 1 ? (size_t)p.S * E * D * 4 : 0);
     p.total = off;
     return p;
 }
@@ -522,7 +550,7 @@ cudaError_t bw_gemm(const BwGemm& g, int grid_x, int grid_z, cudaStream_t s) {
 }  // namespace
 
 extern "C" size_t moe_backward_workspace_size(const moe_dims* dims) {
-    if (!dims || dims->tile_m < 1) return 0;
+    if (!dims) return 0;
     const moe_dims f = bw_dims(dims);
     const size_t sub = moe_workspace_size(&f, nullptr);
     if (sub == 0) return 0;
@@ -581,7 +609,10 @@ extern "C" moe_status moe_backward(const moe_bf16* x, const moe_bf16* W_r, const
     cudaError_t e = launch_gather_rows(dy16, row_token, R, D, H(P.dyp), false, s);
     const int sms = device_sm_count();
     const int wblocks = sms * 8;   // warp-per-item kernels: 8 warps per block
-    if (e == cudaSuccess) e = launch_kernel(bw_tile_table_kernel, dim3(1), dim3(32), 0, s, false, (const int*)counts, E, tiles);
+    int32_t* slices = Iw(P.slices);
+    if (e == cudaSuccess)
+        e = launch_kernel(bw_tile_table_kernel, dim3(1), dim3(32), 0, s, false, (const int*)counts, E, tiles, T, P.S,
+                          slices);
     if (e == cudaSuccess)
         e = launch_kernel(bw_row_weight_kernel, dim3(std::min(wblocks, (T + 7) / 8)), dim3(256), 0, s, false,
                           (const float*)logits, topk_idx, (const int32_t*)slot_row, T, E, k, norm, R, F(P.row_w));
@@ -623,10 +654,18 @@ extern "C" moe_status moe_backward(const moe_bf16* x, const moe_bf16* W_r, const
         e = launch_kernel(bw_route_kernel, dim3(std::min(wblocks, (T + 7) / 8)), dim3(256), 0, s, false,
                           (const float*)logits, topk_idx, (const int32_t*)slot_row, (const float*)F(P.dw_row),
                           dlogits_add, T, E, k, norm, R, P.Epad, dlog, H(P.dl16), dw);
-    // dW_r = dl^T x  (one group of T rows)
+    // dW_r = dl^T x: S token slices as K groups, then their sum in slice order
     if (e == cudaSuccess) {
-        BwGemm g{H(P.dl16), P.Epad, 0, x16, D, 0, dW_r, D, 0, E, D, T, P.Epad, 0, 1, nullptr, nullptr, nullptr};
-        e = bw_gemm<false, false, true>(g, (E + kBwBM - 1) / kBwBM, 1, s);
+        float* dst = P.S > 1 ? F(P.dwr_part) : dW_r;
+        BwGemm g{H(P.dl16), P.Epad, 0, x16, D, 0, dst, D, (long long)E * D, E, D, T, P.Epad, 0, P.S, slices,
+                 slices + P.S, nullptr};
+        e = bw_gemm<false, false, true>(g, (E + kBwBM - 1) / kBwBM, P.S, s);
+        if (e == cudaSuccess && P.S > 1) {
+            const long long n = (long long)E * D;
+            const int blocks = (int)std::min<long long>((n / 4 + 255) / 256, (long long)sms * 8);
+            e = launch_kernel(bw_slice_sum_kernel, dim3(blocks), dim3(256), 0, s, false, (const float*)F(P.dwr_part),
+                              P.S, n, dW_r);
+        }
     }
     // dx (router part) = dl W_r
     if (e == cudaSuccess) {
