@@ -134,3 +134,15 @@ def test_backward_bad_index_is_reported():
     torch.cuda.synchronize()
     assert B.moe_get_device_status(ws) == B.MOE_ERR_INVALID_ARG
     assert torch.ones(4, device="cuda").sum().item() == 4.0
+
+
+def test_backward_keras_shape_unpadded_E():
+    """E=60 (not a multiple of 8: the logit-gradient operand is zero-padded to 64 columns and
+    W_r's rows beyond 60 are not read), k=4, I=1408 (22 tiles of 2I), 40 tokens."""
+    run_case("keras", T=40)
+
+
+@pytest.mark.parametrize("T", [1, 3])
+def test_backward_one_and_three_tokens(T):
+    """T=1 and a ragged T=3 at the D=2048, E=128, k=8, I=768 layer: one row per chosen expert."""
+    run_case("decode", T=T)
