@@ -17,9 +17,11 @@
 // Work: the forward's router and a stable permutation (tile_m = 1) of the given routing,
 // permuted copies of x and dy, then seven grouped bf16 GEMMs with FP32 accumulation on warp
 // MMAs (m16n8k16, operands staged in shared memory by cp.async, ldmatrix with or without
-// transpose for each operand's major-ness) and four small FP32 kernels.  Every sum runs in a
-// fixed order: results are bitwise reproducible.  GEMM operands that the backward computes
-// (h, dg/du, w dy, dl) are rounded to bf16 once; all outputs are FP32.
+// transpose for each operand's major-ness) and small FP32 kernels: the tile and slice tables,
+// routing weights per row, the SwiGLU backward, the routing backward, the bias gradient, the
+// router-weight gradient's slice sum and the dx sum.  Every sum runs in a fixed order that
+// depends only on the shapes: results are bitwise reproducible.  GEMM operands that the
+// backward computes (h, dg/du, w dy, dl) are rounded to bf16 once; all outputs are FP32.
 #include <algorithm>
 
 #include "../../include/moe_b200.h"
