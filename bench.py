@@ -545,47 +545,51 @@ def measure(name, args, rank, world, device, peaks, with_e2e):
         del bw_ws
 
     # end to end through the public API with host buffers (eager, copies inside the region):
-    # each pass's input goes up on one copy stream and its output comes back on another, so
-    # the copies of one pass overlap the other passes' forwards, as a pipelining caller's do;
-    # events order every buffer's reuse from one step to the next
+    # each pass's input goes up on one copy stream and its output comes back on another, and
+    # consecutive steps alternate between two sets of device buffers, so copies overlap the
+    # other passes' and the neighbouring steps' forwards, as a pipelining caller's do; events
+    # order every buffer's reuse
     if with_e2e and not chain:
         hx = [p["x"].cpu().pin_memory() for p in passes]
         hy = [torch.empty(p["out"].shape, dtype=p["out"].dtype).pin_memory() for p in passes]
-        dx = [torch.empty_like(p["x"]) for p in passes]
+        NB = 2
+        dx = [[torch.empty_like(p["x"]) for p in passes] for _ in range(NB)]
+        dout = [[torch.empty_like(p["out"]) for p in passes] for _ in range(NB)]
         main = torch.cuda.current_stream()
         up, down = torch.cuda.Stream(device=device), torch.cuda.Stream(device=device)
-        in_ready = [torch.cuda.Event() for _ in passes]
-        fwd_done = [torch.cuda.Event() for _ in passes]
-        out_read = [torch.cuda.Event() for _ in passes]
+        in_ready = [[torch.cuda.Event() for _ in passes] for _ in range(NB)]
+        fwd_done = [[torch.cuda.Event() for _ in passes] for _ in range(NB)]
+        out_read = [[torch.cuda.Event() for _ in passes] for _ in range(NB)]
 
-        def e2e_step():
+        def e2e_step(b):
             for n in range(len(passes)):
                 with torch.cuda.stream(up):
-                    up.wait_event(fwd_done[n])       # the previous step's forward n read dx[n]
-                    dx[n].copy_(hx[n], non_blocking=True)
-                    in_ready[n].record(up)
+                    up.wait_event(fwd_done[b][n])    # the forward that last read dx[b][n]
+                    dx[b][n].copy_(hx[n], non_blocking=True)
+                    in_ready[b][n].record(up)
             for n, p in enumerate(passes):
-                main.wait_event(in_ready[n])
-                main.wait_event(out_read[n])         # the previous step's copy of out n is done
+                main.wait_event(in_ready[b][n])
+                main.wait_event(out_read[b][n])      # the last copy back of out[b][n] is done
                 w = p["w"]
-                B.moe_forward_ex(dx[n], w["W_r"], w["W_gate_up"], w["W_down"], cfg.k, cfg.norm_topk_prob,
-                                 out=p["out"], ws=p["ws"], opts=p["opts"])
-                fwd_done[n].record(main)
+                B.moe_forward_ex(dx[b][n], w["W_r"], w["W_gate_up"], w["W_down"], cfg.k, cfg.norm_topk_prob,
+                                 out=dout[b][n], ws=p["ws"], opts=p["opts"])
+                fwd_done[b][n].record(main)
                 with torch.cuda.stream(down):
-                    down.wait_event(fwd_done[n])
-                    hy[n].copy_(p["out"], non_blocking=True)
-                    out_read[n].record(down)
+                    down.wait_event(fwd_done[b][n])
+                    hy[n].copy_(dout[b][n], non_blocking=True)
+                    out_read[b][n].record(down)
 
-        for _ in range(max(1, args.warmup)):
-            e2e_step()
+        for i in range(max(1, args.warmup)):
+            e2e_step(i % NB)
         torch.cuda.synchronize()
         s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         s0.record(main)
         up.wait_event(s0)                            # no copy starts before the region
-        for _ in range(K):
-            e2e_step()
-        for ev in out_read:                          # ... and the region ends after the last one
-            main.wait_event(ev)
+        for i in range(K):
+            e2e_step(i % NB)
+        for evs_b in out_read:                       # ... and the region ends after the last one
+            for ev in evs_b:
+                main.wait_event(ev)
         s1.record(main)
         torch.cuda.synchronize()
         e_ms = s0.elapsed_time(s1)
@@ -596,7 +600,8 @@ def measure(name, args, rank, world, device, peaks, with_e2e):
         bytes_in = sum(p["x"].numel() * 2 for p in passes)
         res["e2e"] = dict(value=round(world * tokens_per_step * K / (e_ms / 1e3), 1), unit="tokens/s",
                           h2d_bytes_per_step=bytes_in, d2h_bytes_per_step=bytes_in,
-                          timing="eager; copies on two copy streams, overlapping other passes' forwards")
+                          timing="eager; copies on two copy streams and two buffer sets, overlapping "
+                                 "other passes' and neighbouring steps' forwards")
     del passes, W, x0, evs
     torch.cuda.synchronize()
     torch.cuda.empty_cache()
