@@ -191,7 +191,9 @@ moe_status moe_aux_loss(const float *logits, const int32_t *topk_idx, int T, int
  * dlogits are rounded to bf16 once as GEMM operands; all sums run in a fixed order (bitwise
  * reproducible).  No shared expert.  Shapes as for moe_forward (dims->tile_m is ignored);
  * 16-byte aligned bf16/FP32 matrices, workspace of moe_backward_workspace_size(dims) bytes,
- * 256-byte aligned.  Enqueued on `stream`. */
+ * 256-byte aligned.  Enqueued on `stream`; allocates and synchronises nothing, so a call can
+ * be captured in a CUDA graph once the same shape has run eagerly (the first call of a shape
+ * sets kernel attributes). */
 size_t moe_backward_workspace_size(const moe_dims *dims);
 moe_status moe_backward(const moe_bf16 *x, const moe_bf16 *W_r, const float *bias,
                         const moe_bf16 *W_gate_up, const moe_bf16 *W_down, const moe_bf16 *dy,

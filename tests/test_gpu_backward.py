@@ -146,3 +146,27 @@ def test_backward_keras_shape_unpadded_E():
 def test_backward_one_and_three_tokens(T):
     """T=1 and a ragged T=3 at the D=2048, E=128, k=8, I=768 layer: one row per chosen expert."""
     run_case("decode", T=T)
+
+
+def test_backward_captured_in_a_cuda_graph():
+    """moe_backward allocates and synchronises nothing, so it can be captured in a CUDA graph
+    (after one eager call on the same shape); the replay is bitwise equal to the eager call."""
+    cfg, L, G = layer("tiny", 1024)
+    dy = inputs.upstream_grad(cfg, 1024).cuda()
+    _, idx, _ = O.route(L["x"], L["W_r"], cfg.k, True)
+    idx = torch.from_numpy(idx).cuda()
+    import ctypes
+    dims = B.make_dims(1024, cfg.D, cfg.E, cfg.k, cfg.I, True)
+    ws = torch.empty(int(B.load().moe_backward_workspace_size(ctypes.byref(dims))), dtype=torch.uint8, device="cuda")
+    eager = B.moe_backward(G["x"], G["W_r"], G["W_gate_up"], G["W_down"], dy, idx, True, ws=ws)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    with torch.cuda.graph(g, stream=s):
+        captured = B.moe_backward(G["x"], G["W_r"], G["W_gate_up"], G["W_down"], dy, idx, True, ws=ws)
+    g.replay()
+    torch.cuda.synchronize()
+    for key, v in eager.items():
+        if v is not None:
+            assert torch.equal(v, captured[key]), key
+    del g
